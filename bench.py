@@ -1,0 +1,354 @@
+#!/usr/bin/env python
+"""Benchmark of the fused ELMO classifier-head training step on B200.
+
+One step is one pass of the whole hot path (label preparation, X
+quantisation, logits and gradient, input gradient, weight gradient fused with
+the stochastic-rounding update) over one batch of synthetic input, through the
+C ABI of libelmo.  Default workload: the 3M-label FP8 head (L = 3,000,000,
+d = 768, B = 256, chunk 131,072, lr 0.1), shaped like the Amazon-3M result of
+"ELMO: Efficiency via Low-precision and Peak Memory Optimization in Large
+Output Spaces"; the data are synthetic (the dataset is not available).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl elmo|reference]
+                    [--workload NAME]
+
+Prints one JSON line (rank 0).  For N > 1 the ranks run independent replicas
+of the step (weak scaling, no collective on the data path); the time is the
+max over ranks.  `--impl reference` times the CPU oracle (a deliberately
+plain program) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused XMC head train step: label-rows/s, TFLOP/s and % roofline (1×B200)"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="elmo", choices=["elmo", "reference"])
+    p.add_argument("--workload", default="product3m_fp8")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the oracle sample")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                "sm_max_mhz": pk.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def step_costs(w):
+    """Algorithmic work of one step: flops of the three contractions and the
+    weight bytes that must cross HBM (read + write once)."""
+    s_w = 2 if w.dtype == "bf16" else 1
+    return {"flops": 6.0 * w.B * w.L * w.d, "w_bytes": 2.0 * w.L * w.d * s_w}
+
+
+def tensor_peak_tflops(peaks, dtype, sustained=True):
+    base = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    return base * (2.0 if dtype == "fp8" else 1.0)   # fp8 dense = 2 x bf16 dense (nominal ratio)
+
+
+def alu_peak_tflops(peaks):
+    # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
+    return 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+
+
+def cpu_baseline(w, W_rows_host, X, rowptr, cols, target_s):
+    """The oracle as it stands, on a bounded label sample of the same workload."""
+    import oracle
+    oracle.build()
+    nthreads = os.cpu_count() or 1
+    probe = min(w.L, 64)
+    t = time.perf_counter()
+    oracle.train_step(W_rows_host[:probe], X, rowptr, cols, w.lr, 0, 0, w.dtype, 0, probe, L=w.L, nthreads=nthreads)
+    per = (time.perf_counter() - t) / probe
+    n = int(max(probe, min(W_rows_host.shape[0], target_s / max(per, 1e-9))))
+    t = time.perf_counter()
+    oracle.train_step(W_rows_host[:n], X, rowptr, cols, w.lr, 0, 0, w.dtype, 0, n, L=w.L, nthreads=nthreads)
+    dt = time.perf_counter() - t
+    return {"value": n / dt, "unit": "label-rows/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"labels [0, {n}) of the {w.L}-label step (full B={w.B}, d={w.d}), {dt:.1f} s",
+            "tflops": 6.0 * w.B * n * w.d / dt / 1e12}
+
+
+def run_reference(args, w):
+    import oracle
+    from synthetic import make_labels, make_W_bf16, make_W_f32, make_X
+    oracle.build()
+    nthreads = os.cpu_count() or 1
+    X = make_X(w, 0)
+    rowptr, cols = make_labels(w, 0)
+    # sample size: about 5 s of oracle work per step
+    probe = 64
+    Wp = make_W_f32(w, rows=probe)
+    Wq = oracle.sr_round(Wp, "fp8", 0, 2**64 - 1) if w.dtype == "fp8" else make_W_bf16(w)[:probe]
+    t = time.perf_counter()
+    oracle.train_step(Wq, X, rowptr, cols, w.lr, 0, 0, w.dtype, 0, probe, L=w.L, nthreads=nthreads)
+    per = (time.perf_counter() - t) / probe
+    budget = max(30.0, 150.0 / max(1, args.steps + args.warmup))
+    n = int(max(probe, min(w.L, budget / 3 / max(per, 1e-9))))
+    Wf = make_W_f32(w, rows=n)
+    Wq = oracle.sr_round(Wf, "fp8", 0, 2**64 - 1) if w.dtype == "fp8" else oracle.rne_bf16(Wf)
+    for s in range(args.warmup):
+        oracle.train_step(Wq, make_X(w, s), *make_labels(w, s), w.lr, 0, s, w.dtype, 0, n, L=w.L, nthreads=nthreads)
+    t = time.perf_counter()
+    for s in range(args.warmup, args.warmup + args.steps):
+        oracle.train_step(Wq, make_X(w, s), *make_labels(w, s), w.lr, 0, s, w.dtype, 0, n, L=w.L, nthreads=nthreads)
+    dt = time.perf_counter() - t
+    value = n * args.steps / dt
+    line = {
+        "metric": METRIC, "value": value, "unit": "label-rows/s", "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "L": w.L, "d": w.d, "B": w.B, "w_dtype": w.dtype, "chunk": w.chunk,
+                   "sample_labels": n},
+        "cpu_baseline": {"value": value, "unit": "label-rows/s", "cores": nthreads, "kind": "oracle",
+                         "sample": f"labels [0, {n}) of each {w.L}-label step (full B={w.B}, d={w.d})"},
+        "e2e": {"value": value, "unit": "label-rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from synthetic import workload
+    w = workload(args.workload)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import precision_label_chunk_b200 as elmo
+    from synthetic import make_labels, make_X
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    costs = step_costs(w)
+
+    # model state: W resident in HBM, filled on the device (SR of N(0, 0.02^2))
+    wdt = torch.int16 if w.dtype == "bf16" else torch.uint8
+    W = torch.empty(w.L, w.d, dtype=wdt, device=dev)
+    head = elmo.elmo_init_head(W, w.dtype, fill=True, init_std=0.02, seed=0)
+    nsteps = args.warmup + args.steps
+    host_batches = []
+    for s in range(nsteps):
+        X = make_X(w, s)
+        rowptr, cols = make_labels(w, s)
+        host_batches.append((X, rowptr, cols))
+    dev_batches = [(torch.from_numpy(X.view(np.int16)).to(dev), torch.from_numpy(rp).to(dev),
+                    torch.from_numpy(cl).to(dev)) for X, rp, cl in host_batches]
+    dX = torch.empty(w.B, w.d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(s, batch):
+        Xd, rp, cl = batch
+        elmo.elmo_train_step_chunked(head, Xd, rp, cl, w.lr, w.chunk, 0, s, dX)
+
+    for s in range(args.warmup):
+        step(s, dev_batches[s])
+    elmo.elmo_sync_status(head)
+    torch.cuda.synchronize()
+
+    # ---------------------------------------------------------------- timed region
+    sampler = ClockSampler(local)
+    elmo.elmo_profile_reset(head)
+    elmo.elmo_profile_enable(head, True)
+    launches0 = elmo.elmo_launch_count(head)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for s in range(args.warmup, nsteps):
+        step(s, dev_batches[s])
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    elmo.elmo_profile_enable(head, False)
+    elmo.elmo_sync_status(head)
+    gpu_launches = elmo.elmo_launch_count(head) - launches0
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * w.L * args.steps / (ms / 1e3)
+
+    # per-class device time inside the timed region
+    classes = {}
+    for name in elmo.KERNEL_CLASSES:
+        t_ms, n = elmo.elmo_profile_read(head, name)
+        if n:
+            classes[name] = {"ms": t_ms, "launches": n}
+    elmo.elmo_profile_reset(head)
+
+    # roofline of the dominant kernel class
+    dominant = max(classes, key=lambda k: classes[k]["ms"]) if classes else None
+    roof = None
+    if dominant:
+        fl_per_step = {"logits_grad": 2.0, "input_grad": 2.0, "update": 2.0}.get(dominant, 0.0) * w.B * w.L * w.d
+        fused = os.environ.get("ELMO_FUSED_UPDATE_FLOPS")
+        if dominant == "update" and fused:
+            fl_per_step = float(fused) * w.B * w.L * w.d
+        achieved = fl_per_step * args.steps / (classes[dominant]["ms"] / 1e3) / 1e12
+        simt = elmo.kernel_path() == "simt" if hasattr(elmo, "kernel_path") else True
+        if simt:
+            peak, bound, unit, src = alu_peak_tflops(peaks), "alu", "TFLOP/s", "derived: 148 SM x 128 FMA x 2 x max clock"
+        else:
+            peak, bound, unit, src = tensor_peak_tflops(peaks, w.dtype), "tensor", "TFLOP/s", \
+                f"{peaks['source']} bf16 sustained x {'2 (fp8 nominal ratio)' if w.dtype == 'fp8' else '1'}"
+        roof = {"kernel": dominant, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": None, "peak_source": src,
+                "launches_per_step": classes[dominant]["launches"] / args.steps}
+
+    # the step against its own roofline (slower of tensor and HBM time)
+    t_tensor = costs["flops"] / (tensor_peak_tflops(peaks, w.dtype) * 1e12)
+    t_hbm = costs["w_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_tensor, t_hbm)
+    step_roof = {"t_roof_ms": t_roof * 1e3, "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+                 "frac": t_roof / (ms_per_step / 1e3), "tflops": costs["flops"] / (ms_per_step / 1e3) / 1e12,
+                 "peaks": f"{peaks['source']}: {tensor_peak_tflops(peaks, w.dtype):.0f} TFLOP/s "
+                          f"({w.dtype}, sustained), {peaks['hbm_gbs']:.0f} GB/s"}
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    pin = [(torch.from_numpy(X.view(np.int16)).pin_memory(), torch.from_numpy(rp).pin_memory(),
+            torch.from_numpy(cl).pin_memory()) for X, rp, cl in host_batches]
+    dX_host = torch.empty(w.B, w.d, dtype=torch.float32).pin_memory()
+    h2d = sum(X.numel() * 2 + rp.numel() * 4 + cl.numel() * 4 for X, rp, cl in pin[args.warmup:]) / args.steps
+    d2h = dX_host.numel() * 4
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(args.warmup, nsteps):
+        Xh, rph, clh = pin[s]
+        batch = (Xh.to(dev, non_blocking=True), rph.to(dev, non_blocking=True), clh.to(dev, non_blocking=True))
+        step(s, batch)
+        dX_host.copy_(dX, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e = {"value": world * w.L * args.steps / (ms_e2e / 1e3), "unit": "label-rows/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # ---------------------------------------------------------------- CPU oracle baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        Wh = W[: 200_000].cpu().numpy()
+        Wh = Wh.view(np.uint16) if w.dtype == "bf16" else Wh.view(np.uint8)
+        X, rp, cl = host_batches[0]
+        cpu = cpu_baseline(w, Wh, X, rp, cl, args.cpu_seconds)
+
+    peak_mem = torch.cuda.max_memory_allocated(dev) + elmo.elmo_head_workspace_bytes(head)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "label-rows/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8-e4m3" if w.dtype == "fp8" else "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "L": w.L, "d": w.d, "B": w.B, "w_dtype": w.dtype, "chunk": w.chunk,
+                       "lr": w.lr, "positives_per_sample": f"1+Poisson({w.lam})", "zipf_s": w.zipf_s,
+                       "l2": f"inputs larger than L2 (W = {costs['w_bytes'] / 2 / 1e9:.2f} GB per replica)",
+                       "parallelism": "replicas" if world > 1 else "single"},
+            "tflops": step_roof["tflops"], "step_roofline": step_roof, "roofline": roof,
+            "kernels": classes, "gpu_launches": gpu_launches, "e2e": e2e, "cpu_baseline": cpu,
+            "clocks": clocks, "peak_device_bytes": int(peak_mem),
+        }
+        print(json.dumps(line), flush=True)
+    head.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

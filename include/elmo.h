@@ -1,0 +1,230 @@
+/*
+ * elmo.h -- C ABI of the B200 (sm_100a) ELMO classifier-head library.
+ *
+ * What it computes: the training step and the prediction of the extreme
+ * multilabel classifier head of "ELMO: Efficiency via Low-precision and Peak
+ * Memory Optimization in Large Output Spaces" (Zhang, Ullah, Schultheis,
+ * Babbar, ICML 2025; arXiv 2510.11168).  The head W [L x d] is stored in pure
+ * BF16 or unscaled FP8 E4M3 with no FP32 master copy (abstract; atlas summary,
+ * "Approach" and "Surprising findings": E4M3 native range suffices) and is
+ * trained by momentum-free SGD with stochastic rounding, the classifier
+ * gradient fused with the update and the label axis processed in chunks
+ * ("Approach": gradient fusion and chunking to cut transient memory).
+ *
+ * Conventions for every call:
+ *   - Pointers named *_dev are device pointers owned by the caller; the
+ *     library only borrows them for the duration of the work it enqueues.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and is asynchronous: a call returns once the work is
+ *     enqueued.  Argument errors are reported synchronously; data errors found
+ *     by kernels (malformed label lists) and bounded-wait timeouts are written
+ *     to a device status word and surface from elmo_sync_status() or from the
+ *     next call on the same head.
+ *   - Return values are elmo_status codes; elmo_last_error() gives a message
+ *     (thread-local) for the most recent failure on the calling thread.
+ *   - Matrices are row-major and densely packed; every device pointer must be
+ *     16-byte aligned.
+ *   - There is no CPU fallback: on a machine without an sm_100 GPU the calls
+ *     return ELMO_ECUDA or ELMO_EUNSUPPORTED.
+ */
+#ifndef ELMO_H_
+#define ELMO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ELMO_BF16 = 0,      /* bfloat16 weights (8-bit exponent, 7-bit mantissa) */
+  ELMO_FP8_E4M3 = 1   /* OCP E4M3FN weights: max 448, no infinities, saturating */
+} elmo_dtype;
+
+typedef enum {
+  ELMO_OK = 0,
+  ELMO_EINVAL = 1,        /* bad argument: null pointer, shape, alignment, range */
+  ELMO_ENOMEM = 2,        /* workspace allocation failed */
+  ELMO_ECUDA = 3,         /* a CUDA runtime call failed (message has the CUDA error) */
+  ELMO_ETIMEOUT = 4,      /* a kernel's bounded wait ran out; results are invalid */
+  ELMO_EUNSUPPORTED = 5,  /* valid but beyond this build's limits (see each call) */
+  ELMO_EDATA = 6          /* malformed labels: CSR out of order or column out of [0, L) */
+} elmo_status;
+
+/* Opaque handle: a borrowed weight matrix plus the head's workspace. */
+typedef struct elmo_head elmo_head;
+
+/* Limits of this build. */
+#define ELMO_MAX_BATCH 256          /* B of a training step */
+#define ELMO_MAX_NNZ 32768          /* positive labels per training step */
+#define ELMO_MAX_LABELS (1LL << 24) /* L */
+#define ELMO_MAX_TOPK 64            /* k of a prediction */
+#define ELMO_MAX_PREDICT_BATCH 4096 /* B of a prediction */
+
+/*
+ * elmo_init_head -- wrap a caller-owned weight matrix in a head.
+ *
+ * Passage: the classifier head W of L labels and width d, stored in BF16 or in
+ * unscaled E4M3 (abstract; atlas summary "Approach", "Surprising findings").
+ *
+ *   out      : receives the new handle (host pointer).
+ *   W_dev    : device pointer to W [L x d], bf16 bits (dt = ELMO_BF16) or E4M3
+ *              codes (dt = ELMO_FP8_E4M3); row-major, label-major.  Borrowed
+ *              for the life of the head; updated in place by training steps.
+ *   L        : number of labels, 1 <= L < ELMO_MAX_LABELS.
+ *   d        : width, a multiple of 64 in [64, 4096].
+ *   fill     : 0 = keep W as is; 1 = overwrite W with SR(init_std * N(0,1)),
+ *              the normal draws and the rounding both from Philox4x32-10 keyed
+ *              by `seed` (normal draws use step 2^64-2, the rounding step
+ *              2^64-1; the normal transform is not bit-reproducible on a CPU).
+ *   stream   : stream for the fill.
+ * Allocates the head's workspace (device status word and label buckets);
+ * returns ELMO_ENOMEM if that fails.  Larger per-step buffers are allocated on
+ * first use (see elmo_train_step_chunked).
+ */
+elmo_status elmo_init_head(elmo_head** out, void* W_dev, int64_t L, int32_t d, elmo_dtype dt,
+                           int fill, float init_std, uint64_t seed, void* stream);
+
+/* Releases the workspace (synchronising the device first); W is untouched. */
+elmo_status elmo_head_destroy(elmo_head* h);
+
+/*
+ * elmo_train_step_chunked -- one fused SGD step of the head.
+ *
+ * Passage: atlas summary "Approach" (pure low-precision classifier trained by
+ * stochastic rounding without master weights, momentum dropped, "fusing
+ * classifier gradient computation with the SGD update", "chunking the label
+ * dimension to reduce transient memory"); the abstract (gradient fusion and
+ * chunking).  For every label chunk W_c it computes
+ *     Z   = X W_c^T                       (fp32 accumulation)
+ *     G   = sigmoid(Z) - Y                (Y = 1 at the positive labels)
+ *     dX += G W_c                         (OLD W_c, fp32)
+ *     W_c = SR(W_c - lr * G^T X)          (in place, stochastic rounding)
+ * without materialising Z, G or dW for all L labels.  In FP8 mode the tensor
+ * core operands are E4M3: X is quantised with a per-step power-of-two scale
+ * s_X = 2^floor(log2(448 / max|X|)) and G as E4M3(2^8 G); both scales are
+ * undone exactly in fp32.  In BF16 mode G is rounded to bf16 (RNE).
+ * SR of element (l, j) draws u from Philox4x32-10 with key `seed`, counter
+ * (idx >> 3, step), idx = l * d + j (16-bit draw: half idx & 1 of word
+ * (idx >> 1) & 3), and rounds to the upper grid neighbour iff u < f, f the
+ * fractional position between the neighbours.
+ *
+ *   X_dev      : bf16 [B x d] sample embeddings (device).
+ *   B          : 1 <= B <= ELMO_MAX_BATCH.
+ *   rowptr_dev : int32 [B + 1] CSR row pointers of the positive labels, rowptr[0] = 0.
+ *   cols_dev   : int32 [nnz] label ids in [0, L); order within a row free;
+ *                duplicates count once.
+ *   nnz        : number of entries, 0 <= nnz <= ELMO_MAX_NNZ; must equal rowptr[B].
+ *   lr         : learning rate (finite).
+ *   chunk      : labels per chunk, >= 1.  A scheduling knob only: W is bit-for-
+ *                bit independent of it; dX only up to fp32 summation order.
+ *   seed, step : the stochastic-rounding stream; step 2^64-2 and 2^64-1 are
+ *                reserved for the fill of elmo_init_head.
+ *   dX_dev     : fp32 [B x d] (device), overwritten with the input gradient.
+ * The transient per-chunk gradient buffer (min(chunk, 65536) x B operands) is
+ * allocated on the first call that needs it (cudaMalloc: call once before
+ * capturing the step in a CUDA graph).  A malformed CSR sets ELMO_EDATA in the
+ * status word; the step then skips the malformed entries and W is undefined.
+ */
+elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B,
+                                    const int32_t* rowptr_dev, const int32_t* cols_dev, int32_t nnz,
+                                    float lr, int64_t chunk, uint64_t seed, uint64_t step,
+                                    float* dX_dev, void* stream);
+
+/*
+ * elmo_forward_chunk -- inspection: the logits and gradient operands of the
+ * step for labels [l0, l1), exactly as elmo_train_step_chunked forms them
+ * (same operand preparation and kernels), without touching W.
+ *
+ *   Z_dev : fp32 [(l1 - l0) x B] logits, label-major (may be NULL).
+ *   G_dev : fp32 [(l1 - l0) x B] values of the rounded gradient operand (may be NULL).
+ * Other arguments as in elmo_train_step_chunked.
+ */
+elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B,
+                               const int32_t* rowptr_dev, const int32_t* cols_dev, int32_t nnz,
+                               int64_t l0, int64_t l1, float* Z_dev, float* G_dev, void* stream);
+
+/*
+ * elmo_topk_predict -- chunked top-k labels per sample.
+ *
+ * Passage: the P@k evaluation of the atlas summary ("Metrics: P@1 P@3 P@5")
+ * ranks labels by their logit; the label axis is processed in chunks as in
+ * training ("Approach").  Score of (b, l) is the fp32 fused multiply-add chain
+ * s = fma(x[b,j], w[l,j], s) over j = 0..d-1 from s = 0 with x the bf16 value
+ * of X (unquantised) and w the stored weight; labels are ranked by score
+ * descending, ties to the lower label index, NaN after every number.
+ *
+ *   X_dev     : bf16 [B x d] (device), 1 <= B <= ELMO_MAX_PREDICT_BATCH.
+ *   k         : 1 <= k <= min(L, ELMO_MAX_TOPK).
+ *   chunk     : labels per chunk (scheduling only; the result does not depend on it).
+ *   idx_dev   : int32 [B x k] label ids (device), best first.
+ *   score_dev : fp32 [B x k] their exact scores (device).
+ */
+elmo_status elmo_topk_predict(elmo_head* h, const void* X_dev, int32_t B, int32_t k, int64_t chunk,
+                              int32_t* idx_dev, float* score_dev, void* stream);
+
+/*
+ * elmo_sr_round -- standalone stochastic rounding.
+ *
+ * Passage: stochastic rounding of the classifier weights replaces FP32 master
+ * weights (abstract; atlas summary "Approach").  out[i] = SR(in[i]) with the
+ * draw of element index_base + i of stream (seed, step), as in the step.
+ * NaN -> canonical NaN (bf16 0x7FC0, E4M3 0x7F); E4M3: |v| >= 448 and +-inf ->
+ * +-448; bf16: finite |v| above the largest finite -> largest finite, +-inf
+ * kept.  Values on the grid are returned unchanged; -0 stays -0.
+ *
+ *   in_dev  : fp32 [n] (device);  out_dev : bf16 or E4M3 [n] (device).
+ *   n       : >= 0 (0 is a no-op).
+ */
+elmo_status elmo_sr_round(const float* in_dev, void* out_dev, int64_t n, elmo_dtype dt,
+                          uint64_t seed, uint64_t step, uint64_t index_base, void* stream);
+
+/*
+ * elmo_sr_draws -- the 16-bit uniform draws k (u = k / 2^16) that SR uses for
+ * elements index_base .. index_base + n - 1 of stream (seed, step), as uint16
+ * into out_dev [n] (device).  Philox4x32-10 of Salmon et al. (SC'11).
+ */
+elmo_status elmo_sr_draws(uint16_t* out_dev, int64_t n, uint64_t seed, uint64_t step,
+                          uint64_t index_base, void* stream);
+
+/*
+ * elmo_sync_status -- synchronise `stream` and return the head's device status
+ * word (ELMO_OK, ELMO_EDATA or ELMO_ETIMEOUT), clearing it.
+ */
+elmo_status elmo_sync_status(elmo_head* h, void* stream);
+
+/* Bytes of device workspace the head currently holds (for peak-memory reports). */
+elmo_status elmo_head_workspace_bytes(const elmo_head* h, size_t* bytes);
+
+/*
+ * Tracing.  When enabled, every kernel a head launches is bracketed by CUDA
+ * events recorded on its launch stream and filed under one of these classes;
+ * elmo_profile_read synchronises on the recorded events and returns the summed
+ * device time and the number of launches of a class since the last reset.
+ * elmo_launch_count counts every kernel launch of the head (tracing on or off).
+ */
+typedef enum {
+  ELMO_K_PREP = 0,        /* label sort / validation, X quantisation */
+  ELMO_K_LOGITS_GRAD = 1, /* Z = X W_c^T and G = sigmoid(Z) - Y for a label range */
+  ELMO_K_INPUT_GRAD = 2,  /* dX contributions of a label range */
+  ELMO_K_UPDATE = 3,      /* weight gradient fused with the SR update (and dX where fused) */
+  ELMO_K_TOPK_SCORE = 4,  /* top-k scoring of label segments */
+  ELMO_K_TOPK_MERGE = 5,  /* top-k merge / exact rescoring */
+  ELMO_K_OTHER = 6,       /* fill, clears */
+  ELMO_K_COUNT = 7
+} elmo_kernel_class;
+
+elmo_status elmo_profile_enable(elmo_head* h, int enable);
+elmo_status elmo_profile_reset(elmo_head* h);
+elmo_status elmo_profile_read(elmo_head* h, int kernel_class, double* ms_total, int64_t* launches);
+elmo_status elmo_launch_count(const elmo_head* h, int64_t* launches);
+
+/* Message of the most recent failure on the calling thread ("" if none). */
+const char* elmo_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ELMO_H_ */

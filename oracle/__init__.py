@@ -173,17 +173,20 @@ def fp8_x_scale(X) -> float:
 
 # ---------------------------------------------------------------- the step
 def train_step(W, X, rowptr, cols, lr, seed, step, dtype, l0=0, l1=None,
-               want_dx=True, want_zg=False, nthreads=0):
+               want_dx=True, want_zg=False, nthreads=0, L=None):
     """One step over labels [l0, l1).  W: [L, d] uint16 (bf16) or uint8 (E4M3)
     codes; X: [B, d] bf16 bits.  Returns dict(W=[l1-l0, d] codes, dX=[B, d] fp32
-    (contributions of those labels), Z/G=[l1-l0, B] fp32 when asked)."""
+    (contributions of those labels), Z/G=[l1-l0, B] fp32 when asked).
+    L: total label count when W holds only the rows [0, l1) of a larger head."""
     dt = _DT[dtype]
     W = _c(W, np.uint16 if dt == BF16 else np.uint8)
     X = _c(X, np.uint16)
-    L, d = W.shape
+    Lw, d = W.shape
+    L = Lw if L is None else L
     B = X.shape[0]
     assert X.shape[1] == d
-    l1 = L if l1 is None else l1
+    l1 = Lw if l1 is None else l1
+    assert l1 <= Lw
     rowptr, cols = _c(rowptr, np.int32), _c(cols, np.int32)
     Wout = np.zeros((l1 - l0, d), W.dtype)
     dX = np.zeros((B, d), np.float32) if want_dx else None

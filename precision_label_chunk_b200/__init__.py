@@ -1,0 +1,234 @@
+"""Python binding of libelmo, the B200 (sm_100a) ELMO classifier-head library.
+
+Argument marshalling only: every call below forwards device pointers of
+torch tensors and the current CUDA stream to the C ABI declared in
+include/elmo.h, whose kernels do all of the work.  There is no fallback: if
+libelmo.so is missing or cannot be loaded, importing the library functions
+raises.
+
+The names match the C entry points:
+  elmo_init_head, elmo_head_destroy, elmo_train_step_chunked,
+  elmo_forward_chunk, elmo_topk_predict, elmo_sr_round, elmo_sr_draws,
+  elmo_sync_status, elmo_head_workspace_bytes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "ElmoError", "Head", "BF16", "FP8_E4M3", "MAX_BATCH", "MAX_NNZ", "MAX_TOPK", "MAX_PREDICT_BATCH",
+    "library_path", "load", "elmo_init_head", "elmo_head_destroy", "elmo_train_step_chunked",
+    "elmo_forward_chunk", "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws",
+    "elmo_sync_status", "elmo_head_workspace_bytes", "elmo_profile_enable", "elmo_profile_reset",
+    "elmo_profile_read", "elmo_launch_count", "KERNEL_CLASSES",
+]
+
+BF16 = 0
+FP8_E4M3 = 1
+MAX_BATCH = 256
+MAX_NNZ = 32768
+MAX_TOPK = 64
+MAX_PREDICT_BATCH = 4096
+
+STATUS_NAMES = {0: "ELMO_OK", 1: "ELMO_EINVAL", 2: "ELMO_ENOMEM", 3: "ELMO_ECUDA", 4: "ELMO_ETIMEOUT",
+                5: "ELMO_EUNSUPPORTED", 6: "ELMO_EDATA"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+_lock = threading.Lock()
+
+
+class ElmoError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libelmo.so")
+
+
+def load():
+    """Load libelmo.so (built in-tree by __graft_entry__.build())."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise ImportError(f"libelmo.so not found at {path}; build it with "
+                                  "`python -m precision_label_chunk_b200._build`")
+            lib = ctypes.CDLL(path)
+            _declare(lib)
+            _lib = lib
+    return _lib
+
+
+def _declare(L):
+    P, i32, i64, u64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float
+    st = ctypes.c_int
+    L.elmo_last_error.restype = ctypes.c_char_p
+    L.elmo_init_head.argtypes = [ctypes.POINTER(P), P, i64, i32, ctypes.c_int, ctypes.c_int, f32, u64, P]
+    L.elmo_head_destroy.argtypes = [P]
+    L.elmo_train_step_chunked.argtypes = [P, P, i32, P, P, i32, f32, i64, u64, u64, P, P]
+    L.elmo_forward_chunk.argtypes = [P, P, i32, P, P, i32, i64, i64, P, P, P]
+    L.elmo_topk_predict.argtypes = [P, P, i32, i32, i64, P, P, P]
+    L.elmo_sr_round.argtypes = [P, P, i64, ctypes.c_int, u64, u64, u64, P]
+    L.elmo_sr_draws.argtypes = [P, i64, u64, u64, u64, P]
+    L.elmo_sync_status.argtypes = [P, P]
+    L.elmo_head_workspace_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+    L.elmo_profile_enable.argtypes = [P, ctypes.c_int]
+    L.elmo_profile_reset.argtypes = [P]
+    L.elmo_profile_read.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]
+    L.elmo_launch_count.argtypes = [P, ctypes.POINTER(i64)]
+    for name in ("elmo_profile_enable", "elmo_profile_reset", "elmo_profile_read", "elmo_launch_count","elmo_init_head", "elmo_head_destroy", "elmo_train_step_chunked", "elmo_forward_chunk",
+                 "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws", "elmo_sync_status",
+                 "elmo_head_workspace_bytes"):
+        getattr(L, name).restype = st
+
+
+def _check(rc: int):
+    if rc != 0:
+        msg = load().elmo_last_error().decode(errors="replace")
+        raise ElmoError(rc, msg)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(dtype) -> int:
+    if dtype in (BF16, "bf16", torch.bfloat16):
+        return BF16
+    if dtype in (FP8_E4M3, "fp8", "e4m3", torch.float8_e4m3fn):
+        return FP8_E4M3
+    raise ValueError(f"unknown dtype {dtype!r}")
+
+
+class Head:
+    """A borrowed weight matrix W [L, d] plus the library's workspace."""
+
+    def __init__(self, handle: ctypes.c_void_p, W: torch.Tensor, dtype: int):
+        self.handle = handle
+        self.W = W
+        self.dtype = dtype
+        self.L, self.d = W.shape
+
+    def close(self):
+        if self.handle:
+            _check(load().elmo_head_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def elmo_init_head(W: torch.Tensor, dtype=None, fill: bool = False, init_std: float = 0.02, seed: int = 0,
+                   stream=None) -> Head:
+    """W: [L, d] CUDA tensor (bfloat16, or float8_e4m3fn / uint8 codes)."""
+    if dtype is None:
+        dtype = BF16 if W.dtype in (torch.bfloat16, torch.int16) else FP8_E4M3
+    dt = _dt(dtype)
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [L, d]")
+    if W.element_size() != (2 if dt == BF16 else 1):
+        raise ValueError("W element size does not match dtype")
+    h = ctypes.c_void_p()
+    _check(load().elmo_init_head(ctypes.byref(h), _ptr(W), W.shape[0], W.shape[1], dt, int(bool(fill)),
+                                 float(init_std), int(seed) & (2**64 - 1), _stream(stream)))
+    return Head(h, W, dt)
+
+
+def elmo_head_destroy(head: Head):
+    head.close()
+
+
+def elmo_train_step_chunked(head: Head, X: torch.Tensor, rowptr: torch.Tensor, cols: torch.Tensor, lr: float,
+                            chunk: int, seed: int, step: int, dX: torch.Tensor, stream=None):
+    B = X.shape[0]
+    nnz = cols.numel()
+    _check(load().elmo_train_step_chunked(head.handle, _ptr(X), B, _ptr(rowptr), _ptr(cols) if nnz else None,
+                                          nnz, float(lr), int(chunk), int(seed) & (2**64 - 1),
+                                          int(step) & (2**64 - 1), _ptr(dX), _stream(stream)))
+
+
+def elmo_forward_chunk(head: Head, X: torch.Tensor, rowptr: torch.Tensor, cols: torch.Tensor, l0: int, l1: int,
+                       Z: torch.Tensor | None = None, G: torch.Tensor | None = None, stream=None):
+    nnz = cols.numel()
+    _check(load().elmo_forward_chunk(head.handle, _ptr(X), X.shape[0], _ptr(rowptr), _ptr(cols) if nnz else None,
+                                     nnz, int(l0), int(l1), _ptr(Z), _ptr(G), _stream(stream)))
+
+
+def elmo_topk_predict(head: Head, X: torch.Tensor, k: int, chunk: int, idx: torch.Tensor, score: torch.Tensor,
+                      stream=None):
+    _check(load().elmo_topk_predict(head.handle, _ptr(X), X.shape[0], int(k), int(chunk), _ptr(idx), _ptr(score),
+                                    _stream(stream)))
+
+
+def elmo_sr_round(inp: torch.Tensor, out: torch.Tensor, dtype, seed: int, step: int, index_base: int = 0,
+                  stream=None):
+    _check(load().elmo_sr_round(_ptr(inp), _ptr(out), inp.numel(), _dt(dtype), int(seed) & (2**64 - 1),
+                                int(step) & (2**64 - 1), int(index_base) & (2**64 - 1), _stream(stream)))
+
+
+def elmo_sr_draws(out: torch.Tensor, seed: int, step: int, index_base: int = 0, stream=None):
+    _check(load().elmo_sr_draws(_ptr(out), out.numel(), int(seed) & (2**64 - 1), int(step) & (2**64 - 1),
+                                int(index_base) & (2**64 - 1), _stream(stream)))
+
+
+def elmo_sync_status(head: Head, stream=None):
+    _check(load().elmo_sync_status(head.handle, _stream(stream)))
+
+
+KERNEL_CLASSES = {"prep": 0, "logits_grad": 1, "input_grad": 2, "update": 3, "topk_score": 4, "topk_merge": 5,
+                  "other": 6}
+
+
+def elmo_profile_enable(head: Head, enable: bool = True):
+    _check(load().elmo_profile_enable(head.handle, int(bool(enable))))
+
+
+def elmo_profile_reset(head: Head):
+    _check(load().elmo_profile_reset(head.handle))
+
+
+def elmo_profile_read(head: Head, kernel_class) -> tuple[float, int]:
+    """(summed device milliseconds, launches) of one kernel class since the last reset."""
+    cls = KERNEL_CLASSES[kernel_class] if isinstance(kernel_class, str) else int(kernel_class)
+    ms, n = ctypes.c_double(), ctypes.c_int64()
+    _check(load().elmo_profile_read(head.handle, cls, ctypes.byref(ms), ctypes.byref(n)))
+    return float(ms.value), int(n.value)
+
+
+def elmo_launch_count(head: Head) -> int:
+    n = ctypes.c_int64()
+    _check(load().elmo_launch_count(head.handle, ctypes.byref(n)))
+    return int(n.value)
+
+
+def elmo_head_workspace_bytes(head: Head) -> int:
+    n = ctypes.c_size_t()
+    _check(load().elmo_head_workspace_bytes(head.handle, ctypes.byref(n)))
+    return int(n.value)

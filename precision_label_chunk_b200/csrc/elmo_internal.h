@@ -1,0 +1,85 @@
+// elmo_internal.h -- host-side structures and kernel launchers of libelmo.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/elmo.h"
+
+struct elmo_prof_rec {
+  int cls;
+  cudaEvent_t start, stop;
+};
+
+struct elmo_head {
+  void* W = nullptr;           // borrowed [L x d] bf16 bits or E4M3 codes
+  int64_t L = 0;
+  int32_t d = 0;
+  elmo_dtype dt = ELMO_BF16;
+  int device = 0;
+  int num_sms = 0;
+  // workspace owned by the head
+  int32_t* status = nullptr;   // [4]: status code, first bad index, spare
+  uint32_t* keys = nullptr;    // [ELMO_MAX_NNZ] sorted (label << 8 | sample) positives
+  int32_t* nkeys = nullptr;    // [1] number of valid keys
+  float* xscale = nullptr;     // [2] s_X, 1/s_X (fp8 mode)
+  uint8_t* xq = nullptr;       // [ELMO_MAX_BATCH x d] E4M3 codes of X * s_X (fp8 mode)
+  void* gbuf = nullptr;        // per-chunk gradient operands
+  size_t gbuf_bytes = 0;
+  void* cand = nullptr;        // top-k candidates
+  size_t cand_bytes = 0;
+  size_t base_bytes = 0;       // bytes of the fixed part of the workspace
+  // tracing
+  bool prof = false;
+  std::vector<elmo_prof_rec> prof_recs;
+  std::vector<cudaEvent_t> prof_pool;
+  int64_t launches = 0;
+};
+
+namespace elmo {
+// Brackets the kernel launches of one class with events when tracing is on,
+// and counts launches.  `n` is the number of kernels launched inside.
+struct KernelScope {
+  elmo_head* h;
+  cudaStream_t s;
+  elmo_prof_rec rec{};
+  bool on;
+  KernelScope(elmo_head* h_, int cls, cudaStream_t s_, int n = 1);
+  ~KernelScope();
+};
+}  // namespace elmo
+
+namespace elmo {
+
+constexpr int kTileLabels = 128;        // labels per tensor-core tile
+constexpr int64_t kSubChunk = 65536;    // largest label range per pass (L2-resident G)
+
+// prep.cu
+cudaError_t launch_prep_labels(elmo_head* h, const int32_t* rowptr, const int32_t* cols, int32_t B,
+                               int32_t nnz, cudaStream_t s);
+cudaError_t launch_prep_x(elmo_head* h, const uint16_t* X, int32_t B, cudaStream_t s);
+
+// step_simt.cu -- reference-order kernels (first correct path)
+cudaError_t launch_grad_simt(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
+                             void* gbuf, float* Zout, float* Gout, cudaStream_t s);
+cudaError_t launch_dx_simt(const elmo_head* h, int32_t B, int64_t l0, int64_t l1, const void* gbuf,
+                           float* dX, cudaStream_t s);
+cudaError_t launch_update_simt(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
+                               const void* gbuf, float lr, uint64_t seed, uint64_t step, cudaStream_t s);
+
+// topk_simt.cu
+size_t topk_workspace_bytes(const elmo_head* h, int32_t B, int32_t k);
+cudaError_t launch_topk_simt(elmo_head* h, const uint16_t* X, int32_t B, int32_t k, int64_t chunk,
+                             int32_t* idx, float* score, cudaStream_t s);
+
+// sr.cu
+cudaError_t launch_sr_round(const float* in, void* out, int64_t n, elmo_dtype dt, uint64_t seed,
+                            uint64_t step, uint64_t base, cudaStream_t s);
+cudaError_t launch_sr_draws(uint16_t* out, int64_t n, uint64_t seed, uint64_t step, uint64_t base,
+                            cudaStream_t s);
+cudaError_t launch_fill(void* W, int64_t n, elmo_dtype dt, float std, uint64_t seed, cudaStream_t s);
+
+}  // namespace elmo

@@ -1,0 +1,122 @@
+// sr.cu -- standalone stochastic rounding, its random draws, and the head fill.
+//
+// Stochastic rounding replaces FP32 master weights for the ELMO classifier
+// ("ELMO: Efficiency via Low-precision and Peak Memory Optimization in Large
+// Output Spaces", abstract; atlas summary "Approach").  One thread serves one
+// Philox block, i.e. 8 consecutive elements of the stream.
+#include "elmo_common.cuh"
+#include "elmo_internal.h"
+
+namespace elmo {
+namespace {
+
+__global__ void __launch_bounds__(256) sr_round_kernel(const float* __restrict__ in, void* __restrict__ out,
+                                                       int64_t n, int dt, uint64_t seed, uint64_t step,
+                                                       uint64_t base) {
+  const uint64_t first_blk = base >> 3;
+  const uint64_t last_blk = (base + (uint64_t)n - 1) >> 3;
+  for (uint64_t q = first_blk + blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; q <= last_blk;
+       q += (uint64_t)gridDim.x * blockDim.x) {
+    const u32x4 r = sr_block(seed, step, q);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint64_t idx = q * 8 + e;
+      if (idx < base || idx >= base + (uint64_t)n) continue;
+      const uint32_t word = sr_word(r, e >> 1);
+      const uint32_t k = (e & 1) ? (word >> 16) : (word & 0xFFFFu);
+      const int64_t i = (int64_t)(idx - base);
+      const float v = in[i];
+      if (dt == ELMO_BF16) static_cast<uint16_t*>(out)[i] = sr_bf16(v, k);
+      else static_cast<uint8_t*>(out)[i] = sr_e4m3(v, k);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) sr_draws_kernel(uint16_t* __restrict__ out, int64_t n, uint64_t seed,
+                                                       uint64_t step, uint64_t base) {
+  const uint64_t first_blk = base >> 3;
+  const uint64_t last_blk = (base + (uint64_t)n - 1) >> 3;
+  for (uint64_t q = first_blk + blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; q <= last_blk;
+       q += (uint64_t)gridDim.x * blockDim.x) {
+    const u32x4 r = sr_block(seed, step, q);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint64_t idx = q * 8 + e;
+      if (idx < base || idx >= base + (uint64_t)n) continue;
+      const uint32_t word = sr_word(r, e >> 1);
+      out[idx - base] = (uint16_t)((e & 1) ? (word >> 16) : (word & 0xFFFFu));
+    }
+  }
+}
+
+// W[i] = SR(std * n_i): n_i standard normal by the Box-Muller transform of two
+// 32-bit Philox words (block i >> 2 of step 2^64-2 serves elements 4q..4q+3),
+// rounded with the SR draw of element i at step 2^64-1.
+__global__ void __launch_bounds__(256) fill_kernel(void* __restrict__ W, int64_t n, int dt, float std,
+                                                   uint64_t seed) {
+  const uint64_t nblk = ((uint64_t)n + 7) >> 3;
+  for (uint64_t q = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; q < nblk;
+       q += (uint64_t)gridDim.x * blockDim.x) {
+    float nv[8];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint64_t nb = q * 2 + h;
+      const u32x4 r = philox10((uint32_t)nb, (uint32_t)(nb >> 32), 0xFFFFFFFEu, 0xFFFFFFFFu,
+                               (uint32_t)seed, (uint32_t)(seed >> 32));
+      const uint32_t wd[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const float u1 = ((float)wd[2 * p] + 1.0f) * 2.3283064365386963e-10f;  // (0, 1]
+        const float u2 = (float)wd[2 * p + 1] * 2.3283064365386963e-10f;
+        const float rad = sqrtf(-2.0f * logf(fminf(u1, 1.0f)));
+        float sn, cs;
+        sincospif(2.0f * u2, &sn, &cs);
+        nv[h * 4 + 2 * p] = rad * cs;
+        nv[h * 4 + 2 * p + 1] = rad * sn;
+      }
+    }
+    const u32x4 r = sr_block(seed, ~0ull, q);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint64_t i = q * 8 + e;
+      if (i >= (uint64_t)n) break;
+      const uint32_t word = sr_word(r, e >> 1);
+      const uint32_t k = (e & 1) ? (word >> 16) : (word & 0xFFFFu);
+      const float v = std * nv[e];
+      if (dt == ELMO_BF16) static_cast<uint16_t*>(W)[i] = sr_bf16(v, k);
+      else static_cast<uint8_t*>(W)[i] = sr_e4m3(v, k);
+    }
+  }
+}
+
+int grid_for(uint64_t work, int per_block) {
+  uint64_t g = (work + per_block - 1) / per_block;
+  if (g > 148ull * 64) g = 148ull * 64;
+  return (int)(g > 0 ? g : 1);
+}
+
+}  // namespace
+
+cudaError_t launch_sr_round(const float* in, void* out, int64_t n, elmo_dtype dt, uint64_t seed,
+                            uint64_t step, uint64_t base, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const uint64_t blocks = (((base + n - 1) >> 3) - (base >> 3)) + 1;
+  sr_round_kernel<<<grid_for(blocks, 256), 256, 0, s>>>(in, out, n, (int)dt, seed, step, base);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sr_draws(uint16_t* out, int64_t n, uint64_t seed, uint64_t step, uint64_t base,
+                            cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const uint64_t blocks = (((base + n - 1) >> 3) - (base >> 3)) + 1;
+  sr_draws_kernel<<<grid_for(blocks, 256), 256, 0, s>>>(out, n, seed, step, base);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill(void* W, int64_t n, elmo_dtype dt, float std, uint64_t seed, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  fill_kernel<<<grid_for(((uint64_t)n + 7) >> 3, 256), 256, 0, s>>>(W, n, (int)dt, std, seed);
+  return cudaGetLastError();
+}
+
+}  // namespace elmo

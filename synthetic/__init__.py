@@ -91,10 +91,11 @@ def make_X(w: Workload, step: int) -> np.ndarray:
     return bf16_bits(x)
 
 
-def make_W_f32(w: Workload, std: float = 0.02) -> np.ndarray:
-    """W [L, d] ~ N(0, std^2) as fp32 (before any rounding to the storage grid)."""
+def make_W_f32(w: Workload, std: float = 0.02, rows: int | None = None) -> np.ndarray:
+    """W [L, d] ~ N(0, std^2) as fp32 (before any rounding to the storage grid).
+    rows: only the first `rows` label rows (the same values as the full draw)."""
     rng = np.random.default_rng([2000 + w.index])
-    out = rng.standard_normal((w.L, w.d), dtype=np.float32)
+    out = rng.standard_normal((w.L if rows is None else min(rows, w.L), w.d), dtype=np.float32)
     out *= np.float32(std)
     return out
 

@@ -1,0 +1,54 @@
+"""The C-ABI library loads and exports every entry point include/elmo.h declares."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "elmo.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(elmo_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for must in ["elmo_init_head", "elmo_train_step_chunked", "elmo_topk_predict", "elmo_sr_round",
+                 "elmo_head_destroy", "elmo_sync_status", "elmo_last_error"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    import precision_label_chunk_b200 as elmo
+    from precision_label_chunk_b200 import _build
+    _build.build()
+    lib = ctypes.CDLL(elmo.library_path())
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"libelmo.so does not export {name}"
+
+
+def test_header_compiles_as_c():
+    import shutil
+    import subprocess
+    import tempfile
+    gcc = shutil.which("gcc")
+    if not gcc:
+        pytest.skip("no C compiler")
+    with tempfile.TemporaryDirectory() as d:
+        src = os.path.join(d, "t.c")
+        open(src, "w").write('#include "elmo.h"\nint main(void) { return (int)ELMO_OK; }\n')
+        subprocess.check_call([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                               "-c", src, "-o", os.path.join(d, "t.o")])
+
+
+def test_binding_without_gpu_fails_loudly():
+    import torch
+    import precision_label_chunk_b200 as elmo
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    W = torch.zeros(128, 64, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, elmo.ElmoError)):
+        elmo.elmo_init_head(W, "bf16")

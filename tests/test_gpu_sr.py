@@ -1,0 +1,79 @@
+"""GPU stochastic rounding and its random draws are bit-exact with the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from tests.gpu_common import need_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _adversarial(dtype, rng):
+    import ml_dtypes
+    if dtype == "bf16":
+        g = np.arange(0, 0x7F80, dtype=np.uint16).view(ml_dtypes.bfloat16).astype(np.float32)
+        step = np.abs(np.diff(g.astype(np.float64)))
+        mids = (g[:-1].astype(np.float64) + step / 2).astype(np.float32)
+    else:
+        g = np.arange(0, 127, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float32)
+        mids = ((g[:-1].astype(np.float64) + g[1:]) / 2).astype(np.float32)
+    near = np.concatenate([np.nextafter(g, np.float32(np.inf)), np.nextafter(g, np.float32(0))])
+    special = np.array([0.0, -0.0, np.inf, -np.inf, np.nan, 448.0, 447.99, 448.01, 480.0, 1e30, 3.4e38,
+                        3.3895313892515355e38, 1e-45, -1e-45, 1e-39, 2.0 ** -10, 2.0 ** -9, 2.0 ** -6,
+                        2.0 ** -7 + 2.0 ** -12], np.float32)
+    x = np.concatenate([g, mids, near, special])
+    x = np.concatenate([x, -x])
+    rnd = (rng.standard_normal(1 << 20) * 0.05).astype(np.float32)
+    wide = (rng.random(1 << 18) * 2 - 1).astype(np.float32) * np.exp2(rng.integers(-140, 120, 1 << 18)).astype(np.float32)
+    return np.concatenate([x, rnd, wide]).astype(np.float32)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("seed,step,base", [(0, 0, 0), (0xDEADBEEF12345678, 2**63 + 5, 13), (7, 2**64 - 1, 2**40 + 3)])
+def test_sr_round_bit_exact(orc, dtype, seed, step, base):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    x = _adversarial(dtype, np.random.default_rng(seed & 0xFFFF))
+    ref = orc.sr_round(x, dtype, seed, step, base)
+    xd = torch.from_numpy(x).cuda()
+    out = torch.empty(x.size, dtype=torch.int16 if dtype == "bf16" else torch.uint8, device="cuda")
+    elmo.elmo_sr_round(xd, out, dtype, seed, step, base)
+    got = out.cpu().numpy().view(np.uint16 if dtype == "bf16" else np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, f"{bad.size} mismatches, first x={x[bad[:5]]} got={got[bad[:5]]} ref={ref[bad[:5]]}"
+
+
+def test_sr_round_large_random_bit_exact(orc):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    rng = np.random.default_rng(99)
+    x = (rng.standard_normal(10_000_000) * 0.03).astype(np.float32)
+    for dtype in ("bf16", "fp8"):
+        ref = orc.sr_round(x, dtype, 3, 11, 5)
+        out = torch.empty(x.size, dtype=torch.int16 if dtype == "bf16" else torch.uint8, device="cuda")
+        elmo.elmo_sr_round(torch.from_numpy(x).cuda(), out, dtype, 3, 11, 5)
+        got = out.cpu().numpy().view(np.uint16 if dtype == "bf16" else np.uint8)
+        assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("seed,step,base,n", [(0, 0, 0, 1000), (5, 9, 3, 4097), (2**64 - 1, 2**62, 2**50 + 7, 777)])
+def test_draws_bit_exact(orc, seed, step, base, n):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    out = torch.empty(n, dtype=torch.int16, device="cuda")
+    elmo.elmo_sr_draws(out, seed, step, base)
+    got = out.cpu().numpy().view(np.uint16).astype(np.uint32)
+    assert np.array_equal(got, orc.draw16(seed, step, base, n))
+
+
+def test_sr_round_empty_and_errors():
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    x = torch.zeros(0, device="cuda")
+    out = torch.zeros(0, dtype=torch.uint8, device="cuda")
+    elmo.elmo_sr_round(x, out, "fp8", 0, 0)          # n = 0 is a no-op
+    lib = elmo.load()
+    assert lib.elmo_sr_round(None, None, 5, 0, 0, 0, 0, None) == 1      # null pointers: EINVAL
+    assert lib.elmo_sr_round(None, None, -1, 0, 0, 0, 0, None) == 1     # n < 0: EINVAL
+    xd = torch.zeros(4, device="cuda")
+    assert lib.elmo_sr_round(xd.data_ptr(), out.data_ptr(), 4, 7, 0, 0, 0, None) == 1  # bad dtype

@@ -1,0 +1,164 @@
+"""The CUDA training step against the oracle (element-wise, seeded inputs)."""
+import numpy as np
+import pytest
+import torch
+
+from synthetic import make_labels, make_W_bf16, make_W_f32, make_X, workload
+from tests.gpu_common import need_gpu, run_step, to_dev_i32, to_dev_u16, w_to_dev, w_to_host
+from tests.parity import assert_rel_close, assert_weights_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(orc, w, step=0):
+    X = make_X(w, step)
+    rowptr, cols = make_labels(w, step)
+    if w.dtype == "bf16":
+        W = make_W_bf16(w)
+    else:
+        W = orc.sr_round(make_W_f32(w), "fp8", seed=0, step=2**64 - 1)
+    return W, X, rowptr, cols
+
+
+CASES = [
+    ("tiny", {}),                                   # B=32, d=64, L=4096 (the tiny workload)
+    ("tiny", {"dtype": "fp8"}),
+    ("tiny", {"L": 1000, "d": 128, "B": 17}),       # ragged label tail, odd B
+    ("tiny", {"L": 777, "d": 192, "B": 1, "dtype": "fp8"}),
+    ("text500k_bf16", {"L": 3000, "B": 256}),       # full width and batch, several tiles
+    ("product3m_fp8", {"L": 2500, "B": 256}),
+]
+
+
+@pytest.mark.parametrize("name,over", CASES)
+def test_step_matches_oracle(orc, name, over):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload(name, **over)
+    W, X, rowptr, cols = _inputs(orc, w)
+    chunk = min(w.chunk, 1024)
+    Wg, dXg = run_step(elmo, W, X, rowptr, cols, w.lr, chunk, 0, 0, w.dtype)
+    r = orc.train_step(W, X, rowptr, cols, w.lr, 0, 0, w.dtype)
+    assert_weights_close(Wg, r["W"], w.dtype, chunk_rows=chunk)
+    assert_rel_close(dXg, r["dX"], w.dtype, what="dX")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_forward_chunk_logits_and_gradients(orc, dtype):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("tiny", dtype=dtype, L=900, d=128, B=40)
+    W, X, rowptr, cols = _inputs(orc, w)
+    l0, l1 = 100, 900
+    Wd = w_to_dev(W, dtype)
+    h = elmo.elmo_init_head(Wd, dtype)
+    Z = torch.empty(l1 - l0, w.B, device="cuda")
+    G = torch.empty(l1 - l0, w.B, device="cuda")
+    elmo.elmo_forward_chunk(h, to_dev_u16(X), to_dev_i32(rowptr), to_dev_i32(cols), l0, l1, Z, G)
+    elmo.elmo_sync_status(h)
+    r = orc.train_step(W, X, rowptr, cols, 0.0, 0, 0, dtype, l0=l0, l1=l1, want_zg=True)
+    assert_rel_close(Z.cpu().numpy(), r["Z"], dtype, axis=None, what="Z")
+    # G is the rounded operand: where the logits agree it agrees to one operand ulp
+    g, go = G.cpu().numpy(), r["G"]
+    ulp = 2.0 ** -8 if dtype == "bf16" else 2.0 ** -4
+    assert np.all(np.abs(g - go) <= ulp * np.maximum(np.abs(go), 2.0 ** -6) + 1e-7)
+    assert np.mean(g == go) > 0.99
+    # W untouched
+    assert np.array_equal(w_to_host(Wd, dtype), W)
+    h.close()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_weights_independent_of_chunk(orc, dtype):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("tiny", dtype=dtype, L=1500, d=128, B=24)
+    W, X, rowptr, cols = _inputs(orc, w)
+    outs = [run_step(elmo, W, X, rowptr, cols, w.lr, c, 4, 9, dtype) for c in (1500, 512, 129, 64)]
+    for Wg, dXg in outs[1:]:
+        assert np.array_equal(Wg, outs[0][0])
+        assert np.allclose(dXg, outs[0][1], rtol=1e-4, atol=1e-5)
+
+
+def test_empty_labels_and_zero_lr(orc):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("tiny", L=600, d=64, B=8)
+    W, X, _, _ = _inputs(orc, w)
+    rowptr = np.zeros(w.B + 1, np.int32)
+    cols = np.zeros(0, np.int32)
+    Wg, dXg = run_step(elmo, W, X, rowptr, cols, 0.0, 256, 1, 1, "bf16")
+    vals = lambda a: (a.astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(vals(Wg), vals(W))
+    r = orc.train_step(W, X, rowptr, cols, 0.0, 1, 1, "bf16")
+    assert_rel_close(dXg, r["dX"], "bf16", what="dX")
+
+
+def test_malformed_labels_report_edata():
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    W = torch.zeros(256, 64, dtype=torch.bfloat16, device="cuda")
+    h = elmo.elmo_init_head(W, "bf16")
+    X = torch.zeros(2, 64, dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty(2, 64, device="cuda")
+    rowptr = torch.tensor([0, 1, 2], dtype=torch.int32, device="cuda")
+    cols = torch.tensor([3, 256], dtype=torch.int32, device="cuda")      # 256 is out of range
+    elmo.elmo_train_step_chunked(h, X, rowptr, cols, 0.1, 128, 0, 0, dX)
+    with pytest.raises(elmo.ElmoError) as ei:
+        elmo.elmo_sync_status(h)
+    assert ei.value.status == 6
+    elmo.elmo_sync_status(h)                      # cleared
+    bad_ptr = torch.tensor([0, 2, 1], dtype=torch.int32, device="cuda")
+    elmo.elmo_train_step_chunked(h, X, bad_ptr, cols, 0.1, 128, 0, 0, dX)
+    with pytest.raises(elmo.ElmoError):
+        elmo.elmo_sync_status(h)
+    with pytest.raises(elmo.ElmoError):       # B above the limit
+        elmo.elmo_train_step_chunked(h, torch.zeros(300, 64, dtype=torch.bfloat16, device="cuda"),
+                                     torch.zeros(301, dtype=torch.int32, device="cuda"), cols, 0.1, 128, 0, 0,
+                                     torch.empty(300, 64, device="cuda"))
+    h.close()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_multistep_teacher_forced(orc, dtype):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("tiny", dtype=dtype, L=1200, d=128, B=32)
+    W, _, _, _ = _inputs(orc, w)
+    Wd = w_to_dev(W, dtype)
+    h = elmo.elmo_init_head(Wd, dtype)
+    dX = torch.empty(w.B, w.d, device="cuda")
+    for s in range(4):
+        X = make_X(w, s)
+        rowptr, cols = make_labels(w, s)
+        W_before = w_to_host(Wd, dtype).copy()
+        elmo.elmo_train_step_chunked(h, to_dev_u16(X), to_dev_i32(rowptr), to_dev_i32(cols), w.lr, 512, 0, s, dX)
+        elmo.elmo_sync_status(h)
+        r = orc.train_step(W_before, X, rowptr, cols, w.lr, 0, s, dtype)
+        assert_weights_close(w_to_host(Wd, dtype), r["W"], dtype, chunk_rows=512)
+        assert_rel_close(dX.cpu().numpy(), r["dX"], dtype, what=f"dX step {s}")
+    h.close()
+
+
+def test_resume_is_exact(orc):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("tiny", dtype="fp8", L=700, d=128, B=16)
+    W, _, _, _ = _inputs(orc, w)
+
+    def run(Wstart, steps):
+        Wd = w_to_dev(Wstart, "fp8")
+        h = elmo.elmo_init_head(Wd, "fp8")
+        dX = torch.empty(w.B, w.d, device="cuda")
+        for s in steps:
+            rp, cl = make_labels(w, s)
+            elmo.elmo_train_step_chunked(h, to_dev_u16(make_X(w, s)), to_dev_i32(rp), to_dev_i32(cl), w.lr, 256, 3,
+                                         s, dX)
+        elmo.elmo_sync_status(h)
+        out = w_to_host(Wd, "fp8").copy()
+        h.close()
+        return out
+
+    straight = run(W, range(6))
+    half = run(W, range(3))
+    assert np.array_equal(run(half, range(3, 6)), straight)
