@@ -6,6 +6,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <new>
 #include <string>
 
@@ -39,6 +40,13 @@ elmo_status cuda_fail(cudaError_t e, const char* what) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Development switch: ELMO_STEP_SIMT=1 runs the CUDA-core kernels of the step
+// instead of the tensor-core ones (both on the GPU).
+bool use_simt() {
+  const char* v = getenv("ELMO_STEP_SIMT");
+  return v && v[0] == '1';
+}
 
 // Fails with the status word's code if an earlier kernel recorded one.
 // Reading it costs a synchronisation, so only elmo_sync_status does.
@@ -288,15 +296,20 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B, const
     ELMO_CUDA(elmo::launch_prep_labels(h, rowptr_dev, cols_dev, B, nnz, s), "prep_labels");
     if (h->dt == ELMO_FP8_E4M3) ELMO_CUDA(elmo::launch_prep_x(h, X, B, s), "prep_x");
   }
-  const size_t esz = h->dt == ELMO_BF16 ? 2 : 1;
-  const int64_t span = l1 - l0 < elmo::kSubChunk ? l1 - l0 : elmo::kSubChunk;
-  if ((st = ensure_gbuf(h, (size_t)span * B * esz)) != ELMO_OK) return st;
+  const bool fp8 = h->dt == ELMO_FP8_E4M3;
+  const size_t esz = fp8 ? 1 : 2;
+  const int32_t Bp = elmo::padded_batch(B, fp8);
+  const bool simt = use_simt();
+  const int64_t sub = simt ? elmo::kSubChunk : elmo::sub_chunk_labels(h->d, Bp, (int)esz);
+  const int64_t span = l1 - l0 < sub ? l1 - l0 : sub;
+  if ((st = ensure_gbuf(h, (size_t)span * Bp * esz)) != ELMO_OK) return st;
   for (int64_t a = l0; a < l1; a += span) {
     const int64_t e = a + span < l1 ? a + span : l1;
     elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
-    ELMO_CUDA(elmo::launch_grad_simt(h, X, B, a, e, h->gbuf, Z_dev ? Z_dev + (a - l0) * B : nullptr,
-                                     G_dev ? G_dev + (a - l0) * B : nullptr, s),
-              "grad");
+    float* Za = Z_dev ? Z_dev + (a - l0) * B : nullptr;
+    float* Ga = G_dev ? G_dev + (a - l0) * B : nullptr;
+    if (simt) ELMO_CUDA(elmo::launch_grad_simt(h, X, B, a, e, h->gbuf, Za, Ga, s), "grad");
+    else ELMO_CUDA(elmo::launch_logits_grad_tc(h, X, B, a, e, h->gbuf, Za, Ga, s), "logits_grad");
   }
   return ELMO_OK;
 }
@@ -320,25 +333,36 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
     ELMO_CUDA(elmo::launch_prep_labels(h, rowptr_dev, cols_dev, B, nnz, s), "prep_labels");
     if (h->dt == ELMO_FP8_E4M3) ELMO_CUDA(elmo::launch_prep_x(h, X, B, s), "prep_x");
   }
-  const size_t esz = h->dt == ELMO_BF16 ? 2 : 1;
-  const int64_t sub = chunk < elmo::kSubChunk ? chunk : elmo::kSubChunk;
+  const bool fp8 = h->dt == ELMO_FP8_E4M3;
+  const size_t esz = fp8 ? 1 : 2;
+  const int32_t Bp = elmo::padded_batch(B, fp8);
+  const bool simt = use_simt();
+  const int64_t sub_max = simt ? elmo::kSubChunk : elmo::sub_chunk_labels(h->d, Bp, (int)esz);
+  const int64_t sub = chunk < sub_max ? chunk : sub_max;
   const int64_t span = h->L < sub ? h->L : sub;
-  if ((st = ensure_gbuf(h, (size_t)span * B * esz)) != ELMO_OK) return st;
+  if ((st = ensure_gbuf(h, (size_t)span * Bp * esz)) != ELMO_OK) return st;
   for (int64_t c0 = 0; c0 < h->L; c0 += chunk) {
     const int64_t c1 = c0 + chunk < h->L ? c0 + chunk : h->L;
     for (int64_t a = c0; a < c1; a += span) {
       const int64_t e = a + span < c1 ? a + span : c1;
-      {
-        elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
-        ELMO_CUDA(elmo::launch_grad_simt(h, X, B, a, e, h->gbuf, nullptr, nullptr, s), "grad");
-      }
-      {
-        elmo::KernelScope ks(h, ELMO_K_INPUT_GRAD, s);
-        ELMO_CUDA(elmo::launch_dx_simt(h, B, a, e, h->gbuf, dX_dev, s), "dx");
-      }
-      {
+      if (simt) {
+        {
+          elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
+          ELMO_CUDA(elmo::launch_grad_simt(h, X, B, a, e, h->gbuf, nullptr, nullptr, s), "grad");
+        }
+        {
+          elmo::KernelScope ks(h, ELMO_K_INPUT_GRAD, s);
+          ELMO_CUDA(elmo::launch_dx_simt(h, B, a, e, h->gbuf, dX_dev, s), "dx");
+        }
         elmo::KernelScope ks(h, ELMO_K_UPDATE, s);
         ELMO_CUDA(elmo::launch_update_simt(h, X, B, a, e, h->gbuf, lr, seed, step, s), "update");
+      } else {
+        {
+          elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
+          ELMO_CUDA(elmo::launch_logits_grad_tc(h, X, B, a, e, h->gbuf, nullptr, nullptr, s), "logits_grad");
+        }
+        elmo::KernelScope ks(h, ELMO_K_UPDATE, s);
+        ELMO_CUDA(elmo::launch_update_tc(h, X, B, a, e, h->gbuf, lr, seed, step, dX_dev, s), "update");
       }
     }
   }

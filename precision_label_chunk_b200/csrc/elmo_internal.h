@@ -57,6 +57,15 @@ namespace elmo {
 constexpr int kTileLabels = 128;        // labels per tensor-core tile
 constexpr int64_t kSubChunk = 65536;    // largest label range per pass (L2-resident G)
 
+// Labels per pass of the tensor-core step: W and G of a pass (about 64 MB)
+// stay resident in the 126 MB L2 between the two kernels.
+inline int64_t sub_chunk_labels(int32_t d, int32_t Bp, int elem_bytes) {
+  const int64_t per_label = (int64_t)(d + Bp) * elem_bytes;
+  int64_t n = (int64_t(64) << 20) / per_label;
+  n = n / 128 * 128;
+  return n < 128 ? 128 : n;
+}
+
 // prep.cu
 cudaError_t launch_prep_labels(elmo_head* h, const int32_t* rowptr, const int32_t* cols, int32_t B,
                                int32_t nnz, cudaStream_t s);
@@ -69,6 +78,13 @@ cudaError_t launch_dx_simt(const elmo_head* h, int32_t B, int64_t l0, int64_t l1
                            float* dX, cudaStream_t s);
 cudaError_t launch_update_simt(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
                                const void* gbuf, float lr, uint64_t seed, uint64_t step, cudaStream_t s);
+
+// step_tc.cu -- tensor-core step
+int32_t padded_batch(int32_t B, bool fp8);
+cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
+                                  void* gbuf, float* Zout, float* Gout, cudaStream_t s);
+cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
+                             const void* gbuf, float lr, uint64_t seed, uint64_t step, float* dX, cudaStream_t s);
 
 // topk_simt.cu
 size_t topk_workspace_bytes(const elmo_head* h, int32_t B, int32_t k);
