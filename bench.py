@@ -43,6 +43,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="elmo", choices=["elmo", "reference"])
     p.add_argument("--workload", default="product3m_fp8")
+    p.add_argument("--labels", type=int, default=0, help="override L (smaller cases for profiling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the oracle sample")
     return p.parse_args()
@@ -182,7 +183,7 @@ def run_reference(args, w):
 def main():
     args = parse()
     from synthetic import workload
-    w = workload(args.workload)
+    w = workload(args.workload, **({"L": args.labels} if args.labels else {}))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -268,23 +269,23 @@ def main():
             classes[name] = {"ms": t_ms, "launches": n}
     elmo.elmo_profile_reset(head)
 
-    # roofline of the dominant kernel class
+    # roofline of the dominant kernel class: algorithmic flops of the
+    # contractions it performs per step (2 B L d each) over its device time
+    simt = os.environ.get("ELMO_STEP_SIMT", "0") == "1"
+    contractions = {"logits_grad": 1, "input_grad": 1, "update": 1 if simt else 2}
     dominant = max(classes, key=lambda k: classes[k]["ms"]) if classes else None
     roof = None
-    if dominant:
-        fl_per_step = {"logits_grad": 2.0, "input_grad": 2.0, "update": 2.0}.get(dominant, 0.0) * w.B * w.L * w.d
-        fused = os.environ.get("ELMO_FUSED_UPDATE_FLOPS")
-        if dominant == "update" and fused:
-            fl_per_step = float(fused) * w.B * w.L * w.d
+    if dominant in contractions:
+        fl_per_step = contractions[dominant] * 2.0 * w.B * w.L * w.d
         achieved = fl_per_step * args.steps / (classes[dominant]["ms"] / 1e3) / 1e12
-        simt = elmo.kernel_path() == "simt" if hasattr(elmo, "kernel_path") else True
         if simt:
-            peak, bound, unit, src = alu_peak_tflops(peaks), "alu", "TFLOP/s", "derived: 148 SM x 128 FMA x 2 x max clock"
+            peak, bound, src = alu_peak_tflops(peaks), "alu", "derived: 148 SM x 128 FMA x 2 x max clock"
         else:
-            peak, bound, unit, src = tensor_peak_tflops(peaks, w.dtype), "tensor", "TFLOP/s", \
-                f"{peaks['source']} bf16 sustained x {'2 (fp8 nominal ratio)' if w.dtype == 'fp8' else '1'}"
-        roof = {"kernel": dominant, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            peak, bound = tensor_peak_tflops(peaks, w.dtype), "tensor"
+            src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype == "fp8" else ""))
+        roof = {"kernel": dominant, "bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": None, "peak_source": src,
+                "flops_per_launch": fl_per_step / (classes[dominant]["launches"] / args.steps),
                 "launches_per_step": classes[dominant]["launches"] / args.steps}
 
     # the step against its own roofline (slower of tensor and HBM time)

@@ -7,6 +7,7 @@
 // Spaces", abstract; atlas summary "Approach").
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -27,10 +28,10 @@ __device__ __forceinline__ u32x4 philox10(uint32_t c0, uint32_t c1, uint32_t c2,
   constexpr uint32_t kWeyl0 = 0x9E3779B9u, kWeyl1 = 0xBB67AE85u;
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t hiA = __umulhi(kMulA, c0), loA = kMulA * c0;
-    const uint32_t hiB = __umulhi(kMulB, c2), loB = kMulB * c2;
-    const uint32_t n0 = hiB ^ c1 ^ k0, n2 = hiA ^ c3 ^ k1;
-    c0 = n0; c1 = loB; c2 = n2; c3 = loA;
+    const uint64_t pA = (uint64_t)kMulA * c0;   // one wide multiply gives both halves
+    const uint64_t pB = (uint64_t)kMulB * c2;
+    const uint32_t n0 = (uint32_t)(pB >> 32) ^ c1 ^ k0, n2 = (uint32_t)(pA >> 32) ^ c3 ^ k1;
+    c0 = n0; c1 = (uint32_t)pB; c2 = n2; c3 = (uint32_t)pA;
     k0 += kWeyl0; k1 += kWeyl1;
   }
   return {c0, c1, c2, c3};
@@ -86,42 +87,66 @@ __device__ __forceinline__ uint8_t f32_to_e4m3_rn(float v) {
 // the grid is kept; otherwise with neighbours lo < |v| < hi it returns hi iff
 // u < f = (|v| - lo) / (hi - lo), sign restored.
 //
-// bf16: the bf16 magnitude just below |v| is the top half of |v|'s bit
-// pattern and f * 2^16 is exactly the bottom half (the grid is uniform in the
-// pattern within a binade and across fp32 subnormals), so u < f is k < frac.
+// Both grids are handled by add-and-truncate on the fp32 bit pattern.  If the
+// pattern bits below the target precision hold the fraction F (in units of
+// 2^-n of a grid step), u < f  <=>  2^(n-16) k < F  <=>  adding
+// 2^n - 1 - 2^(n-16) k carries into the first kept bit.  bf16 keeps the top
+// 16 bits (n = 16, F exact).  E4M3 keeps 3 mantissa bits (n = 20) for
+// |v| >= 2^-6; below 2^-6 (the subnormal range, spacing 2^-9) |v| is first
+// moved into the binade [2^-6, 2^-5), whose spacing is also 2^-9, by adding
+// 2^-6 rounded toward +inf: that keeps ceil(F), and for an integer 2^4 k,
+// 2^4 k < F <=> 2^4 k < ceil(F), so the carry test stays exact; 2^-6 is
+// subtracted again exactly afterwards.
 __device__ __forceinline__ uint16_t sr_bf16(float v, uint32_t k) {
   const uint32_t b = __float_as_uint(v);
   const uint32_t mag = b & 0x7FFFFFFFu;
   const uint32_t sign = (b >> 16) & 0x8000u;
-  if (mag > 0x7F800000u) return 0x7FC0;            // NaN
-  uint32_t r = mag >> 16;
-  if (mag < 0x7F800000u) {
-    r += (k < (mag & 0xFFFFu)) ? 1u : 0u;
-    r = min(r, 0x7F7Fu);                            // never round a finite value to inf
-  }
-  return (uint16_t)(sign | r);
+  uint32_t r = min((mag + 0xFFFFu - k) >> 16, 0x7F7Fu);   // never round a finite value to inf
+  r = (mag >= 0x7F800000u) ? ((mag == 0x7F800000u) ? 0x7F80u : 0x7FC0u) : r;
+  return (uint16_t)((mag > 0x7F800000u) ? r : (sign | r));
 }
 
-// E4M3: with e' = max(floor(log2 |v|), -6) the grid spacing near |v| is
-// 2^(e'-3), so t = |v| * 2^(3-e') is exact, lo = floor(t) and f = t - lo are
-// exact, and the code is (e' + 6) * 8 + lo + [u < f] (lo runs 8..15 in a
-// normal binade, 0..7 below 2^-6; a carry to 16 moves to the next binade).
-__device__ __forceinline__ uint8_t sr_e4m3(float v, uint32_t k) {
+// The SR result as an fp32 value on the E4M3 grid (|v| >= 448 and inf are
+// left above 448 for the saturating conversion; NaN becomes +NaN).
+__device__ __forceinline__ float sr_e4m3_value(float v, uint32_t k) {
   const uint32_t b = __float_as_uint(v);
   const uint32_t mag = b & 0x7FFFFFFFu;
-  const uint8_t sign = (uint8_t)((b >> 24) & 0x80u);
-  if (mag > 0x7F800000u) return 0x7F;              // NaN
   const float a = __uint_as_float(mag);
-  if (a >= 448.0f) return sign | 0x7E;              // saturate (inf included)
-  const int eb = (int)(mag >> 23);                  // biased exponent (0 for fp32 subnormals)
-  const int e = max(eb - 127, -6);
-  const float scale = __uint_as_float((uint32_t)(130 - e) << 23);  // 2^(3 - e)
-  const float t = __fmul_rn(a, scale);
-  const float lo = truncf(t);
-  const float f = __fsub_rn(t, lo);
-  const float u = __fmul_rn((float)k, 1.52587890625e-05f);          // k * 2^-16, exact
-  const int code = (e + 6) * 8 + (int)lo + (u < f ? 1 : 0);
-  return sign | (uint8_t)code;
+  const float c = (a < 0.015625f) ? 0.015625f : 0.0f;       // 2^-6 below the normal range
+  const float s = __fadd_ru(a, c);
+  const uint32_t t = (__float_as_uint(s) + 0xFFFFFu - (k << 4)) & 0xFFF00000u;
+  const float r = __fsub_rn(__uint_as_float(t), c);
+  const float out = __uint_as_float(__float_as_uint(r) | (b & 0x80000000u));
+  return (mag > 0x7F800000u) ? __uint_as_float(0x7FC00000u) : out;
+}
+
+// Two fp32 values -> two E4M3 codes (hi in the upper byte), RNE + saturating.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float hi, float lo) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two fp32 values -> two bf16 (hi in the upper half), RNE.
+__device__ __forceinline__ uint32_t pack_bf16x2(float hi, float lo) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ uint8_t sr_e4m3(float v, uint32_t k) {
+  return (uint8_t)(pack_e4m3x2(0.0f, sr_e4m3_value(v, k)) & 0xFF);
+}
+
+// Four E4M3 codes (byte i = element i) -> fp32 values, exact.
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&o)[4]) {
+  uint32_t h01, h23;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"((uint16_t)(w & 0xFFFF)));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"((uint16_t)(w >> 16)));
+  o[0] = __half2float(__ushort_as_half((unsigned short)(h01 & 0xFFFF)));
+  o[1] = __half2float(__ushort_as_half((unsigned short)(h01 >> 16)));
+  o[2] = __half2float(__ushort_as_half((unsigned short)(h23 & 0xFFFF)));
+  o[3] = __half2float(__ushort_as_half((unsigned short)(h23 >> 16)));
 }
 
 }  // namespace elmo

@@ -25,6 +25,7 @@ struct elmo_head {
   int32_t* status = nullptr;   // [4]: status code, first bad index, spare
   uint32_t* keys = nullptr;    // [ELMO_MAX_NNZ] sorted (label << 8 | sample) positives
   int32_t* nkeys = nullptr;    // [1] number of valid keys
+  int32_t* tile_ptr = nullptr; // [ceil(L/128) + 1] first key of every 128-label tile
   float* xscale = nullptr;     // [2] s_X, 1/s_X (fp8 mode)
   uint8_t* xq = nullptr;       // [ELMO_MAX_BATCH x d] E4M3 codes of X * s_X (fp8 mode)
   void* gbuf = nullptr;        // per-chunk gradient operands

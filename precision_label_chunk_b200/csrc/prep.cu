@@ -31,21 +31,25 @@ __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t
                                                                    int32_t nnz, int64_t L, int32_t npow2,
                                                                    uint32_t* __restrict__ keys_out,
                                                                    int32_t* __restrict__ nkeys,
+                                                                   int32_t* __restrict__ tile_ptr,
                                                                    int32_t* __restrict__ status) {
   extern __shared__ uint32_t sk[];
   __shared__ int bad_rows;
   __shared__ int nvalid;
+  __shared__ int32_t rp[ELMO_MAX_BATCH + 1];
   const int tid = threadIdx.x;
-  if (tid == 0) {
-    bad_rows = (rowptr[0] != 0 || rowptr[B] != nnz) ? 1 : 0;
-    nvalid = 0;
-  }
+  for (int b = tid; b <= B; b += blockDim.x) rp[b] = rowptr[b];
+  if (tid == 0) nvalid = 0;
+  __syncthreads();
+  if (tid == 0) bad_rows = (rp[0] != 0 || rp[B] != nnz) ? 1 : 0;
   __syncthreads();
   for (int b = tid; b < B; b += blockDim.x)
-    if (rowptr[b + 1] < rowptr[b]) bad_rows = 1;
+    if (rp[b + 1] < rp[b]) bad_rows = 1;
   __syncthreads();
+  const int ntg = (int)((L + 127) >> 7);     // 128-label tiles of the head
   if (bad_rows) {
     if (tid == 0) { set_status(status, ELMO_EDATA, -1); *nkeys = 0; }
+    for (int g = tid; g <= ntg; g += blockDim.x) tile_ptr[g] = 0;
     return;
   }
   for (int i = tid; i < npow2; i += blockDim.x) {
@@ -54,7 +58,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t
       int lo = 0, hi = B;                     // sample b with rowptr[b] <= i < rowptr[b+1]
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (rowptr[mid] <= i) lo = mid; else hi = mid;
+        if (rp[mid] <= i) lo = mid; else hi = mid;
       }
       const int32_t c = cols[i];
       if (c >= 0 && (int64_t)c < L) key = ((uint32_t)c << 8) | (uint32_t)lo;
@@ -84,9 +88,21 @@ __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t
   }
   atomicAdd(&nvalid, cnt);
   __syncthreads();
-  if (tid == 0) *nkeys = nvalid;
+  const int nv = nvalid;
+  if (tid == 0) *nkeys = nv;
+  // tile_ptr[g] = first key whose label is in tile g or later (keys are label << 8 | sample)
+  for (int g = tid; g <= ntg; g += blockDim.x) {
+    int lo = 0, hi = nv;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((int)(sk[mid] >> 15) < g) lo = mid + 1; else hi = mid;
+    }
+    tile_ptr[g] = lo;
+  }
 }
 
+// One CTA: max |X| with 16-byte loads, the power-of-two scale, then the E4M3
+// codes of X * s_X (second pass mostly from L1/L2).  n is a multiple of 64.
 __global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __restrict__ X, int64_t n,
                                                               float* __restrict__ xscale,
                                                               uint8_t* __restrict__ xq) {
@@ -96,14 +112,21 @@ __global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __
   const int tid = threadIdx.x;
   if (tid == 0) nonfinite = 0;
   __syncthreads();
-  float m = 0.0f;
-  for (int64_t i = tid; i < n; i += blockDim.x) {
-    const float a = fabsf(bf16_to_f32(X[i]));
-    if (!(a <= 3.4028234663852886e38f)) nonfinite = 1;
-    else m = fmaxf(m, a);
+  const uint4* X4 = reinterpret_cast<const uint4*>(X);
+  const int64_t n8 = n / 8;
+  uint32_t mbits = 0;       // max of |x| bit patterns (monotone for non-negative floats)
+  for (int64_t i = tid; i < n8; i += blockDim.x) {
+    const uint4 v = X4[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t lo = (w[e] << 16) & 0x7FFFFFFFu, hi = w[e] & 0x7FFF0000u;
+      mbits = max(mbits, max(lo, hi));
+    }
   }
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  if ((tid & 31) == 0) red[tid >> 5] = m;
+  if (mbits >= 0x7F800000u) nonfinite = 1;
+  for (int o = 16; o > 0; o >>= 1) mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, o));
+  if ((tid & 31) == 0) red[tid >> 5] = __uint_as_float(mbits);
   __syncthreads();
   if (tid == 0) {
     float amax = 0.0f;
@@ -123,7 +146,19 @@ __global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __
   }
   __syncthreads();
   const float s = s_scale;
-  for (int64_t i = tid; i < n; i += blockDim.x) xq[i] = f32_to_e4m3_rn(__fmul_rn(bf16_to_f32(X[i]), s));
+  uint2* Q2 = reinterpret_cast<uint2*>(xq);
+  for (int64_t i = tid; i < n8; i += blockDim.x) {
+    const uint4 v = X4[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t q[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float x0 = __fmul_rn(__uint_as_float(w[2 * h] << 16), s), x1 = __fmul_rn(__uint_as_float(w[2 * h] & 0xFFFF0000u), s);
+      const float x2 = __fmul_rn(__uint_as_float(w[2 * h + 1] << 16), s), x3 = __fmul_rn(__uint_as_float(w[2 * h + 1] & 0xFFFF0000u), s);
+      q[h] = pack_e4m3x2(x1, x0) | (pack_e4m3x2(x3, x2) << 16);
+    }
+    Q2[i] = make_uint2(q[0], q[1]);
+  }
 }
 
 }  // namespace
@@ -137,7 +172,7 @@ cudaError_t launch_prep_labels(elmo_head* h, const int32_t* rowptr, const int32_
                                        (int)(sizeof(uint32_t) * ELMO_MAX_NNZ));
   if (e != cudaSuccess) return e;
   prep_labels_kernel<<<1, kPrepThreads, smem, s>>>(rowptr, cols, B, nnz, h->L, npow2, h->keys, h->nkeys,
-                                                   h->status);
+                                                   h->tile_ptr, h->status);
   return cudaGetLastError();
 }
 

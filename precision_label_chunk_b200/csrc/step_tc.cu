@@ -19,9 +19,11 @@
 //                    W  = SR(W - lr dW)                           (epilogue, in place)
 //                    one fp32 atomic flush of dX^T per run of tiles.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
-// issues MMAs (one elected thread), warps 2-5 are the epilogue (warp w reads
-// TMEM lanes 32*(w%4) .. +31).  Every wait is bounded; a wait that runs out
+// Warp roles (576 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
+// issues MMAs (one elected thread), warps 2-17 are the epilogue: warp w reads
+// TMEM lanes 32*(w%4) .. +31 and the 32-column chunks c with c % 4 == (w-2)/4,
+// so every SM sub-partition runs four epilogue warps (enough to hide the
+// TMEM-load and special-function latencies of one warp's chain).  Every wait is bounded; a wait that runs out
 // records ELMO_ETIMEOUT in the status word and the CTA winds down.
 #include <cuda.h>
 
@@ -34,7 +36,8 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 576;                    // 18 warps: TMA, MMA, 16 epilogue
+constexpr int kEpiWarps = 16;
 constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 2 GHz: only a broken pipeline waits this long
 constexpr uint32_t kBox = 16384;                  // one 128-row x 128-byte TMA box
 
@@ -60,17 +63,175 @@ __device__ __forceinline__ void label_mask(const uint32_t* __restrict__ keys, in
   }
 }
 
-// First key whose label is >= lab.
-__device__ __forceinline__ int lower_bound_label(const uint32_t* keys, int n, int64_t lab) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if ((int64_t)(__ldg(keys + mid) >> 8) < lab) lo = mid + 1; else hi = mid;
-  }
-  return lo;
+
+__device__ __forceinline__ float exp2f_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcpf_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-__device__ __forceinline__ float sigmoidf_fast(float z) { return __frcp_rn(1.0f + __expf(-z)); }
+// ---------------------------------------------------------------- epilogue pieces
+// G = sigmoid(Z) - Y for 16 samples b0 .. b0+15 of one label row, written as
+// the next contraction's operand (bf16, or E4M3 of 2^8 G); padded samples get 0.
+// sigmoid(z) = 1 / (1 + 2^(-z log2 e)) with z = acc / s_X: the scale, log2 e
+// and (E4M3) the 2^8 operand scale fold into `neg_l2e_over_sx` and `gscale`.
+template <int kFp8>
+__device__ __forceinline__ void grad16(const uint32_t* r, float neg_l2e_over_sx, float inv_sx, uint32_t ybits,
+                                       int b0, int B, void* __restrict__ grow, float* __restrict__ Zrow,
+                                       float* __restrict__ Grow) {
+  constexpr float gscale = kFp8 ? 256.0f : 1.0f;
+  float g[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float e = exp2f_approx(__fmul_rn(__uint_as_float(r[i]), neg_l2e_over_sx));
+    g[i] = rcpf_approx(__fmaf_rn(e, 1.0f / gscale, 1.0f / gscale));   // gscale * sigmoid(z)
+  }
+  if (ybits) {                        // positives are rare: subtract y where set
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if ((ybits >> i) & 1u) g[i] -= gscale;
+  }
+  if (b0 + 16 > B) {                  // batch padding
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (b0 + i >= B) g[i] = 0.0f;
+  }
+  uint32_t packed[8];
+  if (kFp8) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      packed[i] = pack_e4m3x2(g[4 * i + 1], g[4 * i]) | (pack_e4m3x2(g[4 * i + 3], g[4 * i + 2]) << 16);
+    *reinterpret_cast<uint4*>(grow) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(g[2 * i + 1], g[2 * i]);
+    uint4* dst = reinterpret_cast<uint4*>(grow);
+    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  }
+  if (Grow) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (b0 + i < B)
+        Grow[i] = kFp8 ? e4m3_to_f32((uint8_t)(packed[i >> 2] >> (8 * (i & 3)))) * 0.00390625f
+                       : bf16_to_f32((uint16_t)(packed[i >> 1] >> (16 * (i & 1))));
+  }
+  if (Zrow) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (b0 + i < B) Zrow[i] = __fmul_rn(__uint_as_float(r[i]), inv_sx);
+  }
+}
+
+// Positive-label bits of samples b0 .. b0+15 from the 256-bit mask.
+__device__ __forceinline__ uint32_t mask16(const uint32_t (&m)[8], int b0) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w = ((b0 >> 5) == i) ? m[i] : w;
+  return (w >> (b0 & 16)) & 0xFFFFu;
+}
+
+// W[l, j0 .. j0+15] = SR(W - lrs * acc) for one label row: old weights from the
+// 128B-swizzled W tile in shared memory (row `row`, tile column jl), draws from
+// the two Philox blocks of elements l*d + j0 .. +15.
+template <int kFp8>
+__device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint8_t* __restrict__ wtile, int row, int jl,
+                                         int64_t l, int32_t d, int j0, float lrs, uint64_t seed, uint64_t step,
+                                         void* __restrict__ Wglob) {
+  float wv[16];
+  if (kFp8) {
+    const uint4 x = *reinterpret_cast<const uint4*>(wtile + row * 128 + (((jl >> 4) ^ (row & 7)) << 4));
+    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float f4[4];
+      e4m3x4_to_f32(xw[e], f4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) wv[4 * e + i] = f4[i];
+    }
+  } else {
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int c16 = ((jl & 63) >> 3) + v;
+      const uint4 x = *reinterpret_cast<const uint4*>(wtile + (jl >> 6) * kBox + row * 128 + ((c16 ^ (row & 7)) << 4));
+      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        wv[8 * v + 2 * e] = __uint_as_float(xw[e] << 16);
+        wv[8 * v + 2 * e + 1] = __uint_as_float(xw[e] & 0xFFFF0000u);
+      }
+    }
+  }
+  // v = w - lr dW, and a probe that turns NaN when any v is NaN or infinite
+  // (bf16: or |v| >= 2^127, where rounding could reach the largest finite
+  // value); such groups take the exact per-element path
+  float vv[16];
+  float probe = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
+    probe = __fmaf_rn(kFp8 ? vv[i] : __fmul_rn(vv[i], 2.0f), 0.0f, probe);
+  }
+  const uint64_t blk = ((uint64_t)l * (uint64_t)d + (uint64_t)j0) >> 3;
+  const u32x4 r0 = sr_block(seed, step, blk), r1 = sr_block(seed, step, blk + 1);
+  const uint32_t rw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+  uint32_t wnew[8];
+  if (probe == 0.0f) {
+    if (kFp8) {
+      // |v| < 2^-6: shift into [2^-6, 2^-5) rounding up, add-and-truncate at 20
+      // bits, shift back.  sat = [|v| < 2^-6] comes from a saturated FMA:
+      // (2^-6 - |v|) 2^100 is >= 2^70 below 2^-6 and <= 0 from 2^-6 up.
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t word = rw[2 * q4 + (e >> 1)];
+          const uint32_t k16 = (e & 1) ? __umulhi(word, 0x10000u) : (word & 0xFFFFu);
+          const uint32_t radd = 0xFFFFFu - k16 * 16u;          // 2^20 - 1 - 16 k
+          const float v = vv[4 * q4 + e];
+          const float a = fabsf(v);
+          const float sat = __saturatef(__fmaf_rn(-a, 0x1p100f, 0x1p94f));
+          const float sh = __fmaf_ru(sat, 0.015625f, a);
+          const uint32_t t = (__float_as_uint(sh) + radd) & 0xFFF00000u;
+          o[e] = copysignf(__fmaf_rn(sat, -0.015625f, __uint_as_float(t)), v);
+        }
+        wnew[q4] = pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16);
+      }
+    } else {
+      // add-and-truncate at 16 bits directly on the signed patterns
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const uint32_t word = rw[p];
+        const uint32_t t0 = __float_as_uint(vv[2 * p]) + (0xFFFFu - (word & 0xFFFFu));
+        const uint32_t t1 = __float_as_uint(vv[2 * p + 1]) + (0xFFFFu - (word >> 16));
+        wnew[p] = __byte_perm(t0, t1, 0x7632);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      if (kFp8) {
+        if (p < 4) {
+          const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
+          const float o0 = sr_e4m3_value(vv[4 * p], w0 & 0xFFFFu), o1 = sr_e4m3_value(vv[4 * p + 1], w0 >> 16);
+          const float o2 = sr_e4m3_value(vv[4 * p + 2], w1 & 0xFFFFu), o3 = sr_e4m3_value(vv[4 * p + 3], w1 >> 16);
+          wnew[p] = pack_e4m3x2(o1, o0) | (pack_e4m3x2(o3, o2) << 16);
+        }
+      } else {
+        wnew[p] = (uint32_t)sr_bf16(vv[2 * p], rw[p] & 0xFFFFu) | ((uint32_t)sr_bf16(vv[2 * p + 1], rw[p] >> 16) << 16);
+      }
+    }
+  }
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(Wglob) + ((size_t)l * d + j0) * (kFp8 ? 1 : 2));
+  dst[0] = make_uint4(wnew[0], wnew[1], wnew[2], wnew[3]);
+  if (!kFp8) dst[1] = make_uint4(wnew[4], wnew[5], wnew[6], wnew[7]);
+}
 
 // ============================================================================
 // Kernel A: logits and gradient operand of a label range.
@@ -88,7 +249,7 @@ template <int kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     logits_grad_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int64_t L,
                    int32_t d, int32_t B, int32_t Bp, int64_t l0, int64_t l1, const uint32_t* __restrict__ keys,
-                   const int32_t* __restrict__ nkeys, const float* __restrict__ xscale, void* __restrict__ gbuf,
+                   const int32_t* __restrict__ tile_ptr, const float* __restrict__ xscale, void* __restrict__ gbuf,
                    float* __restrict__ Zout, float* __restrict__ Gout, int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -103,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesA; ++s) { mbar_init(&S->full[s], 1); mbar_init(&S->empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&S->tfull[b], 1); mbar_init(&S->tempty[b], 4); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&S->tfull[b], 1); mbar_init(&S->tempty[b], kEpiWarps); }
     S->abort = 0;
     fence_barrier_init();
   }
@@ -158,79 +319,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // epilogue: thread owns TMEM lane (label row) 32*(warp%4) + lane
+    // epilogue: thread owns TMEM lane (label row) 32*(warp%4) + lane and the
+    // 32-column chunks c with c % 4 == (warp - 2) / 4
     const int q = warp & 3;
+    const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const float inv_sx = kFp8 ? xscale[1] : 1.0f;
-    const int nk = *nkeys;
+    const float nl2e = -1.4426950408889634f * inv_sx;     // -log2(e) / s_X
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
       const uint32_t buf = tc & 1, use = tc >> 1;
       const int64_t lt0 = l0 + (int64_t)t * 128;
       const int64_t l = lt0 + row;
       const bool valid = (l - l0) < span;
-      const int k0 = lower_bound_label(keys, nk, lt0);
-      const int k1 = lower_bound_label(keys, nk, lt0 + 128);
+      // positives of the 128-label tiles that overlap [lt0, lt0 + 128)
+      const int k0 = __ldg(tile_ptr + (lt0 >> 7));
+      const int k1 = __ldg(tile_ptr + min((lt0 + 127) >> 7, (L - 1) >> 7) + 1);
       uint32_t mask[8];
       label_mask(keys, k0, k1, l, mask);
       if (!mbar_wait(&S->tfull[buf], use & 1, abort, kWaitCycles)) { record_timeout(status, abort, 4); break; }
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * 256;
-      for (int c = 0; c < Bp / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(taddr + c * 32, r);
+      // this warp's 32-column chunks c = sub, sub + 4 (Bp <= 256): one load and wait each
+      for (int c = sub; c < Bp / 32; c += 4) {
+        uint32_t ra[32];
+        tmem_ld32(taddr + c * 32, ra);
         tmem_wait_ld();
-        uint32_t mw = 0;
+        if (!valid) continue;
+        const size_t rowoff = (size_t)(l - l0);
 #pragma unroll
-        for (int w = 0; w < 8; ++w) mw = (c == w) ? mask[w] : mw;
-        float z[32], g[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          z[i] = __fmul_rn(__uint_as_float(r[i]), inv_sx);
-          const float y = ((mw >> i) & 1u) ? 1.0f : 0.0f;
-          g[i] = (c * 32 + i < B) ? sigmoidf_fast(z[i]) - y : 0.0f;
-        }
-        if (valid) {
-          if (kFp8) {
-            uint32_t packed[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              uint32_t v = 0;
-#pragma unroll
-              for (int e = 0; e < 4; ++e) v |= (uint32_t)f32_to_e4m3_rn(g[4 * i + e] * 256.0f) << (8 * e);
-              packed[i] = v;
-            }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(gbuf) + (size_t)(l - l0) * Bp + c * 32);
-            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-            if (Gout) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (c * 32 + i < B)
-                  Gout[(size_t)(l - l0) * B + c * 32 + i] =
-                      e4m3_to_f32((uint8_t)(packed[i >> 2] >> (8 * (i & 3)))) * 0.00390625f;
-            }
-          } else {
-            uint32_t packed[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              packed[i] = (uint32_t)f32_to_bf16_rn(g[2 * i]) | ((uint32_t)f32_to_bf16_rn(g[2 * i + 1]) << 16);
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(gbuf) + (size_t)(l - l0) * Bp + c * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-            if (Gout) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (c * 32 + i < B)
-                  Gout[(size_t)(l - l0) * B + c * 32 + i] = bf16_to_f32((uint16_t)(packed[i >> 1] >> (16 * (i & 1))));
-            }
-          }
-          if (Zout) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c * 32 + i < B) Zout[(size_t)(l - l0) * B + c * 32 + i] = z[i];
-          }
+        for (int k = 0; k < 2; ++k) {
+          const int b0 = c * 32 + k * 16;
+          grad16<kFp8>(ra + k * 16, nl2e, inv_sx, mask16(mask, b0), b0, B,
+                       static_cast<uint8_t*>(gbuf) + (rowoff * Bp + b0) * (kFp8 ? 1 : 2),
+                       Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
         }
       }
       tc_fence_before();
@@ -240,6 +362,164 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   if (*abort) __nanosleep(20000);   // let copies in flight land before the shared memory goes away
+  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+}
+
+// ============================================================================
+// Kernel A, resident-X variant: a panel of PN samples of X (all d columns) is
+// loaded once per CTA and kept in shared memory; only W k-blocks stream from
+// HBM, through a small ring.  Used whenever a panel of at least 64 samples
+// fits (d * bytes <= 3 KB); several panels re-read W from L2.
+// ============================================================================
+constexpr uint32_t kPanelBytes = 196608;   // 192 KB of X
+constexpr int kStagesP = 2;
+
+struct SmemP {
+  uint64_t wfull[kStagesP], wempty[kStagesP], xfull, xempty, tfull[2], tempty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int kFp8>
+__global__ void __launch_bounds__(kThreads, 1)
+    logits_grad_panel_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                         int64_t L, int32_t d, int32_t B, int32_t Bp, int32_t PN, int64_t l0, int64_t l1,
+                         const uint32_t* __restrict__ keys, const int32_t* __restrict__ tile_ptr,
+                         const float* __restrict__ xscale, void* __restrict__ gbuf, float* __restrict__ Zout,
+                         float* __restrict__ Gout, int32_t* __restrict__ status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xs = base;                          // nkb k-blocks of [PN rows x 128 B]
+  uint8_t* wst = base + kPanelBytes;           // kStagesP W k-blocks
+  SmemP* S = reinterpret_cast<SmemP*>(wst + kStagesP * kBox);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t span = l1 - l0;
+  const int ntiles = (int)((span + 127) / 128);
+  const int kb_elems = kFp8 ? 128 : 64;
+  const int nkb = (d + kb_elems - 1) / kb_elems;
+  const int npanels = Bp / PN;
+  const uint32_t xkb_bytes = (uint32_t)PN * 128u;
+  volatile int* abort = &S->abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStagesP; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
+    mbar_init(&S->xfull, 1); mbar_init(&S->xempty, 1);
+    for (int b = 0; b < 2; ++b) { mbar_init(&S->tfull[b], 1); mbar_init(&S->tempty[b], kEpiWarps); }
+    S->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(&S->tmem_base, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S->tmem_base;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      tma_prefetch_desc(&tmW);
+      tma_prefetch_desc(&tmX);
+      uint32_t it = 0;
+      for (int p = 0; p < npanels && !*abort; ++p) {
+        if (!mbar_wait(&S->xempty, (p & 1) ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 41); break; }
+        mbar_arrive_expect_tx(&S->xfull, (uint32_t)nkb * xkb_bytes);
+        for (int kb = 0; kb < nkb; ++kb) tma_load_2d(xs + kb * xkb_bytes, &tmX, &S->xfull, kb * kb_elems, p * PN);
+        for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+          if (p == 0 && t == (int)blockIdx.x) {
+            // warm L2 with this CTA's next tiles: HBM latency then hides behind the short ring
+            for (int t2 = t; t2 < ntiles && t2 < t + 3 * (int)gridDim.x; t2 += gridDim.x)
+              for (int kb = 0; kb < nkb; ++kb)
+                tma_prefetch_l2(&tmW, kb * kb_elems, (int32_t)(l0 + (int64_t)t2 * 128));
+          } else if (p == 0 && t + 2 * (int)gridDim.x < ntiles) {
+            for (int kb = 0; kb < nkb; ++kb)
+              tma_prefetch_l2(&tmW, kb * kb_elems, (int32_t)(l0 + (int64_t)(t + 2 * gridDim.x) * 128));
+          }
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % kStagesP;
+            const uint32_t ph = (it / kStagesP) & 1;
+            if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 42); break; }
+            mbar_arrive_expect_tx(&S->wfull[s], kBox);
+            tma_load_2d(wst + s * kBox, &tmW, &S->wfull[s], kb * kb_elems, (int32_t)(l0 + (int64_t)t * 128));
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, (uint32_t)PN) : make_idesc(1, 1, 0, 0, 128, (uint32_t)PN);
+      uint32_t it = 0, tc = 0;
+      for (int p = 0; p < npanels && !*abort; ++p) {
+        if (!mbar_wait(&S->xfull, p & 1, abort, kWaitCycles)) { record_timeout(status, abort, 43); break; }
+        tc_fence_after();
+        for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
+          const uint32_t buf = tc & 1, use = tc >> 1;
+          if (!mbar_wait(&S->tempty[buf], (use & 1) ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 44); break; }
+          tc_fence_after();
+          const uint32_t dcol = tmem + buf * 256;
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % kStagesP;
+            const uint32_t ph = (it / kStagesP) & 1;
+            if (!mbar_wait(&S->wfull[s], ph, abort, kWaitCycles)) { record_timeout(status, abort, 45); break; }
+            tc_fence_after();
+            const uint32_t a = smem_u32(wst + s * kBox);
+            const uint32_t xb = smem_u32(xs + kb * xkb_bytes);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = sw128_desc(a + k * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(xb + k * 32, 16, 1024);
+              if (kFp8) mma_e4m3(dcol, ad, bd, idesc, (kb | k) != 0);
+              else mma_bf16(dcol, ad, bd, idesc, (kb | k) != 0);
+            }
+            mma_commit(&S->wempty[s]);
+          }
+          mma_commit(&S->tfull[buf]);
+        }
+        mma_commit(&S->xempty);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int sub = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    const float inv_sx = kFp8 ? xscale[1] : 1.0f;
+    const float nl2e = -1.4426950408889634f * inv_sx;     // -log2(e) / s_X
+    uint32_t tc = 0;
+    for (int p = 0; p < npanels && !*abort; ++p) {
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
+        const uint32_t buf = tc & 1, use = tc >> 1;
+        const int64_t lt0 = l0 + (int64_t)t * 128;
+        const int64_t l = lt0 + row;
+        const bool valid = (l - l0) < span;
+        const int k0 = __ldg(tile_ptr + (lt0 >> 7));
+        const int k1 = __ldg(tile_ptr + min((lt0 + 127) >> 7, (L - 1) >> 7) + 1);
+        uint32_t mask[8];
+        label_mask(keys, k0, k1, l, mask);
+        if (!mbar_wait(&S->tfull[buf], use & 1, abort, kWaitCycles)) { record_timeout(status, abort, 46); break; }
+        tc_fence_after();
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * 256;
+        // this warp's 32-column chunks c = sub, sub + 4 of the panel: one load and wait each
+        for (int c = sub; c < PN / 32; c += 4) {
+          uint32_t ra[32];
+          tmem_ld32(taddr + c * 32, ra);
+          tmem_wait_ld();
+          if (!valid) continue;
+          const size_t rowoff = (size_t)(l - l0);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int cb = c * 32 + k * 16;             // panel column
+            const int b0 = p * PN + cb;                 // sample
+            grad16<kFp8>(ra + k * 16, nl2e, inv_sx, mask16(mask, b0), b0, B,
+                         static_cast<uint8_t*>(gbuf) + (rowoff * Bp + b0) * (kFp8 ? 1 : 2),
+                         Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S->tempty[buf]);
+      }
+    }
+  }
+  __syncthreads();
+  if (*abort) __nanosleep(20000);
   if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 512); }
 }
 
@@ -293,10 +573,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&S->xfull, 1); mbar_init(&S->xempty, 1);
-    mbar_init(&S->dxfull, 1); mbar_init(&S->dxempty, 4);
-    for (int s = 0; s < kWSlots; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 4); }
+    mbar_init(&S->dxfull, 1); mbar_init(&S->dxempty, kEpiWarps);
+    for (int s = 0; s < kWSlots; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kEpiWarps); }
     for (int s = 0; s < kGSlots; ++s) { mbar_init(&S->gfull[s], 1); mbar_init(&S->gempty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&S->dwfull[b], 1); mbar_init(&S->dwempty[b], 4); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&S->dwfull[b], 1); mbar_init(&S->dwempty[b], kEpiWarps); }
     S->abort = 0;
     fence_barrier_init();
   }
@@ -419,8 +699,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     const int q = warp & 3;
+    const int sub = (warp - 2) >> 2;           // dW columns 32*sub .. +31; dX^T chunks c % 4 == sub
     const int row = q * 32 + lane;             // label row of dW; column of d for dX^T
-    const float dw_scale = kFp8 ? 0.00390625f * xscale[1] : 1.0f;
+    // lr * dW with dW = acc * 2^-8 / s_X (fp8) folds into one exact power-of-two scaled lr
+    const float lrs = kFp8 ? lr * (0.00390625f * xscale[1]) : lr;
     const float dx_scale = kFp8 ? 0.00390625f : 1.0f;
     int run = 0;
     uint32_t wit = 0, dwit = 0;
@@ -440,58 +722,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool valid = (l - l0) < span;
         const uint8_t* wrow = ws + sw * kWSlotBytes;
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + 256 + db * 128;
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(taddr + c * 32, r);
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          const int jl = sub * 32 + hh * 16;               // column within the 128-column slice
+          uint32_t r[16];
+          tmem_ld16(taddr + jl, r);
           tmem_wait_ld();
-          const int j0 = D0 + c * 32;
+          const int j0 = D0 + jl;
           if (!valid || j0 >= d) continue;
-          // old weights of (row, j0 .. j0+31) from the swizzled W tile
-          uint32_t wold[kFp8 ? 8 : 16];
-          if (kFp8) {
-#pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              const int chunk16 = c * 2 + v;
-              const uint4 x = *reinterpret_cast<const uint4*>(wrow + row * 128 + ((chunk16 ^ (row & 7)) << 4));
-              wold[4 * v] = x.x; wold[4 * v + 1] = x.y; wold[4 * v + 2] = x.z; wold[4 * v + 3] = x.w;
-            }
-          } else {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int chunk16 = (c & 1) * 4 + v;
-              const uint4 x = *reinterpret_cast<const uint4*>(wrow + (c >> 1) * kBox + row * 128 +
-                                                              ((chunk16 ^ (row & 7)) << 4));
-              wold[4 * v] = x.x; wold[4 * v + 1] = x.y; wold[4 * v + 2] = x.z; wold[4 * v + 3] = x.w;
-            }
-          }
-          uint32_t wnew[kFp8 ? 8 : 16];
-#pragma unroll
-          for (int g8 = 0; g8 < 4; ++g8) {
-            const uint64_t idx0 = (uint64_t)l * (uint64_t)d + (uint64_t)(j0 + 8 * g8);
-            const u32x4 rb = sr_block(seed, step, idx0 >> 3);
-            const uint32_t rw[4] = {rb.x, rb.y, rb.z, rb.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int i = 8 * g8 + e;
-              const float dw = __fmul_rn(__uint_as_float(r[i]), dw_scale);
-              float w;
-              if (kFp8) w = e4m3_to_f32((uint8_t)(wold[i >> 2] >> (8 * (i & 3))));
-              else w = bf16_to_f32((uint16_t)(wold[i >> 1] >> (16 * (i & 1))));
-              const float v = __fsub_rn(w, __fmul_rn(lr, dw));
-              const uint32_t k16 = (e & 1) ? (rw[e >> 1] >> 16) : (rw[e >> 1] & 0xFFFFu);
-              if (kFp8) {
-                const uint32_t cde = sr_e4m3(v, k16);
-                if ((i & 3) == 0) wnew[i >> 2] = cde; else wnew[i >> 2] |= cde << (8 * (i & 3));
-              } else {
-                const uint32_t cde = sr_bf16(v, k16);
-                if ((i & 1) == 0) wnew[i >> 1] = cde; else wnew[i >> 1] |= cde << 16;
-              }
-            }
-          }
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(Wglob) + ((size_t)l * d + j0) * kElem);
-#pragma unroll
-          for (int v = 0; v < (kFp8 ? 2 : 4); ++v)
-            dst[v] = make_uint4(wnew[4 * v], wnew[4 * v + 1], wnew[4 * v + 2], wnew[4 * v + 3]);
+          update16<kFp8>(r, wrow, row, jl, l, d, j0, lrs, seed, step, Wglob);
         }
         tc_fence_before();
         __syncwarp();
@@ -503,15 +742,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int j = D0 + row;
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
-      for (int c = 0; c < Bp / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(taddr + c * 32, r);
+      for (int c = sub; c < Bp / 32; c += 4) {
+        uint32_t ra[32];
+        tmem_ld32(taddr + c * 32, ra);
         tmem_wait_ld();
         if (j < d) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int b = c * 32 + i;
-            if (b < B) atomicAdd(dX + (size_t)b * d + j, __uint_as_float(r[i]) * dx_scale);
+            if (b < B) atomicAdd(dX + (size_t)b * d + j, __uint_as_float(ra[i]) * dx_scale);
           }
         }
       }
@@ -561,7 +800,9 @@ cudaError_t make_map(CUtensorMap* m, const void* ptr, int elem_bytes, uint64_t c
 
 constexpr size_t kSmemA = 1024 + kStagesA * kStageABytes + sizeof(SmemA);
 constexpr size_t kSmemB = 1024 + kXBytes + kWSlots * kWSlotBytes + kGSlots * kGSlotBytes + sizeof(SmemB);
+constexpr size_t kSmemP = 1024 + kPanelBytes + kStagesP * kBox + sizeof(SmemP);
 static_assert(kSmemA <= 232448, "kernel A shared memory");
+static_assert(kSmemP <= 232448, "kernel A (resident X) shared memory");
 static_assert(kSmemB <= 232448, "kernel B shared memory");
 
 }  // namespace
@@ -588,10 +829,28 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((l1 - l0 + 127) / 128);
   const int grid = ntiles < h->num_sms ? ntiles : h->num_sms;
+  // resident-X panels: the largest multiple of 64 samples (dividing Bp) whose X fits in 192 KB
+  const int kb_elems = fp8 ? 128 : 64;
+  const int64_t xrow = (int64_t)((h->d + kb_elems - 1) / kb_elems) * 128;   // bytes of one sample, k-block padded
+  int32_t PN = (int32_t)((int64_t)kPanelBytes / xrow) / 64 * 64;
+  if (PN > 256) PN = 256;
+  while (PN >= 64 && Bp % PN != 0) PN -= 64;
+  if (PN >= 64) {
+    CUtensorMap tmXp;
+    e = make_map(&tmXp, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
+                 (uint64_t)B, (uint64_t)h->d, (uint32_t)PN);
+    if (e != cudaSuccess) return e;
+    auto kp = fp8 ? logits_grad_panel_tc<1> : logits_grad_panel_tc<0>;
+    e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemP);
+    if (e != cudaSuccess) return e;
+    kp<<<grid, kThreads, kSmemP, s>>>(tmW, tmXp, h->L, h->d, B, Bp, PN, l0, l1, h->keys, h->tile_ptr, h->xscale, gbuf,
+                                      Zout, Gout, h->status);
+    return cudaGetLastError();
+  }
   auto kern = fp8 ? logits_grad_tc<1> : logits_grad_tc<0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemA);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemA, s>>>(tmW, tmX, h->L, h->d, B, Bp, l0, l1, h->keys, h->nkeys, h->xscale, gbuf, Zout,
+  kern<<<grid, kThreads, kSmemA, s>>>(tmW, tmX, h->L, h->d, B, Bp, l0, l1, h->keys, h->tile_ptr, h->xscale, gbuf, Zout,
                                       Gout, h->status);
   return cudaGetLastError();
 }
