@@ -220,6 +220,48 @@ elmo_status elmo_profile_reset(elmo_head* h);
 elmo_status elmo_profile_read(elmo_head* h, int kernel_class, double* ms_total, int64_t* launches);
 elmo_status elmo_launch_count(const elmo_head* h, int64_t* launches);
 
+/*
+ * elmo_train_step_noalloc -- the training step of elmo_train_step_chunked for
+ * callers that cannot allocate device memory.  The paper has no counterpart:
+ * this entry point exists for deployment, not for the method.
+ *
+ * Who needs it: code that issues the step while a stream is being captured
+ * into a CUDA graph (allocation cannot be captured), runtimes that give the
+ * library a fixed memory budget, and hosts whose device allocator belongs to
+ * someone else.  Such callers cannot create an elmo_head (its workspace is
+ * allocated) nor let the head grow its gradient buffer on first use.
+ *
+ * This call takes W directly and allocates nothing.  Its scratch (sorted
+ * positives, the tile index, quantised X and the per-range gradient operands)
+ * is one static device array of 10 MiB (ELMO_NOALLOC_SCRATCH_BYTES) that every
+ * GPU loading the library holds until the process exits.  It supports the
+ * same sizes as the head-based step -- 1 <= L < 2^24, d a multiple of 64 up to
+ * 4096, 1 <= B <= 256, 0 <= nnz <= 32768 -- and rejects anything beyond them
+ * with ELMO_EUNSUPPORTED; the label range per pass shrinks so that its gradient
+ * operands fit the 8 MiB gradient part of the scratch (W stays bit-identical to
+ * the head-based step; dX differs only by fp32 summation order).
+ *
+ * The first call on a device looks up the device address of the scratch array
+ * (loading the library's device code on that device if needed); make that
+ * first call before capturing any stream.  Every call on a device shares the
+ * one array and each call rewrites it before reading it: calls whose work
+ * overlaps on the GPU (different streams, or the same graph launched
+ * concurrently) race on it and give wrong results -- serialise them.
+ *
+ *   W_dev, L, d, dt : the weights, as in elmo_init_head (updated in place).
+ *   X_dev ... dX_dev: as in elmo_train_step_chunked.
+ *   status_dev      : int32 [2] (device), zeroed by the call; a malformed label
+ *                     list leaves ELMO_EDATA in [0] (and the first bad entry in
+ *                     [1]) once the step has run.
+ * Errors: ELMO_EINVAL / ELMO_EUNSUPPORTED synchronously (message in
+ * elmo_last_error()), ELMO_ECUDA if a launch fails.
+ */
+#define ELMO_NOALLOC_SCRATCH_BYTES (10u << 20)
+elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d, elmo_dtype dt, const void* X_dev,
+                                    int32_t B, const int32_t* rowptr_dev, const int32_t* cols_dev, int32_t nnz,
+                                    float lr, int64_t chunk, uint64_t seed, uint64_t step, float* dX_dev,
+                                    int32_t* status_dev, void* stream);
+
 /* Message of the most recent failure on the calling thread ("" if none). */
 const char* elmo_last_error(void);
 

@@ -24,7 +24,7 @@ __all__ = [
     "library_path", "load", "elmo_init_head", "elmo_head_destroy", "elmo_train_step_chunked",
     "elmo_forward_chunk", "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws",
     "elmo_sync_status", "elmo_head_workspace_bytes", "elmo_profile_enable", "elmo_profile_reset",
-    "elmo_profile_read", "elmo_launch_count", "KERNEL_CLASSES",
+    "elmo_profile_read", "elmo_launch_count", "KERNEL_CLASSES", "elmo_train_step_noalloc",
 ]
 
 BF16 = 0
@@ -80,6 +80,8 @@ def _declare(L):
     L.elmo_sr_draws.argtypes = [P, i64, u64, u64, u64, P]
     L.elmo_sync_status.argtypes = [P, P]
     L.elmo_head_workspace_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+    L.elmo_train_step_noalloc.argtypes = [P, i64, i32, ctypes.c_int, P, i32, P, P, i32, f32, i64, u64, u64, P, P, P]
+    L.elmo_train_step_noalloc.restype = st
     L.elmo_profile_enable.argtypes = [P, ctypes.c_int]
     L.elmo_profile_reset.argtypes = [P]
     L.elmo_profile_read.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]
@@ -172,6 +174,20 @@ def elmo_train_step_chunked(head: Head, X: torch.Tensor, rowptr: torch.Tensor, c
     _check(load().elmo_train_step_chunked(head.handle, _ptr(X), B, _ptr(rowptr), _ptr(cols) if nnz else None,
                                           nnz, float(lr), int(chunk), int(seed) & (2**64 - 1),
                                           int(step) & (2**64 - 1), _ptr(dX), _stream(stream)))
+
+
+def elmo_train_step_noalloc(W: torch.Tensor, dtype, X: torch.Tensor, rowptr: torch.Tensor, cols: torch.Tensor,
+                            lr: float, chunk: int, seed: int, step: int, dX: torch.Tensor, status: torch.Tensor,
+                            stream=None):
+    """The training step without a head and without any device allocation, for
+    callers that must not allocate (stream capture, fixed memory budgets).
+    W: [L, d] weights (updated in place); status: int32 [2] device tensor that
+    receives ELMO_EDATA for malformed labels.  See include/elmo.h."""
+    nnz = cols.numel()
+    _check(load().elmo_train_step_noalloc(_ptr(W), W.shape[0], W.shape[1], _dt(dtype), _ptr(X), X.shape[0],
+                                          _ptr(rowptr), _ptr(cols) if nnz else None, nnz, float(lr), int(chunk),
+                                          int(seed) & (2**64 - 1), int(step) & (2**64 - 1), _ptr(dX), _ptr(status),
+                                          _stream(stream)))
 
 
 def elmo_forward_chunk(head: Head, X: torch.Tensor, rowptr: torch.Tensor, cols: torch.Tensor, l0: int, l1: int,

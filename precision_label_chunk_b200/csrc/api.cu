@@ -100,6 +100,8 @@ elmo_status check_labels_args(const elmo_head* h, const void* X, int32_t B, cons
 
 namespace elmo {
 
+void set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
 KernelScope::KernelScope(elmo_head* h_, int cls, cudaStream_t s_, int n) : h(h_), s(s_), on(h_ && h_->prof) {
   if (h) h->launches += n;
   if (!on) return;

@@ -67,6 +67,9 @@ inline int64_t sub_chunk_labels(int32_t d, int32_t Bp, int elem_bytes) {
   return n < 128 ? 128 : n;
 }
 
+// api.cu: the thread-local message elmo_last_error() returns
+void set_last_error(const char* msg);
+
 // prep.cu
 cudaError_t launch_prep_labels(elmo_head* h, const int32_t* rowptr, const int32_t* cols, int32_t B,
                                int32_t nnz, cudaStream_t s);
