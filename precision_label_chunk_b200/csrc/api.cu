@@ -306,7 +306,7 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B, const
   const bool simt = use_simt();
   const int64_t sub = simt ? elmo::kSubChunk : elmo::sub_chunk_labels(h->d, Bp, (int)esz);
   const int64_t span = l1 - l0 < sub ? l1 - l0 : sub;
-  if ((st = ensure_gbuf(h, (size_t)span * Bp * esz)) != ELMO_OK) return st;
+  if ((st = ensure_gbuf(h, (size_t)((span + 127) / 128 * 128) * Bp * esz)) != ELMO_OK) return st;  // whole tiles
   for (int64_t a = l0; a < l1; a += span) {
     const int64_t e = a + span < l1 ? a + span : l1;
     elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
@@ -344,7 +344,7 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
   const int64_t sub_max = simt ? elmo::kSubChunk : elmo::sub_chunk_labels(h->d, Bp, (int)esz);
   const int64_t sub = chunk < sub_max ? chunk : sub_max;
   const int64_t span = h->L < sub ? h->L : sub;
-  if ((st = ensure_gbuf(h, (size_t)span * Bp * esz)) != ELMO_OK) return st;
+  if ((st = ensure_gbuf(h, (size_t)((span + 127) / 128 * 128) * Bp * esz)) != ELMO_OK) return st;  // whole tiles
   for (int64_t c0 = 0; c0 < h->L; c0 += chunk) {
     const int64_t c1 = c0 + chunk < h->L ? c0 + chunk : h->L;
     for (int64_t a = c0; a < c1; a += span) {

@@ -19,6 +19,13 @@
 //                    W  = SR(W - lr dW)                           (epilogue, in place)
 //                    one fp32 atomic flush of dX^T per run of tiles.
 //
+// The gradient operands of a label range are stored tile by tile (128 labels
+// x Bp samples) as 8-label x 16-byte core matrices: chunk j of samples and
+// label group i sit at byte (j * 16 + i) * 128 of the tile, so the epilogue of
+// kernel A writes 512 contiguous bytes per warp store, kernel B fetches a tile
+// part with one bulk copy, and the same shared-memory block is the K-major
+// dW operand (labels x samples) and the MN-major dX^T operand (samples x labels).
+//
 // Warp roles (576 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
 // issues MMAs (one elected thread), warps 2-17 are the epilogue: warp w reads
 // TMEM lanes 32*(w%4) .. +31 and the 32-column chunks c with c % 4 == (w-2)/4,
@@ -82,8 +89,8 @@ __device__ __forceinline__ float rcpf_approx(float x) {
 // and (E4M3) the 2^8 operand scale fold into `neg_l2e_over_sx` and `gscale`.
 template <int kFp8>
 __device__ __forceinline__ void grad16(const uint32_t* r, float neg_l2e_over_sx, float inv_sx, uint32_t ybits,
-                                       int b0, int B, void* __restrict__ grow, float* __restrict__ Zrow,
-                                       float* __restrict__ Grow) {
+                                       int b0, int B, uint8_t* __restrict__ gtile, int row, bool row_invalid,
+                                       float* __restrict__ Zrow, float* __restrict__ Grow) {
   constexpr float gscale = kFp8 ? 256.0f : 1.0f;
   float g[16];
 #pragma unroll
@@ -96,32 +103,36 @@ __device__ __forceinline__ void grad16(const uint32_t* r, float neg_l2e_over_sx,
     for (int i = 0; i < 16; ++i)
       if ((ybits >> i) & 1u) g[i] -= gscale;
   }
-  if (b0 + 16 > B) {                  // batch padding
-#pragma unroll
+  if (b0 + 16 > B || row_invalid) {  // batch padding, and label rows past the range (their G
+#pragma unroll                        // must be 0: kernel B reads whole tiles)
     for (int i = 0; i < 16; ++i)
-      if (b0 + i >= B) g[i] = 0.0f;
+      if (b0 + i >= B || row_invalid) g[i] = 0.0f;
   }
   uint32_t packed[8];
   if (kFp8) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       packed[i] = pack_e4m3x2(g[4 * i + 1], g[4 * i]) | (pack_e4m3x2(g[4 * i + 3], g[4 * i + 2]) << 16);
-    *reinterpret_cast<uint4*>(grow) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    const int j = b0 >> 4;                                   // 16-byte chunk of samples
+    *reinterpret_cast<uint4*>(gtile + ((j * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
+        make_uint4(packed[0], packed[1], packed[2], packed[3]);
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(g[2 * i + 1], g[2 * i]);
-    uint4* dst = reinterpret_cast<uint4*>(grow);
-    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    const int j = b0 >> 3;                                   // first of two 16-byte chunks
+    *reinterpret_cast<uint4*>(gtile + ((j * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
+        make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    *reinterpret_cast<uint4*>(gtile + (((j + 1) * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
+        make_uint4(packed[4], packed[5], packed[6], packed[7]);
   }
-  if (Grow) {
+  if (Grow && !row_invalid) {
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       if (b0 + i < B)
         Grow[i] = kFp8 ? e4m3_to_f32((uint8_t)(packed[i >> 2] >> (8 * (i & 3)))) * 0.00390625f
                        : bf16_to_f32((uint16_t)(packed[i >> 1] >> (16 * (i & 1))));
   }
-  if (Zrow) {
+  if (Zrow && !row_invalid) {
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       if (b0 + i < B) Zrow[i] = __fmul_rn(__uint_as_float(r[i]), inv_sx);
@@ -345,13 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ra[32];
         tmem_ld32(taddr + c * 32, ra);
         tmem_wait_ld();
-        if (!valid) continue;
         const size_t rowoff = (size_t)(l - l0);
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int b0 = c * 32 + k * 16;
           grad16<kFp8>(ra + k * 16, nl2e, inv_sx, mask16(mask, b0), b0, B,
-                       static_cast<uint8_t*>(gbuf) + (rowoff * Bp + b0) * (kFp8 ? 1 : 2),
+                       static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                        Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
         }
       }
@@ -501,14 +511,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t ra[32];
           tmem_ld32(taddr + c * 32, ra);
           tmem_wait_ld();
-          if (!valid) continue;
           const size_t rowoff = (size_t)(l - l0);
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             const int cb = c * 32 + k * 16;             // panel column
             const int b0 = p * PN + cb;                 // sample
             grad16<kFp8>(ra + k * 16, nl2e, inv_sx, mask16(mask, b0), b0, B,
-                         static_cast<uint8_t*>(gbuf) + (rowoff * Bp + b0) * (kFp8 ? 1 : 2),
+                         static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                          Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
           }
         }
@@ -548,7 +557,7 @@ struct UnitRange {
 template <int kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     update_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-              const __grid_constant__ CUtensorMap tmG, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
+              const uint8_t* __restrict__ gbuf, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
               int32_t Bp, int64_t l0, int64_t l1, const float* __restrict__ xscale, float lr, uint64_t seed,
               uint64_t step, float* __restrict__ dX, int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -588,7 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (elect_one()) {
-      tma_prefetch_desc(&tmW); tma_prefetch_desc(&tmX); tma_prefetch_desc(&tmG);
+      tma_prefetch_desc(&tmW); tma_prefetch_desc(&tmX);
+      const size_t tile_bytes = (size_t)128 * Bp * kElem;
       int run = 0;
       uint32_t wit = 0, git = 0;
       for (int u = u0; u < u1 && !*abort;) {
@@ -623,13 +633,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ph = (git / kGSlots) & 1;
             ++git;
             if (!mbar_wait(&S->gempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 13); break; }
-            const int c0 = p * kPart;
-            int nb = 0;
-            for (int q = 0; q < 2; ++q) nb += (c0 + q * kBoxCols < Bp);
-            mbar_arrive_expect_tx(&S->gfull[s], (uint32_t)nb * kBox);
-            for (int q = 0; q < 2; ++q)
-              if (c0 + q * kBoxCols < Bp)
-                tma_load_2d(gs + s * kGSlotBytes + q * kBox, &tmG, &S->gfull[s], c0 + q * kBoxCols, t * 128);
+            // samples [p*kPart, p*kPart + np) of tile t: a contiguous run of 16-byte chunks
+            const int np = min(kPart, Bp - p * kPart);
+            const uint32_t bytes = (uint32_t)np * kElem * 128u;
+            mbar_arrive_expect_tx(&S->gfull[s], bytes);
+            bulk_load(gs + s * kGSlotBytes, gbuf + (size_t)t * tile_bytes + (size_t)p * kPart * kElem * 128u, bytes,
+                      &S->gfull[s]);
           }
         }
         ++run;
@@ -673,7 +682,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
             for (int k = 0; k < 128 / kK; ++k) {
               const uint64_t ad = sw128_desc(wa + k * kK * 128, kBox, 1024);
-              const uint64_t bd = sw128_desc(ga + k * kK * 128, kBox, 1024);
+              // G part as MN-major B (N = samples, K = labels): label groups 128 B apart,
+              // 16-byte sample chunks 2048 B apart; kK labels = kK / 8 groups per MMA
+              const uint64_t bd = nosw_desc(ga + k * (kK / 8) * 128, 128, 2048);
               if (kFp8) mma_e4m3(dxcol, ad, bd, idesc_dx, !(first && k == 0));
               else mma_bf16(dxcol, ad, bd, idesc_dx, !(first && k == 0));
             }
@@ -681,8 +692,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dwcol = tmem + 256 + db * 128;
 #pragma unroll 1
             for (int k = 0; k < np / kK; ++k) {
-              const int kb = (k * kK * kElem) / 128, kin = (k * kK * kElem) % 128;
-              const uint64_t ad = sw128_desc(ga + kb * kBox + kin, 16, 1024);
+              // G part as K-major A (M = labels, K = samples): 16-byte K chunks 2048 B
+              // apart, label groups 128 B apart; one MMA reads 32 bytes = 2 chunks of K
+              const uint64_t ad = nosw_desc(ga + k * 2 * 2048, 2048, 128);
               const uint64_t bd = sw128_desc(xa + (p * kPart + k * kK) * 128, 32768, 1024);
               if (kFp8) mma_e4m3(dwcol, ad, bd, idesc_dw, (p | k) != 0);
               else mma_bf16(dwcol, ad, bd, idesc_dw, (p | k) != 0);
@@ -861,13 +873,11 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
   const bool fp8 = h->dt == ELMO_FP8_E4M3;
   const int eb = fp8 ? 1 : 2;
   const int32_t Bp = padded_batch(B, fp8);
-  CUtensorMap tmW, tmX, tmG;
+  CUtensorMap tmW, tmX;
   cudaError_t e = make_map(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, 128);
   if (e != cudaSuccess) return e;
   e = make_map(&tmX, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
                (uint64_t)B, (uint64_t)h->d, (uint32_t)Bp);
-  if (e != cudaSuccess) return e;
-  e = make_map(&tmG, gbuf, eb, (uint64_t)Bp, (uint64_t)(l1 - l0), (uint64_t)Bp, 128);
   if (e != cudaSuccess) return e;
   const int T = (int)((l1 - l0 + 127) / 128);
   const int units = T * ((h->d + 127) / 128);
@@ -875,7 +885,7 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
   auto kern = fp8 ? update_tc<1> : update_tc<0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemB, s>>>(tmW, tmX, tmG, h->W, h->L, h->d, B, Bp, l0, l1, h->xscale, lr, seed, step, dX,
+  kern<<<grid, kThreads, kSmemB, s>>>(tmW, tmX, static_cast<const uint8_t*>(gbuf), h->W, h->L, h->d, B, Bp, l0, l1, h->xscale, lr, seed, step, dX,
                                       h->status);
   return cudaGetLastError();
 }
