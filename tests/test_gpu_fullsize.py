@@ -1,0 +1,67 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py uses
+(label chunks of the workload), on outputs the oracle can compute one by one:
+weight rows of sampled label ranges and dX rows of sampled samples (each a
+function of its own row), and top-k rows of sampled queries."""
+import numpy as np
+import pytest
+import torch
+
+from synthetic import make_labels, make_X, workload
+from tests.gpu_common import need_gpu, to_dev_i32, to_dev_u16, w_to_host
+from tests.parity import assert_rel_close, assert_weights_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _device_head(elmo, w):
+    """W of the workload filled on the device by the library (Philox normal of
+    std 0.02, stochastically rounded to the storage grid), as bench.py does;
+    the oracle then starts from a host copy of exactly those weights."""
+    Wd = torch.empty(w.L, w.d, dtype=torch.int16 if w.dtype == "bf16" else torch.uint8, device="cuda")
+    return Wd, elmo.elmo_init_head(Wd, w.dtype, fill=True, init_std=0.02, seed=0)
+
+
+def _label_ranges(L, chunk):
+    # the first labels, a range straddling a chunk boundary, and the ragged tail
+    mid = (L // chunk // 2) * chunk
+    return [(0, 256), (max(0, mid - 128), mid + 128), (L - 300, L)]
+
+
+@pytest.mark.parametrize("name", ["text500k_bf16", "product3m_fp8", "keyword8m6_bf16"])
+def test_step_full_size_sampled(orc, name):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload(name)
+    Wd, h = _device_head(elmo, w)
+    W0 = w_to_host(Wd, w.dtype)
+    X = make_X(w, 0)
+    rowptr, cols = make_labels(w, 0)
+    dX = torch.empty(w.B, w.d, device="cuda")
+    elmo.elmo_train_step_chunked(h, to_dev_u16(X), to_dev_i32(rowptr), to_dev_i32(cols), w.lr, w.chunk, 0, 0, dX)
+    elmo.elmo_sync_status(h)
+    for l0, l1 in _label_ranges(w.L, w.chunk):
+        r = orc.train_step(W0[:l1], X, rowptr, cols, w.lr, 0, 0, w.dtype, l0=l0, l1=l1, want_dx=False, L=w.L)
+        assert_weights_close(w_to_host(Wd[l0:l1], w.dtype), r["W"], w.dtype)
+    if w.L <= 3_000_000:          # dX rows need every label; the 8.6M head checks weights only
+        samples = [0, w.B // 2, w.B - 1]
+        ref = orc.dx_rows(W0, X, rowptr, cols, samples, w.dtype)
+        assert_rel_close(dX.cpu().numpy()[samples], ref, w.dtype, what="dX rows")
+    h.close()
+
+
+def test_topk_full_size_sampled(orc):
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("topk5_3m_fp8")
+    Wd = torch.empty(w.L, w.d, dtype=torch.uint8, device="cuda")
+    h = elmo.elmo_init_head(Wd, "fp8", fill=True, init_std=0.02, seed=0)
+    X = make_X(w, 0)
+    idx = torch.empty(w.B, w.topk, dtype=torch.int32, device="cuda")
+    sc = torch.empty(w.B, w.topk, device="cuda")
+    elmo.elmo_topk_predict(h, to_dev_u16(X), w.topk, w.chunk, idx, sc)
+    torch.cuda.synchronize()
+    rows = [0, 511, 1023]
+    ri, rs = orc.topk(w_to_host(Wd, "fp8"), X, w.topk, "fp8", rows=rows)
+    assert np.array_equal(idx.cpu().numpy()[rows], ri)
+    assert np.array_equal(sc.cpu().numpy()[rows].view(np.uint32), rs.view(np.uint32))
+    h.close()
