@@ -122,8 +122,10 @@ elmo_status elmo_head_destroy(elmo_head* h);
  *   seed, step : the stochastic-rounding stream; step 2^64-2 and 2^64-1 are
  *                reserved for the fill of elmo_init_head.
  *   dX_dev     : fp32 [B x d] (device), overwritten with the input gradient.
- * The transient per-chunk gradient buffer (min(chunk, 65536) x B operands) is
- * allocated on the first call that needs it (cudaMalloc: call once before
+ * The transient gradient buffer of one label range (the chunk, capped so that
+ * its operands stay within 128 MB; B padded to 64 (bf16) or 128 (E4M3) samples,
+ * one operand byte (E4M3) or two (bf16) per label and sample) is allocated on
+ * the first call that needs it (cudaMalloc: call once before
  * capturing the step in a CUDA graph).  A malformed CSR sets ELMO_EDATA in the
  * status word; the step then skips the malformed entries and W is undefined.
  */

@@ -58,11 +58,13 @@ namespace elmo {
 constexpr int kTileLabels = 128;        // labels per tensor-core tile
 constexpr int64_t kSubChunk = 65536;    // largest label range per pass (L2-resident G)
 
-// Labels per pass of the tensor-core step: W and G of a pass (about 64 MB)
-// stay resident in the 126 MB L2 between the two kernels.
+// Labels per pass of the tensor-core step: the caller's chunk, capped so that
+// the gradient operands of one pass (the transient buffer chunking bounds)
+// stay within 128 MB.  Longer passes amortise each kernel's fill and drain.
 inline int64_t sub_chunk_labels(int32_t d, int32_t Bp, int elem_bytes) {
-  const int64_t per_label = (int64_t)(d + Bp) * elem_bytes;
-  int64_t n = (int64_t(64) << 20) / per_label;
+  (void)d;
+  const int64_t per_label = (int64_t)Bp * elem_bytes;
+  int64_t n = (int64_t(128) << 20) / per_label;
   n = n / 128 * 128;
   return n < 128 ? 128 : n;
 }

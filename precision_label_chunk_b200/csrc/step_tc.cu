@@ -381,11 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // HBM, through a small ring.  Used whenever a panel of at least 64 samples
 // fits (d * bytes <= 3 KB); several panels re-read W from L2.
 // ============================================================================
-constexpr uint32_t kPanelBytes = 196608;   // 192 KB of X
-constexpr int kStagesP = 2;
+constexpr uint32_t kPanelSmem = 229376;    // X panel + W ring (224 KB)
+constexpr int kMaxStagesP = 8;
 
 struct SmemP {
-  uint64_t wfull[kStagesP], wempty[kStagesP], xfull, xempty, tfull[2], tempty[2];
+  uint64_t wfull[kMaxStagesP], wempty[kMaxStagesP], xfull, xempty, tfull[2], tempty[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -393,26 +393,27 @@ struct SmemP {
 template <int kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     logits_grad_panel_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                         int64_t L, int32_t d, int32_t B, int32_t Bp, int32_t PN, int64_t l0, int64_t l1,
+                         int64_t L, int32_t d, int32_t B, int32_t Bp, int32_t PN, int32_t nstages, int64_t l0,
+                         int64_t l1,
                          const uint32_t* __restrict__ keys, const int32_t* __restrict__ tile_ptr,
                          const float* __restrict__ xscale, void* __restrict__ gbuf, float* __restrict__ Zout,
                          float* __restrict__ Gout, int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* xs = base;                          // nkb k-blocks of [PN rows x 128 B]
-  uint8_t* wst = base + kPanelBytes;           // kStagesP W k-blocks
-  SmemP* S = reinterpret_cast<SmemP*>(wst + kStagesP * kBox);
+  const int kb_elems = kFp8 ? 128 : 64;
+  const int nkb = (d + kb_elems - 1) / kb_elems;
+  uint8_t* xs = base;                                          // nkb k-blocks of [PN rows x 128 B]
+  uint8_t* wst = base + (size_t)nkb * PN * 128;                // nstages W k-blocks
+  SmemP* S = reinterpret_cast<SmemP*>(base + kPanelSmem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t span = l1 - l0;
   const int ntiles = (int)((span + 127) / 128);
-  const int kb_elems = kFp8 ? 128 : 64;
-  const int nkb = (d + kb_elems - 1) / kb_elems;
   const int npanels = Bp / PN;
   const uint32_t xkb_bytes = (uint32_t)PN * 128u;
   volatile int* abort = &S->abort;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStagesP; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
+    for (int s = 0; s < nstages; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
     mbar_init(&S->xfull, 1); mbar_init(&S->xempty, 1);
     for (int b = 0; b < 2; ++b) { mbar_init(&S->tfull[b], 1); mbar_init(&S->tempty[b], kEpiWarps); }
     S->abort = 0;
@@ -444,8 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_prefetch_l2(&tmW, kb * kb_elems, (int32_t)(l0 + (int64_t)(t + 2 * gridDim.x) * 128));
           }
           for (int kb = 0; kb < nkb; ++kb, ++it) {
-            const int s = it % kStagesP;
-            const uint32_t ph = (it / kStagesP) & 1;
+            const int s = it % nstages;
+            const uint32_t ph = (it / nstages) & 1;
             if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 42); break; }
             mbar_arrive_expect_tx(&S->wfull[s], kBox);
             tma_load_2d(wst + s * kBox, &tmW, &S->wfull[s], kb * kb_elems, (int32_t)(l0 + (int64_t)t * 128));
@@ -466,8 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t dcol = tmem + buf * 256;
           for (int kb = 0; kb < nkb; ++kb, ++it) {
-            const int s = it % kStagesP;
-            const uint32_t ph = (it / kStagesP) & 1;
+            const int s = it % nstages;
+            const uint32_t ph = (it / nstages) & 1;
             if (!mbar_wait(&S->wfull[s], ph, abort, kWaitCycles)) { record_timeout(status, abort, 45); break; }
             tc_fence_after();
             const uint32_t a = smem_u32(wst + s * kBox);
@@ -812,7 +813,7 @@ cudaError_t make_map(CUtensorMap* m, const void* ptr, int elem_bytes, uint64_t c
 
 constexpr size_t kSmemA = 1024 + kStagesA * kStageABytes + sizeof(SmemA);
 constexpr size_t kSmemB = 1024 + kXBytes + kWSlots * kWSlotBytes + kGSlots * kGSlotBytes + sizeof(SmemB);
-constexpr size_t kSmemP = 1024 + kPanelBytes + kStagesP * kBox + sizeof(SmemP);
+constexpr size_t kSmemP = 1024 + kPanelSmem + sizeof(SmemP);
 static_assert(kSmemA <= 232448, "kernel A shared memory");
 static_assert(kSmemP <= 232448, "kernel A (resident X) shared memory");
 static_assert(kSmemB <= 232448, "kernel B shared memory");
@@ -841,12 +842,18 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((l1 - l0 + 127) / 128);
   const int grid = ntiles < h->num_sms ? ntiles : h->num_sms;
-  // resident-X panels: the largest multiple of 64 samples (dividing Bp) whose X fits in 192 KB
+  // resident-X panels: the largest multiple of 64 samples dividing Bp whose X
+  // leaves room for a W ring of at least two 16 KB stages (measured: one large
+  // panel with a short ring beats two panels with a deep ring, which re-read W)
   const int kb_elems = fp8 ? 128 : 64;
   const int64_t xrow = (int64_t)((h->d + kb_elems - 1) / kb_elems) * 128;   // bytes of one sample, k-block padded
-  int32_t PN = (int32_t)((int64_t)kPanelBytes / xrow) / 64 * 64;
-  if (PN > 256) PN = 256;
-  while (PN >= 64 && Bp % PN != 0) PN -= 64;
+  int32_t PN = 0, nst = 0;
+  for (int32_t pn = (Bp < 256 ? Bp : 256); pn >= 64; pn -= 64) {
+    if (Bp % pn) continue;
+    const int64_t free_bytes = (int64_t)kPanelSmem - xrow * pn;
+    const int st = (int)(free_bytes / kBox);
+    if (st >= 2) { PN = pn; nst = st < kMaxStagesP ? st : kMaxStagesP; break; }
+  }
   if (PN >= 64) {
     CUtensorMap tmXp;
     e = make_map(&tmXp, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
@@ -855,8 +862,8 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
     auto kp = fp8 ? logits_grad_panel_tc<1> : logits_grad_panel_tc<0>;
     e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemP);
     if (e != cudaSuccess) return e;
-    kp<<<grid, kThreads, kSmemP, s>>>(tmW, tmXp, h->L, h->d, B, Bp, PN, l0, l1, h->keys, h->tile_ptr, h->xscale, gbuf,
-                                      Zout, Gout, h->status);
+    kp<<<grid, kThreads, kSmemP, s>>>(tmW, tmXp, h->L, h->d, B, Bp, PN, nst, l0, l1, h->keys, h->tile_ptr, h->xscale,
+                                      gbuf, Zout, Gout, h->status);
     return cudaGetLastError();
   }
   auto kern = fp8 ? logits_grad_tc<1> : logits_grad_tc<0>;
