@@ -81,22 +81,40 @@ __device__ __forceinline__ float rcpf_approx(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float tanhf_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // ---------------------------------------------------------------- epilogue pieces
 // G = sigmoid(Z) - Y for 16 samples b0 .. b0+15 of one label row, written as
 // the next contraction's operand (bf16, or E4M3 of 2^8 G); padded samples get 0.
-// sigmoid(z) = 1 / (1 + 2^(-z log2 e)) with z = acc / s_X: the scale, log2 e
-// and (E4M3) the 2^8 operand scale fold into `neg_l2e_over_sx` and `gscale`.
+// z = acc / s_X.  The special-function unit (16 results per clock per SM) is
+// the epilogue's narrowest pipe, so each form uses as few of its ops as its
+// operand precision allows:
+//   bf16: sigmoid(z) = 1 / (1 + 2^(-z log2 e)), an ex2 and a rcp, both to
+//         about 2^-22 relative, far below the bf16 rounding of G;
+//   E4M3: 2^8 sigmoid(z) = 2^7 + 2^7 tanh(z / 2), a single tanh.  Its
+//         relative error of about 2^-11 is an absolute error of at most 2^-4
+//         in units of 2^8 G, below half the E4M3 spacing (2^-3 or more)
+//         wherever 2^8 |G| >= 1; only the codes of negatives with
+//         sigmoid(z) < 2^-8 (z < -5.5) can move by more than one step.
+// `zmul` is -log2(e) / s_X (bf16) or 1 / (2 s_X) (E4M3).
 template <int kFp8>
-__device__ __forceinline__ void grad16(const uint32_t* r, float neg_l2e_over_sx, float inv_sx, uint32_t ybits,
+__device__ __forceinline__ void grad16(const uint32_t* r, float zmul, float inv_sx, uint32_t ybits,
                                        int b0, int B, uint8_t* __restrict__ gtile, int row, bool row_invalid,
                                        float* __restrict__ Zrow, float* __restrict__ Grow) {
   constexpr float gscale = kFp8 ? 256.0f : 1.0f;
   float g[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float e = exp2f_approx(__fmul_rn(__uint_as_float(r[i]), neg_l2e_over_sx));
-    g[i] = rcpf_approx(__fmaf_rn(e, 1.0f / gscale, 1.0f / gscale));   // gscale * sigmoid(z)
+    if (kFp8) {
+      g[i] = __fmaf_rn(tanhf_approx(__fmul_rn(__uint_as_float(r[i]), zmul)), 128.0f, 128.0f);
+    } else {
+      const float e = exp2f_approx(__fmul_rn(__uint_as_float(r[i]), zmul));
+      g[i] = rcpf_approx(__fadd_rn(e, 1.0f));
+    }
   }
   if (ybits) {                        // positives are rare: subtract y where set
 #pragma unroll
@@ -336,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const float inv_sx = kFp8 ? xscale[1] : 1.0f;
-    const float nl2e = -1.4426950408889634f * inv_sx;     // -log2(e) / s_X
+    const float zmul = kFp8 ? 0.5f * inv_sx : -1.4426950408889634f;   // see grad16
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
       const uint32_t buf = tc & 1, use = tc >> 1;
@@ -360,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int b0 = c * 32 + k * 16;
-          grad16<kFp8>(ra + k * 16, nl2e, inv_sx, mask16(mask, b0), b0, B,
+          grad16<kFp8>(ra + k * 16, zmul, inv_sx, mask16(mask, b0), b0, B,
                        static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                        Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
         }
@@ -492,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const float inv_sx = kFp8 ? xscale[1] : 1.0f;
-    const float nl2e = -1.4426950408889634f * inv_sx;     // -log2(e) / s_X
+    const float zmul = kFp8 ? 0.5f * inv_sx : -1.4426950408889634f;   // see grad16
     uint32_t tc = 0;
     for (int p = 0; p < npanels && !*abort; ++p) {
       for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
@@ -517,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 2; ++k) {
             const int cb = c * 32 + k * 16;             // panel column
             const int b0 = p * PN + cb;                 // sample
-            grad16<kFp8>(ra + k * 16, nl2e, inv_sx, mask16(mask, b0), b0, B,
+            grad16<kFp8>(ra + k * 16, zmul, inv_sx, mask16(mask, b0), b0, B,
                          static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                          Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
           }
