@@ -123,6 +123,31 @@ def alu_peak_tflops(peaks):
     return 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
 
 
+def profiled_traffic(kernel, workload):
+    """DRAM bytes (read + write) of one full launch of `kernel`, from the ncu
+    summary committed under profiles/, with the labels that launch covered.
+    None when there is no summary or when the kernel source has changed since
+    the counters were taken (the summary records the source's sha256)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    try:
+        src, digest = fields["source"].split()
+        with open(os.path.join(ROOT, src), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != digest:
+                return None
+        return {"bytes": float(fields["dram bytes per launch"]), "labels": int(fields["labels per launch"])}
+    except (KeyError, ValueError, OSError):
+        return None
+
+
 def cpu_baseline(w, W_rows_host, X, rowptr, cols, target_s):
     """The oracle as it stands, on a bounded label sample of the same workload."""
     import oracle
@@ -180,8 +205,147 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_topk(args, w, rank, world, local):
+    """Chunked top-k prediction (X [B x d] bf16 against the whole head): one
+    step is one elmo_topk_predict call over all L labels."""
+    import torch
+    import precision_label_chunk_b200 as elmo
+    from synthetic import make_X
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    wdt = torch.int16 if w.dtype == "bf16" else torch.uint8
+    W = torch.empty(w.L, w.d, dtype=wdt, device=dev)
+    head = elmo.elmo_init_head(W, w.dtype, fill=True, init_std=0.02, seed=0)
+    nsteps = args.warmup + args.steps
+    Xh = [make_X(w, s) for s in range(nsteps)]
+    Xd = [torch.from_numpy(x.view(np.int16)).to(dev) for x in Xh]
+    idx = torch.empty(w.B, w.topk, dtype=torch.int32, device=dev)
+    sc = torch.empty(w.B, w.topk, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for s in range(args.warmup):
+        elmo.elmo_topk_predict(head, Xd[s], w.topk, w.chunk, idx, sc)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    launches0 = elmo.elmo_launch_count(head)
+    sampler.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for s in range(args.warmup, nsteps):
+        elmo.elmo_topk_predict(head, Xd[s], w.topk, w.chunk, idx, sc)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    gpu_launches = elmo.elmo_launch_count(head) - launches0
+    ms = ev0.elapsed_time(ev1) / args.steps
+    # per-kernel pass (events around every launch, outside the timed region)
+    elmo.elmo_profile_reset(head)
+    elmo.elmo_profile_enable(head, True)
+    for s in range(args.warmup, nsteps):
+        elmo.elmo_topk_predict(head, Xd[s], w.topk, w.chunk, idx, sc)
+    torch.cuda.synchronize()
+    elmo.elmo_profile_enable(head, False)
+    classes = {}
+    for name in elmo.KERNEL_CLASSES:
+        t_ms, n = elmo.elmo_profile_read(head, name)
+        if n:
+            classes[name] = {"ms": t_ms, "launches": n}
+    flops = 2.0 * w.B * w.L * w.d
+    dominant = max(classes, key=lambda k: classes[k]["ms"]) if classes else None
+    roof = None
+    if dominant == "topk_score":
+        t_k = classes[dominant]["ms"] / 1e3 / args.steps
+        peak, bound, src = alu_peak_tflops(peaks), "alu", "derived: 148 SM x 128 FMA x 2 x max clock"
+        roof = {"kernel": dominant, "bound": bound, "achieved": flops / t_k / 1e12, "peak": peak, "unit": "TFLOP/s",
+                "frac": flops / t_k / 1e12 / peak, "traffic": None, "peak_source": src}
+    # end to end: X from pinned host memory, indices and scores back every step
+    pin = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in Xh]
+    idx_h = torch.empty(w.B, w.topk, dtype=torch.int32).pin_memory()
+    sc_h = torch.empty(w.B, w.topk, dtype=torch.float32).pin_memory()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(args.warmup, nsteps):
+        elmo.elmo_topk_predict(head, pin[s].to(dev, non_blocking=True), w.topk, w.chunk, idx, sc)
+        idx_h.copy_(idx, non_blocking=True)
+        sc_h.copy_(sc, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / args.steps
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        Wh = W.cpu().numpy().view(np.uint8 if w.dtype == "fp8" else np.uint16)
+        nthreads = os.cpu_count() or 1
+        t = time.perf_counter()
+        oracle.topk(Wh, Xh[0], w.topk, w.dtype, rows=[0], nthreads=nthreads)
+        dt = time.perf_counter() - t
+        cpu = {"value": w.L / dt, "unit": "query-labels/s", "cores": nthreads, "kind": "oracle",
+               "sample": f"query row 0 against all {w.L} labels, {dt:.1f} s"}
+    if rank == 0:
+        line = {
+            "metric": "chunked top-k predict: query-labels/s", "value": world * w.B * w.L / (ms / 1e3),
+            "unit": "query-labels/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "L": w.L, "d": w.d, "B": w.B, "w_dtype": w.dtype, "k": w.topk,
+                       "chunk": w.chunk, "l2": f"inputs larger than L2 (W = {w.L * w.d / 1e9:.2f} GB)"},
+            "tflops": flops / (ms / 1e3) / 1e12, "roofline": roof, "kernels": classes,
+            "gpu_launches": gpu_launches,
+            "e2e": {"value": world * w.B * w.L / (ms_e2e / 1e3), "unit": "query-labels/s",
+                    "h2d_bytes_per_step": w.B * w.d * 2, "d2h_bytes_per_step": w.B * w.topk * 8},
+            "cpu_baseline": cpu, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    head.close()
+
+
+def run_sr(args, local):
+    """Standalone stochastic rounding of 2^28 fp32 values to E4M3 and to bf16:
+    an HBM-bound pass (4 bytes read and 1 or 2 bytes written per value)."""
+    import torch
+    import precision_label_chunk_b200 as elmo
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    n = 1 << 28
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    x = torch.randn(n, generator=g, device=dev) * 0.02
+    res = {}
+    for dt, odt, ob in (("fp8", torch.uint8, 1), ("bf16", torch.int16, 2)):
+        out = torch.empty(n, dtype=odt, device=dev)
+        for s in range(args.warmup):
+            elmo.elmo_sr_round(x, out, dt, 0, s)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for s in range(args.steps):
+            elmo.elmo_sr_round(x, out, dt, 0, args.warmup + s)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        gbs = n * (4 + ob) / (ms / 1e3) / 1e9
+        res[dt] = {"ms": ms, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]}
+    line = {"metric": "standalone SR: values/s", "value": n / (res["fp8"]["ms"] / 1e3), "unit": "values/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["fp8"]["ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "sr_round", "n": n, "l2": "inputs larger than L2 (1 GiB fp32)"},
+            "roofline": {"kernel": "sr_round", "bound": "hbm", "achieved": res["fp8"]["GB/s"],
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": res["fp8"]["frac"], "traffic": None,
+                         "peak_source": f"{peaks['source']} copy bandwidth"},
+            "per_dtype": res}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.workload == "sr_round":
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_sr(args, int(os.environ.get("LOCAL_RANK", "0")))
+        return
     from synthetic import workload
     w = workload(args.workload, **({"L": args.labels} if args.labels else {}))
     rank = int(os.environ.get("RANK", "0"))
@@ -191,6 +355,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, w)
+        return
+
+    if w.topk > 0:
+        run_topk(args, w, rank, world, local)
         return
 
     import torch
@@ -233,8 +401,6 @@ def main():
 
     # ---------------------------------------------------------------- timed region
     sampler = ClockSampler(local)
-    elmo.elmo_profile_reset(head)
-    elmo.elmo_profile_enable(head, True)
     launches0 = elmo.elmo_launch_count(head)
     if world > 1:
         dist.barrier()
@@ -250,7 +416,6 @@ def main():
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    elmo.elmo_profile_enable(head, False)
     elmo.elmo_sync_status(head)
     gpu_launches = elmo.elmo_launch_count(head) - launches0
     ms = ev0.elapsed_time(ev1)
@@ -261,13 +426,31 @@ def main():
     ms_per_step = ms / args.steps
     value = world * w.L * args.steps / (ms / 1e3)
 
-    # per-class device time inside the timed region
+    # ---------------------------------------------------------------- per-kernel pass
+    # The same K steps again, with the library recording a CUDA event pair on
+    # the launch stream around every kernel.  An event between two kernels
+    # costs a few microseconds of device time (the next launch can no longer
+    # be overlapped with the previous kernel's drain), so these events stay
+    # out of the timed region above; `kernels_pass_ms_per_step` reports what
+    # the pass itself took.
+    elmo.elmo_profile_reset(head)
+    elmo.elmo_profile_enable(head, True)
+    torch.cuda.synchronize()
+    pv0, pv1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pv0.record(stream)
+    for s in range(args.warmup, nsteps):
+        step(nsteps + s, dev_batches[s])
+    pv1.record(stream)
+    torch.cuda.synchronize()
+    elmo.elmo_profile_enable(head, False)
+    elmo.elmo_sync_status(head)
     classes = {}
     for name in elmo.KERNEL_CLASSES:
         t_ms, n = elmo.elmo_profile_read(head, name)
         if n:
             classes[name] = {"ms": t_ms, "launches": n}
     elmo.elmo_profile_reset(head)
+    kernels_pass_ms = pv0.elapsed_time(pv1) / args.steps
 
     # roofline of the dominant kernel class: algorithmic flops of the
     # contractions it performs per step (2 B L d each) over its device time
@@ -283,8 +466,15 @@ def main():
         else:
             peak, bound = tensor_peak_tflops(peaks, w.dtype), "tensor"
             src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype == "fp8" else ""))
+        # ncu DRAM bytes of one full launch, scaled to the mean launch of this
+        # run by the labels it covers (the kernel's traffic is linear in them)
+        tr = profiled_traffic({"update": "update_tc", "logits_grad": "logits_grad_tc"}.get(dominant, dominant),
+                              w.name)
+        traffic = None
+        if tr is not None:
+            traffic = tr["bytes"] * (w.L / (classes[dominant]["launches"] / args.steps)) / tr["labels"]
         roof = {"kernel": dominant, "bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "peak_source": src,
+                "frac": achieved / peak, "traffic": traffic, "peak_source": src,
                 "flops_per_launch": fl_per_step / (classes[dominant]["launches"] / args.steps),
                 "launches_per_step": classes[dominant]["launches"] / args.steps}
 
@@ -342,7 +532,7 @@ def main():
                        "l2": f"inputs larger than L2 (W = {costs['w_bytes'] / 2 / 1e9:.2f} GB per replica)",
                        "parallelism": "replicas" if world > 1 else "single"},
             "tflops": step_roof["tflops"], "step_roofline": step_roof, "roofline": roof,
-            "kernels": classes, "gpu_launches": gpu_launches, "e2e": e2e, "cpu_baseline": cpu,
+            "kernels": classes, "kernels_pass_ms_per_step": kernels_pass_ms, "gpu_launches": gpu_launches, "e2e": e2e, "cpu_baseline": cpu,
             "clocks": clocks, "peak_device_bytes": int(peak_mem),
         }
         print(json.dumps(line), flush=True)

@@ -140,6 +140,62 @@ __device__ __forceinline__ uint8_t sr_e4m3(float v, uint32_t k) {
   return (uint8_t)(pack_e4m3x2(0.0f, sr_e4m3_value(v, k)) & 0xFF);
 }
 
+// Eight values rounded with the eight 16-bit draws of one Philox block (draw
+// e is half e & 1 of word e >> 1).  The common case is add-and-truncate on
+// the fp32 bit pattern: adding 2^m - 1 - k (m = 16 discarded bits for bf16,
+// 20 for E4M3) carries into the first kept bit exactly when k < f 2^16, f the
+// discarded fraction, which is the rule u < (v - lo) / (hi - lo) with
+// u = k / 2^16.  E4M3 values below 2^-6 (its subnormal range, spacing 2^-9)
+// are first moved into [2^-6, 2^-5), which has the same spacing, by an add
+// rounded toward +inf (exact there) and moved back after the truncation.  A
+// group holding a NaN or an infinity (bf16: or a magnitude of 2^127 or more,
+// where the carry could reach the exponent's top) takes the per-element path.
+__device__ __forceinline__ uint4 sr8_bf16(const float (&v)[8], const u32x4& r) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+  float probe = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) probe = __fmaf_rn(__fmul_rn(v[i], 2.0f), 0.0f, probe);
+  uint32_t o[4];
+  if (probe == 0.0f) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t t0 = __float_as_uint(v[2 * p]) + (0xFFFFu - (w[p] & 0xFFFFu));
+      const uint32_t t1 = __float_as_uint(v[2 * p + 1]) + (0xFFFFu - (w[p] >> 16));
+      o[p] = __byte_perm(t0, t1, 0x7632);
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+      o[p] = (uint32_t)sr_bf16(v[2 * p], w[p] & 0xFFFFu) | ((uint32_t)sr_bf16(v[2 * p + 1], w[p] >> 16) << 16);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ uint2 sr8_e4m3(const float (&v)[8], const u32x4& r) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+  float probe = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) probe = __fmaf_rn(v[i], 0.0f, probe);
+  float o[8];
+  if (probe == 0.0f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t k = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+      const float a = fabsf(v[e]);
+      // sat = 1 when |v| < 2^-6: (2^-6 - |v|) 2^100 is then >= 2^70, else <= 0
+      const float sat = __saturatef(__fmaf_rn(-a, 0x1p100f, 0x1p94f));
+      const float sh = __fmaf_ru(sat, 0.015625f, a);
+      const uint32_t t = (__float_as_uint(sh) + (0xFFFFFu - (k << 4))) & 0xFFF00000u;
+      o[e] = copysignf(__fmaf_rn(sat, -0.015625f, __uint_as_float(t)), v[e]);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = sr_e4m3_value(v[e], (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu));
+  }
+  return make_uint2(pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16),
+                    pack_e4m3x2(o[5], o[4]) | (pack_e4m3x2(o[7], o[6]) << 16));
+}
+
 // Four E4M3 codes (byte i = element i) -> fp32 values, exact.
 __device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&o)[4]) {
   uint32_t h01, h23;

@@ -1,11 +1,13 @@
 // prep.cu -- per-step preparation of the sparse labels and of the X operand.
 //
 // Labels: the positives of a step arrive as CSR (rowptr, cols).  The kernels
-// that form G = sigmoid(Z) - Y need them by label, so they are turned into
-// sorted keys (label << 8 | sample) once per step; a label tile then finds its
-// positives by binary search.  Malformed input (rowptr not monotone, rowptr[B]
-// != nnz, a column outside [0, L)) is recorded in the head's status word as
-// ELMO_EDATA and the offending entries are dropped.
+// that form G = sigmoid(Z) - Y need them by label tile, so they are bucketed
+// once per step by a counting sort on the 128-label tile: keys
+// (label << 8 | sample) grouped by tile, tile g's keys at
+// [tile_ptr[g], tile_ptr[g+1]) in no particular order within the tile.
+// Malformed input (rowptr not monotone, rowptr[B] != nnz, a column outside
+// [0, L)) is recorded in the head's status word as ELMO_EDATA and the
+// offending entries are dropped.
 //
 // X in FP8 mode: the pages train the classifier in E4M3 without tensor
 // scaling of the weights ("ELMO: Efficiency via Low-precision and Peak Memory
@@ -26,19 +28,26 @@ __device__ __forceinline__ void set_status(int32_t* status, int code, int32_t de
 
 constexpr int kPrepThreads = 1024;
 
+// One CTA.  Shared memory holds the keys and each key's slot in its tile
+// (nnz <= 32768, so a slot fits 16 bits); the per-tile counters and their
+// prefix sums live in tile_ptr itself ([ntg + 1] entries in global memory).
 __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t* __restrict__ rowptr,
                                                                    const int32_t* __restrict__ cols, int32_t B,
-                                                                   int32_t nnz, int64_t L, int32_t npow2,
+                                                                   int32_t nnz, int64_t L,
                                                                    uint32_t* __restrict__ keys_out,
                                                                    int32_t* __restrict__ nkeys,
                                                                    int32_t* __restrict__ tile_ptr,
                                                                    int32_t* __restrict__ status) {
-  extern __shared__ uint32_t sk[];
+  extern __shared__ uint32_t sk[];                                   // [nnz] keys
+  uint16_t* slot = reinterpret_cast<uint16_t*>(sk + nnz);            // [nnz] slot within the tile
   __shared__ int bad_rows;
   __shared__ int nvalid;
   __shared__ int32_t rp[ELMO_MAX_BATCH + 1];
+  __shared__ int32_t part[kPrepThreads];
   const int tid = threadIdx.x;
+  const int ntg = (int)((L + 127) >> 7);     // 128-label tiles of the head
   for (int b = tid; b <= B; b += blockDim.x) rp[b] = rowptr[b];
+  for (int g = tid; g <= ntg; g += blockDim.x) tile_ptr[g] = 0;
   if (tid == 0) nvalid = 0;
   __syncthreads();
   if (tid == 0) bad_rows = (rp[0] != 0 || rp[B] != nnz) ? 1 : 0;
@@ -46,59 +55,57 @@ __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t
   for (int b = tid; b < B; b += blockDim.x)
     if (rp[b + 1] < rp[b]) bad_rows = 1;
   __syncthreads();
-  const int ntg = (int)((L + 127) >> 7);     // 128-label tiles of the head
   if (bad_rows) {
     if (tid == 0) { set_status(status, ELMO_EDATA, -1); *nkeys = 0; }
-    for (int g = tid; g <= ntg; g += blockDim.x) tile_ptr[g] = 0;
-    return;
+    return;                                  // tile_ptr is all zero: no positives anywhere
   }
-  for (int i = tid; i < npow2; i += blockDim.x) {
+  // keys and per-tile counts (counts of tile g accumulate in tile_ptr[g + 1])
+  int cnt = 0;
+  for (int i = tid; i < nnz; i += blockDim.x) {
+    int lo = 0, hi = B;                       // sample b with rowptr[b] <= i < rowptr[b+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (rp[mid] <= i) lo = mid; else hi = mid;
+    }
+    const int32_t c = cols[i];
     uint32_t key = 0xFFFFFFFFu;
-    if (i < nnz) {
-      int lo = 0, hi = B;                     // sample b with rowptr[b] <= i < rowptr[b+1]
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (rp[mid] <= i) lo = mid; else hi = mid;
-      }
-      const int32_t c = cols[i];
-      if (c >= 0 && (int64_t)c < L) key = ((uint32_t)c << 8) | (uint32_t)lo;
-      else set_status(status, ELMO_EDATA, i);
+    if (c >= 0 && (int64_t)c < L) {
+      key = ((uint32_t)c << 8) | (uint32_t)lo;
+      slot[i] = (uint16_t)atomicAdd(&tile_ptr[(c >> 7) + 1], 1);
+      ++cnt;
+    } else {
+      set_status(status, ELMO_EDATA, i);
     }
     sk[i] = key;
   }
-  __syncthreads();
-  // bitonic sort, ascending
-  for (int size = 2; size <= npow2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < npow2; i += blockDim.x) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const uint32_t a = sk[i], c = sk[j];
-          const bool up = (i & size) == 0;
-          if ((a > c) == up) { sk[i] = c; sk[j] = a; }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  int cnt = 0;
-  for (int i = tid; i < nnz; i += blockDim.x) {
-    keys_out[i] = sk[i];
-    cnt += sk[i] != 0xFFFFFFFFu;
-  }
   atomicAdd(&nvalid, cnt);
   __syncthreads();
-  const int nv = nvalid;
-  if (tid == 0) *nkeys = nv;
-  // tile_ptr[g] = first key whose label is in tile g or later (keys are label << 8 | sample)
-  for (int g = tid; g <= ntg; g += blockDim.x) {
-    int lo = 0, hi = nv;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if ((int)(sk[mid] >> 15) < g) lo = mid + 1; else hi = mid;
-    }
-    tile_ptr[g] = lo;
+  // inclusive scan of tile_ptr[1 .. ntg]: each thread a contiguous run, then the runs' totals
+  const int n = ntg + 1;
+  const int per = (n + kPrepThreads - 1) / kPrepThreads;
+  const int g0 = tid * per, g1 = min(n, g0 + per);
+  int32_t run = 0;
+  for (int g = g0; g < g1; ++g) run += __ldcg(tile_ptr + g);   // the counts were formed by L2 atomics
+  part[tid] = run;
+  __syncthreads();
+  for (int o = 1; o < kPrepThreads; o <<= 1) {   // Hillis-Steele scan of the run totals
+    const int32_t v = tid >= o ? part[tid - o] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
   }
+  int32_t acc = part[tid] - run;                 // exclusive prefix of this run
+  for (int g = g0; g < g1; ++g) {
+    acc += __ldcg(tile_ptr + g);
+    tile_ptr[g] = acc;
+  }
+  __syncthreads();
+  // scatter: tile g's keys land in [tile_ptr[g], tile_ptr[g + 1])
+  for (int i = tid; i < nnz; i += blockDim.x) {
+    const uint32_t key = sk[i];
+    if (key != 0xFFFFFFFFu) keys_out[__ldcg(tile_ptr + (key >> 15)) + slot[i]] = key;
+  }
+  if (tid == 0) *nkeys = nvalid;
 }
 
 // One CTA: max |X| with 16-byte loads, the power-of-two scale, then the E4M3
@@ -165,14 +172,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __
 
 cudaError_t launch_prep_labels(elmo_head* h, const int32_t* rowptr, const int32_t* cols, int32_t B,
                                int32_t nnz, cudaStream_t s) {
-  int32_t npow2 = 1;
-  while (npow2 < nnz) npow2 <<= 1;
-  const size_t smem = sizeof(uint32_t) * (size_t)npow2;
+  const size_t smem = (sizeof(uint32_t) + sizeof(uint16_t)) * (size_t)(nnz > 0 ? nnz : 1);
   cudaError_t e = cudaFuncSetAttribute(prep_labels_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)(sizeof(uint32_t) * ELMO_MAX_NNZ));
+                                       (int)((sizeof(uint32_t) + sizeof(uint16_t)) * ELMO_MAX_NNZ));
   if (e != cudaSuccess) return e;
-  prep_labels_kernel<<<1, kPrepThreads, smem, s>>>(rowptr, cols, B, nnz, h->L, npow2, h->keys, h->nkeys,
-                                                   h->tile_ptr, h->status);
+  prep_labels_kernel<<<1, kPrepThreads, smem, s>>>(rowptr, cols, B, nnz, h->L, h->keys, h->nkeys, h->tile_ptr,
+                                                   h->status);
   return cudaGetLastError();
 }
 

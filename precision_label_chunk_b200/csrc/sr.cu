@@ -32,6 +32,22 @@ __global__ void __launch_bounds__(256) sr_round_kernel(const float* __restrict__
   }
 }
 
+// Whole Philox blocks: thread t rounds the 8 values of block q0 + t, read as
+// two 16-byte loads and written as one 8-byte (E4M3) or 16-byte (bf16) store,
+// all streaming (the data are touched once).
+template <int kFp8>
+__global__ void __launch_bounds__(256) sr_round_vec_kernel(const float4* __restrict__ in, void* __restrict__ out,
+                                                           int64_t nblk, uint64_t seed, uint64_t step,
+                                                           uint64_t q0) {
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < nblk; t += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = __ldcs(in + 2 * t), b = __ldcs(in + 2 * t + 1);
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const u32x4 r = sr_block(seed, step, q0 + (uint64_t)t);
+    if (kFp8) __stcs(reinterpret_cast<uint2*>(out) + t, sr8_e4m3(v, r));
+    else __stcs(reinterpret_cast<uint4*>(out) + t, sr8_bf16(v, r));
+  }
+}
+
 __global__ void __launch_bounds__(256) sr_draws_kernel(uint16_t* __restrict__ out, int64_t n, uint64_t seed,
                                                        uint64_t step, uint64_t base) {
   const uint64_t first_blk = base >> 3;
@@ -100,8 +116,39 @@ int grid_for(uint64_t work, int per_block) {
 cudaError_t launch_sr_round(const float* in, void* out, int64_t n, elmo_dtype dt, uint64_t seed,
                             uint64_t step, uint64_t base, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  const uint64_t blocks = (((base + n - 1) >> 3) - (base >> 3)) + 1;
-  sr_round_kernel<<<grid_for(blocks, 256), 256, 0, s>>>(in, out, n, (int)dt, seed, step, base);
+  const size_t esz = dt == ELMO_BF16 ? 2 : 1;
+  const bool aligned = (base & 7) == 0 && (reinterpret_cast<uintptr_t>(in) & 15) == 0 &&
+                       (reinterpret_cast<uintptr_t>(out) & (8 * esz - 1)) == 0;
+  int64_t done = 0;
+  if (aligned && n >= 8) {
+    const int64_t nblk = n / 8;
+    static int per_sm[2] = {0, 0};                  // resident CTAs per SM of each instance
+    const int which = dt == ELMO_BF16 ? 0 : 1;
+    if (!per_sm[which]) {
+      int m = 0;
+      if (dt == ELMO_BF16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, sr_round_vec_kernel<0>, 256, 0);
+      else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, sr_round_vec_kernel<1>, 256, 0);
+      per_sm[which] = m > 0 ? m : 4;
+    }
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    int64_t grid = (nblk + 255) / 256;
+    if (grid > (int64_t)nsm * per_sm[which]) grid = (int64_t)nsm * per_sm[which];
+    const float4* in4 = reinterpret_cast<const float4*>(in);
+    if (dt == ELMO_BF16) sr_round_vec_kernel<0><<<(int)grid, 256, 0, s>>>(in4, out, nblk, seed, step, base >> 3);
+    else sr_round_vec_kernel<1><<<(int)grid, 256, 0, s>>>(in4, out, nblk, seed, step, base >> 3);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    done = nblk * 8;
+    if (done == n) return cudaSuccess;
+  }
+  // values not in whole aligned blocks: one thread per Philox block, element by element
+  const int64_t m = n - done;
+  const uint64_t b0 = base + (uint64_t)done;
+  const uint64_t blocks = (((b0 + m - 1) >> 3) - (b0 >> 3)) + 1;
+  sr_round_kernel<<<grid_for(blocks, 256), 256, 0, s>>>(in + done, static_cast<uint8_t*>(out) + done * esz, m,
+                                                        (int)dt, seed, step, b0);
   return cudaGetLastError();
 }
 

@@ -12,14 +12,13 @@
 namespace elmo {
 namespace {
 
-__device__ __forceinline__ bool is_positive(const uint32_t* keys, int32_t nkeys, int64_t l, int b) {
+// Keys are grouped by 128-label tile (tile g at [tile_ptr[g], tile_ptr[g+1])).
+__device__ __forceinline__ bool is_positive(const uint32_t* keys, const int32_t* tile_ptr, int64_t l, int b) {
   const uint32_t key = ((uint32_t)l << 8) | (uint32_t)b;
-  int lo = 0, hi = nkeys;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (keys[mid] < key) lo = mid + 1; else hi = mid;
-  }
-  return lo < nkeys && keys[lo] == key;
+  const int64_t g = l >> 7;
+  for (int i = tile_ptr[g]; i < tile_ptr[g + 1]; ++i)
+    if (keys[i] == key) return true;
+  return false;
 }
 
 __device__ __forceinline__ float w_at(const void* W, int dt, int64_t i) {
@@ -40,11 +39,10 @@ __device__ __forceinline__ float g_at(const void* gbuf, int dt, int64_t i) {
 __global__ void grad_simt_kernel(const void* __restrict__ W, int dt, int32_t d, const uint16_t* __restrict__ X,
                                  const uint8_t* __restrict__ xq, const float* __restrict__ xscale, int32_t B,
                                  int64_t l0, int64_t l1, const uint32_t* __restrict__ keys,
-                                 const int32_t* __restrict__ nkeys, void* __restrict__ gbuf,
+                                 const int32_t* __restrict__ tile_ptr, void* __restrict__ gbuf,
                                  float* __restrict__ Zout, float* __restrict__ Gout) {
   const int64_t n = (l1 - l0) * B;
   const float inv_sx = dt == ELMO_BF16 ? 1.0f : xscale[1];
-  const int32_t nk = *nkeys;
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < n; t += (int64_t)gridDim.x * blockDim.x) {
     const int64_t l = l0 + t / B;
     const int b = (int)(t % B);
@@ -53,7 +51,7 @@ __global__ void grad_simt_kernel(const void* __restrict__ W, int dt, int32_t d, 
       acc = __fmaf_rn(x_at(X, xq, dt, (int64_t)b * d + j), w_at(W, dt, l * d + j), acc);
     const float z = __fmul_rn(acc, inv_sx);
     const float sig = 1.0f / (1.0f + expf(-z));
-    const float g = sig - (is_positive(keys, nk, l, b) ? 1.0f : 0.0f);
+    const float g = sig - (is_positive(keys, tile_ptr, l, b) ? 1.0f : 0.0f);
     float gv;
     if (dt == ELMO_BF16) {
       const uint16_t c = f32_to_bf16_rn(g);
@@ -123,7 +121,7 @@ cudaError_t launch_grad_simt(const elmo_head* h, const uint16_t* X, int32_t B, i
                              void* gbuf, float* Zout, float* Gout, cudaStream_t s) {
   if (l1 <= l0) return cudaSuccess;
   grad_simt_kernel<<<grid_cap((l1 - l0) * B, 256), 256, 0, s>>>(h->W, (int)h->dt, h->d, X, h->xq, h->xscale, B,
-                                                                 l0, l1, h->keys, h->nkeys, gbuf, Zout, Gout);
+                                                                 l0, l1, h->keys, h->tile_ptr, gbuf, Zout, Gout);
   return cudaGetLastError();
 }
 

@@ -56,6 +56,28 @@ def test_sr_round_large_random_bit_exact(orc):
         assert np.array_equal(got, ref)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("base,off,tail", [(8, 0, 5), (2**35, 0, 0), (0, 1, 3), (16, 4, 7), (2**60 + 8, 0, 1)])
+def test_sr_round_whole_blocks_and_tails(orc, dtype, base, off, tail):
+    """Whole 8-value blocks at 8-aligned indices and 16-byte aligned buffers take
+    the vectorised kernel; a ragged tail, an unaligned index base or a buffer
+    that starts off a 16-byte boundary take the per-value kernel: all must give
+    the oracle's codes."""
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    x = _adversarial(dtype, np.random.default_rng(base & 0xFFFF))
+    n = (x.size // 8) * 8 - 8 + tail
+    ref = orc.sr_round(x[off:off + n], dtype, 21, 4, base)
+    xd = torch.from_numpy(x).cuda()[off:off + n]          # off > 0: the input starts 4*off bytes past alignment
+    odt = torch.int16 if dtype == "bf16" else torch.uint8
+    out_full = torch.empty(n + off, dtype=odt, device="cuda")
+    out = out_full[off:]
+    elmo.elmo_sr_round(xd, out, dtype, 21, 4, base)
+    got = out.cpu().numpy().view(np.uint16 if dtype == "bf16" else np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, f"{bad.size} mismatches, first at {bad[:5]}"
+
+
 @pytest.mark.parametrize("seed,step,base,n", [(0, 0, 0, 1000), (5, 9, 3, 4097), (2**64 - 1, 2**62, 2**50 + 7, 777)])
 def test_draws_bit_exact(orc, seed, step, base, n):
     need_gpu()
