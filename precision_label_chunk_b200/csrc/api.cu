@@ -43,6 +43,13 @@ cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 // Development switch: ELMO_STEP_SIMT=1 runs the CUDA-core kernels of the step
 // instead of the tensor-core ones (both on the GPU).
+// ELMO_TOPK_SIMT=1 runs top-k prediction on CUDA cores only (every score by
+// its exact chain), the comparison path of the tensor-core screening.
+bool use_topk_simt() {
+  const char* v = getenv("ELMO_TOPK_SIMT");
+  return v && v[0] == '1';
+}
+
 bool use_simt() {
   const char* v = getenv("ELMO_STEP_SIMT");
   return v && v[0] == '1';
@@ -384,10 +391,16 @@ elmo_status elmo_topk_predict(elmo_head* h, const void* X_dev, int32_t B, int32_
   if (!aligned16(X_dev)) return fail(ELMO_EINVAL, "X is not 16-byte aligned");
   elmo_status st = check_device(h);
   if (st != ELMO_OK) return st;
-  if ((st = ensure_cand(h, elmo::topk_workspace_bytes(h, B, k))) != ELMO_OK) return st;
+  const uint16_t* X = static_cast<const uint16_t*>(X_dev);
+  if (elmo::topk_tc_supported(h) && !use_topk_simt()) {
+    if ((st = ensure_cand(h, elmo::topk_tc_workspace_bytes(h, B, k))) != ELMO_OK) return st;
+    ELMO_CUDA(elmo::launch_topk_tc(h, X, B, k, idx_dev, score_dev, as_stream(stream)), "topk");
+    return ELMO_OK;
+  }
+  if ((st = ensure_cand(h, elmo::topk_simt_workspace_bytes(h, B, k))) != ELMO_OK) return st;
   elmo::KernelScope ks(h, ELMO_K_TOPK_SCORE, as_stream(stream), 2);
-  ELMO_CUDA(elmo::launch_topk_simt(h, static_cast<const uint16_t*>(X_dev), B, k, chunk, idx_dev, score_dev,
-                                   as_stream(stream)),
+  ELMO_CUDA(elmo::launch_topk_simt_rows(h, X, B, k, nullptr, nullptr, h->cand, idx_dev, score_dev,
+                                        as_stream(stream)),
             "topk");
   return ELMO_OK;
 }

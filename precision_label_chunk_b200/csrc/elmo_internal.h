@@ -9,6 +9,8 @@
 
 #include "../../include/elmo.h"
 
+struct CUtensorMap_st;   // cuda.h's TMA descriptor (CUtensorMap)
+
 struct elmo_prof_rec {
   int cls;
   cudaEvent_t start, stop;
@@ -86,16 +88,28 @@ cudaError_t launch_update_simt(const elmo_head* h, const uint16_t* X, int32_t B,
                                const void* gbuf, float lr, uint64_t seed, uint64_t step, cudaStream_t s);
 
 // step_tc.cu -- tensor-core step
+// 2-D row-major TMA map [rows x cols] of 1- or 2-byte elements, box = 128 bytes
+// x box_rows, 128-byte swizzle, zero fill outside the tensor.
+cudaError_t make_tma_map_2d(CUtensorMap_st* m, const void* ptr, int elem_bytes, uint64_t cols, uint64_t rows,
+                            uint64_t row_stride_elems, uint32_t box_rows);
 int32_t padded_batch(int32_t B, bool fp8);
 cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
                                   void* gbuf, float* Zout, float* Gout, cudaStream_t s);
 cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
                              const void* gbuf, float lr, uint64_t seed, uint64_t step, float* dX, cudaStream_t s);
 
-// topk_simt.cu
-size_t topk_workspace_bytes(const elmo_head* h, int32_t B, int32_t k);
-cudaError_t launch_topk_simt(elmo_head* h, const uint16_t* X, int32_t B, int32_t k, int64_t chunk,
-                             int32_t* idx, float* score, cudaStream_t s);
+// topk_simt.cu -- exact top-k on CUDA cores, for all rows (rows == null) or
+// for the *nrows rows listed in rows (a list whose length lives on the device)
+size_t topk_simt_workspace_bytes(const elmo_head* h, int32_t B, int32_t k);
+cudaError_t launch_topk_simt_rows(const elmo_head* h, const uint16_t* X, int32_t B, int32_t k, const int32_t* rows,
+                                  const int32_t* nrows, void* cand, int32_t* idx, float* score, cudaStream_t s);
+
+// topk_tc.cu -- tensor-core screening, exact rescoring and certificate, with
+// the CUDA-core path for the rows the certificate does not clear
+bool topk_tc_supported(const elmo_head* h);
+size_t topk_tc_workspace_bytes(const elmo_head* h, int32_t B, int32_t k);
+cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k, int32_t* idx, float* score,
+                           cudaStream_t s);
 
 // sr.cu
 cudaError_t launch_sr_round(const float* in, void* out, int64_t n, elmo_dtype dt, uint64_t seed,

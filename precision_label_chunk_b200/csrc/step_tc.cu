@@ -797,11 +797,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
+constexpr size_t kSmemA = 1024 + kStagesA * kStageABytes + sizeof(SmemA);
+constexpr size_t kSmemB = 1024 + kXBytes + kWSlots * kWSlotBytes + kGSlots * kGSlotBytes + sizeof(SmemB);
+constexpr size_t kSmemP = 1024 + kPanelSmem + sizeof(SmemP);
+static_assert(kSmemA <= 232448, "kernel A shared memory");
+static_assert(kSmemP <= 232448, "kernel A (resident X) shared memory");
+static_assert(kSmemB <= 232448, "kernel B shared memory");
+
+}  // namespace
+
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeFn encode_fn() {
+static EncodeFn encode_fn() {
   static EncodeFn fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -814,7 +823,7 @@ EncodeFn encode_fn() {
 }
 
 // 2-D row-major map [rows x cols] of 1- or 2-byte elements, box = 128 bytes x box_rows, 128B swizzle.
-cudaError_t make_map(CUtensorMap* m, const void* ptr, int elem_bytes, uint64_t cols, uint64_t rows,
+cudaError_t make_tma_map_2d(CUtensorMap* m, const void* ptr, int elem_bytes, uint64_t cols, uint64_t rows,
                      uint64_t row_stride_elems, uint32_t box_rows) {
   EncodeFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -828,15 +837,6 @@ cudaError_t make_map(CUtensorMap* m, const void* ptr, int elem_bytes, uint64_t c
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
-
-constexpr size_t kSmemA = 1024 + kStagesA * kStageABytes + sizeof(SmemA);
-constexpr size_t kSmemB = 1024 + kXBytes + kWSlots * kWSlotBytes + kGSlots * kGSlotBytes + sizeof(SmemB);
-constexpr size_t kSmemP = 1024 + kPanelSmem + sizeof(SmemP);
-static_assert(kSmemA <= 232448, "kernel A shared memory");
-static_assert(kSmemP <= 232448, "kernel A (resident X) shared memory");
-static_assert(kSmemB <= 232448, "kernel B shared memory");
-
-}  // namespace
 
 // Samples are padded to whole 128-byte swizzle atoms of the operand type
 // (64 bf16 or 128 E4M3 values): padded rows of X are zero-filled by TMA and
@@ -853,9 +853,9 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
   const int eb = fp8 ? 1 : 2;
   const int32_t Bp = padded_batch(B, fp8);
   CUtensorMap tmW, tmX;
-  cudaError_t e = make_map(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, 128);
+  cudaError_t e = make_tma_map_2d(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, 128);
   if (e != cudaSuccess) return e;
-  e = make_map(&tmX, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
+  e = make_tma_map_2d(&tmX, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
                (uint64_t)B, (uint64_t)h->d, (uint32_t)Bp);
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((l1 - l0 + 127) / 128);
@@ -874,7 +874,7 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
   }
   if (PN >= 64) {
     CUtensorMap tmXp;
-    e = make_map(&tmXp, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
+    e = make_tma_map_2d(&tmXp, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
                  (uint64_t)B, (uint64_t)h->d, (uint32_t)PN);
     if (e != cudaSuccess) return e;
     auto kp = fp8 ? logits_grad_panel_tc<1> : logits_grad_panel_tc<0>;
@@ -899,9 +899,9 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
   const int eb = fp8 ? 1 : 2;
   const int32_t Bp = padded_batch(B, fp8);
   CUtensorMap tmW, tmX;
-  cudaError_t e = make_map(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, 128);
+  cudaError_t e = make_tma_map_2d(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, 128);
   if (e != cudaSuccess) return e;
-  e = make_map(&tmX, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
+  e = make_tma_map_2d(&tmX, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
                (uint64_t)B, (uint64_t)h->d, (uint32_t)Bp);
   if (e != cudaSuccess) return e;
   const int T = (int)((l1 - l0 + 127) / 128);

@@ -55,3 +55,61 @@ def test_topk_exact_ties(orc):
     ri, rs = orc.topk(W, X, k, "fp8")
     assert np.array_equal(idx, ri)
     assert np.array_equal(sc, rs)
+
+
+def _topk_dev(elmo, Wd, h, X, k, chunk=131072):
+    idx = torch.empty(X.shape[0], k, dtype=torch.int32, device="cuda")
+    sc = torch.empty(X.shape[0], k, dtype=torch.float32, device="cuda")
+    elmo.elmo_topk_predict(h, to_dev_u16(X), k, chunk, idx, sc)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), sc.cpu().numpy()
+
+
+@pytest.mark.parametrize("dtype,L,d,B,k", [("bf16", 6000, 768, 40, 5), ("fp8", 9001, 768, 300, 17),
+                                           ("fp8", 65, 64, 3, 5), ("bf16", 130, 192, 129, 64),
+                                           ("fp8", 40000, 512, 1024, 1)])
+def test_topk_tensor_core_screening_matches_oracle(orc, dtype, L, d, B, k, monkeypatch):
+    """Shapes that stress the screening layout: the widest A operand (d = 768),
+    several query panels with a partial last one, heads smaller than a
+    candidate list, k above 16 (64 candidates per range) and k = 1.  The
+    result must equal the oracle's, and the CUDA-core path's."""
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("topk5_3m_fp8", L=L, d=d, B=B)
+    X = make_X(w, 3)
+    W = orc.sr_round(make_W_f32(w), dtype, 1, 2**64 - 1)
+    Wd = w_to_dev(W, dtype)
+    h = elmo.elmo_init_head(Wd, dtype)
+    idx, sc = _topk_dev(elmo, Wd, h, X, k)
+    rows = np.arange(B) if B <= 64 else np.array([0, 1, 127, 128, B // 2, B - 1])
+    ri, rs = orc.topk(W, X, k, dtype, rows=rows)
+    assert np.array_equal(idx[rows], ri)
+    assert np.array_equal(sc[rows].view(np.uint32), rs.view(np.uint32))
+    monkeypatch.setenv("ELMO_TOPK_SIMT", "1")
+    si, ss = _topk_dev(elmo, Wd, h, X, k)
+    assert np.array_equal(si, idx)
+    assert np.array_equal(ss.view(np.uint32), sc.view(np.uint32))
+    h.close()
+
+
+@pytest.mark.parametrize("case", ["nan_weight", "inf_query"])
+def test_topk_uncertified_rows_take_exact_path(orc, case):
+    """A NaN weight leaves no finite bound on |W|: every row must be recomputed
+    exactly (NaN scores rank last).  An infinite query value voids that row's
+    bound only."""
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("topk5_3m_fp8", L=3000, d=128, B=20)
+    X = make_X(w, 4)
+    W = orc.sr_round(make_W_f32(w), "fp8", 2, 2**64 - 1)
+    if case == "nan_weight":
+        W[17, 5] = 0x7F
+    else:
+        X[3, 9] = 0x7F80
+    Wd = w_to_dev(W, "fp8")
+    h = elmo.elmo_init_head(Wd, "fp8")
+    idx, sc = _topk_dev(elmo, Wd, h, X, 5)
+    ri, rs = orc.topk(W, X, 5, "fp8")
+    assert np.array_equal(idx, ri)
+    assert np.array_equal(sc.view(np.uint32), rs.view(np.uint32))
+    h.close()
