@@ -10,7 +10,8 @@
 //
 //   1. screening (tcgen05): approximate scores S~ = X W^T for all labels, each
 //      CTA keeping, per query, the kp best approximate scores of its label
-//      range (kp >= k) and the best score it did not keep;
+//      range (kp >= k) and the smallest of them, which bounds every score of
+//      the range it did not keep;
 //   2. selection: per query, the kp best candidates over all ranges, their
 //      exact chain scores, the top-k of those, and a certificate: if the k-th
 //      exact score exceeds every non-candidate's approximate score by more
@@ -189,6 +190,47 @@ __global__ void __launch_bounds__(256) topk_wmax_kernel(const uint4* __restrict_
 }
 
 // ---------------------------------------------------------------- stage 1: tensor-core screening
+// Each epilogue thread keeps its query's best kp approximate scores of the
+// CTA's label range as a binary min-heap in shared memory (element i of the
+// thread in column r at [i * 128 + r]): the root is the admission threshold,
+// and a new score above it replaces the root and sifts down (log2 kp steps).
+__device__ __forceinline__ void heap_sift_down(float* hs, int32_t* hl, int r, int i, int kp) {
+  const float v = hs[i * 128 + r];
+  const int32_t vl = hl[i * 128 + r];
+  while (true) {
+    int c = 2 * i + 1;
+    if (c >= kp) break;
+    float cv = hs[c * 128 + r];
+    if (c + 1 < kp) {
+      const float c2 = hs[(c + 1) * 128 + r];
+      if (c2 < cv) { cv = c2; ++c; }
+    }
+    if (!(cv < v)) break;
+    hs[i * 128 + r] = cv;
+    hl[i * 128 + r] = hl[c * 128 + r];
+    i = c;
+  }
+  hs[i * 128 + r] = v;
+  hl[i * 128 + r] = vl;
+}
+
+// Adds (z, lab) as the cnt-th kept score (cnt < kp: the heap is still being
+// filled) or in place of the root; returns the new threshold: -inf until kp
+// scores are kept, then the smallest kept score.
+__device__ __noinline__ float keep_candidate(float* hs, int32_t* hl, int r, int cnt, int kp, float z, int32_t lab) {
+  if (cnt < kp) {
+    hs[cnt * 128 + r] = z;
+    hl[cnt * 128 + r] = lab;
+    if (cnt + 1 < kp) return -INFINITY;
+    for (int i = kp / 2 - 1; i >= 0; --i) heap_sift_down(hs, hl, r, i, kp);
+    return hs[r];
+  }
+  hs[r] = z;
+  hl[r] = lab;
+  heap_sift_down(hs, hl, r, 0, kp);
+  return hs[r];
+}
+
 template <int kFp8>
 __global__ void __launch_bounds__(kSThreads, 1)
     topk_screen_tc(const __grid_constant__ CUtensorMap tmW, int64_t L, int32_t d, int32_t B, int32_t kp,
@@ -298,7 +340,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     const int row = p * 128 + r;
     const bool live = row < B;
     for (int i = 0; i < kp; ++i) { ls[i * 128 + r] = -INFINITY; li[i * 128 + r] = -1; }
-    float tau = -INFINITY;   // the kp-th kept (scaled) score once kp are kept
+    float tau = -INFINITY;   // the smallest kept (scaled) score once kp are kept
     int cnt = 0;
     uint32_t tc = 0;
     for (int64_t t = t0; t < t1 && !*abort; ++t, ++tc) {
@@ -318,18 +360,9 @@ __global__ void __launch_bounds__(kSThreads, 1)
 #pragma unroll
       for (int c = 0; c < kSN; ++c) {
         const float z = __uint_as_float(c < 32 ? v0[c] : v1[c - 32]);
-        if (z > tau && lb + c < L) {
-          // insert; equal scores keep the earlier (lower) label first
-          int pos = cnt < kp ? cnt : kp - 1;
+        if (z > tau && lb + c < L) {   // equal scores never displace an earlier (lower) label
+          tau = keep_candidate(ls, li, r, cnt, kp, z, (int32_t)(lb + c));
           if (cnt < kp) ++cnt;
-          while (pos > 0 && ls[(pos - 1) * 128 + r] < z) {
-            ls[pos * 128 + r] = ls[(pos - 1) * 128 + r];
-            li[pos * 128 + r] = li[(pos - 1) * 128 + r];
-            --pos;
-          }
-          ls[pos * 128 + r] = z;
-          li[pos * 128 + r] = (int32_t)(lb + c);
-          if (cnt == kp) tau = ls[(kp - 1) * 128 + r];
         }
       }
     }
