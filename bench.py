@@ -256,9 +256,17 @@ def run_topk(args, w, rank, world, local):
     roof = None
     if dominant == "topk_score":
         t_k = classes[dominant]["ms"] / 1e3 / args.steps
-        peak, bound, src = alu_peak_tflops(peaks), "alu", "derived: 148 SM x 128 FMA x 2 x max clock"
+        if os.environ.get("ELMO_TOPK_SIMT", "0") == "1":
+            peak, bound, src = alu_peak_tflops(peaks), "alu", "derived: 148 SM x 128 FMA x 2 x max clock"
+        else:
+            # tensor-core screening: the algorithmic 2 B L d flops against the dense
+            # peak of the operand type (E4M3 heads issue the contraction twice, for
+            # the two E4M3 parts of the bf16 queries, so their ceiling is frac = 0.5)
+            peak, bound = tensor_peak_tflops(peaks, w.dtype), "tensor"
+            src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype == "fp8" else ""))
         roof = {"kernel": dominant, "bound": bound, "achieved": flops / t_k / 1e12, "peak": peak, "unit": "TFLOP/s",
-                "frac": flops / t_k / 1e12 / peak, "traffic": None, "peak_source": src}
+                "frac": flops / t_k / 1e12 / peak, "traffic": None, "peak_source": src,
+                "mma_passes": 2 if (w.dtype == "fp8" and bound == "tensor") else 1}
     # end to end: X from pinned host memory, indices and scores back every step
     pin = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in Xh]
     idx_h = torch.empty(w.B, w.topk, dtype=torch.int32).pin_memory()

@@ -60,9 +60,10 @@ namespace {
 using namespace tc;
 
 constexpr int kSThreads = 192;                   // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
+constexpr int kN = 64;                           // labels per tile (the MMA's N)
+constexpr uint32_t kSBox = kN * 128;             // one W k-block: 64 labels x 128 bytes
 constexpr int kSStages = 16;
-constexpr uint32_t kSBox = 8192;                 // one W k-block: 64 labels x 128 bytes
-constexpr int kSN = 64;                          // labels per tile (MMA N)
+constexpr int kNBuf = 2;                         // accumulator buffers
 constexpr uint32_t kSAcc = 384;                  // first accumulator column (A operands below)
 constexpr long long kSWait = 4000000000LL;       // ~2 s at 2 GHz
 constexpr int32_t kEmpty = 0x7FFFFFFF;
@@ -70,7 +71,7 @@ constexpr int kPrepT = 128;
 constexpr int kSelThreads = 512;
 
 struct SmemS {
-  uint64_t wfull[kSStages], wempty[kSStages], tfull[2], tempty[2];
+  uint64_t wfull[kSStages], wempty[kSStages], tfull[kNBuf], tempty[kNBuf];
   uint32_t tmem_base;
   int abort;
 };
@@ -111,11 +112,13 @@ __global__ void __launch_bounds__(kPrepT) topk_xprep_kernel(const uint16_t* __re
                                                             uint8_t* __restrict__ xa, uint8_t* __restrict__ xb,
                                                             float* __restrict__ xinv, float* __restrict__ n1,
                                                             float* __restrict__ r1, int32_t* __restrict__ rflag,
-                                                            uint32_t* __restrict__ wmax, int32_t* __restrict__ nfail) {
+                                                            uint32_t* __restrict__ wmax, int32_t* __restrict__ nfail,
+                                                            uint32_t* __restrict__ tshare) {
   __shared__ float red[kPrepT / 32];
   __shared__ uint32_t mx;
   const int b = blockIdx.x, tid = threadIdx.x;
   if (b == 0 && tid == 0) { *wmax = 0; *nfail = 0; }
+  if (tid == 0) tshare[b] = 0;
   if (tid == 0) mx = 0;
   __syncthreads();
   const uint16_t* xr = X + (size_t)b * d;
@@ -217,7 +220,7 @@ __device__ __forceinline__ void heap_sift_down(float* hs, int32_t* hl, int r, in
 // Adds (z, lab) as the cnt-th kept score (cnt < kp: the heap is still being
 // filled) or in place of the root; returns the new threshold: -inf until kp
 // scores are kept, then the smallest kept score.
-__device__ __noinline__ float keep_candidate(float* hs, int32_t* hl, int r, int cnt, int kp, float z, int32_t lab) {
+__device__ __forceinline__ float keep_candidate(float* hs, int32_t* hl, int r, int cnt, int kp, float z, int32_t lab) {
   if (cnt < kp) {
     hs[cnt * 128 + r] = z;
     hl[cnt * 128 + r] = lab;
@@ -231,22 +234,40 @@ __device__ __noinline__ float keep_candidate(float* hs, int32_t* hl, int r, int 
   return hs[r];
 }
 
+// Float <-> unsigned key with the same order (for atomicMax on a threshold);
+// key 0 stands for "no threshold yet" (-inf).
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord_value(uint32_t k) {
+  return k == 0 ? -INFINITY : __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Every label range of a query publishes its heap threshold (once its heap is
+// full) to tshare[query]; all ranges reject scores at or below the largest
+// published one.  That is sound for the certificate: a label not kept has an
+// approximate score at most the threshold that was in force, and the output
+// thr of a range is the largest threshold it used.
+// Tiles of 64 labels (the MMA's N) with two accumulator buffers: the A
+// operands take 384 of the 512 TMEM columns.
 template <int kFp8>
 __global__ void __launch_bounds__(kSThreads, 1)
     topk_screen_tc(const __grid_constant__ CUtensorMap tmW, int64_t L, int32_t d, int32_t B, int32_t kp,
                    int32_t ngroups, const uint8_t* __restrict__ xa, const uint8_t* __restrict__ xb,
                    const float* __restrict__ xinv, float* __restrict__ cand_s, int32_t* __restrict__ cand_i,
-                   float* __restrict__ thr, int32_t* __restrict__ status) {
+                   float* __restrict__ thr, uint32_t* __restrict__ tshare, int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = base;                                                   // kSStages W k-blocks
-  float* ls = reinterpret_cast<float*>(base + kSStages * kSBox);          // [kp][128] kept scores (scaled)
+  float* zs = reinterpret_cast<float*>(base + kSStages * kSBox);          // [kN][128] a tile's scores
+  float* ls = zs + kN * 128;                                              // [kp][128] kept scores (scaled)
   int32_t* li = reinterpret_cast<int32_t*>(ls + (size_t)kp * 128);        // [kp][128] their labels
   SmemS* S = reinterpret_cast<SmemS*>(li + (size_t)kp * 128);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int P = (B + 127) / 128;
   const int p = blockIdx.x % P, g = blockIdx.x / P;
-  const int64_t T = (L + kSN - 1) / kSN;
+  const int64_t T = (L + kN - 1) / kN;
   const int64_t t0 = T * g / ngroups, t1 = T * (g + 1) / ngroups;
   const int kbe = kFp8 ? 128 : 64;                  // elements of one 128-byte k-block
   const int nkb = (d + kbe - 1) / kbe;
@@ -256,7 +277,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSStages; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
-    for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], 4); }
+    for (int b2 = 0; b2 < kNBuf; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], 4); }
     S->abort = 0;
     fence_barrier_init();
   }
@@ -301,19 +322,19 @@ __global__ void __launch_bounds__(kSThreads, 1)
           const uint32_t ph = (it / kSStages) & 1;
           if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kSWait)) { record_timeout(status, abort, 61); break; }
           mbar_arrive_expect_tx(&S->wfull[s], kSBox);
-          tma_load_2d(ring + s * kSBox, &tmW, &S->wfull[s], kb * kbe, (int32_t)(t * kSN));
+          tma_load_2d(ring + s * kSBox, &tmW, &S->wfull[s], kb * kbe, (int32_t)(t * kN));
         }
       }
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, kSN) : make_idesc(1, 1, 0, 0, 128, kSN);
+      const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, kN) : make_idesc(1, 1, 0, 0, 128, kN);
       uint32_t it = 0, tc = 0;
       for (int64_t t = t0; t < t1 && !*abort; ++t, ++tc) {
-        const uint32_t buf = tc & 1, use = tc >> 1;
+        const uint32_t buf = tc % kNBuf, use = tc / kNBuf;
         if (!mbar_wait(&S->tempty[buf], (use & 1) ^ 1, abort, kSWait)) { record_timeout(status, abort, 62); break; }
         tc_fence_after();
-        const uint32_t dcol = tmem + kSAcc + buf * kSN;
+        const uint32_t dcol = tmem + kSAcc + buf * kN;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = (int)(it % kSStages);
           const uint32_t ph = (it / kSStages) & 1;
@@ -341,30 +362,49 @@ __global__ void __launch_bounds__(kSThreads, 1)
     const bool live = row < B;
     for (int i = 0; i < kp; ++i) { ls[i * 128 + r] = -INFINITY; li[i * 128 + r] = -1; }
     float tau = -INFINITY;   // the smallest kept (scaled) score once kp are kept
+    float tused = -INFINITY; // the largest rejection threshold used so far
     int cnt = 0;
     uint32_t tc = 0;
     for (int64_t t = t0; t < t1 && !*abort; ++t, ++tc) {
-      const uint32_t buf = tc & 1, use = tc >> 1;
+      const uint32_t buf = tc % kNBuf, use = tc / kNBuf;
       if (!mbar_wait(&S->tfull[buf], use & 1, abort, kSWait)) { record_timeout(status, abort, 64); break; }
       tc_fence_after();
-      uint32_t v0[32], v1[32];
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + kSAcc + buf * kSN;
-      tmem_ld32(taddr, v0);
-      tmem_ld32(taddr + 32, v1);
+      uint32_t v[kN / 32][32];
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + kSAcc + buf * kN;
+#pragma unroll
+      for (int h = 0; h < kN / 32; ++h) tmem_ld32(taddr + 32 * h, v[h]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->tempty[buf]);
       if (!live) continue;
-      const int64_t lb = t * kSN;
+      const int64_t lb = t * kN;
+      float teff = fmaxf(tau, ord_value(__ldcg(tshare + row)));
+      // scores above the threshold, as a bit mask (the selection code below is
+      // kept out of the unrolled scan so that it exists once in the binary)
+      uint64_t mask = 0;
 #pragma unroll
-      for (int c = 0; c < kSN; ++c) {
-        const float z = __uint_as_float(c < 32 ? v0[c] : v1[c - 32]);
-        if (z > tau && lb + c < L) {   // equal scores never displace an earlier (lower) label
-          tau = keep_candidate(ls, li, r, cnt, kp, z, (int32_t)(lb + c));
-          if (cnt < kp) ++cnt;
+      for (int c = 0; c < kN; ++c)
+        mask |= (uint64_t)(__uint_as_float(v[c >> 5][c & 31]) > teff) << c;
+      if (lb + kN > L) mask &= L - lb >= 64 ? ~0ull : ((1ull << (L - lb)) - 1);
+      if (mask) {
+#pragma unroll
+        for (int c = 0; c < kN; ++c) zs[c * 128 + r] = __uint_as_float(v[c >> 5][c & 31]);
+        while (mask) {
+          const int c = __ffsll((long long)mask) - 1;
+          mask &= mask - 1;
+          const float z = zs[c * 128 + r];
+          if (z > teff) {   // labels arrive in order: equal scores never displace an earlier (lower) label
+            tau = keep_candidate(ls, li, r, cnt, kp, z, (int32_t)(lb + c));
+            if (cnt < kp) ++cnt;
+            if (tau > teff) {
+              teff = tau;
+              atomicMax(tshare + row, ord_key(tau));
+            }
+          }
         }
       }
+      tused = fmaxf(tused, teff);
     }
     if (live) {
       const float inv = xinv[row];
@@ -374,7 +414,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
         cand_s[o + i] = id >= 0 ? __fmul_rn(ls[i * 128 + r], inv) : -INFINITY;
         cand_i[o + i] = id >= 0 ? id : kEmpty;
       }
-      thr[(size_t)row * ngroups + g] = cnt == kp ? __fmul_rn(tau, inv) : -INFINITY;
+      thr[(size_t)row * ngroups + g] = __fmul_rn(tused, inv);
     }
   }
   __syncthreads();
@@ -502,20 +542,21 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(
 }
 
 struct TopkLayout {
-  int P, G, kp, npow2;
-  size_t xa, xb, xinv, n1, r1, rflag, wmax, nfail, fail, cs, ci, thr, simt, total;
+  int P, G, kp, npow2, N;
+  size_t xa, xb, xinv, n1, r1, rflag, wmax, nfail, fail, cs, ci, thr, tshare, simt, total;
 };
 
 TopkLayout topk_layout(const elmo_head* h, int32_t B, int32_t k) {
   TopkLayout o{};
   const bool fp8 = h->dt == ELMO_FP8_E4M3;
   o.P = (B + 127) / 128;
-  const int64_t T = (h->L + kSN - 1) / kSN;
+  o.N = kN;
+  const int64_t T = (h->L + o.N - 1) / o.N;
   int64_t G = h->num_sms / o.P;
   if (G < 1) G = 1;
   if (G > T) G = T;
   o.G = (int)G;
-  o.kp = k <= 16 ? 32 : 64;
+  o.kp = k <= 8 ? 16 : (k <= 16 ? 32 : 64);
   o.npow2 = 1;
   while (o.npow2 < o.G * o.kp) o.npow2 <<= 1;
   size_t off = 0;
@@ -532,12 +573,14 @@ TopkLayout topk_layout(const elmo_head* h, int32_t B, int32_t k) {
   o.cs = take(sizeof(float) * (size_t)B * o.G * o.kp);
   o.ci = take(sizeof(int32_t) * (size_t)B * o.G * o.kp);
   o.thr = take(sizeof(float) * (size_t)B * o.G);
+  o.tshare = take(sizeof(uint32_t) * (size_t)B);
   o.simt = take(topk_simt_workspace_bytes(h, B, k));
   o.total = off;
   return o;
 }
 
-constexpr size_t kScreenSmem = 1024 + kSStages * kSBox + 2 * sizeof(float) * 64 * 128 + sizeof(SmemS);
+constexpr size_t kScreenSmem = 1024 + kSStages * kSBox + sizeof(float) * kN * 128 + 2 * sizeof(float) * 64 * 128 +
+                                sizeof(SmemS);
 static_assert(kScreenSmem <= 232448, "screening kernel shared memory");
 
 }  // namespace
@@ -567,11 +610,12 @@ cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k
   float* cs = reinterpret_cast<float*>(ws + o.cs);
   int32_t* ci = reinterpret_cast<int32_t*>(ws + o.ci);
   float* thr = reinterpret_cast<float*>(ws + o.thr);
+  uint32_t* tshare = reinterpret_cast<uint32_t*>(ws + o.tshare);
 
   // stage 0
   KernelScope* scope = new KernelScope(h, ELMO_K_PREP, s, 2);
-  if (fp8) topk_xprep_kernel<1><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail);
-  else topk_xprep_kernel<0><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail);
+  if (fp8) topk_xprep_kernel<1><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail, tshare);
+  else topk_xprep_kernel<0><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail, tshare);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t n16 = h->L * (int64_t)h->d * (fp8 ? 1 : 2) / 16;
@@ -584,16 +628,17 @@ cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k
   // stage 1
   CUtensorMap tmW;
   const int eb = fp8 ? 1 : 2;
-  e = make_tma_map_2d(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, (uint32_t)kSN);
+  e = make_tma_map_2d(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, (uint32_t)o.N);
   if (e != cudaSuccess) return e;
-  const size_t smem = 1024 + kSStages * kSBox + 2 * sizeof(float) * (size_t)o.kp * 128 + sizeof(SmemS);
+  const size_t smem = 1024 + kSStages * kSBox + sizeof(float) * kN * 128 + 2 * sizeof(float) * (size_t)o.kp * 128 +
+                      sizeof(SmemS);
   auto ks = fp8 ? topk_screen_tc<1> : topk_screen_tc<0>;
   e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScreenSmem);
   if (e != cudaSuccess) return e;
   {
     KernelScope sc(h, ELMO_K_TOPK_SCORE, s, 1);
     ks<<<o.P * o.G, kSThreads, smem, s>>>(tmW, h->L, h->d, B, o.kp, o.G,
-                                          fp8 ? xa : reinterpret_cast<const uint8_t*>(X), xb, xinv, cs, ci, thr,
+                                          fp8 ? xa : reinterpret_cast<const uint8_t*>(X), xb, xinv, cs, ci, thr, tshare,
                                           h->status);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
