@@ -239,6 +239,9 @@ elmo_status elmo_head_destroy(elmo_head* h) {
   if (h->gbuf) cudaFree(h->gbuf);
   if (h->cand) cudaFree(h->cand);
   if (h->status) cudaFree(h->status);
+  if (h->side) cudaStreamDestroy(h->side);
+  if (h->fork) cudaEventDestroy(h->fork);
+  if (h->join) cudaEventDestroy(h->join);
   for (auto& r : h->prof_recs) { cudaEventDestroy(r.start); cudaEventDestroy(r.stop); }
   for (auto e : h->prof_pool) cudaEventDestroy(e);
   delete h;

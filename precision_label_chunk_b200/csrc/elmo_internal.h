@@ -25,9 +25,11 @@ struct elmo_head {
   int num_sms = 0;
   // workspace owned by the head
   int32_t* status = nullptr;   // [4]: status code, first bad index, spare
-  uint32_t* keys = nullptr;    // [ELMO_MAX_NNZ] sorted (label << 8 | sample) positives
+  uint32_t* keys = nullptr;    // [ELMO_MAX_NNZ] (label << 8 | sample) positives grouped by label tile
   int32_t* nkeys = nullptr;    // [1] number of valid keys
   int32_t* tile_ptr = nullptr; // [ceil(L/128) + 1] first key of every 128-label tile
+  cudaStream_t side = nullptr; // second stream for work that overlaps a kernel of the caller's stream
+  cudaEvent_t fork = nullptr, join = nullptr;
   float* xscale = nullptr;     // [2] s_X, 1/s_X (fp8 mode)
   uint8_t* xq = nullptr;       // [ELMO_MAX_BATCH x d] E4M3 codes of X * s_X (fp8 mode)
   void* gbuf = nullptr;        // per-chunk gradient operands

@@ -613,17 +613,34 @@ cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k
   uint32_t* tshare = reinterpret_cast<uint32_t*>(ws + o.tshare);
 
   // stage 0
-  KernelScope* scope = new KernelScope(h, ELMO_K_PREP, s, 2);
-  if (fp8) topk_xprep_kernel<1><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail, tshare);
-  else topk_xprep_kernel<0><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail, tshare);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  {
+    KernelScope sc(h, ELMO_K_PREP, s, 1);
+    if (fp8) topk_xprep_kernel<1><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail, tshare);
+    else topk_xprep_kernel<0><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail, tshare);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
-  const int64_t n16 = h->L * (int64_t)h->d * (fp8 ? 1 : 2) / 16;
-  const int wgrid = h->num_sms * 8;
-  if (fp8) topk_wmax_kernel<1><<<wgrid, 256, 0, s>>>(static_cast<const uint4*>(h->W), n16, wmax);
-  else topk_wmax_kernel<0><<<wgrid, 256, 0, s>>>(static_cast<const uint4*>(h->W), n16, wmax);
-  delete scope;
+
+  // max|W| streams the head from HBM while the screening kernel (tensor-bound,
+  // light on HBM) runs: a second stream, forked after the clears of stage 0
+  // and joined before the selection
+  if (!h->side) {
+    if ((e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&h->join, cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  if ((e = cudaEventRecord(h->fork, s)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(h->side, h->fork, 0)) != cudaSuccess) return e;
+  {
+    KernelScope sc(h, ELMO_K_PREP, h->side, 1);
+    const int64_t n16 = h->L * (int64_t)h->d * (fp8 ? 1 : 2) / 16;
+    const int wgrid = h->num_sms * 4;
+    if (fp8) topk_wmax_kernel<1><<<wgrid, 256, 0, h->side>>>(static_cast<const uint4*>(h->W), n16, wmax);
+    else topk_wmax_kernel<0><<<wgrid, 256, 0, h->side>>>(static_cast<const uint4*>(h->W), n16, wmax);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = cudaEventRecord(h->join, h->side)) != cudaSuccess) return e;
 
   // stage 1
   CUtensorMap tmW;
@@ -650,6 +667,7 @@ cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k
   const size_t ssmem = sizeof(float) * (2 * (size_t)o.npow2 + (size_t)h->d + 4 * (size_t)o.kp);
   e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
   if (e != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(s, h->join, 0)) != cudaSuccess) return e;
   KernelScope sc(h, ELMO_K_TOPK_MERGE, s, 3);
   topk_select_kernel<<<B, kSelThreads, ssmem, s>>>(cs, ci, thr, o.G, o.kp, k, o.npow2, X, h->W, (int)h->dt, h->d,
                                                    gamma, n1, r1, rflag, wmax, idx, score, fail, nfail);
