@@ -371,12 +371,13 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
         elmo::KernelScope ks(h, ELMO_K_UPDATE, s);
         ELMO_CUDA(elmo::launch_update_simt(h, X, B, a, e, h->gbuf, lr, seed, step, s), "update");
       } else {
+        // every kernel but the first follows one of the step's own kernels: programmatic launches
         {
           elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
-          ELMO_CUDA(elmo::launch_logits_grad_tc(h, X, B, a, e, h->gbuf, nullptr, nullptr, s), "logits_grad");
+          ELMO_CUDA(elmo::launch_logits_grad_tc(h, X, B, a, e, h->gbuf, nullptr, nullptr, s, a > 0), "logits_grad");
         }
         elmo::KernelScope ks(h, ELMO_K_UPDATE, s);
-        ELMO_CUDA(elmo::launch_update_tc(h, X, B, a, e, h->gbuf, lr, seed, step, dX_dev, s), "update");
+        ELMO_CUDA(elmo::launch_update_tc(h, X, B, a, e, h->gbuf, lr, seed, step, dX_dev, s, true), "update");
       }
     }
   }

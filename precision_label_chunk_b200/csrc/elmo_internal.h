@@ -95,10 +95,14 @@ cudaError_t launch_update_simt(const elmo_head* h, const uint16_t* X, int32_t B,
 cudaError_t make_tma_map_2d(CUtensorMap_st* m, const void* ptr, int elem_bytes, uint64_t cols, uint64_t rows,
                             uint64_t row_stride_elems, uint32_t box_rows);
 int32_t padded_batch(int32_t B, bool fp8);
+// pdl: launch programmatically dependent on the previous kernel in the stream,
+// which must be this step's kernel B (for A) or A (for B); the kernels wait
+// for it before touching what it produces or consumes.
 cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
-                                  void* gbuf, float* Zout, float* Gout, cudaStream_t s);
+                                  void* gbuf, float* Zout, float* Gout, cudaStream_t s, bool pdl = false);
 cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
-                             const void* gbuf, float lr, uint64_t seed, uint64_t step, float* dX, cudaStream_t s);
+                             const void* gbuf, float lr, uint64_t seed, uint64_t step, float* dX, cudaStream_t s,
+                             bool pdl = false);
 
 // topk_simt.cu -- exact top-k on CUDA cores, for all rows (rows == null) or
 // for the *nrows rows listed in rows (a list whose length lives on the device)

@@ -129,8 +129,8 @@ extern "C" elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d
     const int64_t c1 = c0 + chunk < L ? c0 + chunk : L;
     for (int64_t a = c0; e == cudaSuccess && a < c1; a += sub) {
       const int64_t b = a + sub < c1 ? a + sub : c1;
-      e = elmo::launch_logits_grad_tc(&h, X, B, a, b, gbuf, nullptr, nullptr, st);
-      if (e == cudaSuccess) e = elmo::launch_update_tc(&h, X, B, a, b, gbuf, lr, seed, step, dX_dev, st);
+      e = elmo::launch_logits_grad_tc(&h, X, B, a, b, gbuf, nullptr, nullptr, st, a > 0);
+      if (e == cudaSuccess) e = elmo::launch_update_tc(&h, X, B, a, b, gbuf, lr, seed, step, dX_dev, st, true);
     }
   }
   if (e != cudaSuccess) return fail(ELMO_ECUDA, "elmo_train_step_noalloc: %s", cudaGetErrorString(e));

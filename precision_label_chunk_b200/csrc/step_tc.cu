@@ -33,6 +33,9 @@
 // TMEM-load and special-function latencies of one warp's chain).  Every wait is bounded; a wait that runs out
 // records ELMO_ETIMEOUT in the status word and the CTA winds down.
 #include <cuda.h>
+#include <stdlib.h>
+
+#include <utility>
 
 #include "elmo_common.cuh"
 #include "elmo_internal.h"
@@ -280,6 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    int32_t d, int32_t B, int32_t Bp, int64_t l0, int64_t l1, const uint32_t* __restrict__ keys,
                    const int32_t* __restrict__ tile_ptr, const float* __restrict__ xscale, void* __restrict__ gbuf,
                    float* __restrict__ Zout, float* __restrict__ Gout, int32_t* __restrict__ status) {
+  pdl_wait();      // G is written below: the previous range's kernel B must be done
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   SmemA* S = reinterpret_cast<SmemA*>(base + kStagesA * kStageABytes);
@@ -416,6 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const uint32_t* __restrict__ keys, const int32_t* __restrict__ tile_ptr,
                          const float* __restrict__ xscale, void* __restrict__ gbuf, float* __restrict__ Zout,
                          float* __restrict__ Gout, int32_t* __restrict__ status) {
+  pdl_wait();      // G is written below: the previous range's kernel B must be done
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int kb_elems = kFp8 ? 128 : 64;
@@ -552,6 +559,248 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ============================================================================
+// Kernel A with X in tensor memory.  Z[samples x 64 labels] = X W_tile^T with
+// X (up to 256 samples as 128-row M-blocks) as the MMA's A operand in TMEM,
+// so shared memory holds a 16-stage ring of W k-blocks (64 labels x 128 B)
+// instead of X.  The epilogue thread of sample b forms G = sigmoid(Z) - Y for
+// its row of the tile and stores it sample-major: in each 128-label tile of
+// the gradient buffer the 16-byte label chunk lc of sample b sits at byte
+// ((b/8) * nlc + lc) * 128 + (b%8) * 16 (nlc = 8 chunks of 16 E4M3 or 16 of 8
+// bf16 labels), i.e. core matrices of 8 samples x 16 bytes, which kernel B
+// reads as the MN-major dW operand and the K-major dX^T operand.  Used when X fits the 384 TMEM columns below the
+// accumulators: E4M3 with B <= 256 or bf16 with B <= 128, d <= 768.
+// ============================================================================
+constexpr int kXtThreads = 320;            // warp 0 TMA, warp 1 MMA + TMEM, warps 2-9 epilogue
+constexpr int kXtEpi = 8;
+constexpr int kXtN = 64;                   // labels per tile (the MMA's N)
+constexpr uint32_t kXtBox = kXtN * 128;    // one W k-block: 64 labels x 128 bytes
+constexpr int kXtStages = 16;
+constexpr uint32_t kXtAcc = 384;           // first accumulator column
+
+struct SmemXt {
+  uint64_t wfull[kXtStages], wempty[kXtStages], tfull[2], tempty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int kFp8>
+__global__ void __launch_bounds__(kXtThreads, 1)
+    logits_grad_xt(const __grid_constant__ CUtensorMap tmW, int64_t L, int32_t d, int32_t B, int32_t Bp, int64_t l0,
+                   int64_t l1, const uint8_t* __restrict__ xop, const uint32_t* __restrict__ keys,
+                   const int32_t* __restrict__ tile_ptr, const float* __restrict__ xscale, void* __restrict__ gbuf,
+                   float* __restrict__ Zout, float* __restrict__ Gout, int32_t* __restrict__ status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = base;
+  SmemXt* S = reinterpret_cast<SmemXt*>(base + kXtStages * kXtBox);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t span = l1 - l0;
+  const int T = 2 * (int)((span + 127) / 128);              // 64-label tiles of whole 128-label tiles
+  const int t0 = (int)((int64_t)T * blockIdx.x / gridDim.x);
+  const int t1 = (int)((int64_t)T * (blockIdx.x + 1) / gridDim.x);
+  const int kbe = kFp8 ? 128 : 64;                          // elements of one 128-byte k-block
+  const int nkb = (d + kbe - 1) / kbe;
+  const uint32_t opcols = (uint32_t)nkb * 32;               // TMEM columns of one M-block of X
+  const int nmb = (Bp + 127) / 128;                         // M-blocks of samples: 1 or 2
+  // Two accumulator slots of 64 columns.  One M-block: the slots alternate
+  // between tiles.  Two M-blocks: slot mb holds M-block mb of every tile, and
+  // the MMAs run M-block by M-block, so the epilogue of one M-block overlaps
+  // the MMAs of the other.  Either way the u-th use of the slots is slot u & 1.
+  volatile int* abort = &S->abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kXtStages; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
+    for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], nmb == 2 ? 4 : kXtEpi); }
+    S->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(&S->tmem_base, 512); tmem_relinquish(); }
+  pdl_trigger();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S->tmem_base;
+
+  // X into TMEM: sample mb*128 + r of M-block mb in lane r, columns mb*opcols ...
+  if (warp >= 2) {
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    if (h < nmb) {
+      const int b = h * 128 + q * 32 + lane;
+      const size_t rowbytes = (size_t)d * (kFp8 ? 1 : 2);
+      const uint8_t* src = xop + (size_t)b * rowbytes;
+      for (uint32_t c0 = 0; c0 < opcols; c0 += 64) {   // 64 columns (16 loads in flight) per round
+        uint32_t v[2][32];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const size_t off = (size_t)(c0 + 4 * u) * 4;
+          uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
+          if (b < B && off < rowbytes) w4 = *reinterpret_cast<const uint4*>(src + off);
+          v[u >> 3][4 * (u & 7)] = w4.x; v[u >> 3][4 * (u & 7) + 1] = w4.y;
+          v[u >> 3][4 * (u & 7) + 2] = w4.z; v[u >> 3][4 * (u & 7) + 3] = w4.w;
+        }
+        tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)h * opcols + c0, v[0]);
+        if (c0 + 32 < opcols) tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)h * opcols + c0 + 32, v[1]);
+      }
+      tmem_wait_st();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp == 0) {
+    if (elect_one()) {
+      tma_prefetch_desc(&tmW);
+      uint32_t it = 0;
+      for (int t = t0; t < t1 && !*abort; ++t) {
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = (int)(it % kXtStages);
+          const uint32_t ph = (it / kXtStages) & 1;
+          if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 71); break; }
+          mbar_arrive_expect_tx(&S->wfull[s], kXtBox);
+          tma_load_2d(ring + s * kXtBox, &tmW, &S->wfull[s], kb * kbe, (int32_t)(l0 + (int64_t)t * kXtN));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, kXtN) : make_idesc(1, 1, 0, 0, 128, kXtN);
+      uint32_t it = 0, u = 0;
+      for (int t = t0; t < t1 && !*abort; ++t) {
+        for (int mb = 0; mb < nmb && !*abort; ++mb, ++u) {
+          const uint32_t slot = u & 1, ph = (u >> 1) & 1;
+          if (!mbar_wait(&S->tempty[slot], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 72); break; }
+          tc_fence_after();
+          const uint32_t dcol = tmem + kXtAcc + slot * kXtN;
+          for (int kb = 0; kb < nkb; ++kb) {
+            const uint32_t its = it + (uint32_t)kb;             // the tile's kb-th W k-block
+            const int s = (int)(its % kXtStages);
+            if (mb == 0) {
+              if (!mbar_wait(&S->wfull[s], (its / kXtStages) & 1, abort, kWaitCycles)) {
+                record_timeout(status, abort, 73);
+                break;
+              }
+              tc_fence_after();
+            }
+            const uint32_t bsm = smem_u32(ring + s * kXtBox);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {   // 32 bytes of K per MMA
+              const uint32_t a = tmem + (uint32_t)mb * opcols + (uint32_t)kb * 32 + (uint32_t)k * 8;
+              const uint64_t bd = sw128_desc(bsm + k * 32, 16, 1024);
+              if (kFp8) mma_e4m3_ts(dcol, a, bd, idesc, (kb | k) != 0);
+              else mma_bf16_ts(dcol, a, bd, idesc, (kb | k) != 0);
+            }
+            if (mb == nmb - 1) mma_commit(&S->wempty[s]);   // the k-block's last reader
+          }
+          mma_commit(&S->tfull[slot]);
+        }
+        it += (uint32_t)nkb;
+      }
+    }
+  } else {
+    // two warps per TMEM lane quadrant: with two M-blocks warp h takes M-block
+    // h (all 64 labels), with one it takes label columns 32h .. 32h+31
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    const int mb = nmb == 2 ? h : 0;
+    const int c_lo = nmb == 2 ? 0 : 32 * h;
+    const int ncol = nmb == 2 ? 64 : 32;
+    const int b = mb * 128 + q * 32 + lane;                  // sample
+    const bool bvalid = b < B;
+    const bool bstore = b < Bp;
+    const float inv_sx = kFp8 ? xscale[1] : 1.0f;
+    const float zmul = kFp8 ? 0.5f * inv_sx : -1.4426950408889634f;   // see grad16
+    constexpr int kEl = kFp8 ? 1 : 2;
+    constexpr int kChunk = 16 / kEl;                          // labels per 16-byte chunk
+    constexpr int kNlc = 128 / kChunk;                        // chunks per 128-label tile
+    // the gradient buffer is free once the previous range's kernel B is done;
+    // everything before the first store (X, W, the MMAs) overlaps its tail
+    pdl_wait();
+    uint32_t tc = 0;
+    for (int t = t0; t < t1 && !*abort; ++t, ++tc) {
+      const uint32_t u = nmb == 2 ? 2 * tc + (uint32_t)mb : tc;   // this thread's use of the slots
+      const uint32_t buf = u & 1;
+      if (!mbar_wait(&S->tfull[buf], (u >> 1) & 1, abort, kWaitCycles)) { record_timeout(status, abort, 74); break; }
+      tc_fence_after();
+      uint32_t v[64];
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + kXtAcc + buf * kXtN + (uint32_t)c_lo;
+      tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(v));
+      if (ncol == 64) tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S->tempty[buf]);
+      // labels lc0 .. lc0 + ncol - 1 of this thread's row
+      const int64_t lc0 = l0 + (int64_t)t * kXtN + c_lo;
+      // positives of sample b among them, from the keys of the 128-label tiles they touch
+      uint64_t pm = 0;
+      {
+        const int k0 = __ldg(tile_ptr + (lc0 >> 7));
+        const int k1 = __ldg(tile_ptr + min((lc0 + ncol - 1) >> 7, (L - 1) >> 7) + 1);
+        for (int i = k0; i < k1; ++i) {
+          const uint32_t key = __ldg(keys + i);
+          const int64_t dl = (int64_t)(key >> 8) - lc0;
+          if ((int)(key & 0xFFu) == b && dl >= 0 && dl < ncol) pm |= 1ull << dl;
+        }
+      }
+      uint8_t* gtile = static_cast<uint8_t*>(gbuf) + (size_t)(t >> 1) * 128 * Bp * kEl;
+      const int lt = (t & 1) * kXtN + c_lo;                   // first label column within the 128-label tile
+      for (int j = 0; j < ncol; j += 16) {
+        float g[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float z = __uint_as_float(v[j + i]);
+          float gv;
+          if (kFp8) {
+            gv = __fmaf_rn(tanhf_approx(__fmul_rn(z, zmul)), 128.0f, 128.0f);
+            if ((pm >> (j + i)) & 1) gv -= 256.0f;
+          } else {
+            gv = rcpf_approx(__fadd_rn(exp2f_approx(__fmul_rn(z, zmul)), 1.0f));
+            if ((pm >> (j + i)) & 1) gv -= 1.0f;
+          }
+          const int64_t l = lc0 + j + i;
+          g[i] = (bvalid && l < l1) ? gv : 0.0f;
+        }
+        uint32_t pk[8];
+        if (kFp8) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) pk[i] = pack_e4m3x2(g[4 * i + 1], g[4 * i]) | (pack_e4m3x2(g[4 * i + 3], g[4 * i + 2]) << 16);
+          if (bstore) {
+            const int lc = (lt + j) / kChunk;
+            *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(g[2 * i + 1], g[2 * i]);
+          if (bstore) {
+            const int lc = (lt + j) / kChunk;
+            *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc + 1) * 128 + (b & 7) * 16) =
+                make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+        if ((Zout || Gout) && bvalid) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int64_t l = lc0 + j + i;
+            if (l >= l1) break;
+            const size_t o = (size_t)(l - l0) * B + b;
+            if (Zout) Zout[o] = __fmul_rn(__uint_as_float(v[j + i]), inv_sx);
+            if (Gout)
+              Gout[o] = kFp8 ? e4m3_to_f32((uint8_t)(pk[i >> 2] >> (8 * (i & 3)))) * 0.00390625f
+                             : bf16_to_f32((uint16_t)(pk[i >> 1] >> (16 * (i & 1))));
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (*abort) __nanosleep(20000);
+  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+}
+
+// ============================================================================
 // Kernel B: input gradient, weight gradient and the SR update.
 // ============================================================================
 constexpr int kWSlots = 2;
@@ -578,7 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     update_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
               const uint8_t* __restrict__ gbuf, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
               int32_t Bp, int64_t l0, int64_t l1, const float* __restrict__ xscale, float lr, uint64_t seed,
-              uint64_t step, float* __restrict__ dX, int32_t* __restrict__ status) {
+              uint64_t step, float* __restrict__ dX, int gsm, int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = base;
@@ -608,6 +857,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     S->abort = 0;
     fence_barrier_init();
   }
+  pdl_trigger();
   if (warp == 1) { tmem_alloc(&S->tmem_base, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -618,6 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (elect_one()) {
       tma_prefetch_desc(&tmW); tma_prefetch_desc(&tmX);
       const size_t tile_bytes = (size_t)128 * Bp * kElem;
+      bool g_ready = false;   // G comes from this range's kernel A: wait for it once, before the first read
       int run = 0;
       uint32_t wit = 0, git = 0;
       for (int u = u0; u < u1 && !*abort;) {
@@ -655,6 +906,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // samples [p*kPart, p*kPart + np) of tile t: a contiguous run of 16-byte chunks
             const int np = min(kPart, Bp - p * kPart);
             const uint32_t bytes = (uint32_t)np * kElem * 128u;
+            if (!g_ready) { pdl_wait(); g_ready = true; }
             mbar_arrive_expect_tx(&S->gfull[s], bytes);
             bulk_load(gs + s * kGSlotBytes, gbuf + (size_t)t * tile_bytes + (size_t)p * kPart * kElem * 128u, bytes,
                       &S->gfull[s]);
@@ -665,7 +917,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const uint32_t idesc_dw = kFp8 ? make_idesc(0, 0, 0, 1, 128, 128) : make_idesc(1, 1, 0, 1, 128, 128);
+      // G stored label-major (kernel A with resident X) or sample-major (X in TMEM):
+      // the same core matrices then serve as K- or MN-major operands
+      const uint32_t gmn = gsm ? 1u : 0u;
+      const uint32_t idesc_dw = kFp8 ? make_idesc(0, 0, gmn, 1, 128, 128) : make_idesc(1, 1, gmn, 1, 128, 128);
+      const uint32_t gstride = (uint32_t)(kFp8 ? 8 : 16) * 128u;   // sample-major: bytes between sample groups
       int run = 0;
       uint32_t wit = 0, git = 0, dwit = 0;
       for (int u = u0; u < u1 && !*abort;) {
@@ -695,15 +951,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ga = smem_u32(gs + sg * kGSlotBytes);
             const int np = min(kPart, Bp - p * kPart);   // samples in this part (multiple of 32)
             // dX^T[slice, part] += W^T G^T : M = 128 (columns of d), N = np, K = 128 labels
-            const uint32_t idesc_dx = kFp8 ? make_idesc(0, 0, 1, 1, 128, (uint32_t)np)
-                                           : make_idesc(1, 1, 1, 1, 128, (uint32_t)np);
+            const uint32_t idesc_dx = kFp8 ? make_idesc(0, 0, 1, gmn ^ 1u, 128, (uint32_t)np)
+                                           : make_idesc(1, 1, 1, gmn ^ 1u, 128, (uint32_t)np);
             const uint32_t dxcol = tmem + (uint32_t)(p * kPart);
 #pragma unroll 1
             for (int k = 0; k < 128 / kK; ++k) {
               const uint64_t ad = sw128_desc(wa + k * kK * 128, kBox, 1024);
-              // G part as MN-major B (N = samples, K = labels): label groups 128 B apart,
-              // 16-byte sample chunks 2048 B apart; kK labels = kK / 8 groups per MMA
-              const uint64_t bd = nosw_desc(ga + k * (kK / 8) * 128, 128, 2048);
+              // G part as B (N = samples, K = labels).  Label-major: MN-major, label
+              // groups 128 B apart, 16-byte sample chunks 2048 B apart, kK / 8 groups per
+              // MMA.  Sample-major: K-major, 16-byte label chunks 128 B apart, sample
+              // groups gstride apart, 2 chunks per MMA.
+              const uint64_t bd = gsm ? nosw_desc(ga + k * 2 * 128, 128, gstride)
+                                      : nosw_desc(ga + k * (kK / 8) * 128, 128, 2048);
               if (kFp8) mma_e4m3(dxcol, ad, bd, idesc_dx, !(first && k == 0));
               else mma_bf16(dxcol, ad, bd, idesc_dx, !(first && k == 0));
             }
@@ -711,9 +970,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dwcol = tmem + 256 + db * 128;
 #pragma unroll 1
             for (int k = 0; k < np / kK; ++k) {
-              // G part as K-major A (M = labels, K = samples): 16-byte K chunks 2048 B
-              // apart, label groups 128 B apart; one MMA reads 32 bytes = 2 chunks of K
-              const uint64_t ad = nosw_desc(ga + k * 2 * 2048, 2048, 128);
+              // G part as A (M = labels, K = samples).  Label-major: K-major, 16-byte
+              // sample chunks 2048 B apart, label groups 128 B apart, 2 chunks per MMA.
+              // Sample-major: MN-major, sample groups gstride apart, 16-byte label
+              // chunks 128 B apart, kK / 8 groups per MMA.
+              const uint64_t ad = gsm ? nosw_desc(ga + k * (kK / 8) * gstride, gstride, 128)
+                                      : nosw_desc(ga + k * 2 * 2048, 2048, 128);
               const uint64_t bd = sw128_desc(xa + (p * kPart + k * kK) * 128, 32768, 1024);
               if (kFp8) mma_e4m3(dwcol, ad, bd, idesc_dw, (p | k) != 0);
               else mma_bf16(dwcol, ad, bd, idesc_dw, (p | k) != 0);
@@ -846,12 +1108,57 @@ int32_t padded_batch(int32_t B, bool fp8) {
   return (B + a - 1) / a * a;
 }
 
+// Launch with programmatic stream serialisation when `pdl` (the kernel's
+// prologue then overlaps the tail of the previous kernel in the stream; each
+// kernel orders its dependent accesses with griddepcontrol.wait).
+template <typename... Params, typename... Args>
+cudaError_t launch_k(void (*kern)(Params...), int grid, int block, size_t smem, cudaStream_t s, bool pdl,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Kernel A keeps X in tensor memory (and stores G sample-major) when X fits
+// the 384 TMEM columns below its accumulators; ELMO_STEP_XT=0 turns it off.
+bool g_sample_major(const elmo_head* h, int32_t Bp) {
+  const char* v = getenv("ELMO_STEP_XT");
+  if (v && v[0] == '0') return false;
+  const bool fp8 = h->dt == ELMO_FP8_E4M3;
+  return h->d % 64 == 0 && h->d <= 768 && (fp8 ? Bp <= 256 : Bp <= 128);
+}
+
+constexpr size_t kSmemXt = 1024 + kXtStages * kXtBox + sizeof(SmemXt);
+static_assert(kSmemXt <= 232448, "kernel A (X in TMEM) shared memory");
+
 cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
-                                  void* gbuf, float* Zout, float* Gout, cudaStream_t s) {
+                                  void* gbuf, float* Zout, float* Gout, cudaStream_t s, bool pdl) {
   if (l1 <= l0) return cudaSuccess;
   const bool fp8 = h->dt == ELMO_FP8_E4M3;
   const int eb = fp8 ? 1 : 2;
   const int32_t Bp = padded_batch(B, fp8);
+  if (g_sample_major(h, Bp)) {
+    CUtensorMap tmW64;
+    cudaError_t e = make_tma_map_2d(&tmW64, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, kXtN);
+    if (e != cudaSuccess) return e;
+    const int T = 2 * (int)((l1 - l0 + 127) / 128);
+    const int grid = T < h->num_sms ? T : h->num_sms;
+    auto kx = fp8 ? logits_grad_xt<1> : logits_grad_xt<0>;
+    e = cudaFuncSetAttribute(kx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemXt);
+    if (e != cudaSuccess) return e;
+    const uint8_t* xop = fp8 ? h->xq : reinterpret_cast<const uint8_t*>(X);
+    return launch_k(kx, grid, kXtThreads, kSmemXt, s, pdl, tmW64, h->L, h->d, B, Bp, l0, l1, xop,
+                    (const uint32_t*)h->keys, (const int32_t*)h->tile_ptr, (const float*)h->xscale, gbuf, Zout, Gout,
+                    h->status);
+  }
   CUtensorMap tmW, tmX;
   cudaError_t e = make_tma_map_2d(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, 128);
   if (e != cudaSuccess) return e;
@@ -880,20 +1187,20 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
     auto kp = fp8 ? logits_grad_panel_tc<1> : logits_grad_panel_tc<0>;
     e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemP);
     if (e != cudaSuccess) return e;
-    kp<<<grid, kThreads, kSmemP, s>>>(tmW, tmXp, h->L, h->d, B, Bp, PN, nst, l0, l1, h->keys, h->tile_ptr, h->xscale,
-                                      gbuf, Zout, Gout, h->status);
-    return cudaGetLastError();
+    return launch_k(kp, grid, kThreads, kSmemP, s, pdl, tmW, tmXp, h->L, h->d, B, Bp, PN, nst, l0, l1,
+                    (const uint32_t*)h->keys, (const int32_t*)h->tile_ptr, (const float*)h->xscale, gbuf, Zout, Gout,
+                    h->status);
   }
   auto kern = fp8 ? logits_grad_tc<1> : logits_grad_tc<0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemA);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemA, s>>>(tmW, tmX, h->L, h->d, B, Bp, l0, l1, h->keys, h->tile_ptr, h->xscale, gbuf, Zout,
-                                      Gout, h->status);
-  return cudaGetLastError();
+  return launch_k(kern, grid, kThreads, kSmemA, s, pdl, tmW, tmX, h->L, h->d, B, Bp, l0, l1, (const uint32_t*)h->keys,
+                  (const int32_t*)h->tile_ptr, (const float*)h->xscale, gbuf, Zout, Gout, h->status);
 }
 
 cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
-                             const void* gbuf, float lr, uint64_t seed, uint64_t step, float* dX, cudaStream_t s) {
+                             const void* gbuf, float lr, uint64_t seed, uint64_t step, float* dX, cudaStream_t s,
+                             bool pdl) {
   if (l1 <= l0) return cudaSuccess;
   const bool fp8 = h->dt == ELMO_FP8_E4M3;
   const int eb = fp8 ? 1 : 2;
@@ -910,9 +1217,9 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
   auto kern = fp8 ? update_tc<1> : update_tc<0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemB, s>>>(tmW, tmX, static_cast<const uint8_t*>(gbuf), h->W, h->L, h->d, B, Bp, l0, l1, h->xscale, lr, seed, step, dX,
-                                      h->status);
-  return cudaGetLastError();
+  return launch_k(kern, grid, kThreads, kSmemB, s, pdl, tmW, tmX, static_cast<const uint8_t*>(gbuf), h->W, h->L, h->d,
+                  B, Bp, l0, l1, (const float*)h->xscale, lr, seed, step, dX, g_sample_major(h, Bp) ? 1 : 0,
+                  h->status);
 }
 
 }  // namespace elmo
