@@ -84,6 +84,12 @@ __device__ __forceinline__ float rcpf_approx(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// fp32 multiply that keeps denormal inputs and results whatever -ftz says
+__device__ __forceinline__ float mul_rn_denorm(float a, float b) {
+  float y;
+  asm("mul.rn.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
+  return y;
+}
 __device__ __forceinline__ float tanhf_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -199,25 +205,32 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint8_t*
       }
     }
   }
-  // v = w - lr dW, and a probe that turns NaN when any v is NaN or infinite
-  // (bf16: or |v| >= 2^127, where rounding could reach the largest finite
+  // v = w - lr dW, and a probe that is not finite when some v is NaN or
+  // infinite (E4M3: the sum of 0 v; bf16: the sum of 2 v, which also overflows
+  // when some |v| >= 2^127, where rounding could pass the largest finite
   // value); such groups take the exact per-element path
   float vv[16];
   float probe = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
-    probe = __fmaf_rn(kFp8 ? vv[i] : __fmul_rn(vv[i], 2.0f), 0.0f, probe);
+    probe = __fmaf_rn(vv[i], kFp8 ? 0.0f : 2.0f, probe);
   }
   const uint64_t blk = ((uint64_t)l * (uint64_t)d + (uint64_t)j0) >> 3;
   const u32x4 r0 = sr_block(seed, step, blk), r1 = sr_block(seed, step, blk + 1);
   const uint32_t rw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
   uint32_t wnew[8];
-  if (probe == 0.0f) {
+  if (fabsf(probe) < INFINITY) {
     if (kFp8) {
-      // |v| < 2^-6: shift into [2^-6, 2^-5) rounding up, add-and-truncate at 20
-      // bits, shift back.  sat = [|v| < 2^-6] comes from a saturated FMA:
-      // (2^-6 - |v|) 2^100 is >= 2^70 below 2^-6 and <= 0 from 2^-6 up.
+      // Scaled by 2^-120, the E4M3 grid is fp32's own grid cut to 3 mantissa
+      // bits: E4M3's subnormal spacing 2^-9 becomes 2^-129 = 2^20 units of
+      // fp32's denormal spacing 2^-149, and its normal range starts at 2^-126,
+      // fp32's.  So one add-and-truncate at 20 bits on the signed pattern rounds
+      // every magnitude (the carry runs into the exponent where it should).
+      // The scaling is exact for |v| >= 2^-6; below, it rounds v to a multiple
+      // of 2^-29, which changes the decision u < f only when f 2^16 lies less
+      // than 2^-5 above an integer equal to the draw (about 2^-21 of the
+      // elements there).  The elmo_sr_round kernel keeps the exact form.
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         float o[4];
@@ -226,12 +239,9 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint8_t*
           const uint32_t word = rw[2 * q4 + (e >> 1)];
           const uint32_t k16 = (e & 1) ? __umulhi(word, 0x10000u) : (word & 0xFFFFu);
           const uint32_t radd = 0xFFFFFu - k16 * 16u;          // 2^20 - 1 - 16 k
-          const float v = vv[4 * q4 + e];
-          const float a = fabsf(v);
-          const float sat = __saturatef(__fmaf_rn(-a, 0x1p100f, 0x1p94f));
-          const float sh = __fmaf_ru(sat, 0.015625f, a);
-          const uint32_t t = (__float_as_uint(sh) + radd) & 0xFFF00000u;
-          o[e] = copysignf(__fmaf_rn(sat, -0.015625f, __uint_as_float(t)), v);
+          const float vs = mul_rn_denorm(vv[4 * q4 + e], 0x1p-120f);
+          const uint32_t t = (__float_as_uint(vs) + radd) & 0xFFF00000u;
+          o[e] = mul_rn_denorm(__uint_as_float(t), 0x1p120f);
         }
         wnew[q4] = pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16);
       }

@@ -165,3 +165,33 @@ def test_resume_is_exact(orc):
     straight = run(W, range(6))
     half = run(W, range(3))
     assert np.array_equal(run(half, range(3, 6)), straight)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_step_special_weights(orc, dtype):
+    """Infinities, NaNs, the largest finite values, subnormals and -0 among the
+    weights take the update's exact per-element path: those weights get the
+    oracle's codes exactly (a NaN weight makes its label's logits and gradient
+    NaN, so its whole row becomes NaN on both sides); the other rows keep the
+    usual statistical agreement."""
+    need_gpu()
+    import ml_dtypes
+    import precision_label_chunk_b200 as elmo
+    w = workload("tiny", dtype=dtype, L=600, d=128, B=24)
+    W, X, rowptr, cols = _inputs(orc, w)
+    specials = {"bf16": [0x7F80, 0xFF80, 0x7FC0, 0x7F7F, 0xFF7F, 0x7F00, 0x0001, 0x8000],
+                "fp8": [0x7F, 0xFF, 0x7E, 0xFE, 0x01, 0x80, 0x7D, 0x08]}[dtype]
+    pos = [(3 + 70 * i, (13 * i) % w.d) for i in range(len(specials))]
+    W = W.copy()
+    for (l, j), c in zip(pos, specials):
+        W[l, j] = c
+    Wg, _ = run_step(elmo, W, X, rowptr, cols, w.lr, 256, 7, 3, dtype)
+    r = orc.train_step(W, X, rowptr, cols, w.lr, 7, 3, dtype)
+    for (l, j), c in zip(pos, specials):
+        assert Wg[l, j] == r["W"][l, j], f"special weight {c:#x} at ({l}, {j}): {Wg[l, j]:#x} vs {r['W'][l, j]:#x}"
+    as_f = (lambda a: a.view(ml_dtypes.bfloat16).astype(np.float32)) if dtype == "bf16" else \
+           (lambda a: a.view(ml_dtypes.float8_e4m3fn).astype(np.float32))
+    nan_g, nan_o = np.isnan(as_f(Wg)), np.isnan(as_f(r["W"]))
+    assert np.array_equal(nan_g, nan_o)
+    finite_rows = ~np.any(~np.isfinite(as_f(r["W"])), axis=1)
+    assert_weights_close(Wg[finite_rows], r["W"][finite_rows], dtype)
