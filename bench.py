@@ -143,7 +143,8 @@ def profiled_traffic(kernel, workload):
         with open(os.path.join(ROOT, src), "rb") as f:
             if hashlib.sha256(f.read()).hexdigest() != digest:
                 return None
-        return {"bytes": float(fields["dram bytes per launch"]), "labels": int(fields["labels per launch"])}
+        units = fields.get("labels per launch", fields.get("values per launch"))
+        return {"bytes": float(fields["dram bytes per launch"]), "labels": int(units)}
     except (KeyError, ValueError, OSError):
         return None
 
@@ -264,8 +265,10 @@ def run_topk(args, w, rank, world, local):
             # the two E4M3 parts of the bf16 queries, so their ceiling is frac = 0.5)
             peak, bound = tensor_peak_tflops(peaks, w.dtype), "tensor"
             src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype == "fp8" else ""))
+        tr = profiled_traffic("topk_screen_tc", w.name) if bound == "tensor" else None
         roof = {"kernel": dominant, "bound": bound, "achieved": flops / t_k / 1e12, "peak": peak, "unit": "TFLOP/s",
-                "frac": flops / t_k / 1e12 / peak, "traffic": None, "peak_source": src,
+                "frac": flops / t_k / 1e12 / peak,
+                "traffic": None if tr is None else tr["bytes"] * w.L / tr["labels"], "peak_source": src,
                 "mma_passes": 2 if (w.dtype == "fp8" and bound == "tensor") else 1}
     # end to end: X from pinned host memory, indices and scores back every step
     pin = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in Xh]
@@ -342,7 +345,9 @@ def run_sr(args, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": "sr_round", "n": n, "l2": "inputs larger than L2 (1 GiB fp32)"},
             "roofline": {"kernel": "sr_round", "bound": "hbm", "achieved": res["fp8"]["GB/s"],
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": res["fp8"]["frac"], "traffic": None,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": res["fp8"]["frac"],
+                         "traffic": (lambda tr: None if tr is None else tr["bytes"] * n / tr["labels"])(
+                             profiled_traffic("sr_round_vec", "sr_round")),
                          "peak_source": f"{peaks['source']} copy bandwidth"},
             "per_dtype": res}
     print(json.dumps(line), flush=True)
