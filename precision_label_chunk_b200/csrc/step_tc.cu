@@ -833,7 +833,7 @@ struct UnitRange {
 };
 
 template <int kFp8>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
     update_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
               const uint8_t* __restrict__ gbuf, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
               int32_t Bp, int64_t l0, int64_t l1, const float* __restrict__ xscale, float lr, uint64_t seed,
@@ -855,15 +855,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBoxCols = 128 / kElem;               // elements per 128-byte box row
   constexpr int kPart = kFp8 ? 256 : 128;             // samples per G part
   constexpr int kK = kFp8 ? 32 : 16;                  // MMA K
+  // epilogue warps: E4M3 16 (two 16-column groups each per unit), bf16 8 (two
+  // pairs of groups each, a pair in flight together: measured faster for bf16,
+  // whose cheaper SR leaves the Philox chains' latency exposed with 16 warps)
+  constexpr int kEpiU = kFp8 ? 16 : 8;
+  constexpr int kGrp = kFp8 ? 1 : 2;                  // 16-column groups per epilogue step
   const int nparts = (Bp + kPart - 1) / kPart;
   volatile int* abort = &S->abort;
 
   if (threadIdx.x == 0) {
     mbar_init(&S->xfull, 1); mbar_init(&S->xempty, 1);
-    mbar_init(&S->dxfull, 1); mbar_init(&S->dxempty, kEpiWarps);
-    for (int s = 0; s < kWSlots; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kEpiWarps); }
+    mbar_init(&S->dxfull, 1); mbar_init(&S->dxempty, kEpiU);
+    for (int s = 0; s < kWSlots; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kEpiU); }
     for (int s = 0; s < kGSlots; ++s) { mbar_init(&S->gfull[s], 1); mbar_init(&S->gempty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&S->dwfull[b], 1); mbar_init(&S->dwempty[b], kEpiWarps); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&S->dwfull[b], 1); mbar_init(&S->dwempty[b], kEpiU); }
     S->abort = 0;
     fence_barrier_init();
   }
@@ -1002,7 +1007,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     const int q = warp & 3;
-    const int sub = (warp - 2) >> 2;           // dW columns 32*sub .. +31; dX^T chunks c % 4 == sub
+    const int sub = (warp - 2) >> 2;           // dW columns of width 128/(kEpiU/4); dX^T chunks c % (kEpiU/4) == sub
     const int row = q * 32 + lane;             // label row of dW; column of d for dX^T
     // lr * dW with dW = acc * 2^-8 / s_X (fp8) folds into one exact power-of-two scaled lr
     const float lrs = kFp8 ? lr * (0.00390625f * xscale[1]) : lr;
@@ -1027,13 +1032,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + 256 + db * 128;
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
-          const int jl = sub * 32 + hh * 16;               // column within the 128-column slice
-          uint32_t r[16];
-          tmem_ld16(taddr + jl, r);
+          const int jl = sub * 32 * kGrp + hh * 16 * kGrp;  // column within the 128-column slice
+          uint32_t r[kGrp][16];
+#pragma unroll
+          for (int g = 0; g < kGrp; ++g) tmem_ld16(taddr + jl + 16 * g, r[g]);
           tmem_wait_ld();
           const int j0 = D0 + jl;
           if (!valid || j0 >= d) continue;
-          update16<kFp8>(r, wrow, row, jl, l, d, j0, lrs, seed, step, Wglob);
+#pragma unroll
+          for (int g = 0; g < kGrp; ++g)
+            update16<kFp8>(r[g], wrow, row, jl + 16 * g, l, d, j0 + 16 * g, lrs, seed, step, Wglob);
         }
         tc_fence_before();
         __syncwarp();
@@ -1045,7 +1053,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int j = D0 + row;
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
-      for (int c = sub; c < Bp / 32; c += 4) {
+      for (int c = sub; c < Bp / 32; c += kEpiU / 4) {
         uint32_t ra[32];
         tmem_ld32(taddr + c * 32, ra);
         tmem_wait_ld();
@@ -1227,7 +1235,8 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
   auto kern = fp8 ? update_tc<1> : update_tc<0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB);
   if (e != cudaSuccess) return e;
-  return launch_k(kern, grid, kThreads, kSmemB, s, pdl, tmW, tmX, static_cast<const uint8_t*>(gbuf), h->W, h->L, h->d,
+  return launch_k(kern, grid, fp8 ? kThreads : 320, kSmemB, s, pdl, tmW, tmX, static_cast<const uint8_t*>(gbuf), h->W,
+                  h->L, h->d,
                   B, Bp, l0, l1, (const float*)h->xscale, lr, seed, step, dX, g_sample_major(h, Bp) ? 1 : 0,
                   h->status);
 }
