@@ -481,7 +481,7 @@ def main():
             src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype == "fp8" else ""))
         # ncu DRAM bytes of one full launch, scaled to the mean launch of this
         # run by the labels it covers (the kernel's traffic is linear in them)
-        tr = profiled_traffic({"update": "update_tc", "logits_grad": "logits_grad_tc"}.get(dominant, dominant),
+        tr = profiled_traffic({"update": "update_tc", "logits_grad": "logits_grad_xt"}.get(dominant, dominant),
                               w.name)
         traffic = None
         if tr is not None:
