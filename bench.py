@@ -123,6 +123,24 @@ def alu_peak_tflops(peaks):
     return 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
 
 
+def max_over_ranks(ms, device=None):
+    """The job's time: the largest of the ranks' device times (every rank calls
+    this at the same point; one process: the value itself)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, labels, steps, ms):
+    """Whole-job label-rows/s: every rank (replica) processes all L labels per
+    step, so the job processes world * L * steps label-rows in the max time."""
+    return world * labels * steps / (ms / 1e3)
+
+
 def profiled_traffic(kernel, workload):
     """DRAM bytes (read + write) of one full launch of `kernel`, from the ncu
     summary committed under profiles/, with the labels that launch covered.
@@ -431,13 +449,9 @@ def main():
         dist.barrier()
     elmo.elmo_sync_status(head)
     gpu_launches = elmo.elmo_launch_count(head) - launches0
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_per_step = ms / args.steps
-    value = world * w.L * args.steps / (ms / 1e3)
+    value = job_throughput(world, w.L, args.steps, ms)
 
     # ---------------------------------------------------------------- per-kernel pass
     # The same K steps again, with the library recording a CUDA event pair on
@@ -518,12 +532,8 @@ def main():
         dX_host.copy_(dX, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e = {"value": world * w.L * args.steps / (ms_e2e / 1e3), "unit": "label-rows/s",
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e = {"value": job_throughput(world, w.L, args.steps, ms_e2e), "unit": "label-rows/s",
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     # ---------------------------------------------------------------- CPU oracle baseline

@@ -233,8 +233,9 @@ elmo_status elmo_launch_count(const elmo_head* h, int64_t* launches);
  * someone else.  Such callers cannot create an elmo_head (its workspace is
  * allocated) nor let the head grow its gradient buffer on first use.
  *
- * This call takes W directly and allocates nothing.  Its scratch (sorted
- * positives, the tile index, quantised X and the per-range gradient operands)
+ * This call takes W directly and allocates nothing.  Its scratch (the
+ * positives grouped by label tile, the tile index, quantised X and the
+ * per-range gradient operands)
  * is one static device array of 10 MiB (ELMO_NOALLOC_SCRATCH_BYTES) that every
  * GPU loading the library holds until the process exits.  It supports the
  * same sizes as the head-based step -- 1 <= L < 2^24, d a multiple of 64 up to
@@ -263,6 +264,23 @@ elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d, elmo_dtyp
                                     int32_t B, const int32_t* rowptr_dev, const int32_t* cols_dev, int32_t nnz,
                                     float lr, int64_t chunk, uint64_t seed, uint64_t step, float* dX_dev,
                                     int32_t* status_dev, void* stream);
+
+/*
+ * elmo_check_bounded_wait -- runs, in one CTA, the bounded mbarrier wait that
+ * every pipelined kernel of the library uses, on a barrier nothing ever
+ * arrives on.  The paper has no counterpart: this checks the library's
+ * failure detection without faulting anything.  The wait gives up after about
+ * limit_cycles SM clock cycles, records ELMO_ETIMEOUT in status_dev[0] and
+ * ELMO_WAIT_CHECK_SITE in status_dev[1] exactly as a kernel whose pipeline
+ * stalled would, and the kernel returns normally, so the context stays usable.
+ *
+ *   limit_cycles : 1 .. 2^32 (about 2 s at the B200's clock)
+ *   status_dev   : int32 [2] (device), cleared by the call
+ * Asynchronous on `stream`: read status_dev after synchronising.  Errors:
+ * ELMO_EINVAL (null status_dev, limit out of range), ELMO_ECUDA (launch).
+ */
+#define ELMO_WAIT_CHECK_SITE 99
+elmo_status elmo_check_bounded_wait(int64_t limit_cycles, int32_t* status_dev, void* stream);
 
 /* Message of the most recent failure on the calling thread ("" if none). */
 const char* elmo_last_error(void);

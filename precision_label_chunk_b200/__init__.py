@@ -25,10 +25,12 @@ __all__ = [
     "elmo_forward_chunk", "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws",
     "elmo_sync_status", "elmo_head_workspace_bytes", "elmo_profile_enable", "elmo_profile_reset",
     "elmo_profile_read", "elmo_launch_count", "KERNEL_CLASSES", "elmo_train_step_noalloc",
+    "elmo_check_bounded_wait", "WAIT_CHECK_SITE",
 ]
 
 BF16 = 0
 FP8_E4M3 = 1
+WAIT_CHECK_SITE = 99
 MAX_BATCH = 256
 MAX_NNZ = 32768
 MAX_TOPK = 64
@@ -86,6 +88,7 @@ def _declare(L):
     L.elmo_profile_reset.argtypes = [P]
     L.elmo_profile_read.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]
     L.elmo_launch_count.argtypes = [P, ctypes.POINTER(i64)]
+    L.elmo_check_bounded_wait.argtypes = [i64, P, P]
     for name in ("elmo_profile_enable", "elmo_profile_reset", "elmo_profile_read", "elmo_launch_count","elmo_init_head", "elmo_head_destroy", "elmo_train_step_chunked", "elmo_forward_chunk",
                  "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws", "elmo_sync_status",
                  "elmo_head_workspace_bytes"):
@@ -212,6 +215,13 @@ def elmo_sr_round(inp: torch.Tensor, out: torch.Tensor, dtype, seed: int, step: 
 def elmo_sr_draws(out: torch.Tensor, seed: int, step: int, index_base: int = 0, stream=None):
     _check(load().elmo_sr_draws(_ptr(out), out.numel(), int(seed) & (2**64 - 1), int(step) & (2**64 - 1),
                                 int(index_base) & (2**64 - 1), _stream(stream)))
+
+
+def elmo_check_bounded_wait(limit_cycles: int, status: torch.Tensor, stream=None):
+    """Runs the kernels' bounded mbarrier wait on a barrier nothing arrives on;
+    after synchronising, status (int32 [2], device) holds ELMO_ETIMEOUT and
+    WAIT_CHECK_SITE."""
+    _check(load().elmo_check_bounded_wait(int(limit_cycles), _ptr(status), _stream(stream)))
 
 
 def elmo_sync_status(head: Head, stream=None):

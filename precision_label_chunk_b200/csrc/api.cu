@@ -384,6 +384,15 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
   return ELMO_OK;
 }
 
+elmo_status elmo_check_bounded_wait(int64_t limit_cycles, int32_t* status_dev, void* stream) {
+  g_last_error.clear();
+  if (!status_dev) return fail(ELMO_EINVAL, "null status_dev");
+  if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 32))
+    return fail(ELMO_EINVAL, "limit_cycles = %lld outside [1, 2^32]", (long long)limit_cycles);
+  ELMO_CUDA(elmo::launch_wait_check((long long)limit_cycles, status_dev, as_stream(stream)), "wait check");
+  return ELMO_OK;
+}
+
 elmo_status elmo_topk_predict(elmo_head* h, const void* X_dev, int32_t B, int32_t k, int64_t chunk,
                               int32_t* idx_dev, float* score_dev, void* stream) {
   g_last_error.clear();

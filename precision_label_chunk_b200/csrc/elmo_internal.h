@@ -95,6 +95,7 @@ cudaError_t launch_update_simt(const elmo_head* h, const uint16_t* X, int32_t B,
 cudaError_t make_tma_map_2d(CUtensorMap_st* m, const void* ptr, int elem_bytes, uint64_t cols, uint64_t rows,
                             uint64_t row_stride_elems, uint32_t box_rows);
 int32_t padded_batch(int32_t B, bool fp8);
+cudaError_t launch_wait_check(long long limit_cycles, int32_t* status, cudaStream_t s);
 // pdl: launch programmatically dependent on the previous kernel in the stream,
 // which must be this step's kernel B (for A) or A (for B); the kernels wait
 // for it before touching what it produces or consumes.

@@ -1,0 +1,64 @@
+"""The multi-process plumbing of bench.py on CPU (gloo, world size 2): the job
+time is the max over ranks and the job throughput counts every replica; the
+reference arm runs on rank 0 only.  The GPU work itself is not involved."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    ms = bench.max_over_ranks(10.0 + 5.0 * rank)           # rank 1 is the slow one
+    val = bench.job_throughput(dist.get_world_size(), 1000, 4, ms)
+    out.put((rank, ms, val))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_job_time_is_max_over_ranks_gloo():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ms, val in res:
+        assert ms == 15.0                                   # every rank sees the slowest rank's time
+        assert val == pytest.approx(2 * 1000 * 4 / 0.015)   # both replicas' labels over that time
+
+
+def test_single_process_time_is_its_own():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(7.5) == 7.5
+    assert bench.job_throughput(1, 3_000_000, 10, 1000.0) == pytest.approx(3e7)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "1"], env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
