@@ -74,6 +74,7 @@ def _declare(L):
                                  i64, i64, P, P, P, ctypes.c_int]
     L.orc_dx_rows.argtypes = [P, i64, i32, ctypes.c_int, P, i32, P, P, P, i32, P, ctypes.c_int]
     L.orc_topk.argtypes = [P, i64, i32, ctypes.c_int, P, i32, i32, P, i32, P, P, ctypes.c_int]
+    L.orc_precision_at_k.argtypes = [P, i32, i32, P, P, P]
     L.orc_score.argtypes = [P, ctypes.c_int, i64, P, i32, i32]
     L.orc_score.restype = f32
 
@@ -225,6 +226,16 @@ def topk(W, X, k, dtype, rows=None, nthreads=0):
     sc = np.zeros((n, k), np.float32)
     _check(lib().orc_topk(_p(W), L, d, dt, _p(X), B, k, _p(r), n, _p(idx), _p(sc), nthreads), "topk")
     return idx, sc
+
+
+def precision_at_k(idx, rowptr, cols):
+    """P@1 .. P@k (float64 [k]) of predictions idx [B, k] against CSR positives."""
+    idx = _c(idx, np.int32)
+    B, k = idx.shape
+    p = np.zeros(k, np.float64)
+    _check(lib().orc_precision_at_k(_p(idx), B, k, _p(_c(rowptr, np.int32)), _p(_c(cols, np.int32)), _p(p)),
+           "precision_at_k")
+    return p
 
 
 def score(W, X, l, b, dtype) -> float:

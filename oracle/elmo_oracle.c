@@ -510,6 +510,34 @@ int orc_topk(const void* W, int64_t L, int32_t d, int dt, const uint16_t* X, int
   return ORC_OK;
 }
 
+/*
+ * P@j for j = 1..k ("ELMO: Efficiency via Low-precision and Peak Memory
+ * Optimization in Large Output Spaces", atlas summary, metrics P@1/3/5): the
+ * mean over the B rows of |{first j predicted labels of the row} ∩ Y_b| / j,
+ * with Y_b the row's positive labels cols[rowptr[b] .. rowptr[b+1]).  idx is
+ * [B, k] (each row's predictions in rank order).  p[j-1] = P@j, computed as an
+ * exact integer hit count over j*B in double.
+ */
+int orc_precision_at_k(const int32_t* idx, int32_t B, int32_t k, const int32_t* rowptr, const int32_t* cols,
+                       double* p) {
+  if (!idx || !rowptr || !p || B < 1 || k < 1) return ORC_EINVAL;
+  for (int j = 0; j < k; j++) p[j] = 0.0;
+  int64_t* hits = (int64_t*)calloc((size_t)k, sizeof(int64_t));
+  for (int32_t b = 0; b < B; b++) {
+    int64_t h = 0;
+    for (int32_t i = 0; i < k; i++) {
+      int32_t lab = idx[(size_t)b * k + i];
+      int hit = 0;
+      for (int32_t q = rowptr[b]; q < rowptr[b + 1] && !hit; q++) hit = (cols[q] == lab);
+      h += hit;
+      hits[i] += h;                 /* hits among the first i + 1 predictions */
+    }
+  }
+  for (int j = 0; j < k; j++) p[j] = (double)hits[j] / ((double)(j + 1) * (double)B);
+  free(hits);
+  return ORC_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Array helpers for the Python side (loops over the scalar definitions).   */
 /* ------------------------------------------------------------------------ */
