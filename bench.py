@@ -302,6 +302,14 @@ def run_topk(args, w, rank, world, local):
     e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / args.steps
+    # P@1, P@3, P@5 of the last predictions against the queries' synthetic labels
+    # (random weights: near zero; the point is that the metric runs on the device)
+    from synthetic import make_labels
+    rp, cl = make_labels(w, nsteps - 1)
+    kk = min(5, w.topk)
+    pk = torch.empty(kk, dtype=torch.float32, device=dev)
+    elmo.elmo_precision_at_k(idx[:, :kk].contiguous(), torch.from_numpy(rp).to(dev), torch.from_numpy(cl).to(dev), pk)
+    p_at_k = {f"P@{j}": float(pk[j - 1]) for j in (1, 3, 5) if j <= kk}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -325,7 +333,7 @@ def run_topk(args, w, rank, world, local):
             "gpu_launches": gpu_launches,
             "e2e": {"value": world * w.B * w.L / (ms_e2e / 1e3), "unit": "query-labels/s",
                     "h2d_bytes_per_step": w.B * w.d * 2, "d2h_bytes_per_step": w.B * w.topk * 8},
-            "cpu_baseline": cpu, "clocks": clocks,
+            "cpu_baseline": cpu, "clocks": clocks, "p_at_k": p_at_k,
         }
         print(json.dumps(line), flush=True)
     head.close()

@@ -266,6 +266,25 @@ elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d, elmo_dtyp
                                     int32_t* status_dev, void* stream);
 
 /*
+ * elmo_precision_at_k -- P@1 .. P@k of top-k predictions ("ELMO: Efficiency
+ * via Low-precision and Peak Memory Optimization in Large Output Spaces",
+ * atlas summary, metrics P@1/3/5): p[j-1] = the mean over the B rows of
+ * |{first j predicted labels} ∩ {positive labels}| / j.
+ *
+ *   idx_dev    : int32 [B x k] (device), each row's predictions in rank order
+ *                (the idx output of elmo_topk_predict)
+ *   B, k       : 1 <= B <= ELMO_MAX_PREDICT_BATCH, 1 <= k <= ELMO_MAX_TOPK
+ *   rowptr_dev : int32 [B+1], cols_dev int32 [nnz] (device): each row's
+ *                positive labels (CSR); entries outside [0, nnz) are clamped
+ *   p_dev      : fp32 [k] (device), written: integer hit counts over j*B,
+ *                divided in double and rounded once (independent of order)
+ * Asynchronous on `stream`.  Errors: ELMO_EINVAL (null pointer, B or k out of
+ * range), ELMO_ECUDA (launch).
+ */
+elmo_status elmo_precision_at_k(const int32_t* idx_dev, int32_t B, int32_t k, const int32_t* rowptr_dev,
+                                const int32_t* cols_dev, int32_t nnz, float* p_dev, void* stream);
+
+/*
  * elmo_check_bounded_wait -- runs, in one CTA, the bounded mbarrier wait that
  * every pipelined kernel of the library uses, on a barrier nothing ever
  * arrives on.  The paper has no counterpart: this checks the library's

@@ -25,7 +25,7 @@ __all__ = [
     "elmo_forward_chunk", "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws",
     "elmo_sync_status", "elmo_head_workspace_bytes", "elmo_profile_enable", "elmo_profile_reset",
     "elmo_profile_read", "elmo_launch_count", "KERNEL_CLASSES", "elmo_train_step_noalloc",
-    "elmo_check_bounded_wait", "WAIT_CHECK_SITE",
+    "elmo_check_bounded_wait", "WAIT_CHECK_SITE", "elmo_precision_at_k",
 ]
 
 BF16 = 0
@@ -89,6 +89,7 @@ def _declare(L):
     L.elmo_profile_read.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]
     L.elmo_launch_count.argtypes = [P, ctypes.POINTER(i64)]
     L.elmo_check_bounded_wait.argtypes = [i64, P, P]
+    L.elmo_precision_at_k.argtypes = [P, i32, i32, P, P, i32, P, P]
     for name in ("elmo_profile_enable", "elmo_profile_reset", "elmo_profile_read", "elmo_launch_count","elmo_init_head", "elmo_head_destroy", "elmo_train_step_chunked", "elmo_forward_chunk",
                  "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws", "elmo_sync_status",
                  "elmo_head_workspace_bytes"):
@@ -215,6 +216,14 @@ def elmo_sr_round(inp: torch.Tensor, out: torch.Tensor, dtype, seed: int, step: 
 def elmo_sr_draws(out: torch.Tensor, seed: int, step: int, index_base: int = 0, stream=None):
     _check(load().elmo_sr_draws(_ptr(out), out.numel(), int(seed) & (2**64 - 1), int(step) & (2**64 - 1),
                                 int(index_base) & (2**64 - 1), _stream(stream)))
+
+
+def elmo_precision_at_k(idx: torch.Tensor, rowptr: torch.Tensor, cols: torch.Tensor, p: torch.Tensor, stream=None):
+    """P@1 .. P@k (fp32 [k], device) of predictions idx (int32 [B, k], device)
+    against the CSR positives rowptr/cols (int32, device)."""
+    B, k = idx.shape
+    _check(load().elmo_precision_at_k(_ptr(idx), B, k, _ptr(rowptr), _ptr(cols), cols.numel(), _ptr(p),
+                                      _stream(stream)))
 
 
 def elmo_check_bounded_wait(limit_cycles: int, status: torch.Tensor, stream=None):

@@ -384,6 +384,18 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
   return ELMO_OK;
 }
 
+elmo_status elmo_precision_at_k(const int32_t* idx_dev, int32_t B, int32_t k, const int32_t* rowptr_dev,
+                                const int32_t* cols_dev, int32_t nnz, float* p_dev, void* stream) {
+  g_last_error.clear();
+  if (!idx_dev || !rowptr_dev || !p_dev || (nnz > 0 && !cols_dev)) return fail(ELMO_EINVAL, "null pointer");
+  if (B < 1 || B > ELMO_MAX_PREDICT_BATCH) return fail(ELMO_EINVAL, "B = %d outside [1, %d]", B, ELMO_MAX_PREDICT_BATCH);
+  if (k < 1 || k > ELMO_MAX_TOPK) return fail(ELMO_EINVAL, "k = %d outside [1, %d]", k, ELMO_MAX_TOPK);
+  if (nnz < 0) return fail(ELMO_EINVAL, "nnz = %d < 0", nnz);
+  ELMO_CUDA(elmo::launch_precision_at_k(idx_dev, B, k, rowptr_dev, cols_dev, nnz, p_dev, as_stream(stream)),
+            "precision_at_k");
+  return ELMO_OK;
+}
+
 elmo_status elmo_check_bounded_wait(int64_t limit_cycles, int32_t* status_dev, void* stream) {
   g_last_error.clear();
   if (!status_dev) return fail(ELMO_EINVAL, "null status_dev");

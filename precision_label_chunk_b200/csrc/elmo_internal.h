@@ -118,6 +118,10 @@ size_t topk_tc_workspace_bytes(const elmo_head* h, int32_t B, int32_t k);
 cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k, int32_t* idx, float* score,
                            cudaStream_t s);
 
+// metrics.cu
+cudaError_t launch_precision_at_k(const int32_t* idx, int32_t B, int32_t k, const int32_t* rowptr,
+                                  const int32_t* cols, int32_t nnz, float* p, cudaStream_t s);
+
 // sr.cu
 cudaError_t launch_sr_round(const float* in, void* out, int64_t n, elmo_dtype dt, uint64_t seed,
                             uint64_t step, uint64_t base, cudaStream_t s);

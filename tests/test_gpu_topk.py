@@ -113,3 +113,31 @@ def test_topk_uncertified_rows_take_exact_path(orc, case):
     assert np.array_equal(idx, ri)
     assert np.array_equal(sc.view(np.uint32), rs.view(np.uint32))
     h.close()
+
+
+@pytest.mark.parametrize("B,k,L", [(1024, 5, 3_000_000), (7, 64, 100), (1, 1, 10)])
+def test_precision_at_k_matches_oracle(orc, B, k, L):
+    """P@1..P@k on the GPU equals the oracle's value rounded to fp32, on seeded
+    predictions (distinct labels per row) and the workload's label law."""
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    from synthetic import make_labels
+    rng = np.random.default_rng(B * 131 + k)
+    w = workload("product3m_fp8", L=L, B=B)
+    rowptr, cols = make_labels(w, 1)
+    # predictions: mostly positives of the row at random ranks, the rest random labels
+    idx = np.zeros((B, k), np.int32)
+    for b in range(B):
+        pos = cols[rowptr[b]:rowptr[b + 1]]
+        cand = np.concatenate([rng.permutation(pos)[: rng.integers(0, min(k, pos.size) + 1)],
+                               rng.choice(L, size=min(2 * k, L), replace=False)])
+        _, first = np.unique(cand, return_index=True)
+        row = cand[np.sort(first)][:k]
+        idx[b, : row.size] = rng.permutation(row)
+        if row.size < k:
+            idx[b, row.size:] = -1
+    p = torch.empty(k, dtype=torch.float32, device="cuda")
+    elmo.elmo_precision_at_k(torch.from_numpy(idx).cuda(), torch.from_numpy(rowptr).cuda(),
+                             torch.from_numpy(cols).cuda(), p)
+    want = orc.precision_at_k(idx, rowptr, cols).astype(np.float32)
+    assert np.array_equal(p.cpu().numpy(), want)
