@@ -306,9 +306,8 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B, const
   cudaStream_t s = as_stream(stream);
   const uint16_t* X = static_cast<const uint16_t*>(X_dev);
   {
-    elmo::KernelScope ks(h, ELMO_K_PREP, s, h->dt == ELMO_FP8_E4M3 ? 2 : 1);
-    ELMO_CUDA(elmo::launch_prep_labels(h, rowptr_dev, cols_dev, B, nnz, s), "prep_labels");
-    if (h->dt == ELMO_FP8_E4M3) ELMO_CUDA(elmo::launch_prep_x(h, X, B, s), "prep_x");
+    elmo::KernelScope ks(h, ELMO_K_PREP, s, 1);
+    ELMO_CUDA(elmo::launch_prep_step(h, rowptr_dev, cols_dev, B, nnz, X, s), "prep");
   }
   const bool fp8 = h->dt == ELMO_FP8_E4M3;
   const size_t esz = fp8 ? 1 : 2;
@@ -342,10 +341,9 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
   cudaStream_t s = as_stream(stream);
   const uint16_t* X = static_cast<const uint16_t*>(X_dev);
   {
-    elmo::KernelScope ks(h, ELMO_K_PREP, s, h->dt == ELMO_FP8_E4M3 ? 2 : 1);
+    elmo::KernelScope ks(h, ELMO_K_PREP, s, 1);
     ELMO_CUDA(cudaMemsetAsync(dX_dev, 0, sizeof(float) * (size_t)B * h->d, s), "dX clear");
-    ELMO_CUDA(elmo::launch_prep_labels(h, rowptr_dev, cols_dev, B, nnz, s), "prep_labels");
-    if (h->dt == ELMO_FP8_E4M3) ELMO_CUDA(elmo::launch_prep_x(h, X, B, s), "prep_x");
+    ELMO_CUDA(elmo::launch_prep_step(h, rowptr_dev, cols_dev, B, nnz, X, s), "prep");
   }
   const bool fp8 = h->dt == ELMO_FP8_E4M3;
   const size_t esz = fp8 ? 1 : 2;

@@ -80,6 +80,9 @@ void set_last_error(const char* msg);
 cudaError_t launch_prep_labels(elmo_head* h, const int32_t* rowptr, const int32_t* cols, int32_t B,
                                int32_t nnz, cudaStream_t s);
 cudaError_t launch_prep_x(elmo_head* h, const uint16_t* X, int32_t B, cudaStream_t s);
+// the labels and (E4M3) X of a training step, in one launch
+cudaError_t launch_prep_step(elmo_head* h, const int32_t* rowptr, const int32_t* cols, int32_t B, int32_t nnz,
+                             const uint16_t* X, cudaStream_t s);
 
 // step_simt.cu -- reference-order kernels (first correct path)
 cudaError_t launch_grad_simt(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,

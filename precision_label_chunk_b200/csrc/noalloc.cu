@@ -123,8 +123,7 @@ extern "C" elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d
   // the status word and dX must start at zero; everything else in the scratch is rewritten before it is read
   e = cudaMemsetAsync(status_dev, 0, 2 * sizeof(int32_t), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(dX_dev, 0, sizeof(float) * (size_t)B * d, st);
-  if (e == cudaSuccess) e = elmo::launch_prep_labels(&h, rowptr_dev, cols_dev, B, nnz, st);
-  if (e == cudaSuccess && fp8) e = elmo::launch_prep_x(&h, X, B, st);
+  if (e == cudaSuccess) e = elmo::launch_prep_step(&h, rowptr_dev, cols_dev, B, nnz, X, st);
   for (int64_t c0 = 0; e == cudaSuccess && c0 < L; c0 += chunk) {
     const int64_t c1 = c0 + chunk < L ? c0 + chunk : L;
     for (int64_t a = c0; e == cudaSuccess && a < c1; a += sub) {

@@ -31,7 +31,7 @@ constexpr int kPrepThreads = 1024;
 // One CTA.  Shared memory holds the keys and each key's slot in its tile
 // (nnz <= 32768, so a slot fits 16 bits); the per-tile counters and their
 // prefix sums live in tile_ptr itself ([ntg + 1] entries in global memory).
-__global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t* __restrict__ rowptr,
+__device__ __forceinline__ void prep_labels_body(const int32_t* __restrict__ rowptr,
                                                                    const int32_t* __restrict__ cols, int32_t B,
                                                                    int32_t nnz, int64_t L,
                                                                    uint32_t* __restrict__ keys_out,
@@ -85,7 +85,13 @@ __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t
   const int per = (n + kPrepThreads - 1) / kPrepThreads;
   const int g0 = tid * per, g1 = min(n, g0 + per);
   int32_t run = 0;
-  for (int g = g0; g < g1; ++g) run += __ldcg(tile_ptr + g);   // the counts were formed by L2 atomics
+  for (int g = g0; g < g1; g += 8) {            // 8 independent loads in flight
+    int32_t c[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) c[u] = g + u < g1 ? __ldcg(tile_ptr + g + u) : 0;   // formed by L2 atomics
+#pragma unroll
+    for (int u = 0; u < 8; ++u) run += c[u];
+  }
   part[tid] = run;
   __syncthreads();
   for (int o = 1; o < kPrepThreads; o <<= 1) {   // Hillis-Steele scan of the run totals
@@ -95,9 +101,13 @@ __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t
     __syncthreads();
   }
   int32_t acc = part[tid] - run;                 // exclusive prefix of this run
-  for (int g = g0; g < g1; ++g) {
-    acc += __ldcg(tile_ptr + g);
-    tile_ptr[g] = acc;
+  for (int g = g0; g < g1; g += 8) {
+    int32_t c[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) c[u] = g + u < g1 ? __ldcg(tile_ptr + g + u) : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (g + u < g1) { acc += c[u]; tile_ptr[g + u] = acc; }
   }
   __syncthreads();
   // scatter: tile g's keys land in [tile_ptr[g], tile_ptr[g + 1])
@@ -110,9 +120,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t
 
 // One CTA: max |X| with 16-byte loads, the power-of-two scale, then the E4M3
 // codes of X * s_X (second pass mostly from L1/L2).  n is a multiple of 64.
-__global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __restrict__ X, int64_t n,
-                                                              float* __restrict__ xscale,
-                                                              uint8_t* __restrict__ xq) {
+__device__ __forceinline__ void prep_x_body(const uint16_t* __restrict__ X, int64_t n, float* __restrict__ xscale,
+                                            uint8_t* __restrict__ xq) {
   __shared__ float red[kPrepThreads / 32];
   __shared__ int nonfinite;
   __shared__ float s_scale;
@@ -168,7 +177,50 @@ __global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __
   }
 }
 
+__global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t* __restrict__ rowptr,
+                                                                   const int32_t* __restrict__ cols, int32_t B,
+                                                                   int32_t nnz, int64_t L,
+                                                                   uint32_t* __restrict__ keys_out,
+                                                                   int32_t* __restrict__ nkeys,
+                                                                   int32_t* __restrict__ tile_ptr,
+                                                                   int32_t* __restrict__ status) {
+  prep_labels_body(rowptr, cols, B, nnz, L, keys_out, nkeys, tile_ptr, status);
+}
+
+__global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __restrict__ X, int64_t n,
+                                                              float* __restrict__ xscale,
+                                                              uint8_t* __restrict__ xq) {
+  prep_x_body(X, n, xscale, xq);
+}
+
+// Both preparations of an E4M3 step in one launch: CTA 0 the labels, CTA 1 X.
+__global__ void __launch_bounds__(kPrepThreads) prep_step_kernel(const int32_t* __restrict__ rowptr,
+                                                                 const int32_t* __restrict__ cols, int32_t B,
+                                                                 int32_t nnz, int64_t L,
+                                                                 uint32_t* __restrict__ keys_out,
+                                                                 int32_t* __restrict__ nkeys,
+                                                                 int32_t* __restrict__ tile_ptr,
+                                                                 int32_t* __restrict__ status,
+                                                                 const uint16_t* __restrict__ X, int64_t n,
+                                                                 float* __restrict__ xscale,
+                                                                 uint8_t* __restrict__ xq) {
+  if (blockIdx.x == 0) prep_labels_body(rowptr, cols, B, nnz, L, keys_out, nkeys, tile_ptr, status);
+  else prep_x_body(X, n, xscale, xq);
+}
+
 }  // namespace
+
+cudaError_t launch_prep_step(elmo_head* h, const int32_t* rowptr, const int32_t* cols, int32_t B, int32_t nnz,
+                             const uint16_t* X, cudaStream_t s) {
+  if (h->dt != ELMO_FP8_E4M3) return launch_prep_labels(h, rowptr, cols, B, nnz, s);
+  const size_t smem = (sizeof(uint32_t) + sizeof(uint16_t)) * (size_t)(nnz > 0 ? nnz : 1);
+  cudaError_t e = cudaFuncSetAttribute(prep_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)((sizeof(uint32_t) + sizeof(uint16_t)) * ELMO_MAX_NNZ));
+  if (e != cudaSuccess) return e;
+  prep_step_kernel<<<2, kPrepThreads, smem, s>>>(rowptr, cols, B, nnz, h->L, h->keys, h->nkeys, h->tile_ptr,
+                                                 h->status, X, (int64_t)B * h->d, h->xscale, h->xq);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_prep_labels(elmo_head* h, const int32_t* rowptr, const int32_t* cols, int32_t B,
                                int32_t nnz, cudaStream_t s) {
