@@ -813,10 +813,10 @@ __global__ void __launch_bounds__(kXtThreads, 1)
 // ============================================================================
 // Kernel B: input gradient, weight gradient and the SR update.
 // ============================================================================
-constexpr int kWSlots = 2;
+constexpr int kWSlots = 4;                  // the most W slots (E4M3; bf16 has 2)
 constexpr int kGSlots = 3;
 constexpr uint32_t kXBytes = 2 * 32768;     // X[:, slice]: up to two 64-column boxes of up to 256 rows
-constexpr uint32_t kWSlotBytes = 2 * kBox;  // W[tile, slice]
+constexpr uint32_t kWSlotBytes = 2 * kBox;  // W[tile, slice] (bf16: two boxes)
 constexpr uint32_t kGSlotBytes = 2 * kBox;  // one part of G^T[tile]: two boxes of 128 bytes of samples
 
 struct SmemB {
@@ -840,9 +840,15 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
               uint64_t step, float* __restrict__ dX, int gsm, int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // E4M3 operands take half the bytes, which leaves room for 4 W slots: the
+  // W load of a unit then starts two units ahead of its epilogue, so the
+  // load -> MMA chain (about 2 us) stays off the epilogue's critical path
+  constexpr int kWS = kFp8 ? 4 : 2;
+  constexpr uint32_t kWSB = kFp8 ? kBox : 2 * kBox;           // bytes of one W slot
+  constexpr uint32_t kXB = kFp8 ? 32768u : 2 * 32768u;        // bytes of X[:, slice]
   uint8_t* xs = base;
-  uint8_t* ws = xs + kXBytes;
-  uint8_t* gs = ws + kWSlots * kWSlotBytes;
+  uint8_t* ws = xs + kXB;
+  uint8_t* gs = ws + kWS * kWSB;
   SmemB* S = reinterpret_cast<SmemB*>(gs + kGSlots * kGSlotBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t span = l1 - l0;
@@ -866,7 +872,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
   if (threadIdx.x == 0) {
     mbar_init(&S->xfull, 1); mbar_init(&S->xempty, 1);
     mbar_init(&S->dxfull, 1); mbar_init(&S->dxempty, kEpiU);
-    for (int s = 0; s < kWSlots; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kEpiU); }
+    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kEpiU); }
     for (int s = 0; s < kGSlots; ++s) { mbar_init(&S->gfull[s], 1); mbar_init(&S->gempty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&S->dwfull[b], 1); mbar_init(&S->dwempty[b], kEpiU); }
     S->abort = 0;
@@ -903,15 +909,15 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
           const int t = u - D * T;
           const int32_t row0 = (int32_t)(l0 + (int64_t)t * 128);
           {
-            const int s = wit % kWSlots;
-            const uint32_t ph = (wit / kWSlots) & 1;
+            const int s = wit % kWS;
+            const uint32_t ph = (wit / kWS) & 1;
             ++wit;
             if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 12); break; }
             int nb = 0;
             for (int q = 0; q < 128 / kBoxCols; ++q) nb += (D0 + q * kBoxCols < d);
             mbar_arrive_expect_tx(&S->wfull[s], (uint32_t)nb * kBox);
             for (int q = 0; q < 128 / kBoxCols; ++q)
-              if (D0 + q * kBoxCols < d) tma_load_2d(ws + s * kWSlotBytes + q * kBox, &tmW, &S->wfull[s], D0 + q * kBoxCols, row0);
+              if (D0 + q * kBoxCols < d) tma_load_2d(ws + s * kWSB + q * kBox, &tmW, &S->wfull[s], D0 + q * kBoxCols, row0);
           }
           for (int p = 0; p < nparts; ++p) {
             const int s = git % kGSlots;
@@ -947,15 +953,15 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
         tc_fence_after();
         bool first = true;
         for (; u < ue && !*abort; ++u) {
-          const int sw = wit % kWSlots;
-          const uint32_t phw = (wit / kWSlots) & 1;
+          const int sw = wit % kWS;
+          const uint32_t phw = (wit / kWS) & 1;
           ++wit;
           const uint32_t db = dwit & 1, duse = dwit >> 1;
           ++dwit;
           if (!mbar_wait(&S->wfull[sw], phw, abort, kWaitCycles)) { record_timeout(status, abort, 23); break; }
           if (!mbar_wait(&S->dwempty[db], (duse & 1) ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 24); break; }
           tc_fence_after();
-          const uint32_t wa = smem_u32(ws + sw * kWSlotBytes);
+          const uint32_t wa = smem_u32(ws + sw * kWSB);
           const uint32_t xa = smem_u32(xs);
           for (int p = 0; p < nparts; ++p) {
             const int sg = git % kGSlots;
@@ -1020,7 +1026,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
       const int D0 = D * 128;
       for (; u < ue && !*abort; ++u) {
         const int t = u - D * T;
-        const int sw = wit % kWSlots;
+        const int sw = wit % kWS;
         ++wit;
         const uint32_t db = dwit & 1, duse = dwit >> 1;
         ++dwit;
@@ -1028,7 +1034,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
         tc_fence_after();
         const int64_t l = l0 + (int64_t)t * 128 + row;
         const bool valid = (l - l0) < span;
-        const uint8_t* wrow = ws + sw * kWSlotBytes;
+        const uint8_t* wrow = ws + sw * kWSB;
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + 256 + db * 128;
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
@@ -1078,7 +1084,10 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
 
 // ---------------------------------------------------------------- host side
 constexpr size_t kSmemA = 1024 + kStagesA * kStageABytes + sizeof(SmemA);
-constexpr size_t kSmemB = 1024 + kXBytes + kWSlots * kWSlotBytes + kGSlots * kGSlotBytes + sizeof(SmemB);
+// the bf16 layout (X 64 KB, 2 W slots of 32 KB) is the larger of the two
+// (E4M3: X 32 KB, 4 W slots of 16 KB)
+constexpr size_t kSmemB = 1024 + kXBytes + 2 * kWSlotBytes + kGSlots * kGSlotBytes + sizeof(SmemB);
+static_assert(32768 + kWSlots * kBox <= kXBytes + 2 * kWSlotBytes, "E4M3 kernel B layout");
 constexpr size_t kSmemP = 1024 + kPanelSmem + sizeof(SmemP);
 static_assert(kSmemA <= 232448, "kernel A shared memory");
 static_assert(kSmemP <= 232448, "kernel A (resident X) shared memory");
