@@ -75,6 +75,7 @@ def _declare(L):
     L.orc_dx_rows.argtypes = [P, i64, i32, ctypes.c_int, P, i32, P, P, P, i32, P, ctypes.c_int]
     L.orc_topk.argtypes = [P, i64, i32, ctypes.c_int, P, i32, i32, P, i32, P, P, ctypes.c_int]
     L.orc_precision_at_k.argtypes = [P, i32, i32, P, P, P]
+    L.orc_kahan_sgd.argtypes = [P, P, P, i64, f32]
     L.orc_score.argtypes = [P, ctypes.c_int, i64, P, i32, i32]
     L.orc_score.restype = f32
 
@@ -236,6 +237,18 @@ def precision_at_k(idx, rowptr, cols):
     _check(lib().orc_precision_at_k(_p(idx), B, k, _p(_c(rowptr, np.int32)), _p(_c(cols, np.int32)), _p(p)),
            "precision_at_k")
     return p
+
+
+def kahan_sgd(p, c, g, lr):
+    """One Kahan-compensated SGD step of bf16 parameters p with bf16
+    compensation c and bf16 gradient g (uint16 bit patterns, same shape).
+    Returns the new (p, c)."""
+    p = _c(p, np.uint16).copy()
+    c = _c(c, np.uint16).copy()
+    g = _c(g, np.uint16)
+    assert p.shape == c.shape == g.shape
+    lib().orc_kahan_sgd(_p(p), _p(c), _p(g), p.size, float(lr))
+    return p, c
 
 
 def score(W, X, l, b, dtype) -> float:

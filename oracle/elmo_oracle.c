@@ -539,6 +539,36 @@ int orc_precision_at_k(const int32_t* idx, int32_t B, int32_t k, const int32_t* 
 }
 
 /* ------------------------------------------------------------------------ */
+/* Kahan-compensated SGD of a dense BF16 layer (the encoder side).           */
+/* The pages train the encoder in pure BF16 with Kahan summation in place of */
+/* FP32 master weights (atlas summary "Approach"; abstract).  Reading: the   */
+/* parameters p and the compensation c are stored in bf16, the gradient g   */
+/* arrives in bf16; every operation below is one IEEE fp32 operation and    */
+/* the two stored results are rounded to bf16 to nearest-even:              */
+/*   u  = -(lr * g)               the plain SGD increment                   */
+/*   y  = u + c                   plus what earlier steps could not store   */
+/*   p' = bf16(p + y)             the new parameter                         */
+/*   c' = bf16(y - (p' - p))      what this step could not store            */
+/* Kahan's compensated summation (Kahan 1965) applied to p + sum of u.      */
+/* ------------------------------------------------------------------------ */
+void orc_kahan_sgd(uint16_t* p, uint16_t* c, const uint16_t* g, int64_t n, float lr) {
+  for (int64_t i = 0; i < n; i++) {
+    const float pv = orc_bf16_value(p[i]);
+    const float cv = orc_bf16_value(c[i]);
+    const float gv = orc_bf16_value(g[i]);
+    const float prod = lr * gv;
+    const float u = -prod;
+    const float y = u + cv;
+    const float sum = pv + y;
+    const uint16_t pn = orc_rne_bf16(sum);
+    const float moved = orc_bf16_value(pn) - pv;
+    const float lost = y - moved;
+    c[i] = orc_rne_bf16(lost);
+    p[i] = pn;
+  }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Array helpers for the Python side (loops over the scalar definitions).   */
 /* ------------------------------------------------------------------------ */
 void orc_draw16_array(uint64_t seed, uint64_t step, uint64_t base, int64_t n, uint32_t* out) {
