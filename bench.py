@@ -12,9 +12,11 @@ Output Spaces"; the data are synthetic (the dataset is not available).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl elmo|reference]
                     [--workload NAME]
 
-Prints one JSON line (rank 0).  For N > 1 the ranks run independent replicas
-of the step (weak scaling, no collective on the data path); the time is the
-max over ranks.  `--impl reference` times the CPU oracle (a deliberately
+Prints one JSON line (rank 0).  For N > 1 the ranks hold one head of N * L
+labels split by labels (rank r the rows [r L, (r + 1) L)): every rank runs the
+fused step on its rows for the same batch and the ranks' input gradients are
+summed by one all-reduce of dX per step (weak scaling: L labels per GPU); the
+time is the max over ranks.  `--impl reference` times the CPU oracle (a deliberately
 plain program) on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -136,8 +138,9 @@ def max_over_ranks(ms, device=None):
 
 
 def job_throughput(world, labels, steps, ms):
-    """Whole-job label-rows/s: every rank (replica) processes all L labels per
-    step, so the job processes world * L * steps label-rows in the max time."""
+    """Whole-job label-rows/s: every rank processes its L labels per step (its
+    rows of the split head), so the job processes world * L * steps label-rows
+    in the max time."""
     return world * labels * steps / (ms / 1e3)
 
 
@@ -226,43 +229,59 @@ def run_reference(args, w):
 
 def run_topk(args, w, rank, world, local):
     """Chunked top-k prediction (X [B x d] bf16 against the whole head): one
-    step is one elmo_topk_predict call over all L labels."""
+    step is one elmo_topk_predict call over all L labels.  N > 1: a head of
+    N * L labels split by labels; each rank ranks its L rows, the ranks' lists
+    are gathered and merged on the device."""
     import torch
+    import torch.distributed as dist
     import precision_label_chunk_b200 as elmo
+    from precision_label_chunk_b200.sharded import ShardedHead
     from synthetic import make_X
     torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     dev = torch.device("cuda", local)
     peaks = load_peaks()
     wdt = torch.int16 if w.dtype == "bf16" else torch.uint8
     W = torch.empty(w.L, w.d, dtype=wdt, device=dev)
-    head = elmo.elmo_init_head(W, w.dtype, fill=True, init_std=0.02, seed=0)
+    labels_total = world * w.L
+    sharded = ShardedHead(W, labels_total, w.dtype, fill=True, init_std=0.02, seed=0, label_base=rank * w.L)
+    head = sharded.head
     nsteps = args.warmup + args.steps
     Xh = [make_X(w, s) for s in range(nsteps)]
     Xd = [torch.from_numpy(x.view(np.int16)).to(dev) for x in Xh]
     idx = torch.empty(w.B, w.topk, dtype=torch.int32, device=dev)
     sc = torch.empty(w.B, w.topk, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+    predict = lambda X: sharded.topk_predict(X, w.topk, w.chunk, idx, sc)   # noqa: E731
     for s in range(args.warmup):
-        elmo.elmo_topk_predict(head, Xd[s], w.topk, w.chunk, idx, sc)
+        predict(Xd[s])
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
     launches0 = elmo.elmo_launch_count(head)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for s in range(args.warmup, nsteps):
-        elmo.elmo_topk_predict(head, Xd[s], w.topk, w.chunk, idx, sc)
+        predict(Xd[s])
     ev1.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
-    gpu_launches = elmo.elmo_launch_count(head) - launches0
-    ms = ev0.elapsed_time(ev1) / args.steps
+    if world > 1:
+        dist.barrier()
+    # the head's kernels, plus one merge launch per step when split
+    gpu_launches = elmo.elmo_launch_count(head) - launches0 + (args.steps if world > 1 else 0)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev) / args.steps
     # per-kernel pass (events around every launch, outside the timed region)
     elmo.elmo_profile_reset(head)
     elmo.elmo_profile_enable(head, True)
     for s in range(args.warmup, nsteps):
-        elmo.elmo_topk_predict(head, Xd[s], w.topk, w.chunk, idx, sc)
+        predict(Xd[s])
     torch.cuda.synchronize()
     elmo.elmo_profile_enable(head, False)
     classes = {}
@@ -294,18 +313,21 @@ def run_topk(args, w, rank, world, local):
     sc_h = torch.empty(w.B, w.topk, dtype=torch.float32).pin_memory()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
     e0.record(stream)
     for s in range(args.warmup, nsteps):
-        elmo.elmo_topk_predict(head, pin[s].to(dev, non_blocking=True), w.topk, w.chunk, idx, sc)
+        predict(pin[s].to(dev, non_blocking=True))
         idx_h.copy_(idx, non_blocking=True)
         sc_h.copy_(sc, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1) / args.steps
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
     # P@1, P@3, P@5 of the last predictions against the queries' synthetic labels
     # (random weights: near zero; the point is that the metric runs on the device)
-    from synthetic import make_labels
-    rp, cl = make_labels(w, nsteps - 1)
+    from synthetic import make_labels, workload
+    rp, cl = make_labels(w if world == 1 else workload(w.name, L=labels_total), nsteps - 1)
     kk = min(5, w.topk)
     pk = torch.empty(kk, dtype=torch.float32, device=dev)
     elmo.elmo_precision_at_k(idx[:, :kk].contiguous(), torch.from_numpy(rp).to(dev), torch.from_numpy(cl).to(dev), pk)
@@ -328,7 +350,9 @@ def run_topk(args, w, rank, world, local):
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "L": w.L, "d": w.d, "B": w.B, "w_dtype": w.dtype, "k": w.topk,
-                       "chunk": w.chunk, "l2": f"inputs larger than L2 (W = {w.L * w.d / 1e9:.2f} GB)"},
+                       "chunk": w.chunk, "l2": f"inputs larger than L2 (W = {w.L * w.d / 1e9:.2f} GB per GPU)",
+                       "labels_total": labels_total,
+                       "parallelism": f"label-shards{world} (gather + merge of top-k)" if world > 1 else "single"},
             "tflops": flops / (ms / 1e3) / 1e12, "roofline": roof, "kernels": classes,
             "gpu_launches": gpu_launches,
             "e2e": {"value": world * w.B * w.L / (ms_e2e / 1e3), "unit": "query-labels/s",
@@ -337,6 +361,8 @@ def run_topk(args, w, rank, world, local):
         }
         print(json.dumps(line), flush=True)
     head.close()
+    if world > 1:
+        dist.destroy_process_group()
 
 
 def run_sr(args, local):
@@ -379,11 +405,99 @@ def run_sr(args, local):
     print(json.dumps(line), flush=True)
 
 
+def run_kahan(args, local):
+    """Kahan-compensated SGD of an encoder-sized BF16 parameter vector (110M
+    parameters, a BERT-base-sized encoder): bf16 p, c, g read and p, c written,
+    10 bytes per parameter, HBM-bound.  One step is one update of all
+    parameters; the fp32 dX of the head (B = 256, d = 768) handed over in
+    bf16 is timed beside it."""
+    import torch
+    import precision_label_chunk_b200 as elmo
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    n = 110_000_000
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    P = (torch.randn(n, generator=gen, device=dev) * 0.05).to(torch.bfloat16)
+    C = torch.zeros(n, dtype=torch.bfloat16, device=dev)
+    G = (torch.randn(n, generator=gen, device=dev) * 1e-2).to(torch.bfloat16)
+    lr = 1e-3
+    for _ in range(args.warmup):
+        elmo.elmo_kahan_sgd(P, C, G, lr)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        elmo.elmo_kahan_sgd(P, C, G, lr)
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    gbs = n * 10 / (ms / 1e3) / 1e9
+    # dX of the head to bf16 (small: launch-bound, reported for completeness)
+    dX = torch.randn(256 * 768, generator=gen, device=dev)
+    dXb = torch.empty(256 * 768, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        elmo.elmo_round_bf16(dX, dXb)
+    torch.cuda.synchronize()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record()
+    for _ in range(100):
+        elmo.elmo_round_bf16(dX, dXb)
+    r1.record()
+    torch.cuda.synchronize()
+    # end to end: the gradient from pinned host memory, the parameters back to the host
+    Gh = G.cpu().pin_memory()
+    Ph = torch.empty(n, dtype=torch.bfloat16).pin_memory()
+    torch.cuda.synchronize()
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record()
+    for _ in range(args.steps):
+        elmo.elmo_kahan_sgd(P, C, Gh.to(dev, non_blocking=True), lr)
+        Ph.copy_(P, non_blocking=True)
+    h1.record()
+    torch.cuda.synchronize()
+    ms_e2e = h0.elapsed_time(h1) / args.steps
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        ps, cs, gs = (t.view(torch.int16).cpu().numpy().view(np.uint16) for t in (P, C, G))
+        t, k = time.perf_counter(), 0
+        while k < 3 and time.perf_counter() - t < args.cpu_seconds:     # bounded: at most 3 steps
+            ps, cs = oracle.kahan_sgd(ps, cs, gs, lr)
+            k += 1
+        dt = time.perf_counter() - t
+        cpu = {"value": k * n / dt, "unit": "params/s", "cores": 1, "kind": "oracle",
+               "sample": f"all {n} parameters, {k} step(s), {dt:.1f} s"}
+    tr = profiled_traffic("kahan_sgd_vec", "kahan_sgd")
+    line = {"metric": "Kahan-compensated bf16 SGD: params/s", "value": n / (ms / 1e3), "unit": "params/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (fp32 arithmetic)",
+            "data": "synthetic",
+            "config": {"workload": "kahan_sgd", "n": n, "lr": lr,
+                       "l2": "inputs larger than L2 (660 MB of bf16 p, c, g)"},
+            "roofline": {"kernel": "kahan_sgd_vec", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "traffic": None if tr is None else tr["bytes"] * n / tr["labels"],
+                         "bytes_per_param": 10, "peak_source": f"{peaks['source']} copy bandwidth"},
+            "round_bf16_dx_us": r0.elapsed_time(r1) / 100 * 1e3,
+            "gpu_launches": args.steps,
+            "e2e": {"value": n / (ms_e2e / 1e3), "unit": "params/s", "h2d_bytes_per_step": n * 2,
+                    "d2h_bytes_per_step": n * 2},
+            "cpu_baseline": cpu, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
-    if args.workload == "sr_round":
+    if args.workload in ("sr_round", "kahan_sgd"):
         if int(os.environ.get("RANK", "0")) == 0:
-            run_sr(args, int(os.environ.get("LOCAL_RANK", "0")))
+            (run_sr if args.workload == "sr_round" else run_kahan)(args, int(os.environ.get("LOCAL_RANK", "0")))
         return
     from synthetic import workload
     w = workload(args.workload, **({"L": args.labels} if args.labels else {}))
@@ -404,6 +518,7 @@ def main():
     import torch.distributed as dist
 
     import precision_label_chunk_b200 as elmo
+    from precision_label_chunk_b200.sharded import ShardedHead
     from synthetic import make_labels, make_X
 
     torch.cuda.set_device(local)
@@ -414,15 +529,20 @@ def main():
     peaks = load_peaks()
     costs = step_costs(w)
 
-    # model state: W resident in HBM, filled on the device (SR of N(0, 0.02^2))
+    # model state: W resident in HBM, filled on the device (SR of N(0, 0.02^2)).
+    # N > 1: this rank's L rows of a head of N * L labels; the labels of a
+    # batch are drawn over the whole head
     wdt = torch.int16 if w.dtype == "bf16" else torch.uint8
     W = torch.empty(w.L, w.d, dtype=wdt, device=dev)
-    head = elmo.elmo_init_head(W, w.dtype, fill=True, init_std=0.02, seed=0)
+    labels_total = world * w.L
+    sharded = ShardedHead(W, labels_total, w.dtype, fill=True, init_std=0.02, seed=0, label_base=rank * w.L)
+    head = sharded.head
+    w_labels = w if world == 1 else workload(args.workload, L=labels_total)
     nsteps = args.warmup + args.steps
     host_batches = []
     for s in range(nsteps):
         X = make_X(w, s)
-        rowptr, cols = make_labels(w, s)
+        rowptr, cols = make_labels(w_labels, s)
         host_batches.append((X, rowptr, cols))
     dev_batches = [(torch.from_numpy(X.view(np.int16)).to(dev), torch.from_numpy(rp).to(dev),
                     torch.from_numpy(cl).to(dev)) for X, rp, cl in host_batches]
@@ -431,7 +551,7 @@ def main():
 
     def step(s, batch):
         Xd, rp, cl = batch
-        elmo.elmo_train_step_chunked(head, Xd, rp, cl, w.lr, w.chunk, 0, s, dX)
+        sharded.train_step(Xd, rp, cl, w.lr, w.chunk, 0, s, dX)     # + all-reduce of dX when N > 1
 
     for s in range(args.warmup):
         step(s, dev_batches[s])
@@ -560,8 +680,9 @@ def main():
             "vs_baseline": None, "dtype": "fp8-e4m3" if w.dtype == "fp8" else "bf16", "data": "synthetic",
             "config": {"workload": w.name, "L": w.L, "d": w.d, "B": w.B, "w_dtype": w.dtype, "chunk": w.chunk,
                        "lr": w.lr, "positives_per_sample": f"1+Poisson({w.lam})", "zipf_s": w.zipf_s,
-                       "l2": f"inputs larger than L2 (W = {costs['w_bytes'] / 2 / 1e9:.2f} GB per replica)",
-                       "parallelism": "replicas" if world > 1 else "single"},
+                       "l2": f"inputs larger than L2 (W = {costs['w_bytes'] / 2 / 1e9:.2f} GB per GPU)",
+                       "labels_total": labels_total,
+                       "parallelism": f"label-shards{world} (all-reduce of dX)" if world > 1 else "single"},
             "tflops": step_roof["tflops"], "step_roofline": step_roof, "roofline": roof,
             "kernels": classes, "kernels_pass_ms_per_step": kernels_pass_ms, "gpu_launches": gpu_launches, "e2e": e2e, "cpu_baseline": cpu,
             "clocks": clocks, "peak_device_bytes": int(peak_mem),

@@ -61,6 +61,8 @@ typedef struct elmo_head elmo_head;
 #define ELMO_MAX_LABELS (1LL << 24) /* L */
 #define ELMO_MAX_TOPK 64            /* k of a prediction */
 #define ELMO_MAX_PREDICT_BATCH 4096 /* B of a prediction */
+#define ELMO_MAX_TOTAL_LABELS 2147483647LL /* labels of a head split over devices (int32 ids) */
+#define ELMO_MAX_SHARDS 64          /* lists merged by elmo_topk_merge */
 
 /*
  * elmo_init_head -- wrap a caller-owned weight matrix in a head.
@@ -85,6 +87,35 @@ typedef struct elmo_head elmo_head;
  */
 elmo_status elmo_init_head(elmo_head** out, void* W_dev, int64_t L, int32_t d, elmo_dtype dt,
                            int fill, float init_std, uint64_t seed, void* stream);
+
+/*
+ * elmo_init_head_shard -- wrap the label rows [label_base, label_base + L) of
+ * a head of labels_total labels that is split by labels over several devices.
+ *
+ * Passage: the head is the part of the model that grows with the label count
+ * and dominates its compute and memory (abstract); split by label rows, each
+ * device holds and trains its own rows.  The step of a label depends only on
+ * its own weights, X and whether it is positive, so each device runs the same
+ * step on its rows and the devices' dX add up to the whole head's dX (the
+ * caller sums them, e.g. with one all-reduce).  Stochastic rounding and the
+ * fill draw by the element's index in the whole head, (label_base + l) * d + j,
+ * so the rows come out bit-identical to those of an unsplit head.
+ *
+ *   W_dev        : device pointer to this device's rows, [L x d], as in elmo_init_head.
+ *   L            : rows held here, 1 <= L < ELMO_MAX_LABELS.
+ *   label_base   : label id of row 0; 0 <= label_base <= labels_total - L.
+ *   labels_total : labels of the whole head, <= ELMO_MAX_TOTAL_LABELS.
+ * Training steps take the CSR of the whole head: positives with ids in
+ * [0, labels_total) outside this device's rows are skipped, ids outside
+ * [0, labels_total) set ELMO_EDATA.  elmo_topk_predict ranks this device's
+ * rows and returns label ids of the whole head; elmo_topk_merge combines the
+ * devices' lists.  elmo_forward_chunk's l0, l1 are row numbers of this device.
+ * Other arguments and errors as in elmo_init_head, which is this call with
+ * label_base = 0 and labels_total = L.
+ */
+elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_t d, elmo_dtype dt,
+                                 int64_t label_base, int64_t labels_total, int fill, float init_std,
+                                 uint64_t seed, void* stream);
 
 /* Releases the workspace (synchronising the device first); W is untouched. */
 elmo_status elmo_head_destroy(elmo_head* h);
@@ -160,11 +191,30 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B,
  *   X_dev     : bf16 [B x d] (device), 1 <= B <= ELMO_MAX_PREDICT_BATCH.
  *   k         : 1 <= k <= min(L, ELMO_MAX_TOPK).
  *   chunk     : labels per chunk (scheduling only; the result does not depend on it).
- *   idx_dev   : int32 [B x k] label ids (device), best first.
+ *   idx_dev   : int32 [B x k] label ids (device), best first; label ids of the
+ *               whole head for a head made by elmo_init_head_shard.
  *   score_dev : fp32 [B x k] their exact scores (device).
  */
 elmo_status elmo_topk_predict(elmo_head* h, const void* X_dev, int32_t B, int32_t k, int64_t chunk,
                               int32_t* idx_dev, float* score_dev, void* stream);
+
+/*
+ * elmo_topk_merge -- the top-k of a head split over P devices from the
+ * devices' own top-k lists (each device's elmo_topk_predict, gathered).
+ *
+ * Passage: as elmo_topk_predict.  The label sets of the lists are disjoint, so
+ * the best k of their union, in the same order (score descending, NaN after
+ * every number, ties to the lower label id), is the top-k of the whole head.
+ *
+ *   idx_dev, score_dev : int32 / fp32 [P x B x k] (device), list p of sample b
+ *                        at ((p * B) + b) * k, each sorted best first.
+ *   P                  : 1 <= P <= ELMO_MAX_SHARDS.
+ *   B, k               : 1 <= B <= ELMO_MAX_PREDICT_BATCH, 1 <= k <= ELMO_MAX_TOPK.
+ *   idx_out_dev, score_out_dev : int32 / fp32 [B x k] (device), best first;
+ *                        must not overlap the inputs.
+ */
+elmo_status elmo_topk_merge(const int32_t* idx_dev, const float* score_dev, int32_t P, int32_t B, int32_t k,
+                            int32_t* idx_out_dev, float* score_out_dev, void* stream);
 
 /*
  * elmo_sr_round -- standalone stochastic rounding.
@@ -181,6 +231,34 @@ elmo_status elmo_topk_predict(elmo_head* h, const void* X_dev, int32_t B, int32_
  */
 elmo_status elmo_sr_round(const float* in_dev, void* out_dev, int64_t n, elmo_dtype dt,
                           uint64_t seed, uint64_t step, uint64_t index_base, void* stream);
+
+/*
+ * elmo_kahan_sgd -- one Kahan-compensated SGD step of a dense BF16 layer.
+ *
+ * Passage: the pages train the encoder in pure BF16 with Kahan summation in
+ * place of FP32 master weights (atlas summary "Approach"; abstract).  For
+ * every element, with one IEEE fp32 operation per step and the two stored
+ * results rounded to nearest-even bf16 (NaN -> 0x7FC0):
+ *     u = -(lr g),  y = u + c,  p' = bf16(p + y),  c' = bf16(y - (p' - p))
+ * (Kahan's compensated summation of p and the increments: c carries what the
+ * bf16 grid of p could not take).
+ *
+ *   p_dev : bf16 [n] parameters (device), updated in place.
+ *   c_dev : bf16 [n] compensation (device), updated in place; zero it before
+ *           the first step.
+ *   g_dev : bf16 [n] gradient (device).
+ *   n     : >= 0 (0 is a no-op);  lr : finite.
+ * Buffers may have any alignment (16-byte aligned ones take the vector path).
+ */
+elmo_status elmo_kahan_sgd(void* p_dev, void* c_dev, const void* g_dev, int64_t n, float lr, void* stream);
+
+/*
+ * elmo_round_bf16 -- out[i] = bf16(in[i]), round to nearest-even, NaN -> 0x7FC0:
+ * the head's fp32 dX handed to a BF16 encoder (atlas summary "Approach": the
+ * whole model in pure BF16).
+ *   in_dev : fp32 [n] (device);  out_dev : bf16 [n] (device);  n >= 0.
+ */
+elmo_status elmo_round_bf16(const float* in_dev, void* out_dev, int64_t n, void* stream);
 
 /*
  * elmo_sr_draws -- the 16-bit uniform draws k (u = k / 2^16) that SR uses for

@@ -7,9 +7,12 @@ libelmo.so is missing or cannot be loaded, importing the library functions
 raises.
 
 The names match the C entry points:
-  elmo_init_head, elmo_head_destroy, elmo_train_step_chunked,
-  elmo_forward_chunk, elmo_topk_predict, elmo_sr_round, elmo_sr_draws,
-  elmo_sync_status, elmo_head_workspace_bytes.
+  elmo_init_head, elmo_init_head_shard, elmo_head_destroy,
+  elmo_train_step_chunked, elmo_train_step_noalloc, elmo_forward_chunk,
+  elmo_topk_predict, elmo_topk_merge, elmo_sr_round, elmo_sr_draws,
+  elmo_precision_at_k, elmo_kahan_sgd, elmo_round_bf16,
+  elmo_check_bounded_wait, elmo_sync_status,
+  elmo_head_workspace_bytes and the tracing calls.
 """
 from __future__ import annotations
 
@@ -25,7 +28,8 @@ __all__ = [
     "elmo_forward_chunk", "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws",
     "elmo_sync_status", "elmo_head_workspace_bytes", "elmo_profile_enable", "elmo_profile_reset",
     "elmo_profile_read", "elmo_launch_count", "KERNEL_CLASSES", "elmo_train_step_noalloc",
-    "elmo_check_bounded_wait", "WAIT_CHECK_SITE", "elmo_precision_at_k",
+    "elmo_check_bounded_wait", "WAIT_CHECK_SITE", "elmo_precision_at_k", "elmo_init_head_shard",
+    "elmo_topk_merge", "MAX_SHARDS", "MAX_TOTAL_LABELS", "elmo_kahan_sgd", "elmo_round_bf16",
 ]
 
 BF16 = 0
@@ -35,6 +39,8 @@ MAX_BATCH = 256
 MAX_NNZ = 32768
 MAX_TOPK = 64
 MAX_PREDICT_BATCH = 4096
+MAX_TOTAL_LABELS = 2**31 - 1
+MAX_SHARDS = 64
 
 STATUS_NAMES = {0: "ELMO_OK", 1: "ELMO_EINVAL", 2: "ELMO_ENOMEM", 3: "ELMO_ECUDA", 4: "ELMO_ETIMEOUT",
                 5: "ELMO_EUNSUPPORTED", 6: "ELMO_EDATA"}
@@ -74,6 +80,11 @@ def _declare(L):
     st = ctypes.c_int
     L.elmo_last_error.restype = ctypes.c_char_p
     L.elmo_init_head.argtypes = [ctypes.POINTER(P), P, i64, i32, ctypes.c_int, ctypes.c_int, f32, u64, P]
+    L.elmo_init_head_shard.argtypes = [ctypes.POINTER(P), P, i64, i32, ctypes.c_int, i64, i64, ctypes.c_int, f32,
+                                       u64, P]
+    L.elmo_topk_merge.argtypes = [P, P, i32, i32, i32, P, P, P]
+    L.elmo_kahan_sgd.argtypes = [P, P, P, i64, f32, P]
+    L.elmo_round_bf16.argtypes = [P, P, i64, P]
     L.elmo_head_destroy.argtypes = [P]
     L.elmo_train_step_chunked.argtypes = [P, P, i32, P, P, i32, f32, i64, u64, u64, P, P]
     L.elmo_forward_chunk.argtypes = [P, P, i32, P, P, i32, i64, i64, P, P, P]
@@ -131,13 +142,17 @@ def _dt(dtype) -> int:
 
 
 class Head:
-    """A borrowed weight matrix W [L, d] plus the library's workspace."""
+    """A borrowed weight matrix W [L, d] plus the library's workspace; W holds
+    the label rows [label_base, label_base + L) of a head of labels_total."""
 
-    def __init__(self, handle: ctypes.c_void_p, W: torch.Tensor, dtype: int):
+    def __init__(self, handle: ctypes.c_void_p, W: torch.Tensor, dtype: int, label_base: int = 0,
+                 labels_total: int | None = None):
         self.handle = handle
         self.W = W
         self.dtype = dtype
         self.L, self.d = W.shape
+        self.label_base = label_base
+        self.labels_total = self.L if labels_total is None else labels_total
 
     def close(self):
         if self.handle:
@@ -154,6 +169,13 @@ class Head:
 def elmo_init_head(W: torch.Tensor, dtype=None, fill: bool = False, init_std: float = 0.02, seed: int = 0,
                    stream=None) -> Head:
     """W: [L, d] CUDA tensor (bfloat16, or float8_e4m3fn / uint8 codes)."""
+    return elmo_init_head_shard(W, 0, W.shape[0], dtype, fill, init_std, seed, stream)
+
+
+def elmo_init_head_shard(W: torch.Tensor, label_base: int, labels_total: int, dtype=None, fill: bool = False,
+                         init_std: float = 0.02, seed: int = 0, stream=None) -> Head:
+    """W: this device's label rows [label_base, label_base + L) of a head of
+    labels_total labels split by labels over several devices."""
     if dtype is None:
         dtype = BF16 if W.dtype in (torch.bfloat16, torch.int16) else FP8_E4M3
     dt = _dt(dtype)
@@ -162,9 +184,10 @@ def elmo_init_head(W: torch.Tensor, dtype=None, fill: bool = False, init_std: fl
     if W.element_size() != (2 if dt == BF16 else 1):
         raise ValueError("W element size does not match dtype")
     h = ctypes.c_void_p()
-    _check(load().elmo_init_head(ctypes.byref(h), _ptr(W), W.shape[0], W.shape[1], dt, int(bool(fill)),
-                                 float(init_std), int(seed) & (2**64 - 1), _stream(stream)))
-    return Head(h, W, dt)
+    _check(load().elmo_init_head_shard(ctypes.byref(h), _ptr(W), W.shape[0], W.shape[1], dt, int(label_base),
+                                       int(labels_total), int(bool(fill)), float(init_std), int(seed) & (2**64 - 1),
+                                       _stream(stream)))
+    return Head(h, W, dt, int(label_base), int(labels_total))
 
 
 def elmo_head_destroy(head: Head):
@@ -205,6 +228,29 @@ def elmo_topk_predict(head: Head, X: torch.Tensor, k: int, chunk: int, idx: torc
                       stream=None):
     _check(load().elmo_topk_predict(head.handle, _ptr(X), X.shape[0], int(k), int(chunk), _ptr(idx), _ptr(score),
                                     _stream(stream)))
+
+
+def elmo_topk_merge(idx: torch.Tensor, score: torch.Tensor, idx_out: torch.Tensor, score_out: torch.Tensor,
+                    stream=None):
+    """Top-k of a head split over P devices: idx/score [P, B, k] (each device's
+    list, best first) -> idx_out/score_out [B, k]."""
+    P, B, k = idx.shape
+    _check(load().elmo_topk_merge(_ptr(idx), _ptr(score), P, B, k, _ptr(idx_out), _ptr(score_out), _stream(stream)))
+
+
+def elmo_kahan_sgd(p: torch.Tensor, c: torch.Tensor, g: torch.Tensor, lr: float, stream=None):
+    """One Kahan-compensated SGD step: bf16 parameters p and compensation c
+    (updated in place) with bf16 gradient g, all of the same size."""
+    if not (p.numel() == c.numel() == g.numel()) or any(t.element_size() != 2 for t in (p, c, g)):
+        raise ValueError("p, c and g must be bf16 tensors of the same size")
+    _check(load().elmo_kahan_sgd(_ptr(p), _ptr(c), _ptr(g), p.numel(), float(lr), _stream(stream)))
+
+
+def elmo_round_bf16(inp: torch.Tensor, out: torch.Tensor, stream=None):
+    """out = bf16(inp), round to nearest-even (fp32 dX handed to a bf16 encoder)."""
+    if inp.numel() != out.numel() or out.element_size() != 2:
+        raise ValueError("out must be a 2-byte tensor of inp's size")
+    _check(load().elmo_round_bf16(_ptr(inp), _ptr(out), inp.numel(), _stream(stream)))
 
 
 def elmo_sr_round(inp: torch.Tensor, out: torch.Tensor, dtype, seed: int, step: int, index_base: int = 0,

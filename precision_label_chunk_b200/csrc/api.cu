@@ -180,11 +180,21 @@ const char* elmo_last_error(void) { return g_last_error.c_str(); }
 
 elmo_status elmo_init_head(elmo_head** out, void* W_dev, int64_t L, int32_t d, elmo_dtype dt, int fill,
                            float init_std, uint64_t seed, void* stream) {
+  return elmo_init_head_shard(out, W_dev, L, d, dt, 0, L, fill, init_std, seed, stream);
+}
+
+elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_t d, elmo_dtype dt,
+                                 int64_t label_base, int64_t labels_total, int fill, float init_std, uint64_t seed,
+                                 void* stream) {
   g_last_error.clear();
   if (!out || !W_dev) return fail(ELMO_EINVAL, "null out or W");
   *out = nullptr;
   if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3) return fail(ELMO_EINVAL, "unknown dtype %d", (int)dt);
   if (L < 1 || L >= ELMO_MAX_LABELS) return fail(ELMO_EINVAL, "L = %lld outside [1, 2^24)", (long long)L);
+  if (label_base < 0 || labels_total > ELMO_MAX_TOTAL_LABELS || label_base > labels_total - L)
+    return fail(ELMO_EINVAL, "label rows [%lld, %lld) outside a head of %lld labels (at most %lld)",
+                (long long)label_base, (long long)(label_base + L), (long long)labels_total,
+                (long long)ELMO_MAX_TOTAL_LABELS);
   if (d < 64 || d > 4096 || d % 64 != 0) return fail(ELMO_EINVAL, "d = %d: need a multiple of 64 in [64, 4096]", d);
   if (!aligned16(W_dev)) return fail(ELMO_EINVAL, "W is not 16-byte aligned");
   if (fill && !(init_std >= 0.0f && init_std < 1e30f)) return fail(ELMO_EINVAL, "bad init_std");
@@ -197,6 +207,8 @@ elmo_status elmo_init_head(elmo_head** out, void* W_dev, int64_t L, int32_t d, e
   if (!h) return fail(ELMO_ENOMEM, "host allocation failed");
   h->W = W_dev;
   h->L = L;
+  h->label_base = label_base;
+  h->labels_total = labels_total;
   h->d = d;
   h->dt = dt;
   h->device = dev;
@@ -221,7 +233,7 @@ elmo_status elmo_init_head(elmo_head** out, void* W_dev, int64_t L, int32_t d, e
   cudaError_t e = cudaMemsetAsync(base, 0, 64, s);
   if (e == cudaSuccess && fill) {
     h->launches += 1;
-    e = elmo::launch_fill(W_dev, L * (int64_t)d, dt, init_std, seed, s);
+    e = elmo::launch_fill(W_dev, L * (int64_t)d, dt, init_std, seed, (uint64_t)label_base * (uint64_t)d, s);
   }
   if (e != cudaSuccess) {
     cudaFree(base);
@@ -418,13 +430,46 @@ elmo_status elmo_topk_predict(elmo_head* h, const void* X_dev, int32_t B, int32_
   if (elmo::topk_tc_supported(h) && !use_topk_simt()) {
     if ((st = ensure_cand(h, elmo::topk_tc_workspace_bytes(h, B, k))) != ELMO_OK) return st;
     ELMO_CUDA(elmo::launch_topk_tc(h, X, B, k, idx_dev, score_dev, as_stream(stream)), "topk");
-    return ELMO_OK;
+  } else {
+    if ((st = ensure_cand(h, elmo::topk_simt_workspace_bytes(h, B, k))) != ELMO_OK) return st;
+    elmo::KernelScope ks(h, ELMO_K_TOPK_SCORE, as_stream(stream), 2);
+    ELMO_CUDA(elmo::launch_topk_simt_rows(h, X, B, k, nullptr, nullptr, h->cand, idx_dev, score_dev,
+                                          as_stream(stream)),
+              "topk");
   }
-  if ((st = ensure_cand(h, elmo::topk_simt_workspace_bytes(h, B, k))) != ELMO_OK) return st;
-  elmo::KernelScope ks(h, ELMO_K_TOPK_SCORE, as_stream(stream), 2);
-  ELMO_CUDA(elmo::launch_topk_simt_rows(h, X, B, k, nullptr, nullptr, h->cand, idx_dev, score_dev,
-                                        as_stream(stream)),
-            "topk");
+  if (h->label_base != 0) {     // label ids of the whole head
+    h->launches += 1;
+    ELMO_CUDA(elmo::launch_topk_offset(idx_dev, (int64_t)B * k, h->label_base, as_stream(stream)), "topk offset");
+  }
+  return ELMO_OK;
+}
+
+elmo_status elmo_kahan_sgd(void* p_dev, void* c_dev, const void* g_dev, int64_t n, float lr, void* stream) {
+  g_last_error.clear();
+  if (n < 0) return fail(ELMO_EINVAL, "n = %lld < 0", (long long)n);
+  if (n > 0 && (!p_dev || !c_dev || !g_dev)) return fail(ELMO_EINVAL, "null pointer");
+  if (!(lr > -1e30f && lr < 1e30f)) return fail(ELMO_EINVAL, "lr is not finite");
+  ELMO_CUDA(elmo::launch_kahan_sgd(p_dev, c_dev, g_dev, n, lr, as_stream(stream)), "kahan_sgd");
+  return ELMO_OK;
+}
+
+elmo_status elmo_round_bf16(const float* in_dev, void* out_dev, int64_t n, void* stream) {
+  g_last_error.clear();
+  if (n < 0) return fail(ELMO_EINVAL, "n = %lld < 0", (long long)n);
+  if (n > 0 && (!in_dev || !out_dev)) return fail(ELMO_EINVAL, "null pointer");
+  ELMO_CUDA(elmo::launch_round_bf16(in_dev, out_dev, n, as_stream(stream)), "round_bf16");
+  return ELMO_OK;
+}
+
+elmo_status elmo_topk_merge(const int32_t* idx_dev, const float* score_dev, int32_t P, int32_t B, int32_t k,
+                            int32_t* idx_out_dev, float* score_out_dev, void* stream) {
+  g_last_error.clear();
+  if (!idx_dev || !score_dev || !idx_out_dev || !score_out_dev) return fail(ELMO_EINVAL, "null pointer");
+  if (P < 1 || P > ELMO_MAX_SHARDS) return fail(ELMO_EINVAL, "P = %d outside [1, %d]", P, ELMO_MAX_SHARDS);
+  if (B < 1 || B > ELMO_MAX_PREDICT_BATCH) return fail(ELMO_EINVAL, "B = %d outside [1, %d]", B, ELMO_MAX_PREDICT_BATCH);
+  if (k < 1 || k > ELMO_MAX_TOPK) return fail(ELMO_EINVAL, "k = %d outside [1, %d]", k, ELMO_MAX_TOPK);
+  ELMO_CUDA(elmo::launch_topk_merge(idx_dev, score_dev, P, B, k, idx_out_dev, score_out_dev, as_stream(stream)),
+            "topk merge");
   return ELMO_OK;
 }
 

@@ -19,6 +19,8 @@ struct elmo_prof_rec {
 struct elmo_head {
   void* W = nullptr;           // borrowed [L x d] bf16 bits or E4M3 codes
   int64_t L = 0;
+  int64_t label_base = 0;      // W holds the label rows [label_base, label_base + L) ...
+  int64_t labels_total = 0;    // ... of a head of labels_total labels (0 and L when unsharded)
   int32_t d = 0;
   elmo_dtype dt = ELMO_BF16;
   int device = 0;
@@ -130,6 +132,13 @@ cudaError_t launch_sr_round(const float* in, void* out, int64_t n, elmo_dtype dt
                             uint64_t step, uint64_t base, cudaStream_t s);
 cudaError_t launch_sr_draws(uint16_t* out, int64_t n, uint64_t seed, uint64_t step, uint64_t base,
                             cudaStream_t s);
-cudaError_t launch_fill(void* W, int64_t n, elmo_dtype dt, float std, uint64_t seed, cudaStream_t s);
+cudaError_t launch_fill(void* W, int64_t n, elmo_dtype dt, float std, uint64_t seed, uint64_t index_base,
+                        cudaStream_t s);
+cudaError_t launch_kahan_sgd(void* p, void* c, const void* g, int64_t n, float lr, cudaStream_t s);
+cudaError_t launch_round_bf16(const float* in, void* out, int64_t n, cudaStream_t s);
+// global label ids of a sharded head's top-k (idx += label_base)
+cudaError_t launch_topk_offset(int32_t* idx, int64_t n, int64_t label_base, cudaStream_t s);
+cudaError_t launch_topk_merge(const int32_t* idx, const float* score, int32_t P, int32_t B, int32_t k,
+                              int32_t* idx_out, float* score_out, cudaStream_t s);
 
 }  // namespace elmo

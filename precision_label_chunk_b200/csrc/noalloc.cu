@@ -98,6 +98,7 @@ extern "C" elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d
   elmo_head h;
   h.W = W_dev;
   h.L = L;
+  h.labels_total = L;
   h.d = d;
   h.dt = dt;
   h.device = dev;

@@ -6,8 +6,10 @@
 // (label << 8 | sample) grouped by tile, tile g's keys at
 // [tile_ptr[g], tile_ptr[g+1]) in no particular order within the tile.
 // Malformed input (rowptr not monotone, rowptr[B] != nnz, a column outside
-// [0, L)) is recorded in the head's status word as ELMO_EDATA and the
-// offending entries are dropped.
+// [0, labels_total)) is recorded in the head's status word as ELMO_EDATA and
+// the offending entries are dropped.  A head that holds the label rows
+// [label_base, label_base + L) of a larger head keeps the positives that fall
+// in its rows, as local labels (label - label_base), and skips the others.
 //
 // X in FP8 mode: the pages train the classifier in E4M3 without tensor
 // scaling of the weights ("ELMO: Efficiency via Low-precision and Peak Memory
@@ -34,6 +36,7 @@ constexpr int kPrepThreads = 1024;
 __device__ __forceinline__ void prep_labels_body(const int32_t* __restrict__ rowptr,
                                                                    const int32_t* __restrict__ cols, int32_t B,
                                                                    int32_t nnz, int64_t L,
+                                                                   int64_t label_base, int64_t labels_total,
                                                                    uint32_t* __restrict__ keys_out,
                                                                    int32_t* __restrict__ nkeys,
                                                                    int32_t* __restrict__ tile_ptr,
@@ -69,10 +72,13 @@ __device__ __forceinline__ void prep_labels_body(const int32_t* __restrict__ row
     }
     const int32_t c = cols[i];
     uint32_t key = 0xFFFFFFFFu;
-    if (c >= 0 && (int64_t)c < L) {
-      key = ((uint32_t)c << 8) | (uint32_t)lo;
-      slot[i] = (uint16_t)atomicAdd(&tile_ptr[(c >> 7) + 1], 1);
-      ++cnt;
+    if (c >= 0 && (int64_t)c < labels_total) {
+      const int64_t lc = (int64_t)c - label_base;   // label within this head's rows
+      if (lc >= 0 && lc < L) {
+        key = ((uint32_t)lc << 8) | (uint32_t)lo;
+        slot[i] = (uint16_t)atomicAdd(&tile_ptr[(lc >> 7) + 1], 1);
+        ++cnt;
+      }
     } else {
       set_status(status, ELMO_EDATA, i);
     }
@@ -180,11 +186,12 @@ __device__ __forceinline__ void prep_x_body(const uint16_t* __restrict__ X, int6
 __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t* __restrict__ rowptr,
                                                                    const int32_t* __restrict__ cols, int32_t B,
                                                                    int32_t nnz, int64_t L,
+                                                                   int64_t label_base, int64_t labels_total,
                                                                    uint32_t* __restrict__ keys_out,
                                                                    int32_t* __restrict__ nkeys,
                                                                    int32_t* __restrict__ tile_ptr,
                                                                    int32_t* __restrict__ status) {
-  prep_labels_body(rowptr, cols, B, nnz, L, keys_out, nkeys, tile_ptr, status);
+  prep_labels_body(rowptr, cols, B, nnz, L, label_base, labels_total, keys_out, nkeys, tile_ptr, status);
 }
 
 __global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __restrict__ X, int64_t n,
@@ -197,6 +204,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __
 __global__ void __launch_bounds__(kPrepThreads) prep_step_kernel(const int32_t* __restrict__ rowptr,
                                                                  const int32_t* __restrict__ cols, int32_t B,
                                                                  int32_t nnz, int64_t L,
+                                                                 int64_t label_base, int64_t labels_total,
                                                                  uint32_t* __restrict__ keys_out,
                                                                  int32_t* __restrict__ nkeys,
                                                                  int32_t* __restrict__ tile_ptr,
@@ -204,7 +212,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_step_kernel(const int32_t* 
                                                                  const uint16_t* __restrict__ X, int64_t n,
                                                                  float* __restrict__ xscale,
                                                                  uint8_t* __restrict__ xq) {
-  if (blockIdx.x == 0) prep_labels_body(rowptr, cols, B, nnz, L, keys_out, nkeys, tile_ptr, status);
+  if (blockIdx.x == 0)
+    prep_labels_body(rowptr, cols, B, nnz, L, label_base, labels_total, keys_out, nkeys, tile_ptr, status);
   else prep_x_body(X, n, xscale, xq);
 }
 
@@ -217,8 +226,9 @@ cudaError_t launch_prep_step(elmo_head* h, const int32_t* rowptr, const int32_t*
   cudaError_t e = cudaFuncSetAttribute(prep_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)((sizeof(uint32_t) + sizeof(uint16_t)) * ELMO_MAX_NNZ));
   if (e != cudaSuccess) return e;
-  prep_step_kernel<<<2, kPrepThreads, smem, s>>>(rowptr, cols, B, nnz, h->L, h->keys, h->nkeys, h->tile_ptr,
-                                                 h->status, X, (int64_t)B * h->d, h->xscale, h->xq);
+  prep_step_kernel<<<2, kPrepThreads, smem, s>>>(rowptr, cols, B, nnz, h->L, h->label_base, h->labels_total,
+                                                 h->keys, h->nkeys, h->tile_ptr, h->status, X,
+                                                 (int64_t)B * h->d, h->xscale, h->xq);
   return cudaGetLastError();
 }
 
@@ -228,8 +238,8 @@ cudaError_t launch_prep_labels(elmo_head* h, const int32_t* rowptr, const int32_
   cudaError_t e = cudaFuncSetAttribute(prep_labels_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)((sizeof(uint32_t) + sizeof(uint16_t)) * ELMO_MAX_NNZ));
   if (e != cudaSuccess) return e;
-  prep_labels_kernel<<<1, kPrepThreads, smem, s>>>(rowptr, cols, B, nnz, h->L, h->keys, h->nkeys, h->tile_ptr,
-                                                   h->status);
+  prep_labels_kernel<<<1, kPrepThreads, smem, s>>>(rowptr, cols, B, nnz, h->L, h->label_base, h->labels_total,
+                                                   h->keys, h->nkeys, h->tile_ptr, h->status);
   return cudaGetLastError();
 }
 

@@ -65,18 +65,19 @@ __global__ void __launch_bounds__(256) sr_draws_kernel(uint16_t* __restrict__ ou
   }
 }
 
-// W[i] = SR(std * n_i): n_i standard normal by the Box-Muller transform of two
-// 32-bit Philox words (block i >> 2 of step 2^64-2 serves elements 4q..4q+3),
-// rounded with the SR draw of element i at step 2^64-1.
+// W[i] = SR(std * n_g): g = index_base + i the element's index in the whole
+// head (index_base a multiple of 8), n_g standard normal by the Box-Muller
+// transform of two 32-bit Philox words (block g >> 2 of step 2^64-2 serves
+// elements 4q..4q+3), rounded with the SR draw of element g at step 2^64-1.
 __global__ void __launch_bounds__(256) fill_kernel(void* __restrict__ W, int64_t n, int dt, float std,
-                                                   uint64_t seed) {
+                                                   uint64_t seed, uint64_t blk_base) {
   const uint64_t nblk = ((uint64_t)n + 7) >> 3;
   for (uint64_t q = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; q < nblk;
        q += (uint64_t)gridDim.x * blockDim.x) {
     float nv[8];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint64_t nb = q * 2 + h;
+      const uint64_t nb = (blk_base + q) * 2 + h;
       const u32x4 r = philox10((uint32_t)nb, (uint32_t)(nb >> 32), 0xFFFFFFFEu, 0xFFFFFFFFu,
                                (uint32_t)seed, (uint32_t)(seed >> 32));
       const uint32_t wd[4] = {r.x, r.y, r.z, r.w};
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(256) fill_kernel(void* __restrict__ W, int64_t
         nv[h * 4 + 2 * p + 1] = rad * sn;
       }
     }
-    const u32x4 r = sr_block(seed, ~0ull, q);
+    const u32x4 r = sr_block(seed, ~0ull, blk_base + q);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const uint64_t i = q * 8 + e;
@@ -160,9 +161,11 @@ cudaError_t launch_sr_draws(uint16_t* out, int64_t n, uint64_t seed, uint64_t st
   return cudaGetLastError();
 }
 
-cudaError_t launch_fill(void* W, int64_t n, elmo_dtype dt, float std, uint64_t seed, cudaStream_t s) {
+cudaError_t launch_fill(void* W, int64_t n, elmo_dtype dt, float std, uint64_t seed, uint64_t index_base,
+                        cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  fill_kernel<<<grid_for(((uint64_t)n + 7) >> 3, 256), 256, 0, s>>>(W, n, (int)dt, std, seed);
+  if (index_base & 7) return cudaErrorInvalidValue;
+  fill_kernel<<<grid_for(((uint64_t)n + 7) >> 3, 256), 256, 0, s>>>(W, n, (int)dt, std, seed, index_base >> 3);
   return cudaGetLastError();
 }
 

@@ -83,14 +83,14 @@ __global__ void dx_simt_kernel(const void* __restrict__ W, int dt, int32_t d, in
 __global__ void update_simt_kernel(void* __restrict__ W, int dt, int32_t d, const uint16_t* __restrict__ X,
                                    const uint8_t* __restrict__ xq, const float* __restrict__ xscale, int32_t B,
                                    int64_t l0, int64_t l1, const void* __restrict__ gbuf, float lr,
-                                   uint64_t seed, uint64_t step) {
+                                   uint64_t seed, uint64_t step, uint64_t idx_base) {
   const int64_t groups = (l1 - l0) * (d / 8);
   const float dw_scale = dt == ELMO_BF16 ? 1.0f : 0.00390625f * xscale[1];
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < groups;
        t += (int64_t)gridDim.x * blockDim.x) {
     const int64_t l = l0 + t / (d / 8);
     const int j0 = (int)(t % (d / 8)) * 8;
-    const uint64_t idx0 = (uint64_t)l * d + j0;
+    const uint64_t idx0 = idx_base + (uint64_t)l * d + j0;   // index in the whole head
     const u32x4 r = sr_block(seed, step, idx0 >> 3);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -142,7 +142,8 @@ cudaError_t launch_update_simt(const elmo_head* h, const uint16_t* X, int32_t B,
                                const void* gbuf, float lr, uint64_t seed, uint64_t step, cudaStream_t s) {
   if (l1 <= l0) return cudaSuccess;
   update_simt_kernel<<<grid_cap((l1 - l0) * (h->d / 8), 128), 128, 0, s>>>(
-      h->W, (int)h->dt, h->d, X, h->xq, h->xscale, B, l0, l1, gbuf, lr, seed, step);
+      h->W, (int)h->dt, h->d, X, h->xq, h->xscale, B, l0, l1, gbuf, lr, seed, step,
+      (uint64_t)h->label_base * (uint64_t)h->d);
   return cudaGetLastError();
 }
 

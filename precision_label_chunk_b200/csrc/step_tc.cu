@@ -176,11 +176,13 @@ __device__ __forceinline__ uint32_t mask16(const uint32_t (&m)[8], int b0) {
 
 // W[l, j0 .. j0+15] = SR(W - lrs * acc) for one label row: old weights from the
 // 128B-swizzled W tile in shared memory (row `row`, tile column jl), draws from
-// the two Philox blocks of elements l*d + j0 .. +15.
+// the two Philox blocks of elements l*d + j0 .. +15 (blk_base more blocks in
+// when this head holds the rows of a larger head from label_base on:
+// blk_base = label_base * d / 8).
 template <int kFp8>
 __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint8_t* __restrict__ wtile, int row, int jl,
                                          int64_t l, int32_t d, int j0, float lrs, uint64_t seed, uint64_t step,
-                                         void* __restrict__ Wglob) {
+                                         uint64_t blk_base, void* __restrict__ Wglob) {
   float wv[16];
   if (kFp8) {
     const uint4 x = *reinterpret_cast<const uint4*>(wtile + row * 128 + (((jl >> 4) ^ (row & 7)) << 4));
@@ -216,7 +218,7 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint8_t*
     vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
     probe = __fmaf_rn(vv[i], kFp8 ? 0.0f : 2.0f, probe);
   }
-  const uint64_t blk = ((uint64_t)l * (uint64_t)d + (uint64_t)j0) >> 3;
+  const uint64_t blk = blk_base + (((uint64_t)l * (uint64_t)d + (uint64_t)j0) >> 3);
   const u32x4 r0 = sr_block(seed, step, blk), r1 = sr_block(seed, step, blk + 1);
   const uint32_t rw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
   uint32_t wnew[8];
@@ -837,7 +839,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
     update_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
               const uint8_t* __restrict__ gbuf, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
               int32_t Bp, int64_t l0, int64_t l1, const float* __restrict__ xscale, float lr, uint64_t seed,
-              uint64_t step, float* __restrict__ dX, int gsm, int32_t* __restrict__ status) {
+              uint64_t step, uint64_t blk_base, float* __restrict__ dX, int gsm, int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // E4M3 operands take half the bytes, which leaves room for 4 W slots: the
@@ -1047,7 +1049,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
           if (!valid || j0 >= d) continue;
 #pragma unroll
           for (int g = 0; g < kGrp; ++g)
-            update16<kFp8>(r[g], wrow, row, jl + 16 * g, l, d, j0 + 16 * g, lrs, seed, step, Wglob);
+            update16<kFp8>(r[g], wrow, row, jl + 16 * g, l, d, j0 + 16 * g, lrs, seed, step, blk_base, Wglob);
         }
         tc_fence_before();
         __syncwarp();
@@ -1246,8 +1248,8 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
   if (e != cudaSuccess) return e;
   return launch_k(kern, grid, fp8 ? kThreads : 320, kSmemB, s, pdl, tmW, tmX, static_cast<const uint8_t*>(gbuf), h->W,
                   h->L, h->d,
-                  B, Bp, l0, l1, (const float*)h->xscale, lr, seed, step, dX, g_sample_major(h, Bp) ? 1 : 0,
-                  h->status);
+                  B, Bp, l0, l1, (const float*)h->xscale, lr, seed, step,
+                  (uint64_t)h->label_base * (uint64_t)h->d / 8, dX, g_sample_major(h, Bp) ? 1 : 0, h->status);
 }
 
 }  // namespace elmo
