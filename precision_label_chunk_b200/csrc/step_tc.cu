@@ -591,6 +591,7 @@ constexpr uint32_t kXtAcc = 384;           // first accumulator column
 
 struct SmemXt {
   uint64_t wfull[kXtStages], wempty[kXtStages], tfull[2], tempty[2];
+  uint64_t pmask[kXtEpi][32];   // per epilogue warp: its 32 samples' positives among the tile's labels
   uint32_t tmem_base;
   int abort;
 };
@@ -743,16 +744,27 @@ __global__ void __launch_bounds__(kXtThreads, 1)
       if (lane == 0) mbar_arrive(&S->tempty[buf]);
       // labels lc0 .. lc0 + ncol - 1 of this thread's row
       const int64_t lc0 = l0 + (int64_t)t * kXtN + c_lo;
-      // positives of sample b among them, from the keys of the 128-label tiles they touch
-      uint64_t pm = 0;
+      // positives of sample b among them, from the keys of the 128-label tiles
+      // they touch.  The warp reads the keys together (32 per pass, coalesced)
+      // and each key sets its bit in the mask of its sample, when that sample
+      // is one of the warp's: a tile of a frequent label holds hundreds of keys,
+      // which one thread per sample would each have to walk alone.
+      uint64_t pm;
       {
         const int k0 = __ldg(tile_ptr + (lc0 >> 7));
         const int k1 = __ldg(tile_ptr + min((lc0 + ncol - 1) >> 7, (L - 1) >> 7) + 1);
-        for (int i = k0; i < k1; ++i) {
+        unsigned long long* wm = reinterpret_cast<unsigned long long*>(S->pmask[warp - 2]);
+        wm[lane] = 0;
+        __syncwarp();
+        const int wb = b - lane;                              // the warp's first sample
+        for (int i = k0 + lane; i < k1; i += 32) {
           const uint32_t key = __ldg(keys + i);
+          const int sb = (int)(key & 0xFFu) - wb;
           const int64_t dl = (int64_t)(key >> 8) - lc0;
-          if ((int)(key & 0xFFu) == b && dl >= 0 && dl < ncol) pm |= 1ull << dl;
+          if (sb >= 0 && sb < 32 && dl >= 0 && dl < ncol) atomicOr(wm + sb, 1ull << dl);
         }
+        __syncwarp();
+        pm = wm[lane];
       }
       uint8_t* gtile = static_cast<uint8_t*>(gbuf) + (size_t)(t >> 1) * 128 * Bp * kEl;
       const int lt = (t & 1) * kXtN + c_lo;                   // first label column within the 128-label tile
