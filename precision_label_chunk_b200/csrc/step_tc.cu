@@ -591,6 +591,7 @@ constexpr uint32_t kXtAcc = 384;           // first accumulator column
 
 struct SmemXt {
   uint64_t wfull[kXtStages], wempty[kXtStages], tfull[2], tempty[2];
+  uint64_t xready;              // X is in TMEM (one arrival per epilogue warp)
   uint64_t pmask[kXtEpi][32];   // per epilogue warp: its 32 samples' positives among the tile's labels
   uint32_t tmem_base;
   int abort;
@@ -624,6 +625,7 @@ __global__ void __launch_bounds__(kXtThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kXtStages; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
     for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], nmb == 2 ? 4 : kXtEpi); }
+    mbar_init(&S->xready, kXtEpi);
     S->abort = 0;
     fence_barrier_init();
   }
@@ -656,10 +658,11 @@ __global__ void __launch_bounds__(kXtThreads, 1)
       }
       tmem_wait_st();
     }
+    // only the MMA warp needs X: the W stream starts while X is still filling
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S->xready);
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
 
   if (warp == 0) {
     if (elect_one()) {
@@ -679,6 +682,8 @@ __global__ void __launch_bounds__(kXtThreads, 1)
     if (elect_one()) {
       const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, kXtN) : make_idesc(1, 1, 0, 0, 128, kXtN);
       uint32_t it = 0, u = 0;
+      if (!mbar_wait(&S->xready, 0, abort, kWaitCycles)) record_timeout(status, abort, 75);
+      tc_fence_after();
       for (int t = t0; t < t1 && !*abort; ++t) {
         for (int mb = 0; mb < nmb && !*abort; ++mb, ++u) {
           const uint32_t slot = u & 1, ph = (u >> 1) & 1;
