@@ -31,7 +31,9 @@ _lib = None
 
 BF16 = 0
 FP8_E4M3 = 1
-_DT = {"bf16": BF16, "fp8": FP8_E4M3, BF16: BF16, FP8_E4M3: FP8_E4M3}
+FP8_E4M3_GE5M2 = 2      # E4M3 weights and X, E5M2 gradient operand
+_DT = {"bf16": BF16, "fp8": FP8_E4M3, "fp8_ge5m2": FP8_E4M3_GE5M2, BF16: BF16, FP8_E4M3: FP8_E4M3,
+       FP8_E4M3_GE5M2: FP8_E4M3_GE5M2}
 
 
 def build(force: bool = False) -> str:
@@ -67,6 +69,8 @@ def _declare(L):
     L.orc_rne_bf16_array.argtypes = [P, i64, P]
     L.orc_rne_e4m3_array.argtypes = [P, i64, P]
     L.orc_e4m3_value_array.argtypes = [P, i64, P]
+    L.orc_rne_e5m2_array.argtypes = [P, i64, P]
+    L.orc_e5m2_value_array.argtypes = [P, i64, P]
     L.orc_sr_round.argtypes = [P, P, i64, ctypes.c_int, u64, u64, u64]
     L.orc_fp8_x_scale.argtypes = [P, i64]
     L.orc_fp8_x_scale.restype = f32
@@ -157,6 +161,20 @@ def e4m3_value(codes) -> np.ndarray:
     c = _c(codes, np.uint8)
     o = np.zeros(c.shape, np.float32)
     lib().orc_e4m3_value_array(_p(c), c.size, _p(o))
+    return o
+
+
+def rne_e5m2(x) -> np.ndarray:
+    x = _c(x, np.float32)
+    o = np.zeros(x.shape, np.uint8)
+    lib().orc_rne_e5m2_array(_p(x), x.size, _p(o))
+    return o
+
+
+def e5m2_value(codes) -> np.ndarray:
+    c = _c(codes, np.uint8)
+    o = np.zeros(c.shape, np.float32)
+    lib().orc_e5m2_value_array(_p(c), c.size, _p(o))
     return o
 
 

@@ -52,6 +52,8 @@
 
 #define DT_BF16 0
 #define DT_E4M3 1
+#define DT_E4M3_GE5M2 2   /* E4M3 weights and X, E5M2 gradient operand */
+#define IS_FP8(dt) ((dt) == DT_E4M3 || (dt) == DT_E4M3_GE5M2)
 
 /* ------------------------------------------------------------------------ */
 /* Philox-4xW-10 (Salmon et al. 2011).  One round maps the counter words     */
@@ -160,6 +162,37 @@ uint16_t orc_rne_bf16(float v) {
   return (uint16_t)((sign >> 16) | pick);
 }
 
+/* OCP E5M2: 1 sign, 5 exponent bits (bias 15), 2 mantissa bits; exponent
+ * field 0 is subnormal (m * 2^-16); field 31 is infinity (m = 0) or NaN. */
+float orc_e5m2_value(uint8_t c) {
+  int s = c >> 7, e = (c >> 2) & 31, m = c & 3;
+  float mag;
+  if (e == 31) mag = m ? NAN : INFINITY;
+  else if (e == 0) mag = ldexpf((float)m, -16);
+  else mag = ldexpf(1.0f + (float)m / 4.0f, e - 15);
+  return s ? -mag : mag;
+}
+
+/* Round-to-nearest-even onto the finite E5M2 grid, saturating to +-57344
+ * (the largest finite value; infinities saturate too); NaN -> 0x7F. */
+uint8_t orc_rne_e5m2(float v) {
+  if (isnan(v)) return 0x7F;
+  uint8_t sign = signbit(v) ? 0x80 : 0;
+  double a = fabs((double)v);
+  if (a >= 57344.0) return sign | 0x7B;   /* codes 0x00 .. 0x7B are the finite magnitudes */
+  int lo = 0;
+  while (lo + 1 <= 0x7B && (double)orc_e5m2_value((uint8_t)(lo + 1)) <= a) lo++;
+  double vlo = (double)orc_e5m2_value((uint8_t)lo);
+  if (vlo == a) return sign | (uint8_t)lo;
+  double vhi = (double)orc_e5m2_value((uint8_t)(lo + 1));
+  double dlo = a - vlo, dhi = vhi - a;
+  int pick;
+  if (dlo < dhi) pick = lo;
+  else if (dhi < dlo) pick = lo + 1;
+  else pick = (lo & 1) ? lo + 1 : lo;      /* tie: even code */
+  return sign | (uint8_t)pick;
+}
+
 /* Round-to-nearest-even onto the E4M3 grid, saturating to +-448. */
 uint8_t orc_rne_e4m3(float v) {
   e4m3_table();
@@ -257,10 +290,10 @@ float orc_fp8_x_scale(const uint16_t* X, int64_t n) {
 static float* make_xv(const uint16_t* X, int32_t B, int32_t d, int dt, float* sx_out) {
   float* xv = (float*)malloc(sizeof(float) * (size_t)B * (size_t)d);
   float sx = 1.0f;
-  if (dt == DT_E4M3) sx = orc_fp8_x_scale(X, (int64_t)B * d);
+  if (IS_FP8(dt)) sx = orc_fp8_x_scale(X, (int64_t)B * d);
   for (int64_t i = 0; i < (int64_t)B * d; i++) {
     float x = orc_bf16_value(X[i]);
-    if (dt == DT_E4M3) xv[i] = orc_e4m3_value(orc_rne_e4m3(x * sx)) / sx;
+    if (IS_FP8(dt)) xv[i] = orc_e4m3_value(orc_rne_e4m3(x * sx)) / sx;
     else xv[i] = x;
   }
   if (sx_out) *sx_out = sx;
@@ -310,11 +343,13 @@ static float logit(const float* xq_row, const void* W, int dt, int64_t l, int32_
   return acc * inv_sx;
 }
 
-/* g = sigmoid(z) - y in fp32, then rounded to the operand grid. */
+/* g = sigmoid(z) - y in fp32, then rounded to the operand grid: bf16, or
+ * E4M3 / E5M2 of 2^8 g (the same fixed scale for both FP8 gradient grids). */
 static float grad_operand(float z, int y, int dt) {
   float s = (float)(1.0 / (1.0 + exp(-(double)z)));
   float g = s - (y ? 1.0f : 0.0f);
   if (dt == DT_BF16) return orc_bf16_value(orc_rne_bf16(g));
+  if (dt == DT_E4M3_GE5M2) return orc_e5m2_value(orc_rne_e5m2(g * 256.0f)) / 256.0f;
   return orc_e4m3_value(orc_rne_e4m3(g * 256.0f)) / 256.0f;
 }
 
@@ -339,7 +374,7 @@ int orc_train_step(const void* W, void* W_out, int64_t L, int32_t d, int dt,
                    float lr, uint64_t seed, uint64_t step, int64_t l0, int64_t l1,
                    float* dX, float* Z, float* G, int nthreads) {
   if (!W || !X || !rowptr || B < 0 || d <= 0 || L < 0 || l0 < 0 || l1 > L || l0 > l1) return ORC_EINVAL;
-  if (dt != DT_BF16 && dt != DT_E4M3) return ORC_EINVAL;
+  if (dt != DT_BF16 && !IS_FP8(dt)) return ORC_EINVAL;
   pos_t pos;
   int rc = make_pos(rowptr, cols, B, L, &pos);
   if (rc) return rc;
@@ -582,6 +617,12 @@ void orc_sr_e4m3_array(const float* v, const uint32_t* k, int64_t n, uint8_t* ou
 }
 void orc_rne_bf16_array(const float* v, int64_t n, uint16_t* out) {
   for (int64_t i = 0; i < n; i++) out[i] = orc_rne_bf16(v[i]);
+}
+void orc_rne_e5m2_array(const float* v, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; i++) out[i] = orc_rne_e5m2(v[i]);
+}
+void orc_e5m2_value_array(const uint8_t* c, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; i++) out[i] = orc_e5m2_value(c[i]);
 }
 void orc_rne_e4m3_array(const float* v, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; i++) out[i] = orc_rne_e4m3(v[i]);

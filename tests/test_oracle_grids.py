@@ -66,3 +66,32 @@ def test_fp8_x_scale_is_largest_fitting_power_of_two(orc):
     assert orc.fp8_x_scale(np.zeros(8, np.uint16)) == 1.0
     # a non-finite entry leaves X unscaled
     assert orc.fp8_x_scale(bf16_bits(np.array([1.0, np.inf], np.float32))) == 1.0
+
+
+def test_e5m2_decode_all_codes(orc):
+    codes = np.arange(256, dtype=np.uint8)
+    got = orc.e5m2_value(codes)
+    ref = codes.view(ml_dtypes.float8_e5m2).astype(np.float32)
+    ref_t = torch.from_numpy(codes.copy()).view(torch.float8_e5m2).float().numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.array_equal(got[ok], ref_t[ok])
+    assert np.nanmax(got[np.isfinite(got)]) == 57344.0 and np.nanmin(got[got > 0]) == 2.0 ** -16
+    assert got[0x7C] == np.inf and got[0xFC] == -np.inf
+
+
+def test_rne_e5m2_matches_ml_dtypes(orc):
+    rng = np.random.default_rng(1)
+    grid = orc.e5m2_value(np.arange(0x7C, dtype=np.uint8)).astype(np.float64)   # finite magnitudes
+    mids = ((grid[:-1] + grid[1:]) / 2).astype(np.float32)                      # exact ties
+    x = np.concatenate([_rand_f32(rng, 20000, -20, 16), mids, -mids, grid.astype(np.float32),
+                        np.array([0.0, -0.0, 57343.0, 57344.0, 2.0 ** -17, 2.0 ** -18], np.float32)])
+    x = x[np.abs(x) <= 57344]
+    got = orc.rne_e5m2(x)
+    ref = x.astype(ml_dtypes.float8_e5m2).view(np.uint8)
+    assert np.array_equal(got, ref)
+    # beyond the largest finite value the oracle saturates (satfinite); NaN -> 0x7F
+    assert np.all(orc.rne_e5m2(np.array([61440, 1e9, np.inf], np.float32)) == 0x7B)
+    assert np.all(orc.rne_e5m2(np.array([-61440, -np.inf], np.float32)) == 0xFB)
+    assert orc.rne_e5m2(np.array([np.nan], np.float32))[0] == 0x7F

@@ -25,6 +25,10 @@ def _rne_e4m3_val(x):
     return np.asarray(x, np.float32).astype(ml_dtypes.float8_e4m3fn).astype(np.float32)
 
 
+def _rne_e5m2_val(x):
+    return np.asarray(x, np.float32).astype(ml_dtypes.float8_e5m2).astype(np.float32)
+
+
 def _dyadic_case(rng, B, d, L, dtype):
     # X: integers in [-8, 8] / 8; W: integers in [-8, 8] / 64 (exact in both
     # grids); every sum below is exact in fp32.
@@ -36,7 +40,7 @@ def _dyadic_case(rng, B, d, L, dtype):
     return X, W, xv, wv, _csr(rows)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2"])
 def test_step_exact_dyadic_case(orc, dtype):
     rng = np.random.default_rng(10)
     B, d, L = 6, 16, 40
@@ -49,8 +53,10 @@ def test_step_exact_dyadic_case(orc, dtype):
     g = expit(Z64).astype(np.float32) - Y                   # fp32 sigmoid minus y
     if dtype == "bf16":
         Gh = _rne_bf16_val(g)
-    else:
+    elif dtype == "fp8":
         Gh = _rne_e4m3_val(g * np.float32(256)) / np.float32(256)
+    else:                                                   # E5M2 gradient operand, same 2^8 scale
+        Gh = _rne_e5m2_val(g * np.float32(256)) / np.float32(256)
     assert np.array_equal(r["G"], Gh.T)
     dw = Gh.T.astype(np.float64) @ xv.astype(np.float64)    # [L, d], exact
     v = (wv - (np.float32(lr) * dw.astype(np.float32))).astype(np.float32)
@@ -70,9 +76,9 @@ def _random_case(w_dtype, B=8, d=48, L=300, seed=0):
     return X, W, _csr(rows)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2"])
 def test_step_random_case_within_fp32_bounds(orc, dtype):
-    X, W, (rowptr, cols) = _random_case(dtype)
+    X, W, (rowptr, cols) = _random_case("bf16" if dtype == "bf16" else "fp8")
     L, d = W.shape
     B = X.shape[0]
     r = orc.train_step(W, X, rowptr, cols, 0.05, 1, 2, dtype, want_zg=True)
@@ -92,8 +98,10 @@ def test_step_random_case_within_fp32_bounds(orc, dtype):
     G = r["G"].T.astype(np.float64)
     if dtype == "bf16":
         assert np.all(np.abs(G - g64) <= 2.0 ** -8 * np.abs(g64) + 1e-6)
-    else:
+    elif dtype == "fp8":
         assert np.all(np.abs(G - g64) <= 2.0 ** -4 * np.abs(g64) + 2.0 ** -17 + 1e-6)
+    else:       # E5M2 of 2^8 g: half a spacing is 2^-3 relative, subnormal spacing 2^-16 / 2^8
+        assert np.all(np.abs(G - g64) <= 2.0 ** -3 * np.abs(g64) + 2.0 ** -25 + 1e-6)
     # dX = G W (old W), float64 brute force on the oracle's own operand values
     dX64 = G @ wv
     err_bound = L * 2.0 ** -24 * (np.abs(G) @ np.abs(wv)) + 1e-30
@@ -127,7 +135,7 @@ def test_gradient_matches_finite_difference_of_bce(orc):
     assert np.all(r["G"][Y == 1] < 0) and np.all(r["G"][Y == 0] > 0)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2"])
 def test_special_cases(orc, dtype):
     X, W, (rowptr, cols) = _random_case(dtype, seed=4)
     L, d = W.shape
@@ -146,7 +154,7 @@ def test_special_cases(orc, dtype):
     assert np.array_equal(r["G"], 0.5 - Y)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2"])
 def test_label_range_split_and_dx_rows(orc, dtype):
     X, W, (rowptr, cols) = _random_case(dtype, seed=5)
     L, d = W.shape
