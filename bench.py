@@ -117,7 +117,7 @@ def step_costs(w):
 
 def tensor_peak_tflops(peaks, dtype, sustained=True):
     base = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    return base * (2.0 if dtype == "fp8" else 1.0)   # fp8 dense = 2 x bf16 dense (nominal ratio)
+    return base * (1.0 if dtype == "bf16" else 2.0)   # fp8 dense = 2 x bf16 dense (nominal ratio)
 
 
 def alu_peak_tflops(peaks):
@@ -198,14 +198,14 @@ def run_reference(args, w):
     # sample size: about 5 s of oracle work per step
     probe = 64
     Wp = make_W_f32(w, rows=probe)
-    Wq = oracle.sr_round(Wp, "fp8", 0, 2**64 - 1) if w.dtype == "fp8" else make_W_bf16(w)[:probe]
+    Wq = oracle.sr_round(Wp, "fp8", 0, 2**64 - 1) if w.dtype != "bf16" else make_W_bf16(w)[:probe]
     t = time.perf_counter()
     oracle.train_step(Wq, X, rowptr, cols, w.lr, 0, 0, w.dtype, 0, probe, L=w.L, nthreads=nthreads)
     per = (time.perf_counter() - t) / probe
     budget = max(30.0, 150.0 / max(1, args.steps + args.warmup))
     n = int(max(probe, min(w.L, budget / 3 / max(per, 1e-9))))
     Wf = make_W_f32(w, rows=n)
-    Wq = oracle.sr_round(Wf, "fp8", 0, 2**64 - 1) if w.dtype == "fp8" else oracle.rne_bf16(Wf)
+    Wq = oracle.sr_round(Wf, "fp8", 0, 2**64 - 1) if w.dtype != "bf16" else oracle.rne_bf16(Wf)
     for s in range(args.warmup):
         oracle.train_step(Wq, make_X(w, s), *make_labels(w, s), w.lr, 0, s, w.dtype, 0, n, L=w.L, nthreads=nthreads)
     t = time.perf_counter()
@@ -301,12 +301,12 @@ def run_topk(args, w, rank, world, local):
             # peak of the operand type (E4M3 heads issue the contraction twice, for
             # the two E4M3 parts of the bf16 queries, so their ceiling is frac = 0.5)
             peak, bound = tensor_peak_tflops(peaks, w.dtype), "tensor"
-            src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype == "fp8" else ""))
+            src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype != "bf16" else ""))
         tr = profiled_traffic("topk_screen_tc", w.name) if bound == "tensor" else None
         roof = {"kernel": dominant, "bound": bound, "achieved": flops / t_k / 1e12, "peak": peak, "unit": "TFLOP/s",
                 "frac": flops / t_k / 1e12 / peak,
                 "traffic": None if tr is None else tr["bytes"] * w.L / tr["labels"], "peak_source": src,
-                "mma_passes": 2 if (w.dtype == "fp8" and bound == "tensor") else 1}
+                "mma_passes": 2 if (w.dtype != "bf16" and bound == "tensor") else 1}
     # end to end: X from pinned host memory, indices and scores back every step
     pin = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in Xh]
     idx_h = torch.empty(w.B, w.topk, dtype=torch.int32).pin_memory()
@@ -336,7 +336,7 @@ def run_topk(args, w, rank, world, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        Wh = W.cpu().numpy().view(np.uint8 if w.dtype == "fp8" else np.uint16)
+        Wh = W.cpu().numpy().view(np.uint8 if w.dtype != "bf16" else np.uint16)
         nthreads = os.cpu_count() or 1
         t = time.perf_counter()
         oracle.topk(Wh, Xh[0], w.topk, w.dtype, rows=[0], nthreads=nthreads)
@@ -620,7 +620,7 @@ def main():
             peak, bound, src = alu_peak_tflops(peaks), "alu", "derived: 148 SM x 128 FMA x 2 x max clock"
         else:
             peak, bound = tensor_peak_tflops(peaks, w.dtype), "tensor"
-            src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype == "fp8" else ""))
+            src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype != "bf16" else ""))
         # ncu DRAM bytes of one full launch, scaled to the mean launch of this
         # run by the labels it covers (the kernel's traffic is linear in them)
         tr = profiled_traffic({"update": "update_tc", "logits_grad": "logits_grad_xt"}.get(dominant, dominant),
@@ -677,7 +677,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "label-rows/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "fp8-e4m3" if w.dtype == "fp8" else "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": {"bf16": "bf16", "fp8": "fp8-e4m3", "fp8_ge5m2": "fp8-e4m3 (e5m2 gradient operand)"}[w.dtype], "data": "synthetic",
             "config": {"workload": w.name, "L": w.L, "d": w.d, "B": w.B, "w_dtype": w.dtype, "chunk": w.chunk,
                        "lr": w.lr, "positives_per_sample": f"1+Poisson({w.lam})", "zipf_s": w.zipf_s,
                        "l2": f"inputs larger than L2 (W = {costs['w_bytes'] / 2 / 1e9:.2f} GB per GPU)",

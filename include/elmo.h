@@ -38,8 +38,10 @@ extern "C" {
 #endif
 
 typedef enum {
-  ELMO_BF16 = 0,      /* bfloat16 weights (8-bit exponent, 7-bit mantissa) */
-  ELMO_FP8_E4M3 = 1   /* OCP E4M3FN weights: max 448, no infinities, saturating */
+  ELMO_BF16 = 0,           /* bfloat16 weights (8-bit exponent, 7-bit mantissa) */
+  ELMO_FP8_E4M3 = 1,       /* OCP E4M3FN weights: max 448, no infinities, saturating */
+  ELMO_FP8_E4M3_GE5M2 = 2  /* E4M3 weights (and X) as above; the training step's gradient
+                              operand is OCP E5M2 of 2^8 G instead of E4M3 (heads only) */
 } elmo_dtype;
 
 typedef enum {

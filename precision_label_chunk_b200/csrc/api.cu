@@ -189,7 +189,10 @@ elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_
   g_last_error.clear();
   if (!out || !W_dev) return fail(ELMO_EINVAL, "null out or W");
   *out = nullptr;
-  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3) return fail(ELMO_EINVAL, "unknown dtype %d", (int)dt);
+  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3 && dt != ELMO_FP8_E4M3_GE5M2)
+    return fail(ELMO_EINVAL, "unknown dtype %d", (int)dt);
+  const bool g_e5m2 = dt == ELMO_FP8_E4M3_GE5M2;
+  if (g_e5m2) dt = ELMO_FP8_E4M3;                    // the weights are E4M3
   if (L < 1 || L >= ELMO_MAX_LABELS) return fail(ELMO_EINVAL, "L = %lld outside [1, 2^24)", (long long)L);
   if (label_base < 0 || labels_total > ELMO_MAX_TOTAL_LABELS || label_base > labels_total - L)
     return fail(ELMO_EINVAL, "label rows [%lld, %lld) outside a head of %lld labels (at most %lld)",
@@ -209,6 +212,7 @@ elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_
   h->L = L;
   h->label_base = label_base;
   h->labels_total = labels_total;
+  h->g_e5m2 = g_e5m2;
   h->d = d;
   h->dt = dt;
   h->device = dev;
@@ -325,6 +329,8 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B, const
   const size_t esz = fp8 ? 1 : 2;
   const int32_t Bp = elmo::padded_batch(B, fp8);
   const bool simt = use_simt();
+  if (simt && h->g_e5m2)
+    return fail(ELMO_EUNSUPPORTED, "the CUDA-core development path has no E5M2 gradient operand");
   const int64_t sub = simt ? elmo::kSubChunk : elmo::sub_chunk_labels(h->d, Bp, (int)esz);
   const int64_t span = l1 - l0 < sub ? l1 - l0 : sub;
   if ((st = ensure_gbuf(h, (size_t)((span + 127) / 128 * 128) * Bp * esz)) != ELMO_OK) return st;  // whole tiles
@@ -361,6 +367,8 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
   const size_t esz = fp8 ? 1 : 2;
   const int32_t Bp = elmo::padded_batch(B, fp8);
   const bool simt = use_simt();
+  if (simt && h->g_e5m2)
+    return fail(ELMO_EUNSUPPORTED, "the CUDA-core development path has no E5M2 gradient operand");
   const int64_t sub_max = simt ? elmo::kSubChunk : elmo::sub_chunk_labels(h->d, Bp, (int)esz);
   const int64_t sub = chunk < sub_max ? chunk : sub_max;
   const int64_t span = h->L < sub ? h->L : sub;

@@ -129,6 +129,21 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float hi, float lo) {
   return r;
 }
 
+// Two fp32 values -> two E5M2 codes (hi in the upper byte), RNE + saturating.
+__device__ __forceinline__ uint32_t pack_e5m2x2(float hi, float lo) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// E5M2 code -> value: an E5M2 code is the upper byte of the binary16 value.
+__device__ __forceinline__ float e5m2_to_f32(uint8_t c) {
+  float f;
+  const uint16_t h = (uint16_t)((uint16_t)c << 8);
+  asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
+  return f;
+}
+
 // Two fp32 values -> two bf16 (hi in the upper half), RNE.
 __device__ __forceinline__ uint32_t pack_bf16x2(float hi, float lo) {
   uint32_t r;

@@ -22,7 +22,8 @@ struct elmo_head {
   int64_t label_base = 0;      // W holds the label rows [label_base, label_base + L) ...
   int64_t labels_total = 0;    // ... of a head of labels_total labels (0 and L when unsharded)
   int32_t d = 0;
-  elmo_dtype dt = ELMO_BF16;
+  elmo_dtype dt = ELMO_BF16;    // format of W (and of X and G in the tensor cores): BF16 or E4M3
+  bool g_e5m2 = false;         // E4M3 step whose gradient operand G is E5M2 (ELMO_FP8_E4M3_GE5M2)
   int device = 0;
   int num_sms = 0;
   // workspace owned by the head

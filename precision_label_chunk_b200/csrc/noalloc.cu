@@ -56,7 +56,10 @@ extern "C" elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d
   // ---- arguments (the same limits as the head-based step; the scratch is sized for them)
   if (!W_dev || !X_dev || !rowptr_dev || !dX_dev || !status_dev) return fail(ELMO_EINVAL, "null pointer argument");
   if (nnz > 0 && !cols_dev) return fail(ELMO_EINVAL, "null cols with nnz > 0");
-  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3) return fail(ELMO_EINVAL, "unknown dtype %d", (int)dt);
+  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3 && dt != ELMO_FP8_E4M3_GE5M2)
+    return fail(ELMO_EINVAL, "unknown dtype %d", (int)dt);
+  const bool g_e5m2 = dt == ELMO_FP8_E4M3_GE5M2;
+  if (g_e5m2) dt = ELMO_FP8_E4M3;                    // the weights are E4M3
   if (L < 1 || L >= ELMO_MAX_LABELS)
     return fail(ELMO_EUNSUPPORTED, "L = %lld: the no-allocation step supports 1 <= L < 2^24", (long long)L);
   if (d < 64 || d > 4096 || d % 64 != 0)
@@ -101,6 +104,7 @@ extern "C" elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d
   h.labels_total = L;
   h.d = d;
   h.dt = dt;
+  h.g_e5m2 = g_e5m2;
   h.device = dev;
   h.num_sms = nsm;
   h.status = status_dev;

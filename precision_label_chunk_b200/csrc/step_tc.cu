@@ -110,7 +110,7 @@ __device__ __forceinline__ float tanhf_approx(float x) {
 //         wherever 2^8 |G| >= 1; only the codes of negatives with
 //         sigmoid(z) < 2^-8 (z < -5.5) can move by more than one step.
 // `zmul` is -log2(e) / s_X (bf16) or 1 / (2 s_X) (E4M3).
-template <int kFp8>
+template <int kFp8, int kG5 = 0>
 __device__ __forceinline__ void grad16(const uint32_t* r, float zmul, float inv_sx, uint32_t ybits,
                                        int b0, int B, uint8_t* __restrict__ gtile, int row, bool row_invalid,
                                        float* __restrict__ Zrow, float* __restrict__ Grow) {
@@ -139,7 +139,8 @@ __device__ __forceinline__ void grad16(const uint32_t* r, float zmul, float inv_
   if (kFp8) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      packed[i] = pack_e4m3x2(g[4 * i + 1], g[4 * i]) | (pack_e4m3x2(g[4 * i + 3], g[4 * i + 2]) << 16);
+      packed[i] = kG5 ? pack_e5m2x2(g[4 * i + 1], g[4 * i]) | (pack_e5m2x2(g[4 * i + 3], g[4 * i + 2]) << 16)
+                      : pack_e4m3x2(g[4 * i + 1], g[4 * i]) | (pack_e4m3x2(g[4 * i + 3], g[4 * i + 2]) << 16);
     const int j = b0 >> 4;                                   // 16-byte chunk of samples
     *reinterpret_cast<uint4*>(gtile + ((j * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
         make_uint4(packed[0], packed[1], packed[2], packed[3]);
@@ -156,7 +157,8 @@ __device__ __forceinline__ void grad16(const uint32_t* r, float zmul, float inv_
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       if (b0 + i < B)
-        Grow[i] = kFp8 ? e4m3_to_f32((uint8_t)(packed[i >> 2] >> (8 * (i & 3)))) * 0.00390625f
+        Grow[i] = kFp8 ? (kG5 ? e5m2_to_f32((uint8_t)(packed[i >> 2] >> (8 * (i & 3))))
+                              : e4m3_to_f32((uint8_t)(packed[i >> 2] >> (8 * (i & 3))))) * 0.00390625f
                        : bf16_to_f32((uint16_t)(packed[i >> 1] >> (16 * (i & 1))));
   }
   if (Zrow && !row_invalid) {
@@ -289,7 +291,7 @@ struct SmemA {
   int abort;
 };
 
-template <int kFp8>
+template <int kFp8, int kG5 = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     logits_grad_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int64_t L,
                    int32_t d, int32_t B, int32_t Bp, int64_t l0, int64_t l1, const uint32_t* __restrict__ keys,
@@ -395,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int b0 = c * 32 + k * 16;
-          grad16<kFp8>(ra + k * 16, zmul, inv_sx, mask16(mask, b0), b0, B,
+          grad16<kFp8, kG5>(ra + k * 16, zmul, inv_sx, mask16(mask, b0), b0, B,
                        static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                        Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
         }
@@ -425,7 +427,7 @@ struct SmemP {
   int abort;
 };
 
-template <int kFp8>
+template <int kFp8, int kG5 = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     logits_grad_panel_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                          int64_t L, int32_t d, int32_t B, int32_t Bp, int32_t PN, int32_t nstages, int64_t l0,
@@ -554,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 2; ++k) {
             const int cb = c * 32 + k * 16;             // panel column
             const int b0 = p * PN + cb;                 // sample
-            grad16<kFp8>(ra + k * 16, zmul, inv_sx, mask16(mask, b0), b0, B,
+            grad16<kFp8, kG5>(ra + k * 16, zmul, inv_sx, mask16(mask, b0), b0, B,
                          static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                          Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
           }
@@ -597,7 +599,7 @@ struct SmemXt {
   int abort;
 };
 
-template <int kFp8>
+template <int kFp8, int kG5 = 0>
 __global__ void __launch_bounds__(kXtThreads, 1)
     logits_grad_xt(const __grid_constant__ CUtensorMap tmW, int64_t L, int32_t d, int32_t B, int32_t Bp, int64_t l0,
                    int64_t l1, const uint8_t* __restrict__ xop, const uint32_t* __restrict__ keys,
@@ -792,7 +794,9 @@ __global__ void __launch_bounds__(kXtThreads, 1)
         uint32_t pk[8];
         if (kFp8) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) pk[i] = pack_e4m3x2(g[4 * i + 1], g[4 * i]) | (pack_e4m3x2(g[4 * i + 3], g[4 * i + 2]) << 16);
+          for (int i = 0; i < 4; ++i)
+            pk[i] = kG5 ? pack_e5m2x2(g[4 * i + 1], g[4 * i]) | (pack_e5m2x2(g[4 * i + 3], g[4 * i + 2]) << 16)
+                        : pack_e4m3x2(g[4 * i + 1], g[4 * i]) | (pack_e4m3x2(g[4 * i + 3], g[4 * i + 2]) << 16);
           if (bstore) {
             const int lc = (lt + j) / kChunk;
             *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =
@@ -817,7 +821,8 @@ __global__ void __launch_bounds__(kXtThreads, 1)
             const size_t o = (size_t)(l - l0) * B + b;
             if (Zout) Zout[o] = __fmul_rn(__uint_as_float(v[j + i]), inv_sx);
             if (Gout)
-              Gout[o] = kFp8 ? e4m3_to_f32((uint8_t)(pk[i >> 2] >> (8 * (i & 3)))) * 0.00390625f
+              Gout[o] = kFp8 ? (kG5 ? e5m2_to_f32((uint8_t)(pk[i >> 2] >> (8 * (i & 3))))
+                                    : e4m3_to_f32((uint8_t)(pk[i >> 2] >> (8 * (i & 3))))) * 0.00390625f
                              : bf16_to_f32((uint16_t)(pk[i >> 1] >> (16 * (i & 1))));
           }
         }
@@ -856,7 +861,8 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
     update_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
               const uint8_t* __restrict__ gbuf, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
               int32_t Bp, int64_t l0, int64_t l1, const float* __restrict__ xscale, float lr, uint64_t seed,
-              uint64_t step, uint64_t blk_base, float* __restrict__ dX, int gsm, int32_t* __restrict__ status) {
+              uint64_t step, uint64_t blk_base, float* __restrict__ dX, int gsm, uint32_t gfmt,
+              int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // E4M3 operands take half the bytes, which leaves room for 4 W slots: the
@@ -960,7 +966,8 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
       // G stored label-major (kernel A with resident X) or sample-major (X in TMEM):
       // the same core matrices then serve as K- or MN-major operands
       const uint32_t gmn = gsm ? 1u : 0u;
-      const uint32_t idesc_dw = kFp8 ? make_idesc(0, 0, gmn, 1, 128, 128) : make_idesc(1, 1, gmn, 1, 128, 128);
+      // E4M3 steps: G is E4M3 (gfmt 0) or E5M2 (gfmt 1); W and X are E4M3
+      const uint32_t idesc_dw = kFp8 ? make_idesc(gfmt, 0, gmn, 1, 128, 128) : make_idesc(1, 1, gmn, 1, 128, 128);
       const uint32_t gstride = (uint32_t)(kFp8 ? 8 : 16) * 128u;   // sample-major: bytes between sample groups
       int run = 0;
       uint32_t wit = 0, git = 0, dwit = 0;
@@ -991,7 +998,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
             const uint32_t ga = smem_u32(gs + sg * kGSlotBytes);
             const int np = min(kPart, Bp - p * kPart);   // samples in this part (multiple of 32)
             // dX^T[slice, part] += W^T G^T : M = 128 (columns of d), N = np, K = 128 labels
-            const uint32_t idesc_dx = kFp8 ? make_idesc(0, 0, 1, gmn ^ 1u, 128, (uint32_t)np)
+            const uint32_t idesc_dx = kFp8 ? make_idesc(0, gfmt, 1, gmn ^ 1u, 128, (uint32_t)np)
                                            : make_idesc(1, 1, 1, gmn ^ 1u, 128, (uint32_t)np);
             const uint32_t dxcol = tmem + (uint32_t)(p * kPart);
 #pragma unroll 1
@@ -1197,7 +1204,7 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
     if (e != cudaSuccess) return e;
     const int T = 2 * (int)((l1 - l0 + 127) / 128);
     const int grid = T < h->num_sms ? T : h->num_sms;
-    auto kx = fp8 ? logits_grad_xt<1> : logits_grad_xt<0>;
+    auto kx = fp8 ? (h->g_e5m2 ? logits_grad_xt<1, 1> : logits_grad_xt<1>) : logits_grad_xt<0>;
     e = cudaFuncSetAttribute(kx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemXt);
     if (e != cudaSuccess) return e;
     const uint8_t* xop = fp8 ? h->xq : reinterpret_cast<const uint8_t*>(X);
@@ -1230,14 +1237,14 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
     e = make_tma_map_2d(&tmXp, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
                  (uint64_t)B, (uint64_t)h->d, (uint32_t)PN);
     if (e != cudaSuccess) return e;
-    auto kp = fp8 ? logits_grad_panel_tc<1> : logits_grad_panel_tc<0>;
+    auto kp = fp8 ? (h->g_e5m2 ? logits_grad_panel_tc<1, 1> : logits_grad_panel_tc<1>) : logits_grad_panel_tc<0>;
     e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemP);
     if (e != cudaSuccess) return e;
     return launch_k(kp, grid, kThreads, kSmemP, s, pdl, tmW, tmXp, h->L, h->d, B, Bp, PN, nst, l0, l1,
                     (const uint32_t*)h->keys, (const int32_t*)h->tile_ptr, (const float*)h->xscale, gbuf, Zout, Gout,
                     h->status);
   }
-  auto kern = fp8 ? logits_grad_tc<1> : logits_grad_tc<0>;
+  auto kern = fp8 ? (h->g_e5m2 ? logits_grad_tc<1, 1> : logits_grad_tc<1>) : logits_grad_tc<0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemA);
   if (e != cudaSuccess) return e;
   return launch_k(kern, grid, kThreads, kSmemA, s, pdl, tmW, tmX, h->L, h->d, B, Bp, l0, l1, (const uint32_t*)h->keys,
@@ -1266,7 +1273,8 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
   return launch_k(kern, grid, fp8 ? kThreads : 320, kSmemB, s, pdl, tmW, tmX, static_cast<const uint8_t*>(gbuf), h->W,
                   h->L, h->d,
                   B, Bp, l0, l1, (const float*)h->xscale, lr, seed, step,
-                  (uint64_t)h->label_base * (uint64_t)h->d / 8, dX, g_sample_major(h, Bp) ? 1 : 0, h->status);
+                  (uint64_t)h->label_base * (uint64_t)h->d / 8, dX, g_sample_major(h, Bp) ? 1 : 0,
+                  h->g_e5m2 ? 1u : 0u, h->status);
 }
 
 }  // namespace elmo

@@ -40,7 +40,7 @@ class Workload:
     B: int                # samples per step
     d: int                # embedding width
     L: int                # number of labels
-    dtype: str            # "bf16" or "fp8" (storage type of W)
+    dtype: str            # "bf16" or "fp8" (storage type of W); "fp8_ge5m2": E4M3 W, E5M2 gradient operand
     lam: float            # positives per sample: 1 + Poisson(lam)
     zipf_s: float         # Zipf exponent of the label law
     lr: float
@@ -62,6 +62,9 @@ WORKLOADS = {
                  zipf_s=1.2, lr=0.05, chunk=262_144, steps=10),
         Workload("topk5_3m_fp8", 4, B=1024, d=768, L=3_000_000, dtype="fp8", lam=0,
                  zipf_s=1.0, lr=0.0, chunk=131_072, steps=1, topk=5),
+        # the 3M-label head with an E5M2 gradient operand (same inputs as product3m_fp8)
+        Workload("product3m_fp8_ge5m2", 2, B=256, d=768, L=3_000_000, dtype="fp8_ge5m2", lam=35,
+                 zipf_s=1.0, lr=0.1, chunk=131_072, steps=20),
     ]
 }
 
