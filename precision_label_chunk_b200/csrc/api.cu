@@ -219,7 +219,7 @@ elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_
   h->num_sms = nsm;
   const size_t xq_bytes = (size_t)ELMO_MAX_BATCH * d;
   const size_t tp_bytes = (sizeof(int32_t) * (size_t)((L + 127) / 128 + 1) + 255) / 256 * 256;
-  const size_t bytes = 64 + sizeof(uint32_t) * ELMO_MAX_NNZ + 64 + xq_bytes + tp_bytes;
+  const size_t bytes = 64 + sizeof(uint32_t) * ELMO_MAX_NNZ + 64 + 2 * xq_bytes + tp_bytes;
   char* base = nullptr;
   if (cudaMalloc(&base, bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -232,6 +232,7 @@ elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_
   h->keys = reinterpret_cast<uint32_t*>(base + 64);
   h->xq = reinterpret_cast<uint8_t*>(base + 64 + sizeof(uint32_t) * ELMO_MAX_NNZ + 64);
   h->tile_ptr = reinterpret_cast<int32_t*>(base + 64 + sizeof(uint32_t) * ELMO_MAX_NNZ + 64 + xq_bytes);
+  h->xqt = reinterpret_cast<uint8_t*>(base + 64 + sizeof(uint32_t) * ELMO_MAX_NNZ + 64 + xq_bytes + tp_bytes);
   h->base_bytes = bytes;
   cudaStream_t s = as_stream(stream);
   cudaError_t e = cudaMemsetAsync(base, 0, 64, s);

@@ -35,6 +35,7 @@ struct elmo_head {
   cudaEvent_t fork = nullptr, join = nullptr;
   float* xscale = nullptr;     // [2] s_X, 1/s_X (fp8 mode)
   uint8_t* xq = nullptr;       // [ELMO_MAX_BATCH x d] E4M3 codes of X * s_X (fp8 mode)
+  uint8_t* xqt = nullptr;      // the same codes by 16-byte column chunk: [d/16][ELMO_MAX_BATCH][16]
   void* gbuf = nullptr;        // per-chunk gradient operands
   size_t gbuf_bytes = 0;
   void* cand = nullptr;        // top-k candidates

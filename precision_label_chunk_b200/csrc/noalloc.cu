@@ -26,7 +26,7 @@ constexpr size_t kSmallBytes = 256;                                             
 constexpr size_t kXqBytes = (size_t)ELMO_MAX_BATCH * 4096;                             // E4M3 X
 constexpr size_t kTilePtrBytes = (sizeof(int32_t) * ((ELMO_MAX_LABELS / 128) + 1) + 255) / 256 * 256;
 constexpr size_t kGBytes = 8u << 20;                                                   // gradient operands
-constexpr size_t kScratchBytes = kKeysBytes + kSmallBytes + kXqBytes + kTilePtrBytes + kGBytes;
+constexpr size_t kScratchBytes = kKeysBytes + kSmallBytes + 2 * kXqBytes + kTilePtrBytes + kGBytes;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -113,7 +113,8 @@ extern "C" elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d
   h.xscale = reinterpret_cast<float*>(s + kKeysBytes + 16);
   h.xq = reinterpret_cast<uint8_t*>(s + kKeysBytes + kSmallBytes);
   h.tile_ptr = reinterpret_cast<int32_t*>(s + kKeysBytes + kSmallBytes + kXqBytes);
-  void* gbuf = s + kKeysBytes + kSmallBytes + kXqBytes + kTilePtrBytes;
+  h.xqt = reinterpret_cast<uint8_t*>(s + kKeysBytes + kSmallBytes + kXqBytes + kTilePtrBytes);
+  void* gbuf = s + kKeysBytes + kSmallBytes + 2 * kXqBytes + kTilePtrBytes;
 
   const bool fp8 = dt == ELMO_FP8_E4M3;
   const size_t esz = fp8 ? 1 : 2;

@@ -125,9 +125,14 @@ __device__ __forceinline__ void prep_labels_body(const int32_t* __restrict__ row
 }
 
 // One CTA: max |X| with 16-byte loads, the power-of-two scale, then the E4M3
-// codes of X * s_X (second pass mostly from L1/L2).  n is a multiple of 64.
-__device__ __forceinline__ void prep_x_body(const uint16_t* __restrict__ X, int64_t n, float* __restrict__ xscale,
-                                            uint8_t* __restrict__ xq) {
+// codes of X * s_X (second pass mostly from L1/L2).  n = B d, d a multiple
+// of 64.  The codes go out twice: row-major (xq, [B x d]) and by 16-byte
+// column chunk (xqt: chunk c of row b at byte (c * ELMO_MAX_BATCH + b) * 16),
+// the layout in which a warp reads one chunk of 32 consecutive rows with
+// 512 contiguous bytes when it copies X into tensor memory.
+__device__ __forceinline__ void prep_x_body(const uint16_t* __restrict__ X, int64_t n, int32_t d,
+                                            float* __restrict__ xscale, uint8_t* __restrict__ xq,
+                                            uint8_t* __restrict__ xqt) {
   __shared__ float red[kPrepThreads / 32];
   __shared__ int nonfinite;
   __shared__ float s_scale;
@@ -180,6 +185,8 @@ __device__ __forceinline__ void prep_x_body(const uint16_t* __restrict__ X, int6
       q[h] = pack_e4m3x2(x1, x0) | (pack_e4m3x2(x3, x2) << 16);
     }
     Q2[i] = make_uint2(q[0], q[1]);
+    const int64_t b = (8 * i) / d, j = (8 * i) % d;           // 8 codes of row b from column j
+    *reinterpret_cast<uint2*>(xqt + ((j >> 4) * ELMO_MAX_BATCH + b) * 16 + (j & 15)) = make_uint2(q[0], q[1]);
   }
 }
 
@@ -194,10 +201,10 @@ __global__ void __launch_bounds__(kPrepThreads) prep_labels_kernel(const int32_t
   prep_labels_body(rowptr, cols, B, nnz, L, label_base, labels_total, keys_out, nkeys, tile_ptr, status);
 }
 
-__global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __restrict__ X, int64_t n,
+__global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __restrict__ X, int64_t n, int32_t d,
                                                               float* __restrict__ xscale,
-                                                              uint8_t* __restrict__ xq) {
-  prep_x_body(X, n, xscale, xq);
+                                                              uint8_t* __restrict__ xq, uint8_t* __restrict__ xqt) {
+  prep_x_body(X, n, d, xscale, xq, xqt);
 }
 
 // Both preparations of an E4M3 step in one launch: CTA 0 the labels, CTA 1 X.
@@ -210,11 +217,11 @@ __global__ void __launch_bounds__(kPrepThreads) prep_step_kernel(const int32_t* 
                                                                  int32_t* __restrict__ tile_ptr,
                                                                  int32_t* __restrict__ status,
                                                                  const uint16_t* __restrict__ X, int64_t n,
-                                                                 float* __restrict__ xscale,
-                                                                 uint8_t* __restrict__ xq) {
+                                                                 int32_t d, float* __restrict__ xscale,
+                                                                 uint8_t* __restrict__ xq, uint8_t* __restrict__ xqt) {
   if (blockIdx.x == 0)
     prep_labels_body(rowptr, cols, B, nnz, L, label_base, labels_total, keys_out, nkeys, tile_ptr, status);
-  else prep_x_body(X, n, xscale, xq);
+  else prep_x_body(X, n, d, xscale, xq, xqt);
 }
 
 }  // namespace
@@ -228,7 +235,7 @@ cudaError_t launch_prep_step(elmo_head* h, const int32_t* rowptr, const int32_t*
   if (e != cudaSuccess) return e;
   prep_step_kernel<<<2, kPrepThreads, smem, s>>>(rowptr, cols, B, nnz, h->L, h->label_base, h->labels_total,
                                                  h->keys, h->nkeys, h->tile_ptr, h->status, X,
-                                                 (int64_t)B * h->d, h->xscale, h->xq);
+                                                 (int64_t)B * h->d, h->d, h->xscale, h->xq, h->xqt);
   return cudaGetLastError();
 }
 
@@ -244,7 +251,7 @@ cudaError_t launch_prep_labels(elmo_head* h, const int32_t* rowptr, const int32_
 }
 
 cudaError_t launch_prep_x(elmo_head* h, const uint16_t* X, int32_t B, cudaStream_t s) {
-  prep_x_kernel<<<1, kPrepThreads, 0, s>>>(X, (int64_t)B * h->d, h->xscale, h->xq);
+  prep_x_kernel<<<1, kPrepThreads, 0, s>>>(X, (int64_t)B * h->d, h->d, h->xscale, h->xq, h->xqt);
   return cudaGetLastError();
 }
 

@@ -644,14 +644,18 @@ __global__ void __launch_bounds__(kXtThreads, 1)
     if (h < nmb) {
       const int b = h * 128 + q * 32 + lane;
       const size_t rowbytes = (size_t)d * (kFp8 ? 1 : 2);
-      const uint8_t* src = xop + (size_t)b * rowbytes;
+      // E4M3: xop holds the codes by 16-byte column chunk (chunk c of row b at
+      // (c * 256 + b) * 16), so a warp's load of one chunk covers 512
+      // contiguous bytes; bf16: xop is X itself, row-major
+      const uint8_t* src = kFp8 ? xop + (size_t)b * 16 : xop + (size_t)b * rowbytes;
       for (uint32_t c0 = 0; c0 < opcols; c0 += 64) {   // 64 columns (16 loads in flight) per round
         uint32_t v[2][32];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const size_t off = (size_t)(c0 + 4 * u) * 4;
           uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
-          if (b < B && off < rowbytes) w4 = *reinterpret_cast<const uint4*>(src + off);
+          if (b < B && off < rowbytes)
+            w4 = *reinterpret_cast<const uint4*>(kFp8 ? src + (off >> 4) * (ELMO_MAX_BATCH * 16) : src + off);
           v[u >> 3][4 * (u & 7)] = w4.x; v[u >> 3][4 * (u & 7) + 1] = w4.y;
           v[u >> 3][4 * (u & 7) + 2] = w4.z; v[u >> 3][4 * (u & 7) + 3] = w4.w;
         }
@@ -1207,7 +1211,7 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
     auto kx = fp8 ? (h->g_e5m2 ? logits_grad_xt<1, 1> : logits_grad_xt<1>) : logits_grad_xt<0>;
     e = cudaFuncSetAttribute(kx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemXt);
     if (e != cudaSuccess) return e;
-    const uint8_t* xop = fp8 ? h->xq : reinterpret_cast<const uint8_t*>(X);
+    const uint8_t* xop = fp8 ? h->xqt : reinterpret_cast<const uint8_t*>(X);
     return launch_k(kx, grid, kXtThreads, kSmemXt, s, pdl, tmW64, h->L, h->d, B, Bp, l0, l1, xop,
                     (const uint32_t*)h->keys, (const int32_t*)h->tile_ptr, (const float*)h->xscale, gbuf, Zout, Gout,
                     h->status);
