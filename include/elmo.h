@@ -316,7 +316,7 @@ elmo_status elmo_launch_count(const elmo_head* h, int64_t* launches);
  * This call takes W directly and allocates nothing.  Its scratch (the
  * positives grouped by label tile, the tile index, quantised X and the
  * per-range gradient operands)
- * is one static device array of 10 MiB (ELMO_NOALLOC_SCRATCH_BYTES) that every
+ * is one static device array of 11 MiB (ELMO_NOALLOC_SCRATCH_BYTES) that every
  * GPU loading the library holds until the process exits.  It supports the
  * same sizes as the head-based step -- 1 <= L < 2^24, d a multiple of 64 up to
  * 4096, 1 <= B <= 256, 0 <= nnz <= 32768 -- and rejects anything beyond them
@@ -339,7 +339,7 @@ elmo_status elmo_launch_count(const elmo_head* h, int64_t* launches);
  * Errors: ELMO_EINVAL / ELMO_EUNSUPPORTED synchronously (message in
  * elmo_last_error()), ELMO_ECUDA if a launch fails.
  */
-#define ELMO_NOALLOC_SCRATCH_BYTES (10u << 20)
+#define ELMO_NOALLOC_SCRATCH_BYTES (11u << 20)
 elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d, elmo_dtype dt, const void* X_dev,
                                     int32_t B, const int32_t* rowptr_dev, const int32_t* cols_dev, int32_t nnz,
                                     float lr, int64_t chunk, uint64_t seed, uint64_t step, float* dX_dev,

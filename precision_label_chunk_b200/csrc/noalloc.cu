@@ -27,8 +27,9 @@ constexpr size_t kXqBytes = (size_t)ELMO_MAX_BATCH * 4096;                      
 constexpr size_t kTilePtrBytes = (sizeof(int32_t) * ((ELMO_MAX_LABELS / 128) + 1) + 255) / 256 * 256;
 constexpr size_t kGBytes = 8u << 20;                                                   // gradient operands
 constexpr size_t kScratchBytes = kKeysBytes + kSmallBytes + 2 * kXqBytes + kTilePtrBytes + kGBytes;
+static_assert(kScratchBytes <= ELMO_NOALLOC_SCRATCH_BYTES, "no-alloc scratch layout");
 
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ELMO_NOALLOC_SCRATCH_BYTES];
 
 // Device address of the array, looked up once per device (host code must not
 // use the symbol itself as a pointer: on the host it is only a stand-in).
