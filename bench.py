@@ -195,15 +195,15 @@ def run_reference(args, w):
     nthreads = os.cpu_count() or 1
     X = make_X(w, 0)
     rowptr, cols = make_labels(w, 0)
-    # sample size: about 5 s of oracle work per step
-    probe = 64
+    # sample size: about 120 s of oracle work for the whole run (warm-up steps included)
+    probe = min(w.L, 2048)      # enough labels that fixed costs do not dominate the rate
     Wp = make_W_f32(w, rows=probe)
     Wq = oracle.sr_round(Wp, "fp8", 0, 2**64 - 1) if w.dtype != "bf16" else make_W_bf16(w)[:probe]
     t = time.perf_counter()
     oracle.train_step(Wq, X, rowptr, cols, w.lr, 0, 0, w.dtype, 0, probe, L=w.L, nthreads=nthreads)
     per = (time.perf_counter() - t) / probe
-    budget = max(30.0, 150.0 / max(1, args.steps + args.warmup))
-    n = int(max(probe, min(w.L, budget / 3 / max(per, 1e-9))))
+    per_step_s = 120.0 / max(1, args.steps + args.warmup)
+    n = int(max(probe, min(w.L, per_step_s / max(per, 1e-9))))
     Wf = make_W_f32(w, rows=n)
     Wq = oracle.sr_round(Wf, "fp8", 0, 2**64 - 1) if w.dtype != "bf16" else oracle.rne_bf16(Wf)
     for s in range(args.warmup):
