@@ -29,7 +29,7 @@ __all__ = [
     "elmo_sync_status", "elmo_head_workspace_bytes", "elmo_profile_enable", "elmo_profile_reset",
     "elmo_profile_read", "elmo_launch_count", "KERNEL_CLASSES", "elmo_train_step_noalloc",
     "elmo_check_bounded_wait", "WAIT_CHECK_SITE", "elmo_precision_at_k", "elmo_init_head_shard",
-    "elmo_topk_merge", "MAX_SHARDS", "MAX_TOTAL_LABELS", "elmo_kahan_sgd", "elmo_round_bf16",
+    "elmo_topk_merge", "MAX_SHARDS", "MAX_TOTAL_LABELS", "elmo_kahan_sgd", "elmo_round_bf16", "elmo_last_error",
 ]
 
 BF16 = 0
@@ -108,10 +108,14 @@ def _declare(L):
         getattr(L, name).restype = st
 
 
+def elmo_last_error() -> str:
+    """The message of this thread's last failed call ("" after a success)."""
+    return load().elmo_last_error().decode(errors="replace")
+
+
 def _check(rc: int):
     if rc != 0:
-        msg = load().elmo_last_error().decode(errors="replace")
-        raise ElmoError(rc, msg)
+        raise ElmoError(rc, elmo_last_error())
 
 
 def _stream(stream):

@@ -52,3 +52,17 @@ def test_binding_without_gpu_fails_loudly():
     W = torch.zeros(128, 64, dtype=torch.bfloat16)
     with pytest.raises((ValueError, elmo.ElmoError)):
         elmo.elmo_init_head(W, "bf16")
+
+
+def test_binding_has_every_declared_name():
+    """The Python binding carries the C entry points under the same names."""
+    import precision_label_chunk_b200 as elmo
+    missing = [n for n in declared_symbols() if not callable(getattr(elmo, n, None))]
+    assert not missing, f"no binding for {missing}"
+
+
+def test_binding_rejects_unknown_dtypes():
+    import precision_label_chunk_b200 as elmo
+    assert elmo._dt("fp8_ge5m2") == elmo.FP8_E4M3_GE5M2 == 2
+    with pytest.raises(ValueError):
+        elmo._dt("e5m2")
