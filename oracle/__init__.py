@@ -32,8 +32,9 @@ _lib = None
 BF16 = 0
 FP8_E4M3 = 1
 FP8_E4M3_GE5M2 = 2      # E4M3 weights and X, E5M2 gradient operand
-_DT = {"bf16": BF16, "fp8": FP8_E4M3, "fp8_ge5m2": FP8_E4M3_GE5M2, BF16: BF16, FP8_E4M3: FP8_E4M3,
-       FP8_E4M3_GE5M2: FP8_E4M3_GE5M2}
+FP8_E5M2 = 3            # E5M2 values (standalone stochastic rounding)
+_DT = {"bf16": BF16, "fp8": FP8_E4M3, "fp8_ge5m2": FP8_E4M3_GE5M2, "e5m2": FP8_E5M2, BF16: BF16,
+       FP8_E4M3: FP8_E4M3, FP8_E4M3_GE5M2: FP8_E4M3_GE5M2, FP8_E5M2: FP8_E5M2}
 
 
 def build(force: bool = False) -> str:
@@ -66,6 +67,7 @@ def _declare(L):
     L.orc_draw16_array.argtypes = [u64, u64, u64, i64, P]
     L.orc_sr_bf16_array.argtypes = [P, P, i64, P]
     L.orc_sr_e4m3_array.argtypes = [P, P, i64, P]
+    L.orc_sr_e5m2_array.argtypes = [P, P, i64, P]
     L.orc_rne_bf16_array.argtypes = [P, i64, P]
     L.orc_rne_e4m3_array.argtypes = [P, i64, P]
     L.orc_e4m3_value_array.argtypes = [P, i64, P]
@@ -130,6 +132,9 @@ def sr_with_draws(v, k, dtype) -> np.ndarray:
     if _DT[dtype] == BF16:
         o = np.zeros(v.shape, np.uint16)
         lib().orc_sr_bf16_array(_p(v), _p(k), v.size, _p(o))
+    elif _DT[dtype] == FP8_E5M2:
+        o = np.zeros(v.shape, np.uint8)
+        lib().orc_sr_e5m2_array(_p(v), _p(k), v.size, _p(o))
     else:
         o = np.zeros(v.shape, np.uint8)
         lib().orc_sr_e4m3_array(_p(v), _p(k), v.size, _p(o))

@@ -53,6 +53,7 @@
 #define DT_BF16 0
 #define DT_E4M3 1
 #define DT_E4M3_GE5M2 2   /* E4M3 weights and X, E5M2 gradient operand */
+#define DT_E5M2 3         /* E5M2 values (standalone stochastic rounding) */
 #define IS_FP8(dt) ((dt) == DT_E4M3 || (dt) == DT_E4M3_GE5M2)
 
 /* ------------------------------------------------------------------------ */
@@ -248,6 +249,24 @@ uint8_t orc_sr_e4m3(float v, uint32_t k16) {
   return sign | (uint8_t)((u < f) ? hi : lo);
 }
 
+/* E5M2 has infinities, like bf16: +-inf stays +-inf, a finite |v| above the
+ * largest finite value (57344) saturates to it, NaN -> 0x7F. */
+uint8_t orc_sr_e5m2(float v, uint32_t k16) {
+  if (isnan(v)) return 0x7F;
+  uint8_t sign = signbit(v) ? 0x80 : 0;
+  if (isinf(v)) return sign | 0x7C;
+  double a = fabs((double)v);
+  if (a >= 57344.0) return sign | 0x7B;
+  int lo = 0;                               /* codes 0 .. 0x7B: the finite magnitudes, ascending */
+  while (lo + 1 <= 0x7B && (double)orc_e5m2_value((uint8_t)(lo + 1)) <= a) lo++;
+  double vlo = (double)orc_e5m2_value((uint8_t)lo);
+  if (vlo == a) return sign | (uint8_t)lo;
+  double vhi = (double)orc_e5m2_value((uint8_t)(lo + 1));
+  double f = (a - vlo) / (vhi - vlo);
+  double u = (double)k16 / 65536.0;
+  return sign | (uint8_t)((u < f) ? lo + 1 : lo);
+}
+
 /* out[i] = SR(in[i]) with the draw of element index_base + i. */
 int orc_sr_round(const float* in, void* out, int64_t n, int dt, uint64_t seed,
                  uint64_t step, uint64_t index_base) {
@@ -256,6 +275,7 @@ int orc_sr_round(const float* in, void* out, int64_t n, int dt, uint64_t seed,
     uint32_t k = orc_draw16(seed, step, index_base + (uint64_t)i);
     if (dt == DT_BF16) ((uint16_t*)out)[i] = orc_sr_bf16(in[i], k);
     else if (dt == DT_E4M3) ((uint8_t*)out)[i] = orc_sr_e4m3(in[i], k);
+    else if (dt == DT_E5M2) ((uint8_t*)out)[i] = orc_sr_e5m2(in[i], k);
     else return ORC_EINVAL;
   }
   return ORC_OK;
@@ -611,6 +631,9 @@ void orc_draw16_array(uint64_t seed, uint64_t step, uint64_t base, int64_t n, ui
 }
 void orc_sr_bf16_array(const float* v, const uint32_t* k, int64_t n, uint16_t* out) {
   for (int64_t i = 0; i < n; i++) out[i] = orc_sr_bf16(v[i], k[i]);
+}
+void orc_sr_e5m2_array(const float* v, const uint32_t* k, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; i++) out[i] = orc_sr_e5m2(v[i], k[i]);
 }
 void orc_sr_e4m3_array(const float* v, const uint32_t* k, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; i++) out[i] = orc_sr_e4m3(v[i], k[i]);

@@ -12,6 +12,8 @@ def _grid(dtype):
     """Sorted finite non-negative grid values, enumerated with ml_dtypes."""
     if dtype == "bf16":
         v = np.arange(0, 0x7F80, dtype=np.uint16).view(ml_dtypes.bfloat16).astype(np.float64)
+    elif dtype == "e5m2":
+        v = np.arange(0, 0x7C, dtype=np.uint8).view(ml_dtypes.float8_e5m2).astype(np.float64)
     else:
         v = np.arange(0, 127, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
     return np.unique(v)
@@ -20,10 +22,12 @@ def _grid(dtype):
 def _code_value(codes, dtype):
     if dtype == "bf16":
         return codes.view(ml_dtypes.bfloat16).astype(np.float64)
+    if dtype == "e5m2":
+        return codes.view(ml_dtypes.float8_e5m2).astype(np.float64)
     return codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "e5m2"])
 def test_grid_points_are_fixed(orc, dtype):
     g = _grid(dtype)
     x = np.concatenate([g, -g]).astype(np.float32)
@@ -36,12 +40,12 @@ def test_grid_points_are_fixed(orc, dtype):
     assert np.signbit(_code_value(z, dtype)).tolist() == [True, False]
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "e5m2"])
 def test_result_is_a_neighbour(orc, dtype):
     g = _grid(dtype)
     rng = np.random.default_rng(4)
-    top = 448.0 if dtype == "fp8" else 1e30
-    lo_e = -12 if dtype == "fp8" else -130
+    top = {"fp8": 448.0, "e5m2": 57344.0, "bf16": 1e30}[dtype]
+    lo_e = {"fp8": -12, "e5m2": -19, "bf16": -130}[dtype]
     x = (rng.random(30000) + 1) * np.exp2(rng.integers(lo_e, int(np.log2(top)), 30000))
     x = np.minimum(x, top * 0.999).astype(np.float32)
     x = np.where(rng.random(x.size) < 0.5, -x, x).astype(np.float32)
@@ -55,7 +59,7 @@ def test_result_is_a_neighbour(orc, dtype):
     assert np.all(np.sign(out)[oa > 0] == np.sign(x)[oa > 0])
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "e5m2"])
 def test_probability_of_rounding_up_closed_form(orc, dtype):
     # over all 2^16 draws the count of "hi" is #{k : k/2^16 < f} = ceil(f 2^16)
     g = _grid(dtype)
@@ -76,7 +80,7 @@ def test_probability_of_rounding_up_closed_form(orc, dtype):
             assert Fraction(n_hi, 65536) == f   # exactly unbiased on bf16
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "e5m2"])
 def test_unbiased_over_steps(orc, dtype):
     # mean of 10^4 SR draws (different steps) is within 4 sigma of v
     g = _grid(dtype)
@@ -109,10 +113,22 @@ def test_special_values(orc):
     assert int((out == 1).sum()) == 32768 and int((out == 0).sum()) == 32768
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "e5m2"])
 def test_sr_round_uses_element_draws(orc, dtype):
     rng = np.random.default_rng(8)
     x = (rng.standard_normal(1000) * 0.02).astype(np.float32)
     out = orc.sr_round(x, dtype, seed=5, step=9, index_base=777)
     k = orc.draw16(5, 9, 777, 1000)
     assert np.array_equal(out, orc.sr_with_draws(x, k, dtype))
+
+
+def test_special_values_e5m2(orc):
+    k = np.array([0, 65535], np.uint32)
+    assert orc.sr_with_draws(np.array([np.nan, -np.nan], np.float32), k, "e5m2").tolist() == [0x7F, 0x7F]
+    big = np.array([57344.0, 60000.0, 1e9, np.inf, -57344.0, -61000.0, -np.inf], np.float32)
+    out = orc.sr_with_draws(big, np.zeros(7, np.uint32), "e5m2").tolist()
+    assert out == [0x7B, 0x7B, 0x7B, 0x7C, 0xFB, 0xFB, 0xFC]        # finite saturates, inf stays inf
+    # subnormal range: 2^-17 sits halfway between 0 and 2^-16
+    v = np.full(65536, 2.0 ** -17, np.float32)
+    out = orc.sr_with_draws(v, np.arange(65536, dtype=np.uint32), "e5m2")
+    assert int((out == 1).sum()) == 32768 and int((out == 0).sum()) == 32768
