@@ -366,7 +366,7 @@ def run_topk(args, w, rank, world, local):
 
 
 def run_sr(args, local):
-    """Standalone stochastic rounding of 2^28 fp32 values to E4M3 and to bf16:
+    """Standalone stochastic rounding of 2^28 fp32 values to E4M3, bf16 and E5M2:
     an HBM-bound pass (4 bytes read and 1 or 2 bytes written per value)."""
     import torch
     import precision_label_chunk_b200 as elmo
@@ -378,7 +378,7 @@ def run_sr(args, local):
     g.manual_seed(0)
     x = torch.randn(n, generator=g, device=dev) * 0.02
     res = {}
-    for dt, odt, ob in (("fp8", torch.uint8, 1), ("bf16", torch.int16, 2)):
+    for dt, odt, ob in (("fp8", torch.uint8, 1), ("bf16", torch.int16, 2), ("e5m2", torch.uint8, 1)):
         out = torch.empty(n, dtype=odt, device=dev)
         for s in range(args.warmup):
             elmo.elmo_sr_round(x, out, dt, 0, s)

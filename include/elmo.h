@@ -40,8 +40,9 @@ extern "C" {
 typedef enum {
   ELMO_BF16 = 0,           /* bfloat16 weights (8-bit exponent, 7-bit mantissa) */
   ELMO_FP8_E4M3 = 1,       /* OCP E4M3FN weights: max 448, no infinities, saturating */
-  ELMO_FP8_E4M3_GE5M2 = 2  /* E4M3 weights (and X) as above; the training step's gradient
+  ELMO_FP8_E4M3_GE5M2 = 2, /* E4M3 weights (and X) as above; the training step's gradient
                               operand is OCP E5M2 of 2^8 G instead of E4M3 (heads only) */
+  ELMO_FP8_E5M2 = 3        /* OCP E5M2 values (max 57344, with infinities): elmo_sr_round only */
 } elmo_dtype;
 
 typedef enum {
@@ -224,11 +225,12 @@ elmo_status elmo_topk_merge(const int32_t* idx_dev, const float* score_dev, int3
  * Passage: stochastic rounding of the classifier weights replaces FP32 master
  * weights (abstract; atlas summary "Approach").  out[i] = SR(in[i]) with the
  * draw of element index_base + i of stream (seed, step), as in the step.
- * NaN -> canonical NaN (bf16 0x7FC0, E4M3 0x7F); E4M3: |v| >= 448 and +-inf ->
- * +-448; bf16: finite |v| above the largest finite -> largest finite, +-inf
- * kept.  Values on the grid are returned unchanged; -0 stays -0.
+ * NaN -> canonical NaN (bf16 0x7FC0, E4M3 and E5M2 0x7F); E4M3: |v| >= 448 and
+ * +-inf -> +-448; bf16 and E5M2 (dt = ELMO_FP8_E5M2, largest finite 57344):
+ * finite |v| above the largest finite -> largest finite, +-inf kept.  Values
+ * on the grid are returned unchanged; -0 stays -0.
  *
- *   in_dev  : fp32 [n] (device);  out_dev : bf16 or E4M3 [n] (device).
+ *   in_dev  : fp32 [n] (device);  out_dev : bf16, E4M3 or E5M2 [n] (device).
  *   n       : >= 0 (0 is a no-op).
  */
 elmo_status elmo_sr_round(const float* in_dev, void* out_dev, int64_t n, elmo_dtype dt,

@@ -23,7 +23,7 @@ import threading
 import torch
 
 __all__ = [
-    "ElmoError", "Head", "BF16", "FP8_E4M3", "FP8_E4M3_GE5M2", "MAX_BATCH", "MAX_NNZ", "MAX_TOPK", "MAX_PREDICT_BATCH",
+    "ElmoError", "Head", "BF16", "FP8_E4M3", "FP8_E4M3_GE5M2", "FP8_E5M2", "MAX_BATCH", "MAX_NNZ", "MAX_TOPK", "MAX_PREDICT_BATCH",
     "library_path", "load", "elmo_init_head", "elmo_head_destroy", "elmo_train_step_chunked",
     "elmo_forward_chunk", "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws",
     "elmo_sync_status", "elmo_head_workspace_bytes", "elmo_profile_enable", "elmo_profile_reset",
@@ -35,6 +35,7 @@ __all__ = [
 BF16 = 0
 FP8_E4M3 = 1
 FP8_E4M3_GE5M2 = 2    # E4M3 weights, E5M2 gradient operand in the training step
+FP8_E5M2 = 3          # E5M2 values (elmo_sr_round only)
 WAIT_CHECK_SITE = 99
 MAX_BATCH = 256
 MAX_NNZ = 32768
@@ -145,6 +146,8 @@ def _dt(dtype) -> int:
         return FP8_E4M3
     if dtype in (FP8_E4M3_GE5M2, "fp8_ge5m2"):
         return FP8_E4M3_GE5M2
+    if dtype in (FP8_E5M2, "e5m2", torch.float8_e5m2):
+        return FP8_E5M2
     raise ValueError(f"unknown dtype {dtype!r}")
 
 

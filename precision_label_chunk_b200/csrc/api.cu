@@ -189,6 +189,7 @@ elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_
   g_last_error.clear();
   if (!out || !W_dev) return fail(ELMO_EINVAL, "null out or W");
   *out = nullptr;
+  if (dt == ELMO_FP8_E5M2) return fail(ELMO_EUNSUPPORTED, "E5M2 weights: ELMO_FP8_E5M2 is an SR output grid only");
   if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3 && dt != ELMO_FP8_E4M3_GE5M2)
     return fail(ELMO_EINVAL, "unknown dtype %d", (int)dt);
   const bool g_e5m2 = dt == ELMO_FP8_E4M3_GE5M2;
@@ -292,9 +293,14 @@ elmo_status elmo_sr_round(const float* in_dev, void* out_dev, int64_t n, elmo_dt
   if (n < 0) return fail(ELMO_EINVAL, "n < 0");
   if (n == 0) return ELMO_OK;
   if (!in_dev || !out_dev) return fail(ELMO_EINVAL, "null pointer");
-  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3) return fail(ELMO_EINVAL, "unknown dtype %d", (int)dt);
+  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3 && dt != ELMO_FP8_E5M2)
+    return fail(ELMO_EINVAL, "dtype %d is not an SR output grid", (int)dt);
   if (index_base + (uint64_t)n < index_base) return fail(ELMO_EINVAL, "index range wraps around 2^64");
-  ELMO_CUDA(elmo::launch_sr_round(in_dev, out_dev, n, dt, seed, step, index_base, as_stream(stream)), "sr_round");
+  if (dt == ELMO_FP8_E5M2)
+    ELMO_CUDA(elmo::launch_sr_e5m2(in_dev, static_cast<uint8_t*>(out_dev), n, seed, step, index_base,
+                                   as_stream(stream)), "sr_round");
+  else
+    ELMO_CUDA(elmo::launch_sr_round(in_dev, out_dev, n, dt, seed, step, index_base, as_stream(stream)), "sr_round");
   return ELMO_OK;
 }
 

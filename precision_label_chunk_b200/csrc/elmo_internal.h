@@ -136,6 +136,8 @@ cudaError_t launch_sr_draws(uint16_t* out, int64_t n, uint64_t seed, uint64_t st
                             cudaStream_t s);
 cudaError_t launch_fill(void* W, int64_t n, elmo_dtype dt, float std, uint64_t seed, uint64_t index_base,
                         cudaStream_t s);
+cudaError_t launch_sr_e5m2(const float* in, uint8_t* out, int64_t n, uint64_t seed, uint64_t step, uint64_t base,
+                           cudaStream_t s);
 cudaError_t launch_kahan_sgd(void* p, void* c, const void* g, int64_t n, float lr, cudaStream_t s);
 cudaError_t launch_round_bf16(const float* in, void* out, int64_t n, cudaStream_t s);
 // global label ids of a sharded head's top-k (idx += label_base)

@@ -64,5 +64,6 @@ def test_binding_has_every_declared_name():
 def test_binding_rejects_unknown_dtypes():
     import precision_label_chunk_b200 as elmo
     assert elmo._dt("fp8_ge5m2") == elmo.FP8_E4M3_GE5M2 == 2
+    assert elmo._dt("e5m2") == elmo.FP8_E5M2 == 3
     with pytest.raises(ValueError):
-        elmo._dt("e5m2")
+        elmo._dt("e4m3fnuz")

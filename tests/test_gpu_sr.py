@@ -14,13 +14,17 @@ def _adversarial(dtype, rng):
         g = np.arange(0, 0x7F80, dtype=np.uint16).view(ml_dtypes.bfloat16).astype(np.float32)
         step = np.abs(np.diff(g.astype(np.float64)))
         mids = (g[:-1].astype(np.float64) + step / 2).astype(np.float32)
+    elif dtype == "e5m2":
+        g = np.arange(0, 0x7C, dtype=np.uint8).view(ml_dtypes.float8_e5m2).astype(np.float32)
+        mids = ((g[:-1].astype(np.float64) + g[1:]) / 2).astype(np.float32)
     else:
         g = np.arange(0, 127, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float32)
         mids = ((g[:-1].astype(np.float64) + g[1:]) / 2).astype(np.float32)
     near = np.concatenate([np.nextafter(g, np.float32(np.inf)), np.nextafter(g, np.float32(0))])
     special = np.array([0.0, -0.0, np.inf, -np.inf, np.nan, 448.0, 447.99, 448.01, 480.0, 1e30, 3.4e38,
                         3.3895313892515355e38, 1e-45, -1e-45, 1e-39, 2.0 ** -10, 2.0 ** -9, 2.0 ** -6,
-                        2.0 ** -7 + 2.0 ** -12], np.float32)
+                        2.0 ** -7 + 2.0 ** -12, 57344.0, 57343.99, 57345.0, 61440.0, 2.0 ** -16, 2.0 ** -17,
+                        2.0 ** -14, 2.0 ** -14 + 2.0 ** -30, 2.0 ** -14 - 2.0 ** -30, 3 * 2.0 ** -18], np.float32)
     x = np.concatenate([g, mids, near, special])
     x = np.concatenate([x, -x])
     rnd = (rng.standard_normal(1 << 20) * 0.05).astype(np.float32)
@@ -28,7 +32,7 @@ def _adversarial(dtype, rng):
     return np.concatenate([x, rnd, wide]).astype(np.float32)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "e5m2"])
 @pytest.mark.parametrize("seed,step,base", [(0, 0, 0), (0xDEADBEEF12345678, 2**63 + 5, 13), (7, 2**64 - 1, 2**40 + 3)])
 def test_sr_round_bit_exact(orc, dtype, seed, step, base):
     need_gpu()
@@ -48,7 +52,7 @@ def test_sr_round_large_random_bit_exact(orc):
     import precision_label_chunk_b200 as elmo
     rng = np.random.default_rng(99)
     x = (rng.standard_normal(10_000_000) * 0.03).astype(np.float32)
-    for dtype in ("bf16", "fp8"):
+    for dtype in ("bf16", "fp8", "e5m2"):
         ref = orc.sr_round(x, dtype, 3, 11, 5)
         out = torch.empty(x.size, dtype=torch.int16 if dtype == "bf16" else torch.uint8, device="cuda")
         elmo.elmo_sr_round(torch.from_numpy(x).cuda(), out, dtype, 3, 11, 5)
@@ -56,7 +60,7 @@ def test_sr_round_large_random_bit_exact(orc):
         assert np.array_equal(got, ref)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "e5m2"])
 @pytest.mark.parametrize("base,off,tail", [(8, 0, 5), (2**35, 0, 0), (0, 1, 3), (16, 4, 7), (2**60 + 8, 0, 1)])
 def test_sr_round_whole_blocks_and_tails(orc, dtype, base, off, tail):
     """Whole 8-value blocks at 8-aligned indices and 16-byte aligned buffers take
@@ -66,7 +70,7 @@ def test_sr_round_whole_blocks_and_tails(orc, dtype, base, off, tail):
     need_gpu()
     import precision_label_chunk_b200 as elmo
     x = _adversarial(dtype, np.random.default_rng(base & 0xFFFF))
-    n = (x.size // 8) * 8 - 8 + tail
+    n = ((x.size - off) // 8) * 8 - 8 + tail
     ref = orc.sr_round(x[off:off + n], dtype, 21, 4, base)
     xd = torch.from_numpy(x).cuda()[off:off + n]          # off > 0: the input starts 4*off bytes past alignment
     odt = torch.int16 if dtype == "bf16" else torch.uint8
@@ -99,3 +103,8 @@ def test_sr_round_empty_and_errors():
     assert lib.elmo_sr_round(None, None, -1, 0, 0, 0, 0, None) == 1     # n < 0: EINVAL
     xd = torch.zeros(4, device="cuda")
     assert lib.elmo_sr_round(xd.data_ptr(), out.data_ptr(), 4, 7, 0, 0, 0, None) == 1  # bad dtype
+    # E5M2 is an output grid of the standalone rounding, not a weight format
+    W = torch.zeros(128, 64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(elmo.ElmoError) as ei:
+        elmo.elmo_init_head(W, "e5m2")
+    assert ei.value.status == 5                                                     # ELMO_EUNSUPPORTED
