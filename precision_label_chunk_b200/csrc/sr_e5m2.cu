@@ -55,6 +55,40 @@ __global__ void __launch_bounds__(256) sr_e5m2_kernel(const float* __restrict__ 
   }
 }
 
+// Eight values with the eight draws of one Philox block, without a branch
+// per value.  Below 2^-14 a value is first moved into [2^-14, 2^-13), whose
+// spacing is also 2^-16, by adding 2^-14 rounded toward +inf: in units of the
+// 21 discarded bits that keeps ceil(F), and for an integer 32 k,
+// 32 k < F <=> 32 k < ceil(F), so the carry test stays exact; the 2^-14 is
+// taken off again exactly.  Values at or above 57344 round to at least 57344
+// and the saturating conversion brings them to 57344.  A group holding a NaN
+// or an infinity takes the per-value path.
+__device__ __forceinline__ uint2 sr8_e5m2(const float (&v)[8], const u32x4& r) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+  float probe = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) probe = __fmaf_rn(v[i], 0.0f, probe);
+  if (probe != 0.0f) {
+    uint32_t c[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) c[e] = sr_e5m2_code(v[e], (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu));
+    return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+  }
+  float o[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint32_t k = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+    const float a = fabsf(v[e]);
+    // sub = 1 when |v| < 2^-14: (2^-14 - |v|) 2^100 is then >= 2^62, else <= 0
+    const float sub = __saturatef(__fmaf_rn(-a, 0x1p100f, 0x1p86f));
+    const float sh = __fmaf_ru(sub, 0x1p-14f, a);
+    const uint32_t t = (__float_as_uint(sh) + (0x1FFFFFu - (k << 5))) & 0xFFE00000u;
+    o[e] = copysignf(__fmaf_rn(sub, -0x1p-14f, __uint_as_float(t)), v[e]);
+  }
+  return make_uint2(pack_e5m2x2(o[1], o[0]) | (pack_e5m2x2(o[3], o[2]) << 16),
+                    pack_e5m2x2(o[5], o[4]) | (pack_e5m2x2(o[7], o[6]) << 16));
+}
+
 // Whole Philox blocks: thread t rounds the 8 values of block q0 + t (two
 // 16-byte streaming loads, one 8-byte streaming store).
 __global__ void __launch_bounds__(256) sr_e5m2_vec_kernel(const float4* __restrict__ in, uint2* __restrict__ out,
@@ -62,15 +96,7 @@ __global__ void __launch_bounds__(256) sr_e5m2_vec_kernel(const float4* __restri
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < nblk; t += (int64_t)gridDim.x * blockDim.x) {
     const float4 a = __ldcs(in + 2 * t), b = __ldcs(in + 2 * t + 1);
     const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    const u32x4 r = sr_block(seed, step, q0 + (uint64_t)t);
-    uint32_t c[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const uint32_t word = sr_word(r, e >> 1);
-      c[e] = sr_e5m2_code(v[e], (e & 1) ? (word >> 16) : (word & 0xFFFFu));
-    }
-    __stcs(out + t, make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
-                               c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24)));
+    __stcs(out + t, sr8_e5m2(v, sr_block(seed, step, q0 + (uint64_t)t)));
   }
 }
 
