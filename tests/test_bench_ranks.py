@@ -1,6 +1,7 @@
 """The multi-process plumbing of bench.py on CPU (gloo, world size 2): the job
-time is the max over ranks and the job throughput counts every replica; the
-reference arm runs on rank 0 only.  The GPU work itself is not involved."""
+time is the max over ranks and the job throughput counts every rank's labels
+(its rows of the split head); the reference arm runs on rank 0 only.  The GPU
+work itself is not involved."""
 import os
 import socket
 import subprocess
@@ -46,7 +47,7 @@ def test_job_time_is_max_over_ranks_gloo():
         assert p.exitcode == 0
     for rank, ms, val in res:
         assert ms == 15.0                                   # every rank sees the slowest rank's time
-        assert val == pytest.approx(2 * 1000 * 4 / 0.015)   # both replicas' labels over that time
+        assert val == pytest.approx(2 * 1000 * 4 / 0.015)   # both ranks' labels over that time
 
 
 def test_single_process_time_is_its_own():
