@@ -144,12 +144,23 @@ def job_throughput(world, labels, steps, ms):
     return world * labels * steps / (ms / 1e3)
 
 
+def code_digest(path):
+    """sha256 of a source file's code: comments removed and white space
+    collapsed, so that an edit of the comments keeps the digest."""
+    import hashlib
+    import re
+    with open(path) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()
+
+
 def profiled_traffic(kernel, workload):
     """DRAM bytes (read + write) of one full launch of `kernel`, from the ncu
     summary committed under profiles/, with the labels that launch covered.
-    None when there is no summary or when the kernel source has changed since
-    the counters were taken (the summary records the source's sha256)."""
-    import hashlib
+    None when there is no summary or when the kernel's code has changed since
+    the counters were taken (the summary records code_digest of the source)."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
@@ -161,9 +172,8 @@ def profiled_traffic(kernel, workload):
                 fields[k.strip()] = v.strip().strip("`")
     try:
         src, digest = fields["source"].split()
-        with open(os.path.join(ROOT, src), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != digest:
-                return None
+        if code_digest(os.path.join(ROOT, src)) != digest:
+            return None
         units = fields.get("labels per launch", fields.get("values per launch"))
         return {"bytes": float(fields["dram bytes per launch"]), "labels": int(units)}
     except (KeyError, ValueError, OSError):
