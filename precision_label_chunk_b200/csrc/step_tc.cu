@@ -4,33 +4,38 @@
 // Output Spaces", atlas summary "Approach": per label chunk the classifier
 // gradient is fused with the momentum-free SGD update and applied with
 // stochastic rounding, without FP32 master weights; chunking bounds the
-// transient memory.  A label range (at most a few tens of MB of W and G, so
-// that both stay in L2 between the two kernels) is processed by:
+// transient memory.  A label range (the caller's chunk, split where its
+// gradient operands would pass 128 MB) is processed by two kernels:
 //
-//   logits_grad_tc : Z^T[128 labels x B] = W_tile X^T on tcgen05 (TMEM
-//                    accumulators, TMA-fed shared-memory operands), then
-//                    G = sigmoid(Z) - Y formed in-tile by four epilogue warps
-//                    and written as the next contraction's operand (bf16, or
-//                    E4M3 of 2^8 G).
-//   update_tc      : per (label tile, 128-column slice of d):
-//                    dX^T[slice] += W_tile[:, slice]^T G_tile^T   (old W, TMEM-resident
-//                                                                  across the CTA's tiles)
-//                    dW = G_tile^T X[:, slice]                    (TMEM)
-//                    W  = SR(W - lr dW)                           (epilogue, in place)
-//                    one fp32 atomic flush of dX^T per run of tiles.
+//   kernel A, Z = X W_tile^T and G = sigmoid(Z) - Y, written as the next
+//   contraction's operand (bf16, or E4M3 / E5M2 of 2^8 G):
+//     logits_grad_xt       : X resident in TMEM as the MMA's A operand, 64-label
+//                            W k-blocks streamed by TMA through a 16-stage ring,
+//                            G stored sample-major (E4M3 with B <= 256, bf16
+//                            with B <= 128, d <= 768);
+//     logits_grad_panel_tc : X panel resident in shared memory, Z^T = W X^T
+//                            (bf16 with B > 128, or d > 768 when a panel fits);
+//     logits_grad_tc       : X and W both streamed (the rest).
+//   kernel B, update_tc, per (label tile, 128-column slice of d):
+//     dX^T[slice] += W_tile[:, slice]^T G_tile^T   (old W, TMEM-resident across
+//                                                   the CTA's tiles)
+//     dW = G_tile^T X[:, slice]                    (TMEM)
+//     W  = SR(W - lr dW)                           (epilogue, in place)
+//     one fp32 atomic flush of dX^T per run of tiles.
 //
 // The gradient operands of a label range are stored tile by tile (128 labels
-// x Bp samples) as 8-label x 16-byte core matrices: chunk j of samples and
-// label group i sit at byte (j * 16 + i) * 128 of the tile, so the epilogue of
-// kernel A writes 512 contiguous bytes per warp store, kernel B fetches a tile
-// part with one bulk copy, and the same shared-memory block is the K-major
-// dW operand (labels x samples) and the MN-major dX^T operand (samples x labels).
+// x Bp samples) as 8-row x 16-byte core matrices, label-major (chunk j of
+// samples and label group i at byte (j * 16 + i) * 128 of the tile) or
+// sample-major (label chunk lc of sample b at ((b / 8) * nlc + lc) * 128 +
+// (b % 8) * 16): kernel B fetches a tile part with one bulk copy and uses the
+// same shared-memory block as both of its G operands (K-major for one
+// contraction, MN-major for the other).
 //
-// Warp roles (576 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
-// issues MMAs (one elected thread), warps 2-17 are the epilogue: warp w reads
-// TMEM lanes 32*(w%4) .. +31 and the 32-column chunks c with c % 4 == (w-2)/4,
-// so every SM sub-partition runs four epilogue warps (enough to hide the
-// TMEM-load and special-function latencies of one warp's chain).  Every wait is bounded; a wait that runs out
+// Kernel B's warp roles (576 threads for E4M3, 320 for bf16): warp 0 issues
+// TMA loads, warp 1 allocates TMEM and issues MMAs (one elected thread), the
+// rest are the epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 and an equal
+// share of the 32-column chunks, so every SM sub-partition runs the same
+// number of epilogue warps.  Every wait is bounded; a wait that runs out
 // records ELMO_ETIMEOUT in the status word and the CTA winds down.
 #include <cuda.h>
 #include <stdlib.h>
