@@ -32,7 +32,7 @@ _lib = None
 BF16 = 0
 FP8_E4M3 = 1
 FP8_E4M3_GE5M2 = 2      # E4M3 weights and X, E5M2 gradient operand
-FP8_E5M2 = 3            # E5M2 values (standalone stochastic rounding)
+FP8_E5M2 = 3            # E5M2 values; as a head: E5M2 weights with E4M3 X and gradient operand
 _DT = {"bf16": BF16, "fp8": FP8_E4M3, "fp8_ge5m2": FP8_E4M3_GE5M2, "e5m2": FP8_E5M2, BF16: BF16,
        FP8_E4M3: FP8_E4M3, FP8_E4M3_GE5M2: FP8_E4M3_GE5M2, FP8_E5M2: FP8_E5M2}
 
@@ -188,7 +188,8 @@ def bf16_value(bits) -> np.ndarray:
 
 
 def w_value(W, dtype) -> np.ndarray:
-    return bf16_value(W) if _DT[dtype] == BF16 else e4m3_value(W)
+    dt = _DT[dtype]
+    return bf16_value(W) if dt == BF16 else (e5m2_value(W) if dt == FP8_E5M2 else e4m3_value(W))
 
 
 def fp8_x_scale(X) -> float:

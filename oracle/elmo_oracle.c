@@ -53,8 +53,8 @@
 #define DT_BF16 0
 #define DT_E4M3 1
 #define DT_E4M3_GE5M2 2   /* E4M3 weights and X, E5M2 gradient operand */
-#define DT_E5M2 3         /* E5M2 values (standalone stochastic rounding) */
-#define IS_FP8(dt) ((dt) == DT_E4M3 || (dt) == DT_E4M3_GE5M2)
+#define DT_E5M2 3         /* E5M2 values; as a head: E5M2 weights, E4M3 X and gradient operand */
+#define IS_FP8(dt) ((dt) == DT_E4M3 || (dt) == DT_E4M3_GE5M2 || (dt) == DT_E5M2)
 
 /* ------------------------------------------------------------------------ */
 /* Philox-4xW-10 (Salmon et al. 2011).  One round maps the counter words     */
@@ -285,7 +285,9 @@ int orc_sr_round(const float* in, void* out, int64_t n, int dt, uint64_t seed,
 /* Operand preparation                                                       */
 /* ------------------------------------------------------------------------ */
 static float w_value(const void* W, int dt, int64_t i) {
-  return dt == DT_BF16 ? orc_bf16_value(((const uint16_t*)W)[i]) : orc_e4m3_value(((const uint8_t*)W)[i]);
+  if (dt == DT_BF16) return orc_bf16_value(((const uint16_t*)W)[i]);
+  if (dt == DT_E5M2) return orc_e5m2_value(((const uint8_t*)W)[i]);
+  return orc_e4m3_value(((const uint8_t*)W)[i]);
 }
 
 /* s_X = 2^e with e the largest integer such that 2^e * max|X| <= 448,
@@ -434,6 +436,7 @@ int orc_train_step(const void* W, void* W_out, int64_t L, int32_t d, int dt,
         uint32_t k = orc_draw16(seed, step, (uint64_t)l * (uint64_t)d + (uint64_t)j);
         if (W_out) {
           if (dt == DT_BF16) ((uint16_t*)W_out)[(l - l0) * d + j] = orc_sr_bf16(v, k);
+          else if (dt == DT_E5M2) ((uint8_t*)W_out)[(l - l0) * d + j] = orc_sr_e5m2(v, k);
           else ((uint8_t*)W_out)[(l - l0) * d + j] = orc_sr_e4m3(v, k);
         }
         if (dxp) for (int b = 0; b < B; b++) dxp[(size_t)b * d + j] = dxp[(size_t)b * d + j] + gl[b] * w;

@@ -29,18 +29,26 @@ def _rne_e5m2_val(x):
     return np.asarray(x, np.float32).astype(ml_dtypes.float8_e5m2).astype(np.float32)
 
 
+def _w_codes(wf, dtype):
+    """Weights on the head's grid (RNE): bf16 bits, E4M3 or E5M2 codes."""
+    if dtype == "bf16":
+        return bf16_bits(wf)
+    fmt = ml_dtypes.float8_e5m2 if dtype == "e5m2" else ml_dtypes.float8_e4m3fn
+    return np.asarray(wf, np.float32).astype(fmt).view(np.uint8)
+
+
 def _dyadic_case(rng, B, d, L, dtype):
     # X: integers in [-8, 8] / 8; W: integers in [-8, 8] / 64 (exact in both
     # grids); every sum below is exact in fp32.
     xv = (rng.integers(-8, 9, (B, d)) / 8).astype(np.float32)
     wv = (rng.integers(-8, 9, (L, d)) / 64).astype(np.float32)
     X = bf16_bits(xv)
-    W = bf16_bits(wv) if dtype == "bf16" else wv.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    W = _w_codes(wv, dtype)
     rows = [sorted(set(rng.integers(0, L, 1 + int(rng.integers(0, 4))).tolist())) for _ in range(B)]
     return X, W, xv, wv, _csr(rows)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2", "e5m2"])
 def test_step_exact_dyadic_case(orc, dtype):
     rng = np.random.default_rng(10)
     B, d, L = 6, 16, 40
@@ -53,7 +61,7 @@ def test_step_exact_dyadic_case(orc, dtype):
     g = expit(Z64).astype(np.float32) - Y                   # fp32 sigmoid minus y
     if dtype == "bf16":
         Gh = _rne_bf16_val(g)
-    elif dtype == "fp8":
+    elif dtype in ("fp8", "e5m2"):                          # E4M3 gradient operand (E5M2 heads too)
         Gh = _rne_e4m3_val(g * np.float32(256)) / np.float32(256)
     else:                                                   # E5M2 gradient operand, same 2^8 scale
         Gh = _rne_e5m2_val(g * np.float32(256)) / np.float32(256)
@@ -71,14 +79,14 @@ def _random_case(w_dtype, B=8, d=48, L=300, seed=0):
     rng = np.random.default_rng(seed)
     X = bf16_bits((rng.standard_normal((B, d)) / np.sqrt(d)).astype(np.float32))
     wf = (rng.standard_normal((L, d)) * 0.3).astype(np.float32)
-    W = bf16_bits(wf) if w_dtype == "bf16" else wf.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    W = _w_codes(wf, "e5m2" if w_dtype == "e5m2" else ("bf16" if w_dtype == "bf16" else "fp8"))
     rows = [rng.integers(0, L, 1 + int(rng.integers(0, 5))).tolist() for _ in range(B)]
     return X, W, _csr(rows)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2", "e5m2"])
 def test_step_random_case_within_fp32_bounds(orc, dtype):
-    X, W, (rowptr, cols) = _random_case("bf16" if dtype == "bf16" else "fp8")
+    X, W, (rowptr, cols) = _random_case(dtype)
     L, d = W.shape
     B = X.shape[0]
     r = orc.train_step(W, X, rowptr, cols, 0.05, 1, 2, dtype, want_zg=True)
@@ -98,7 +106,7 @@ def test_step_random_case_within_fp32_bounds(orc, dtype):
     G = r["G"].T.astype(np.float64)
     if dtype == "bf16":
         assert np.all(np.abs(G - g64) <= 2.0 ** -8 * np.abs(g64) + 1e-6)
-    elif dtype == "fp8":
+    elif dtype in ("fp8", "e5m2"):
         assert np.all(np.abs(G - g64) <= 2.0 ** -4 * np.abs(g64) + 2.0 ** -17 + 1e-6)
     else:       # E5M2 of 2^8 g: half a spacing is 2^-3 relative, subnormal spacing 2^-16 / 2^8
         assert np.all(np.abs(G - g64) <= 2.0 ** -3 * np.abs(g64) + 2.0 ** -25 + 1e-6)
@@ -112,6 +120,8 @@ def test_step_random_case_within_fp32_bounds(orc, dtype):
     new = orc.w_value(r["W"], dtype).reshape(L, d).astype(np.float64)
     if dtype == "bf16":
         grid = np.unique(np.arange(0, 0x7F80, dtype=np.uint16).view(ml_dtypes.bfloat16).astype(np.float64))
+    elif dtype == "e5m2":
+        grid = np.unique(np.arange(0, 0x7C, dtype=np.uint8).view(ml_dtypes.float8_e5m2).astype(np.float64))
     else:
         grid = np.unique(np.arange(0, 127, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64))
     a = np.abs(v64)
@@ -135,7 +145,7 @@ def test_gradient_matches_finite_difference_of_bce(orc):
     assert np.all(r["G"][Y == 1] < 0) and np.all(r["G"][Y == 0] > 0)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2", "e5m2"])
 def test_special_cases(orc, dtype):
     X, W, (rowptr, cols) = _random_case(dtype, seed=4)
     L, d = W.shape
@@ -154,7 +164,7 @@ def test_special_cases(orc, dtype):
     assert np.array_equal(r["G"], 0.5 - Y)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "fp8_ge5m2", "e5m2"])
 def test_label_range_split_and_dx_rows(orc, dtype):
     X, W, (rowptr, cols) = _random_case(dtype, seed=5)
     L, d = W.shape

@@ -14,7 +14,7 @@ def _brute(scores, k):
     return order[:k]
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "e5m2"])
 def test_topk_exact_ties_lower_index(orc, dtype):
     rng = np.random.default_rng(20)
     B, d, L, k = 5, 32, 200, 7
@@ -22,7 +22,8 @@ def test_topk_exact_ties_lower_index(orc, dtype):
     wv = (rng.integers(-4, 5, (L, d)) / 32).astype(np.float32)
     wv[150] = wv[10]; wv[151] = wv[10]; wv[3] = wv[199]       # exact ties
     X = bf16_bits(xv)
-    W = bf16_bits(wv) if dtype == "bf16" else wv.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    fmt = ml_dtypes.float8_e5m2 if dtype == "e5m2" else ml_dtypes.float8_e4m3fn     # k/32, |k| <= 4: on both grids
+    W = bf16_bits(wv) if dtype == "bf16" else wv.astype(fmt).view(np.uint8)
     idx, sc = orc.topk(W, X, k, dtype, nthreads=3)
     S = xv.astype(np.float64) @ wv.astype(np.float64).T      # exact
     for b in range(B):
