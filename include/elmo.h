@@ -22,8 +22,9 @@
  *     next call on the same head.
  *   - Return values are elmo_status codes; elmo_last_error() gives a message
  *     (thread-local) for the most recent failure on the calling thread.
- *   - Matrices are row-major and densely packed; every device pointer must be
- *     16-byte aligned.
+ *   - Matrices are row-major and densely packed; device pointers must be
+ *     16-byte aligned unless the call says otherwise (the element-wise calls
+ *     elmo_sr_round, elmo_kahan_sgd and elmo_round_bf16 take any alignment).
  *   - There is no CPU fallback: on a machine without an sm_100 GPU the calls
  *     return ELMO_ECUDA or ELMO_EUNSUPPORTED.
  */
