@@ -52,14 +52,14 @@ typedef enum {
   ELMO_ENOMEM = 2,        /* workspace allocation failed */
   ELMO_ECUDA = 3,         /* a CUDA runtime call failed (message has the CUDA error) */
   ELMO_ETIMEOUT = 4,      /* a kernel's bounded wait ran out; results are invalid */
-  ELMO_EUNSUPPORTED = 5,  /* valid but beyond this build's limits (see each call) */
+  ELMO_EUNSUPPORTED = 5,  /* valid but beyond the library's limits (see each call) */
   ELMO_EDATA = 6          /* malformed labels: CSR out of order or column out of [0, L) */
 } elmo_status;
 
 /* Opaque handle: a borrowed weight matrix plus the head's workspace. */
 typedef struct elmo_head elmo_head;
 
-/* Limits of this build. */
+/* Limits of the library. */
 #define ELMO_MAX_BATCH 256          /* B of a training step */
 #define ELMO_MAX_NNZ 32768          /* positive labels per training step */
 #define ELMO_MAX_LABELS (1LL << 24) /* L */
