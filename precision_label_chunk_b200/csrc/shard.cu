@@ -1,13 +1,14 @@
 // shard.cu -- a head split by labels over several devices.
 //
 // The classifier head is the part of the model whose size grows with the label
-// count ("ELMO: Efficiency via Low-precision and Peak Memory Optimization in
-// Large Output Spaces", abstract: the head becomes the main driver of compute
-// and memory).  Split by label rows, every device runs the same fused step on
-// its rows: the step of a label depends only on that label's weights, X and
-// whether the label is positive, so the only exchange is the sum of the
-// per-device input gradients, and the stochastic rounding stays bit-identical
-// because it draws by the element's index in the whole head.
+// count, and with millions of labels it dominates the model's compute and
+// memory ("ELMO: Efficiency via Low-precision and Peak Memory Optimization in
+// Large Output Spaces", abstract).  Split by label rows, every device runs the
+// same fused step on its rows: the step of a label depends only on that
+// label's weights, X and whether the label is positive, so the only exchange
+// is the sum of the per-device input gradients, and the stochastic rounding
+// stays bit-identical because it draws by the element's index in the whole
+// head.
 //
 // Prediction: every device ranks its own rows; the global top-k of a sample is
 // the best k of the union of the per-device lists, merged here.
