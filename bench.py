@@ -237,6 +237,74 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def _time_reference(args, fn):
+    """Warm-up calls, then the mean seconds per timed call of fn(step)."""
+    for s in range(args.warmup):
+        fn(s)
+    t = time.perf_counter()
+    for s in range(args.warmup, args.warmup + args.steps):
+        fn(s)
+    return (time.perf_counter() - t) / args.steps
+
+
+def run_reference_other(args, w):
+    """--impl reference for the workloads other than the training step: the
+    oracle as it stands, timed on a bounded sample (about 60 s for the run)."""
+    import oracle
+    from synthetic import make_X
+    oracle.build()
+    nthreads = os.cpu_count() or 1
+    per_step_s = 60.0 / max(1, args.steps + args.warmup)
+    rng = np.random.default_rng(0)
+    if args.workload == "sr_round":
+        metric, unit, cores = "standalone SR: values/s", "values/s", 1
+        probe = (rng.standard_normal(1 << 16) * 0.02).astype(np.float32)
+        t = time.perf_counter()
+        oracle.sr_round(probe, "fp8", 0, 0)
+        n = int(min(1 << 28, max(probe.size, per_step_s * probe.size / (time.perf_counter() - t))))
+        x = (rng.standard_normal(n) * 0.02).astype(np.float32)
+        sec = _time_reference(args, lambda s: oracle.sr_round(x, "fp8", 0, s))
+        units, sample, config = n, f"{n} fp32 values to E4M3 per step", {"workload": "sr_round", "n": n}
+    elif args.workload == "kahan_sgd":
+        metric, unit, cores = "Kahan-compensated bf16 SGD: params/s", "params/s", 1
+        bits = lambda a: (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)   # noqa: E731
+        probe = 1 << 16
+        p0, g0 = bits(rng.standard_normal(probe) * 0.05), bits(rng.standard_normal(probe) * 1e-2)
+        t = time.perf_counter()
+        oracle.kahan_sgd(p0, np.zeros(probe, np.uint16), g0, 1e-3)
+        n = int(min(110_000_000, max(probe, per_step_s * probe / (time.perf_counter() - t))))
+        p, c, g = bits(rng.standard_normal(n) * 0.05), np.zeros(n, np.uint16), bits(rng.standard_normal(n) * 1e-2)
+        sec = _time_reference(args, lambda s: oracle.kahan_sgd(p, c, g, 1e-3))
+        units, sample, config = n, f"{n} parameters per step", {"workload": "kahan_sgd", "n": n}
+    else:                                   # top-k prediction
+        metric, unit, cores = "chunked top-k predict: query-labels/s", "query-labels/s", nthreads
+        import torch                        # W codes of N(0, 0.02^2), made block by block (timing only)
+        gen = torch.Generator().manual_seed(0)
+        fp8 = w.dtype != "bf16"
+        Wq = np.empty((w.L, w.d), np.uint8 if fp8 else np.uint16)
+        for r0 in range(0, w.L, 1 << 17):
+            blk = torch.randn(min(1 << 17, w.L - r0), w.d, generator=gen) * 0.02
+            Wq[r0:r0 + blk.shape[0]] = (blk.to(torch.float8_e4m3fn).view(torch.uint8) if fp8
+                                         else blk.to(torch.bfloat16).view(torch.int16)).numpy().view(Wq.dtype)
+        X = make_X(w, 0)
+        t = time.perf_counter()
+        oracle.topk(Wq, X, w.topk, w.dtype, rows=[0], nthreads=nthreads)
+        rows = int(min(w.B, max(1, per_step_s / (time.perf_counter() - t))))
+        sec = _time_reference(args, lambda s: oracle.topk(Wq, X, w.topk, w.dtype, rows=list(range(rows)),
+                                                          nthreads=nthreads))
+        units = rows * w.L
+        sample = f"query rows [0, {rows}) against all {w.L} labels per step"
+        config = {"workload": w.name, "L": w.L, "d": w.d, "B": w.B, "w_dtype": w.dtype, "k": w.topk}
+    value = units / sec
+    print(json.dumps({
+        "metric": metric, "value": value, "unit": unit, "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def run_topk(args, w, rank, world, local):
     """Chunked top-k prediction (X [B x d] bf16 against the whole head): one
     step is one elmo_topk_predict call over all L labels.  N > 1: a head of
@@ -505,6 +573,15 @@ def run_kahan(args, local):
 
 def main():
     args = parse()
+    if args.impl == "reference":            # the oracle on the host cores, rank 0 only
+        if int(os.environ.get("RANK", "0")) == 0:
+            from synthetic import workload
+            if args.workload in ("sr_round", "kahan_sgd"):
+                run_reference_other(args, None)
+            else:
+                w = workload(args.workload, **({"L": args.labels} if args.labels else {}))
+                (run_reference_other if w.topk > 0 else run_reference)(args, w)
+        return
     if args.workload in ("sr_round", "kahan_sgd"):
         if int(os.environ.get("RANK", "0")) == 0:
             (run_sr if args.workload == "sr_round" else run_kahan)(args, int(os.environ.get("LOCAL_RANK", "0")))
@@ -514,11 +591,6 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-
-    if args.impl == "reference":
-        if rank == 0:
-            run_reference(args, w)
-        return
 
     if w.topk > 0:
         run_topk(args, w, rank, world, local)
