@@ -178,7 +178,10 @@ class Head:
 
 def elmo_init_head(W: torch.Tensor, dtype=None, fill: bool = False, init_std: float = 0.02, seed: int = 0,
                    stream=None) -> Head:
-    """W: [L, d] CUDA tensor (bfloat16, or float8_e4m3fn / uint8 codes)."""
+    """A head over W: [L, d] CUDA tensor of bf16 values ("bf16") or E4M3 codes
+    ("fp8"; "fp8_ge5m2" for the step with an E5M2 gradient operand), borrowed
+    and updated in place by the training steps.  fill=True overwrites W with
+    SR(init_std * N(0, 1)) drawn from Philox keyed by seed."""
     return elmo_init_head_shard(W, 0, W.shape[0], dtype, fill, init_std, seed, stream)
 
 
@@ -206,6 +209,10 @@ def elmo_head_destroy(head: Head):
 
 def elmo_train_step_chunked(head: Head, X: torch.Tensor, rowptr: torch.Tensor, cols: torch.Tensor, lr: float,
                             chunk: int, seed: int, step: int, dX: torch.Tensor, stream=None):
+    """One fused SGD step of the head: X bf16 [B, d], CSR positives rowptr
+    [B + 1] / cols [nnz] (int32, label ids of the whole head), chunk labels per
+    chunk; W is updated in place with stochastic rounding of stream (seed,
+    step) and dX (fp32 [B, d]) receives the input gradient."""
     B = X.shape[0]
     nnz = cols.numel()
     _check(load().elmo_train_step_chunked(head.handle, _ptr(X), B, _ptr(rowptr), _ptr(cols) if nnz else None,
@@ -229,6 +236,8 @@ def elmo_train_step_noalloc(W: torch.Tensor, dtype, X: torch.Tensor, rowptr: tor
 
 def elmo_forward_chunk(head: Head, X: torch.Tensor, rowptr: torch.Tensor, cols: torch.Tensor, l0: int, l1: int,
                        Z: torch.Tensor | None = None, G: torch.Tensor | None = None, stream=None):
+    """Inspection: logits Z and rounded gradient operand values G (fp32
+    [l1 - l0, B]) of rows [l0, l1) as the step forms them; W is not touched."""
     nnz = cols.numel()
     _check(load().elmo_forward_chunk(head.handle, _ptr(X), X.shape[0], _ptr(rowptr), _ptr(cols) if nnz else None,
                                      nnz, int(l0), int(l1), _ptr(Z), _ptr(G), _stream(stream)))
@@ -236,6 +245,8 @@ def elmo_forward_chunk(head: Head, X: torch.Tensor, rowptr: torch.Tensor, cols: 
 
 def elmo_topk_predict(head: Head, X: torch.Tensor, k: int, chunk: int, idx: torch.Tensor, score: torch.Tensor,
                       stream=None):
+    """Top-k labels per row of X (bf16 [B, d]): idx int32 [B, k] (label ids of
+    the whole head, best first) and score fp32 [B, k], the exact fp32 chain."""
     _check(load().elmo_topk_predict(head.handle, _ptr(X), X.shape[0], int(k), int(chunk), _ptr(idx), _ptr(score),
                                     _stream(stream)))
 
@@ -265,11 +276,14 @@ def elmo_round_bf16(inp: torch.Tensor, out: torch.Tensor, stream=None):
 
 def elmo_sr_round(inp: torch.Tensor, out: torch.Tensor, dtype, seed: int, step: int, index_base: int = 0,
                   stream=None):
+    """out = SR(inp) onto the "bf16", "fp8" (E4M3) or "e5m2" grid with the draws
+    of elements index_base .. of stream (seed, step)."""
     _check(load().elmo_sr_round(_ptr(inp), _ptr(out), inp.numel(), _dt(dtype), int(seed) & (2**64 - 1),
                                 int(step) & (2**64 - 1), int(index_base) & (2**64 - 1), _stream(stream)))
 
 
 def elmo_sr_draws(out: torch.Tensor, seed: int, step: int, index_base: int = 0, stream=None):
+    """The 16-bit draws (uint16 in a 2-byte tensor) that SR uses for elements index_base .."""
     _check(load().elmo_sr_draws(_ptr(out), out.numel(), int(seed) & (2**64 - 1), int(step) & (2**64 - 1),
                                 int(index_base) & (2**64 - 1), _stream(stream)))
 
@@ -290,6 +304,7 @@ def elmo_check_bounded_wait(limit_cycles: int, status: torch.Tensor, stream=None
 
 
 def elmo_sync_status(head: Head, stream=None):
+    """Synchronise and raise ElmoError if a kernel recorded ELMO_EDATA or ELMO_ETIMEOUT (then cleared)."""
     _check(load().elmo_sync_status(head.handle, _stream(stream)))
 
 
