@@ -33,7 +33,13 @@
  *     +-inf -> +-448; bf16: finite |v| above the largest finite -> largest
  *     finite, +-inf stays +-inf;
  *   - top-k scores are the fp32 fma chain over j = 0..d-1 in order, ranked by
- *     score descending, ties to the lower label index, NaN last.
+ *     score descending, ties to the lower label index, NaN last;
+ *   - the adjacent FP8 choices: an E5M2 gradient operand (E5M2 of 2^8 g, W and
+ *     X E4M3), and an E5M2 head (W stored and rounded on the E5M2 grid, which
+ *     has infinities: +-inf stays, finite values above 57344 saturate; X and
+ *     G E4M3);
+ *   - the encoder side: Kahan-compensated SGD of bf16 parameters with a bf16
+ *     compensation, one IEEE fp32 operation per step, RNE at the stores.
  *
  * Everything here is written for a reader checking it against those
  * definitions: no blocking, no fusion, no reordering.
