@@ -691,18 +691,14 @@ def main():
 
     # roofline of the dominant kernel class: algorithmic flops of the
     # contractions it performs per step (2 B L d each) over its device time
-    simt = os.environ.get("ELMO_STEP_SIMT", "0") == "1"
-    contractions = {"logits_grad": 1, "input_grad": 1, "update": 1 if simt else 2}
+    contractions = {"logits_grad": 1, "update": 2}
     dominant = max(classes, key=lambda k: classes[k]["ms"]) if classes else None
     roof = None
     if dominant in contractions:
         fl_per_step = contractions[dominant] * 2.0 * w.B * w.L * w.d
         achieved = fl_per_step * args.steps / (classes[dominant]["ms"] / 1e3) / 1e12
-        if simt:
-            peak, bound, src = alu_peak_tflops(peaks), "alu", "derived: 148 SM x 128 FMA x 2 x max clock"
-        else:
-            peak, bound = tensor_peak_tflops(peaks, w.dtype), "tensor"
-            src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype != "bf16" else ""))
+        peak, bound = tensor_peak_tflops(peaks, w.dtype), "tensor"
+        src = (f"{peaks['source']} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if w.dtype != "bf16" else ""))
         # ncu DRAM bytes of one full launch, scaled to the mean launch of this
         # run by the labels it covers (the kernel's traffic is linear in them)
         tr = profiled_traffic({"update": "update_tc", "logits_grad": "logits_grad_xt"}.get(dominant, dominant),

@@ -127,11 +127,11 @@ elmo_status elmo_head_destroy(elmo_head* h);
 /*
  * elmo_train_step_chunked -- one fused SGD step of the head.
  *
- * Passage: atlas summary "Approach" (pure low-precision classifier trained by
- * stochastic rounding without master weights, momentum dropped, "fusing
- * classifier gradient computation with the SGD update", "chunking the label
- * dimension to reduce transient memory"); the abstract (gradient fusion and
- * chunking).  For every label chunk W_c it computes
+ * Passage: atlas summary "Approach" (the classifier is trained in pure low
+ * precision by stochastic rounding without master weights or momentum; its
+ * gradient is computed inside the SGD update kernel, and the label dimension
+ * is processed chunk by chunk so that transient memory stays small); the
+ * abstract (gradient fusion and chunking).  For every label chunk W_c it computes
  *     Z   = X W_c^T                       (fp32 accumulation)
  *     G   = sigmoid(Z) - Y                (Y = 1 at the positive labels)
  *     dX += G W_c                         (OLD W_c, fp32)
@@ -185,8 +185,8 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B,
 /*
  * elmo_topk_predict -- chunked top-k labels per sample.
  *
- * Passage: the P@k evaluation of the atlas summary ("Metrics: P@1 P@3 P@5")
- * ranks labels by their logit; the label axis is processed in chunks as in
+ * Passage: the atlas summary's "Experimental setup" evaluates by precision at
+ * 1, 3 and 5, which ranks labels by their logit; the label axis is processed in chunks as in
  * training ("Approach").  Score of (b, l) is the fp32 fused multiply-add chain
  * s = fma(x[b,j], w[l,j], s) over j = 0..d-1 from s = 0 with x the bf16 value
  * of X (unquantised) and w the stored weight; labels are ranked by score
@@ -201,6 +201,39 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B,
  */
 elmo_status elmo_topk_predict(elmo_head* h, const void* X_dev, int32_t B, int32_t k, int64_t chunk,
                               int32_t* idx_dev, float* score_dev, void* stream);
+
+/*
+ * elmo_topk_uncertified_rows -- how many rows of the most recent
+ * elmo_topk_predict(h, ..., B, k, ...) the screening could not certify, so
+ * that their top-k came from the exact CUDA-core path over all labels.
+ *
+ * Passage: as elmo_topk_predict (a measurement of the chunked prediction).
+ *   B, k  : the arguments of that call (they locate its counter).
+ *   rows  : host int32, receives the count.
+ * Synchronises `stream`.  ELMO_EINVAL if no tensor-core prediction ran.
+ */
+elmo_status elmo_topk_uncertified_rows(elmo_head* h, int32_t B, int32_t k, int32_t* rows, void* stream);
+
+/*
+ * elmo_topk_screen_scores -- inspection of the tensor-core screening of
+ * elmo_topk_predict, for tests: the approximate scores it ranks labels
+ * [l0, l1) by, and each row's bound on their distance to the exact score.
+ *
+ * Passage: as elmo_topk_predict.  The prediction keeps, per row, the labels
+ * whose screening scores are highest, rescores them exactly, and accepts the
+ * result when the k-th exact score exceeds every other label's screening
+ * score by more than the row's bound (else the row is recomputed exactly);
+ * this call exposes both quantities so that the bound can be checked.
+ *
+ *   X_dev     : bf16 [B x d] (device), 1 <= B <= ELMO_MAX_PREDICT_BATCH.
+ *   l0, l1    : label rows, 0 <= l0 <= l1 <= L.
+ *   S_dev     : fp32 [B x (l1 - l0)] (device): screening scores.
+ *   bound_dev : fp32 [B] (device): the certificate's bound of each row (NaN
+ *               where the row or the head holds non-finite values).
+ * Uses (and grows) the head's top-k workspace; W is not modified.
+ */
+elmo_status elmo_topk_screen_scores(elmo_head* h, const void* X_dev, int32_t B, int64_t l0, int64_t l1,
+                                    float* S_dev, float* bound_dev, void* stream);
 
 /*
  * elmo_topk_merge -- the top-k of a head split over P devices from the
@@ -297,7 +330,8 @@ typedef enum {
   ELMO_K_TOPK_SCORE = 4,  /* top-k scoring of label segments */
   ELMO_K_TOPK_MERGE = 5,  /* top-k merge / exact rescoring */
   ELMO_K_OTHER = 6,       /* fill, clears */
-  ELMO_K_COUNT = 7
+  ELMO_K_STEP = 7,        /* the whole step in one persistent launch: Z, G, dX, dW and the SR update */
+  ELMO_K_COUNT = 8
 } elmo_kernel_class;
 
 elmo_status elmo_profile_enable(elmo_head* h, int enable);

@@ -10,9 +10,10 @@ Every function cites the passage it follows in the C source.
 
 Parity status: every function below is pinned by CPU tests
 (tests/test_oracle_*.py) against library routines, closed forms, special
-cases or float64 brute force, except the absolute values of the Philox4x32
-multipliers, which only the 4x64 member of the family (same round structure,
-its own constants) pins against numpy's implementation.
+cases or float64 brute force.  Philox4x32-10 itself is pinned bit-exactly
+against cuRAND's host implementation of the same generator (compiled from
+the toolkit header and run, never copied), and the 4x64 member of the family
+against numpy's Philox bit generator.
 """
 from __future__ import annotations
 
@@ -78,10 +79,11 @@ def _declare(L):
     L.orc_fp8_x_scale.restype = f32
     L.orc_train_step.argtypes = [P, P, i64, i32, ctypes.c_int, P, i32, P, P, f32, u64, u64,
                                  i64, i64, P, P, P, ctypes.c_int]
-    L.orc_dx_rows.argtypes = [P, i64, i32, ctypes.c_int, P, i32, P, P, P, i32, P, ctypes.c_int]
+    L.orc_dx_rows.argtypes = [P, i64, i32, ctypes.c_int, P, i32, P, P, P, i32, P, P, P, ctypes.c_int]
     L.orc_topk.argtypes = [P, i64, i32, ctypes.c_int, P, i32, i32, P, i32, P, P, ctypes.c_int]
     L.orc_precision_at_k.argtypes = [P, i32, i32, P, P, P]
     L.orc_kahan_sgd.argtypes = [P, P, P, i64, f32]
+    L.orc_scores.argtypes = [P, i64, i32, ctypes.c_int, P, i32, P, i32, i64, i64, P, ctypes.c_int]
     L.orc_score.argtypes = [P, ctypes.c_int, i64, P, i32, i32]
     L.orc_score.restype = f32
 
@@ -224,18 +226,22 @@ def train_step(W, X, rowptr, cols, lr, seed, step, dtype, l0=0, l1=None,
     return {"W": Wout, "dX": dX, "Z": Z, "G": G}
 
 
-def dx_rows(W, X, rowptr, cols, samples, dtype, nthreads=0):
-    """dX rows of the listed samples over all labels."""
+def dx_rows(W, X, rowptr, cols, samples, dtype, nthreads=0, want_zg=False):
+    """dX rows of the listed samples over all labels; with want_zg also their
+    logits and gradient operand values ([len(samples), L] fp32 each):
+    returns (dX rows, Z rows, G rows)."""
     dt = _DT[dtype]
     W = _c(W, np.uint16 if dt == BF16 else np.uint8)
     X = _c(X, np.uint16)
     L, d = W.shape
     samples = _c(samples, np.int32)
     out = np.zeros((samples.size, d), np.float32)
+    Z = np.zeros((samples.size, L), np.float32) if want_zg else None
+    G = np.zeros((samples.size, L), np.float32) if want_zg else None
     _check(lib().orc_dx_rows(_p(W), L, d, dt, _p(X), X.shape[0], _p(_c(rowptr, np.int32)),
-                             _p(_c(cols, np.int32)), _p(samples), samples.size, _p(out), nthreads),
+                             _p(_c(cols, np.int32)), _p(samples), samples.size, _p(out), _p(Z), _p(G), nthreads),
            "dx_rows")
-    return out
+    return (out, Z, G) if want_zg else out
 
 
 def topk(W, X, k, dtype, rows=None, nthreads=0):
@@ -273,6 +279,20 @@ def kahan_sgd(p, c, g, lr):
     assert p.shape == c.shape == g.shape
     lib().orc_kahan_sgd(_p(p), _p(c), _p(g), p.size, float(lr))
     return p, c
+
+
+def scores(W, X, rows, l0, l1, dtype, nthreads=0) -> np.ndarray:
+    """Exact top-k scores (the fp32 fma chain) of the listed rows of X against
+    labels [l0, l1): fp32 [len(rows), l1 - l0]."""
+    dt = _DT[dtype]
+    W = _c(W, np.uint16 if dt == BF16 else np.uint8)
+    X = _c(X, np.uint16)
+    L, d = W.shape
+    rows = _c(rows, np.int32)
+    out = np.zeros((rows.size, l1 - l0), np.float32)
+    _check(lib().orc_scores(_p(W), L, d, dt, _p(X), X.shape[0], _p(rows), rows.size, l0, l1, _p(out), nthreads),
+           "scores")
+    return out
 
 
 def score(W, X, l, b, dtype) -> float:

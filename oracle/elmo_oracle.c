@@ -465,10 +465,12 @@ int orc_train_step(const void* W, void* W_out, int64_t L, int32_t d, int dt,
 /*
  * Rows of dX for selected samples, over ALL labels: dX[b, :] = sum_l g_hat[b,l] w[l,:].
  * Each row depends only on its own sample, so full-size runs can be sampled.
+ * Z_rows, G_rows ([ns, L] fp32, or NULL): the logits and rounded gradient
+ * operand values of those samples.
  */
 int orc_dx_rows(const void* W, int64_t L, int32_t d, int dt, const uint16_t* X, int32_t B,
                 const int32_t* rowptr, const int32_t* cols, const int32_t* samples, int32_t ns,
-                float* dX_rows, int nthreads) {
+                float* dX_rows, float* Z_rows, float* G_rows, int nthreads) {
   if (!W || !X || !rowptr || !samples || !dX_rows || d <= 0) return ORC_EINVAL;
   pos_t pos;
   int rc = make_pos(rowptr, cols, B, L, &pos);
@@ -494,6 +496,8 @@ int orc_dx_rows(const void* W, int64_t L, int32_t d, int dt, const uint16_t* X, 
       for (int s = 0; s < ns; s++) {
         float z = logit(xq + (size_t)s * d, W, dt, l, d, inv_sx);
         float g = grad_operand(z, is_positive(&pos, samples[s], l), dt);
+        if (Z_rows) Z_rows[(size_t)s * L + l] = z;
+        if (G_rows) G_rows[(size_t)s * L + l] = g;
         for (int j = 0; j < d; j++) p[(size_t)s * d + j] = p[(size_t)s * d + j] + g * w_value(W, dt, l * d + j);
       }
     }
@@ -521,6 +525,18 @@ float orc_score(const void* W, int dt, int64_t l, const uint16_t* X, int32_t b, 
   float s = 0.0f;
   for (int j = 0; j < d; j++) s = fmaf(orc_bf16_value(X[(size_t)b * d + j]), w_value(W, dt, l * d + j), s);
   return s;
+}
+
+/* Exact scores of the listed rows of X against labels [l0, l1): out[r, l - l0]. */
+int orc_scores(const void* W, int64_t L, int32_t d, int dt, const uint16_t* X, int32_t B, const int32_t* rows,
+               int32_t nrows, int64_t l0, int64_t l1, float* out, int nthreads) {
+  if (!W || !X || !rows || !out || l0 < 0 || l1 > L || l0 > l1 || d <= 0) return ORC_EINVAL;
+  for (int r = 0; r < nrows; r++) if (rows[r] < 0 || rows[r] >= B) return ORC_EINVAL;
+  int nt = nthreads_or_default(nthreads);
+#pragma omp parallel for num_threads(nt) schedule(static)
+  for (int64_t l = l0; l < l1; l++)
+    for (int r = 0; r < nrows; r++) out[(size_t)r * (l1 - l0) + (l - l0)] = orc_score(W, dt, l, X, rows[r], d);
+  return ORC_OK;
 }
 
 /*

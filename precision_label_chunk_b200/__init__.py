@@ -25,7 +25,8 @@ import torch
 __all__ = [
     "ElmoError", "Head", "BF16", "FP8_E4M3", "FP8_E4M3_GE5M2", "FP8_E5M2", "MAX_BATCH", "MAX_NNZ", "MAX_TOPK", "MAX_PREDICT_BATCH",
     "library_path", "load", "elmo_init_head", "elmo_head_destroy", "elmo_train_step_chunked",
-    "elmo_forward_chunk", "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws",
+    "elmo_forward_chunk", "elmo_topk_predict", "elmo_topk_uncertified_rows", "elmo_topk_screen_scores",
+    "elmo_sr_round", "elmo_sr_draws",
     "elmo_sync_status", "elmo_head_workspace_bytes", "elmo_profile_enable", "elmo_profile_reset",
     "elmo_profile_read", "elmo_launch_count", "KERNEL_CLASSES", "elmo_train_step_noalloc",
     "elmo_check_bounded_wait", "WAIT_CHECK_SITE", "elmo_precision_at_k", "elmo_init_head_shard",
@@ -91,6 +92,8 @@ def _declare(L):
     L.elmo_train_step_chunked.argtypes = [P, P, i32, P, P, i32, f32, i64, u64, u64, P, P]
     L.elmo_forward_chunk.argtypes = [P, P, i32, P, P, i32, i64, i64, P, P, P]
     L.elmo_topk_predict.argtypes = [P, P, i32, i32, i64, P, P, P]
+    L.elmo_topk_uncertified_rows.argtypes = [P, i32, i32, ctypes.POINTER(i32), P]
+    L.elmo_topk_screen_scores.argtypes = [P, P, i32, i64, i64, P, P, P]
     L.elmo_sr_round.argtypes = [P, P, i64, ctypes.c_int, u64, u64, u64, P]
     L.elmo_sr_draws.argtypes = [P, i64, u64, u64, u64, P]
     L.elmo_sync_status.argtypes = [P, P]
@@ -105,7 +108,7 @@ def _declare(L):
     L.elmo_precision_at_k.argtypes = [P, i32, i32, P, P, i32, P, P]
     for name in ("elmo_profile_enable", "elmo_profile_reset", "elmo_profile_read", "elmo_launch_count","elmo_init_head", "elmo_head_destroy", "elmo_train_step_chunked", "elmo_forward_chunk",
                  "elmo_topk_predict", "elmo_sr_round", "elmo_sr_draws", "elmo_sync_status",
-                 "elmo_head_workspace_bytes"):
+                 "elmo_head_workspace_bytes", "elmo_topk_uncertified_rows", "elmo_topk_screen_scores"):
         getattr(L, name).restype = st
 
 
@@ -251,6 +254,22 @@ def elmo_topk_predict(head: Head, X: torch.Tensor, k: int, chunk: int, idx: torc
                                     _stream(stream)))
 
 
+def elmo_topk_uncertified_rows(head: Head, B: int, k: int, stream=None) -> int:
+    """Rows of the last elmo_topk_predict(B, k) on this head that the screening
+    certificate sent to the exact path."""
+    n = ctypes.c_int32()
+    _check(load().elmo_topk_uncertified_rows(head.handle, int(B), int(k), ctypes.byref(n), _stream(stream)))
+    return int(n.value)
+
+
+def elmo_topk_screen_scores(head: Head, X: torch.Tensor, l0: int, l1: int, S: torch.Tensor, bound: torch.Tensor,
+                            stream=None):
+    """Inspection: the tensor-core screening scores S (fp32 [B, l1 - l0]) of
+    labels [l0, l1) and each row's certificate bound (fp32 [B])."""
+    _check(load().elmo_topk_screen_scores(head.handle, _ptr(X), X.shape[0], int(l0), int(l1), _ptr(S), _ptr(bound),
+                                          _stream(stream)))
+
+
 def elmo_topk_merge(idx: torch.Tensor, score: torch.Tensor, idx_out: torch.Tensor, score_out: torch.Tensor,
                     stream=None):
     """Top-k of a head split over P devices: idx/score [P, B, k] (each device's
@@ -309,7 +328,7 @@ def elmo_sync_status(head: Head, stream=None):
 
 
 KERNEL_CLASSES = {"prep": 0, "logits_grad": 1, "input_grad": 2, "update": 3, "topk_score": 4, "topk_merge": 5,
-                  "other": 6}
+                  "other": 6, "step": 7}
 
 
 def elmo_profile_enable(head: Head, enable: bool = True):

@@ -10,10 +10,22 @@
 #include <new>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/elmo.h"
 #include "elmo_internal.h"
 
 namespace {
+
+// An NVTX range named after the entry point around each call, so that a
+// profiler's timeline groups the kernels of a call under the call's name.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define ELMO_NVTX_RANGE() NvtxRange nvtx_range_(__func__)
 
 thread_local std::string g_last_error;
 
@@ -41,17 +53,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
-// Development switch: ELMO_STEP_SIMT=1 runs the CUDA-core kernels of the step
-// instead of the tensor-core ones (both on the GPU).
 // ELMO_TOPK_SIMT=1 runs top-k prediction on CUDA cores only (every score by
 // its exact chain), the comparison path of the tensor-core screening.
 bool use_topk_simt() {
   const char* v = getenv("ELMO_TOPK_SIMT");
-  return v && v[0] == '1';
-}
-
-bool use_simt() {
-  const char* v = getenv("ELMO_STEP_SIMT");
   return v && v[0] == '1';
 }
 
@@ -75,6 +80,25 @@ elmo_status ensure_gbuf(elmo_head* h, size_t bytes) {
     return fail(ELMO_ENOMEM, "cannot allocate %zu bytes of gradient workspace", bytes);
   }
   h->gbuf_bytes = bytes;
+  return ELMO_OK;
+}
+
+// The persistent step's ring: kRingTiles gradient-operand tiles of up to
+// 128 labels x 256 E4M3 (or 128 bf16) samples, and its two flag arrays.
+elmo_status ensure_ring(elmo_head* h) {
+  const size_t tiles = elmo::kRingTiles;
+  const size_t bytes = tiles * 32768 + 2 * sizeof(int32_t) * tiles;
+  if (h->ring_bytes >= bytes) return ELMO_OK;
+  if (h->ring) cudaFree(h->ring);
+  h->ring = nullptr;
+  h->ring_bytes = 0;
+  if (cudaMalloc(&h->ring, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ELMO_ENOMEM, "cannot allocate %zu bytes of gradient-operand ring", bytes);
+  }
+  h->ring_bytes = bytes;
+  h->ring_tiles = (int32_t)tiles;
+  h->ring_flags = reinterpret_cast<int32_t*>(static_cast<char*>(h->ring) + tiles * 32768);
   return ELMO_OK;
 }
 
@@ -186,6 +210,7 @@ elmo_status elmo_init_head(elmo_head** out, void* W_dev, int64_t L, int32_t d, e
 elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_t d, elmo_dtype dt,
                                  int64_t label_base, int64_t labels_total, int fill, float init_std, uint64_t seed,
                                  void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (!out || !W_dev) return fail(ELMO_EINVAL, "null out or W");
   *out = nullptr;
@@ -251,10 +276,12 @@ elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_
 }
 
 elmo_status elmo_head_destroy(elmo_head* h) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (!h) return ELMO_OK;
   cudaDeviceSynchronize();
   if (h->gbuf) cudaFree(h->gbuf);
+  if (h->ring) cudaFree(h->ring);
   if (h->cand) cudaFree(h->cand);
   if (h->status) cudaFree(h->status);
   if (h->side) cudaStreamDestroy(h->side);
@@ -268,11 +295,12 @@ elmo_status elmo_head_destroy(elmo_head* h) {
 
 elmo_status elmo_head_workspace_bytes(const elmo_head* h, size_t* bytes) {
   if (!h || !bytes) return fail(ELMO_EINVAL, "null argument");
-  *bytes = h->base_bytes + h->gbuf_bytes + h->cand_bytes;
+  *bytes = h->base_bytes + h->gbuf_bytes + h->ring_bytes + h->cand_bytes;
   return ELMO_OK;
 }
 
 elmo_status elmo_sync_status(elmo_head* h, void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (!h) return fail(ELMO_EINVAL, "null head");
   int32_t st[2] = {0, 0};
@@ -289,6 +317,7 @@ elmo_status elmo_sync_status(elmo_head* h, void* stream) {
 
 elmo_status elmo_sr_round(const float* in_dev, void* out_dev, int64_t n, elmo_dtype dt, uint64_t seed,
                           uint64_t step, uint64_t index_base, void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (n < 0) return fail(ELMO_EINVAL, "n < 0");
   if (n == 0) return ELMO_OK;
@@ -306,6 +335,7 @@ elmo_status elmo_sr_round(const float* in_dev, void* out_dev, int64_t n, elmo_dt
 
 elmo_status elmo_sr_draws(uint16_t* out_dev, int64_t n, uint64_t seed, uint64_t step, uint64_t index_base,
                           void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (n < 0) return fail(ELMO_EINVAL, "n < 0");
   if (n == 0) return ELMO_OK;
@@ -318,6 +348,7 @@ elmo_status elmo_sr_draws(uint16_t* out_dev, int64_t n, uint64_t seed, uint64_t 
 elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B, const int32_t* rowptr_dev,
                                const int32_t* cols_dev, int32_t nnz, int64_t l0, int64_t l1, float* Z_dev,
                                float* G_dev, void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (!h) return fail(ELMO_EINVAL, "null head");
   elmo_status st = check_labels_args(h, X_dev, B, rowptr_dev, cols_dev, nnz);
@@ -335,10 +366,7 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B, const
   const bool fp8 = h->dt == ELMO_FP8_E4M3;
   const size_t esz = fp8 ? 1 : 2;
   const int32_t Bp = elmo::padded_batch(B, fp8);
-  const bool simt = use_simt();
-  if (simt && h->g_e5m2)
-    return fail(ELMO_EUNSUPPORTED, "the CUDA-core development path has no E5M2 gradient operand");
-  const int64_t sub = simt ? elmo::kSubChunk : elmo::sub_chunk_labels(h->d, Bp, (int)esz);
+  const int64_t sub = elmo::sub_chunk_labels(h->d, Bp, (int)esz);
   const int64_t span = l1 - l0 < sub ? l1 - l0 : sub;
   if ((st = ensure_gbuf(h, (size_t)((span + 127) / 128 * 128) * Bp * esz)) != ELMO_OK) return st;  // whole tiles
   for (int64_t a = l0; a < l1; a += span) {
@@ -346,8 +374,7 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B, const
     elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
     float* Za = Z_dev ? Z_dev + (a - l0) * B : nullptr;
     float* Ga = G_dev ? G_dev + (a - l0) * B : nullptr;
-    if (simt) ELMO_CUDA(elmo::launch_grad_simt(h, X, B, a, e, h->gbuf, Za, Ga, s), "grad");
-    else ELMO_CUDA(elmo::launch_logits_grad_tc(h, X, B, a, e, h->gbuf, Za, Ga, s), "logits_grad");
+    ELMO_CUDA(elmo::launch_logits_grad_tc(h, X, B, a, e, h->gbuf, Za, Ga, s), "logits_grad");
   }
   return ELMO_OK;
 }
@@ -355,6 +382,7 @@ elmo_status elmo_forward_chunk(elmo_head* h, const void* X_dev, int32_t B, const
 elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, const int32_t* rowptr_dev,
                                     const int32_t* cols_dev, int32_t nnz, float lr, int64_t chunk, uint64_t seed,
                                     uint64_t step, float* dX_dev, void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (!h) return fail(ELMO_EINVAL, "null head");
   elmo_status st = check_labels_args(h, X_dev, B, rowptr_dev, cols_dev, nnz);
@@ -373,10 +401,15 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
   const bool fp8 = h->dt == ELMO_FP8_E4M3;
   const size_t esz = fp8 ? 1 : 2;
   const int32_t Bp = elmo::padded_batch(B, fp8);
-  const bool simt = use_simt();
-  if (simt && h->g_e5m2)
-    return fail(ELMO_EUNSUPPORTED, "the CUDA-core development path has no E5M2 gradient operand");
-  const int64_t sub_max = simt ? elmo::kSubChunk : elmo::sub_chunk_labels(h->d, Bp, (int)esz);
+  if (elmo::fused_step_supported(h, B)) {
+    // one persistent launch; the chunk only bounds transient memory, which
+    // the ring of gradient-operand tiles already does
+    if ((st = ensure_ring(h)) != ELMO_OK) return st;
+    elmo::KernelScope ks(h, ELMO_K_STEP, s);
+    ELMO_CUDA(elmo::launch_step_fused(h, X, B, lr, seed, step, dX_dev, s), "step");
+    return ELMO_OK;
+  }
+  const int64_t sub_max = elmo::sub_chunk_labels(h->d, Bp, (int)esz);
   const int64_t sub = chunk < sub_max ? chunk : sub_max;
   const int64_t span = h->L < sub ? h->L : sub;
   if ((st = ensure_gbuf(h, (size_t)((span + 127) / 128 * 128) * Bp * esz)) != ELMO_OK) return st;  // whole tiles
@@ -384,26 +417,13 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
     const int64_t c1 = c0 + chunk < h->L ? c0 + chunk : h->L;
     for (int64_t a = c0; a < c1; a += span) {
       const int64_t e = a + span < c1 ? a + span : c1;
-      if (simt) {
-        {
-          elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
-          ELMO_CUDA(elmo::launch_grad_simt(h, X, B, a, e, h->gbuf, nullptr, nullptr, s), "grad");
-        }
-        {
-          elmo::KernelScope ks(h, ELMO_K_INPUT_GRAD, s);
-          ELMO_CUDA(elmo::launch_dx_simt(h, B, a, e, h->gbuf, dX_dev, s), "dx");
-        }
-        elmo::KernelScope ks(h, ELMO_K_UPDATE, s);
-        ELMO_CUDA(elmo::launch_update_simt(h, X, B, a, e, h->gbuf, lr, seed, step, s), "update");
-      } else {
-        // every kernel but the first follows one of the step's own kernels: programmatic launches
-        {
-          elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
-          ELMO_CUDA(elmo::launch_logits_grad_tc(h, X, B, a, e, h->gbuf, nullptr, nullptr, s, a > 0), "logits_grad");
-        }
-        elmo::KernelScope ks(h, ELMO_K_UPDATE, s);
-        ELMO_CUDA(elmo::launch_update_tc(h, X, B, a, e, h->gbuf, lr, seed, step, dX_dev, s, true), "update");
+      // every kernel but the first follows one of the step's own kernels: programmatic launches
+      {
+        elmo::KernelScope ks(h, ELMO_K_LOGITS_GRAD, s);
+        ELMO_CUDA(elmo::launch_logits_grad_tc(h, X, B, a, e, h->gbuf, nullptr, nullptr, s, a > 0), "logits_grad");
       }
+      elmo::KernelScope ks(h, ELMO_K_UPDATE, s);
+      ELMO_CUDA(elmo::launch_update_tc(h, X, B, a, e, h->gbuf, lr, seed, step, dX_dev, s, true), "update");
     }
   }
   return ELMO_OK;
@@ -411,6 +431,7 @@ elmo_status elmo_train_step_chunked(elmo_head* h, const void* X_dev, int32_t B, 
 
 elmo_status elmo_precision_at_k(const int32_t* idx_dev, int32_t B, int32_t k, const int32_t* rowptr_dev,
                                 const int32_t* cols_dev, int32_t nnz, float* p_dev, void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (!idx_dev || !rowptr_dev || !p_dev || (nnz > 0 && !cols_dev)) return fail(ELMO_EINVAL, "null pointer");
   if (B < 1 || B > ELMO_MAX_PREDICT_BATCH) return fail(ELMO_EINVAL, "B = %d outside [1, %d]", B, ELMO_MAX_PREDICT_BATCH);
@@ -432,6 +453,7 @@ elmo_status elmo_check_bounded_wait(int64_t limit_cycles, int32_t* status_dev, v
 
 elmo_status elmo_topk_predict(elmo_head* h, const void* X_dev, int32_t B, int32_t k, int64_t chunk,
                               int32_t* idx_dev, float* score_dev, void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (!h) return fail(ELMO_EINVAL, "null head");
   if (!X_dev || !idx_dev || !score_dev) return fail(ELMO_EINVAL, "null pointer");
@@ -459,7 +481,39 @@ elmo_status elmo_topk_predict(elmo_head* h, const void* X_dev, int32_t B, int32_
   return ELMO_OK;
 }
 
+elmo_status elmo_topk_uncertified_rows(elmo_head* h, int32_t B, int32_t k, int32_t* rows, void* stream) {
+  g_last_error.clear();
+  if (!h || !rows) return fail(ELMO_EINVAL, "null argument");
+  if (B < 1 || B > ELMO_MAX_PREDICT_BATCH) return fail(ELMO_EINVAL, "B = %d outside [1, %d]", B, ELMO_MAX_PREDICT_BATCH);
+  if (k < 1 || k > ELMO_MAX_TOPK) return fail(ELMO_EINVAL, "k = %d outside [1, %d]", k, ELMO_MAX_TOPK);
+  if (!elmo::topk_tc_supported(h) || !h->cand || h->cand_bytes < elmo::topk_tc_workspace_bytes(h, B, k))
+    return fail(ELMO_EINVAL, "no tensor-core prediction of this shape has run on this head");
+  ELMO_CUDA(elmo::topk_uncertified_rows(h, B, k, rows, as_stream(stream)), "uncertified rows");
+  return ELMO_OK;
+}
+
+elmo_status elmo_topk_screen_scores(elmo_head* h, const void* X_dev, int32_t B, int64_t l0, int64_t l1,
+                                    float* S_dev, float* bound_dev, void* stream) {
+  ELMO_NVTX_RANGE();
+  g_last_error.clear();
+  if (!h) return fail(ELMO_EINVAL, "null head");
+  if (!X_dev || !S_dev || !bound_dev) return fail(ELMO_EINVAL, "null pointer");
+  if (B < 1 || B > ELMO_MAX_PREDICT_BATCH) return fail(ELMO_EINVAL, "B = %d outside [1, %d]", B, ELMO_MAX_PREDICT_BATCH);
+  if (l0 < 0 || l1 > h->L || l0 > l1) return fail(ELMO_EINVAL, "label range [%lld, %lld) outside [0, %lld]",
+                                                 (long long)l0, (long long)l1, (long long)h->L);
+  if (!aligned16(X_dev)) return fail(ELMO_EINVAL, "X is not 16-byte aligned");
+  if (!elmo::topk_tc_supported(h)) return fail(ELMO_EUNSUPPORTED, "this head has no tensor-core screening");
+  elmo_status st = check_device(h);
+  if (st != ELMO_OK) return st;
+  if (l0 == l1) return ELMO_OK;
+  if ((st = ensure_cand(h, elmo::topk_tc_workspace_bytes(h, B, 1))) != ELMO_OK) return st;
+  ELMO_CUDA(elmo::launch_topk_screen_dump(h, static_cast<const uint16_t*>(X_dev), B, l0, l1, S_dev, bound_dev,
+                                          as_stream(stream)), "screen scores");
+  return ELMO_OK;
+}
+
 elmo_status elmo_kahan_sgd(void* p_dev, void* c_dev, const void* g_dev, int64_t n, float lr, void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (n < 0) return fail(ELMO_EINVAL, "n = %lld < 0", (long long)n);
   if (n > 0 && (!p_dev || !c_dev || !g_dev)) return fail(ELMO_EINVAL, "null pointer");
@@ -469,6 +523,7 @@ elmo_status elmo_kahan_sgd(void* p_dev, void* c_dev, const void* g_dev, int64_t 
 }
 
 elmo_status elmo_round_bf16(const float* in_dev, void* out_dev, int64_t n, void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (n < 0) return fail(ELMO_EINVAL, "n = %lld < 0", (long long)n);
   if (n > 0 && (!in_dev || !out_dev)) return fail(ELMO_EINVAL, "null pointer");
@@ -478,6 +533,7 @@ elmo_status elmo_round_bf16(const float* in_dev, void* out_dev, int64_t n, void*
 
 elmo_status elmo_topk_merge(const int32_t* idx_dev, const float* score_dev, int32_t P, int32_t B, int32_t k,
                             int32_t* idx_out_dev, float* score_out_dev, void* stream) {
+  ELMO_NVTX_RANGE();
   g_last_error.clear();
   if (!idx_dev || !score_dev || !idx_out_dev || !score_out_dev) return fail(ELMO_EINVAL, "null pointer");
   if (P < 1 || P > ELMO_MAX_SHARDS) return fail(ELMO_EINVAL, "P = %d outside [1, %d]", P, ELMO_MAX_SHARDS);

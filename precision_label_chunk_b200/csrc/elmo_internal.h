@@ -38,6 +38,10 @@ struct elmo_head {
   uint8_t* xqt = nullptr;      // the same codes by 16-byte column chunk: [d/16][ELMO_MAX_BATCH][16]
   void* gbuf = nullptr;        // per-chunk gradient operands
   size_t gbuf_bytes = 0;
+  void* ring = nullptr;        // the persistent step's ring of gradient-operand tiles
+  int32_t* ring_flags = nullptr; // [2 * ring_tiles]: ready, then consumed (zeroed every step)
+  int32_t ring_tiles = 0;
+  size_t ring_bytes = 0;
   void* cand = nullptr;        // top-k candidates
   size_t cand_bytes = 0;
   size_t base_bytes = 0;       // bytes of the fixed part of the workspace
@@ -64,7 +68,6 @@ struct KernelScope {
 namespace elmo {
 
 constexpr int kTileLabels = 128;        // labels per tensor-core tile
-constexpr int64_t kSubChunk = 65536;    // largest label range per pass (L2-resident G)
 
 // Labels per pass of the tensor-core step: the caller's chunk, capped so that
 // the gradient operands of one pass (the transient buffer chunking bounds)
@@ -88,14 +91,6 @@ cudaError_t launch_prep_x(elmo_head* h, const uint16_t* X, int32_t B, cudaStream
 cudaError_t launch_prep_step(elmo_head* h, const int32_t* rowptr, const int32_t* cols, int32_t B, int32_t nnz,
                              const uint16_t* X, cudaStream_t s);
 
-// step_simt.cu -- reference-order kernels (first correct path)
-cudaError_t launch_grad_simt(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
-                             void* gbuf, float* Zout, float* Gout, cudaStream_t s);
-cudaError_t launch_dx_simt(const elmo_head* h, int32_t B, int64_t l0, int64_t l1, const void* gbuf,
-                           float* dX, cudaStream_t s);
-cudaError_t launch_update_simt(const elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1,
-                               const void* gbuf, float lr, uint64_t seed, uint64_t step, cudaStream_t s);
-
 // step_tc.cu -- tensor-core step
 // 2-D row-major TMA map [rows x cols] of 1- or 2-byte elements, box = 128 bytes
 // x box_rows, 128-byte swizzle, zero fill outside the tensor.
@@ -112,6 +107,14 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
                              const void* gbuf, float lr, uint64_t seed, uint64_t step, float* dX, cudaStream_t s,
                              bool pdl = false);
 
+// step_fused.cu -- the whole step in one persistent, cooperative launch (role A:
+// logits and gradient operands into a ring of tiles; role B: dX, dW and the SR
+// update), for the shapes whose X fits in TMEM
+bool fused_step_supported(const elmo_head* h, int32_t B);
+constexpr int32_t kRingTiles = 256;      // gradient-operand tiles in the ring
+cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float lr, uint64_t seed, uint64_t step,
+                              float* dX, cudaStream_t s);
+
 // topk_simt.cu -- exact top-k on CUDA cores, for all rows (rows == null) or
 // for the *nrows rows listed in rows (a list whose length lives on the device)
 size_t topk_simt_workspace_bytes(const elmo_head* h, int32_t B, int32_t k);
@@ -124,6 +127,11 @@ bool topk_tc_supported(const elmo_head* h);
 size_t topk_tc_workspace_bytes(const elmo_head* h, int32_t B, int32_t k);
 cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k, int32_t* idx, float* score,
                            cudaStream_t s);
+// rows of the last launch_topk_tc(B, k) that the certificate sent to the exact path (synchronises s)
+cudaError_t topk_uncertified_rows(elmo_head* h, int32_t B, int32_t k, int32_t* rows, cudaStream_t s);
+// inspection: screening scores S [B x (l1 - l0)] and each row's certificate bound [B]
+cudaError_t launch_topk_screen_dump(elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1, float* S,
+                                    float* bound, cudaStream_t s);
 
 // metrics.cu
 cudaError_t launch_precision_at_k(const int32_t* idx, int32_t B, int32_t k, const int32_t* rowptr,

@@ -1,0 +1,323 @@
+// step_common.cuh -- device pieces shared by the kernels of the training step:
+// bounded-wait bookkeeping, the gradient operand G = sigmoid(Z) - Y with its
+// certified rounding, and the stochastic-rounding SGD update of 16 weights.
+//
+// "ELMO: Efficiency via Low-precision and Peak Memory Optimization in Large
+// Output Spaces", atlas summary "Approach": the classifier's gradient is fused
+// with a momentum-free SGD update applied by stochastic rounding onto the BF16
+// or E4M3 grid, without FP32 master weights.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "elmo_common.cuh"
+#include "elmo_internal.h"
+#include "tc_ptx.cuh"
+
+namespace elmo {
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 576;                    // 18 warps: TMA, MMA, 16 epilogue
+constexpr int kEpiWarps = 16;
+constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 2 GHz: only a broken pipeline waits this long
+constexpr uint32_t kBox = 16384;                  // one 128-row x 128-byte TMA box
+
+__device__ __forceinline__ void record_timeout(int32_t* status, volatile int* abort, int site) {
+  *abort = 1;
+  if (atomicCAS(status, 0, (int)ELMO_ETIMEOUT) == 0) status[1] = site;
+}
+
+// Positives of label `l` among the sorted keys (label << 8 | sample) in
+// [k0, k1): a 256-bit sample mask.
+__device__ __forceinline__ void label_mask(const uint32_t* __restrict__ keys, int k0, int k1, int64_t l,
+                                           uint32_t (&m)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = 0;
+  for (int i = k0; i < k1; ++i) {
+    const uint32_t key = __ldg(keys + i);
+    if ((int64_t)(key >> 8) == l) {
+      const uint32_t b = key & 0xFFu;
+#pragma unroll
+      for (int w = 0; w < 8; ++w)
+        if ((b >> 5) == (uint32_t)w) m[w] |= 1u << (b & 31);
+    }
+  }
+}
+
+
+__device__ __forceinline__ float exp2f_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcpf_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// fp32 multiply that keeps denormal inputs and results whatever -ftz says
+__device__ __forceinline__ float mul_rn_denorm(float a, float b) {
+  float y;
+  asm("mul.rn.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
+  return y;
+}
+
+// ---------------------------------------------------------------- epilogue pieces
+// The gradient operand of the next two contractions for 16 elements:
+// G = sigmoid(z) - y rounded to nearest even onto bf16 (kG = 0), or 2^8 G onto
+// E4M3 (kG = 1) or E5M2 (kG = 2), z = acc * inv_sx; y = 1 at the positives.
+// The code is the one that sigmoid(z) = 1 / (1 + e^-z) correctly rounded to
+// fp32 gives.  sigmoid comes from one ex2 and one rcp of the special-function
+// unit, within 2^-21 relative plus |z| 2^-23 from the rounded argument of ex2;
+// each element is rounded from both ends of an interval around its value that
+// is wider than that error, and where the two ends land on different codes
+// (the value lies within that error of a midpoint of the operand grid, about
+// 2^-15 of the elements at the workloads' logits) sigmoid is recomputed in
+// double precision and rounded to fp32 first.  ybits: positives; vbits: valid
+// elements (the others, batch padding and labels past the range, get code 0);
+// out: 4 words of 8-bit codes or 8 words of bf16, element 0 in the low bits.
+template <int kG>
+__device__ __forceinline__ uint32_t grad_pack2(float hi, float lo) {
+  return kG == 0 ? pack_bf16x2(hi, lo) : kG == 1 ? pack_e4m3x2(hi, lo) : pack_e5m2x2(hi, lo);
+}
+
+template <int kG>
+__device__ __noinline__ uint32_t grad_code_exact(float acc, float inv_sx, bool pos) {
+  constexpr float sc = kG ? 256.0f : 1.0f;
+  const float z = __fmul_rn(acc, inv_sx);
+  const float s = (float)(1.0 / (1.0 + exp(-(double)z)));
+  const float x = __fmaf_rn(s, sc, pos ? -sc : 0.0f);     // sc (s - y): the scale is exact
+  return grad_pack2<kG>(0.0f, x) & (kG ? 0xFFu : 0xFFFFu);
+}
+
+template <int kG>
+__device__ __forceinline__ void grad_codes16(const uint32_t* acc, float inv_sx, uint32_t ybits, uint32_t vbits,
+                                             uint32_t* out) {
+  constexpr float sc = kG ? 256.0f : 1.0f;
+  constexpr int kPer = kG ? 4 : 2;                 // codes per 32-bit word
+  constexpr int kBits = 32 / kPer;
+  const float zmul = -1.4426950408889634f * inv_sx;
+  float lo[16], hi[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a = __uint_as_float(acc[i]);
+    const float e = exp2f_approx(__fmul_rn(a, zmul));
+    const float s = rcpf_approx(__fadd_rn(e, 1.0f));
+    const float as = s * sc;
+    const float xc = as - (((ybits >> i) & 1u) ? sc : 0.0f);
+    const float eps = __fmaf_rn(fabsf(__fmul_rn(a, inv_sx)), 0x1p-22f, 0x1p-20f);
+    const float w = __fmaf_rn(fabsf(xc), 0x1p-22f, as * eps);
+    const bool v = (vbits >> i) & 1u;
+    lo[i] = v ? xc - w : 0.0f;
+    hi[i] = v ? xc + w : 0.0f;
+  }
+  uint32_t wlo[16 / kPer], whi[16 / kPer];
+#pragma unroll
+  for (int q = 0; q < 16 / kPer; ++q) {
+    if (kG) {
+      wlo[q] = grad_pack2<kG>(lo[4 * q + 1], lo[4 * q]) | (grad_pack2<kG>(lo[4 * q + 3], lo[4 * q + 2]) << 16);
+      whi[q] = grad_pack2<kG>(hi[4 * q + 1], hi[4 * q]) | (grad_pack2<kG>(hi[4 * q + 3], hi[4 * q + 2]) << 16);
+    } else {
+      wlo[q] = grad_pack2<kG>(lo[2 * q + 1], lo[2 * q]);
+      whi[q] = grad_pack2<kG>(hi[2 * q + 1], hi[2 * q]);
+    }
+  }
+  uint32_t diff = 0;
+#pragma unroll
+  for (int q = 0; q < 16 / kPer; ++q) diff |= wlo[q] ^ whi[q];
+  if (diff) {                                      // rare: a value near a midpoint of the grid
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int q = i / kPer, sh = (i % kPer) * kBits;
+      const uint32_t m = (kG ? 0xFFu : 0xFFFFu) << sh;
+      if ((wlo[q] ^ whi[q]) & m)
+        wlo[q] = (wlo[q] & ~m) | (grad_code_exact<kG>(__uint_as_float(acc[i]), inv_sx, (ybits >> i) & 1u) << sh);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 16 / kPer; ++q) out[q] = wlo[q];
+}
+
+// The operand value of code `c` (G, with 2^-8 undone for the 8-bit formats).
+template <int kG>
+__device__ __forceinline__ float grad_value(uint32_t c) {
+  return kG == 0 ? bf16_to_f32((uint16_t)c)
+                 : (kG == 1 ? e4m3_to_f32((uint8_t)c) : e5m2_to_f32((uint8_t)c)) * 0.00390625f;
+}
+
+// G for 16 samples b0 .. b0+15 of one label row, stored label-major as the
+// next contraction's operand (the resident-X and streamed-X kernels A).
+template <int kFp8, int kG5 = 0>
+__device__ __forceinline__ void grad16(const uint32_t* r, float inv_sx, uint32_t ybits, int b0, int B,
+                                       uint8_t* __restrict__ gtile, int row, bool row_invalid,
+                                       float* __restrict__ Zrow, float* __restrict__ Grow) {
+  constexpr int kG = kFp8 ? (kG5 ? 2 : 1) : 0;
+  uint32_t vbits = 0;
+  if (!row_invalid) vbits = b0 + 16 <= B ? 0xFFFFu : (B > b0 ? (1u << (B - b0)) - 1u : 0u);
+  uint32_t packed[8];
+  grad_codes16<kG>(r, inv_sx, ybits, vbits, packed);
+  if (kFp8) {
+    const int j = b0 >> 4;                                   // 16-byte chunk of samples
+    *reinterpret_cast<uint4*>(gtile + ((j * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
+        make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  } else {
+    const int j = b0 >> 3;                                   // first of two 16-byte chunks
+    *reinterpret_cast<uint4*>(gtile + ((j * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
+        make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    *reinterpret_cast<uint4*>(gtile + (((j + 1) * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
+        make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  }
+  if (Grow && !row_invalid) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (b0 + i < B)
+        Grow[i] = grad_value<kG>(kFp8 ? (packed[i >> 2] >> (8 * (i & 3))) & 0xFFu
+                                      : (packed[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+  }
+  if (Zrow && !row_invalid) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (b0 + i < B) Zrow[i] = __fmul_rn(__uint_as_float(r[i]), inv_sx);
+  }
+}
+
+// Positive-label bits of samples b0 .. b0+15 from the 256-bit mask.
+__device__ __forceinline__ uint32_t mask16(const uint32_t (&m)[8], int b0) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w = ((b0 >> 5) == i) ? m[i] : w;
+  return (w >> (b0 & 16)) & 0xFFFFu;
+}
+
+// ---------------------------------------------------------------- the SR update
+// fp32 product rounded toward +infinity, denormal inputs and results kept
+__device__ __forceinline__ float mul_rp(float a, float b) {
+  float y;
+  asm("mul.rp.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
+  return y;
+}
+
+// The 16 draws of elements l*d + j0 .. +15 (two Philox blocks; blk_base more
+// blocks in when this head holds the rows of a larger head from label_base on:
+// blk_base = label_base * d / 8).  Independent of the gradient, so the update
+// can form them while the MMAs of its tile are still running.
+__device__ __forceinline__ void sr_draws16(uint64_t seed, uint64_t step, uint64_t blk_base, int64_t l, int32_t d,
+                                           int j0, uint32_t (&rw)[8]) {
+  const uint64_t blk = blk_base + (((uint64_t)l * (uint64_t)d + (uint64_t)j0) >> 3);
+  const u32x4 r0 = sr_block(seed, step, blk), r1 = sr_block(seed, step, blk + 1);
+  rw[0] = r0.x; rw[1] = r0.y; rw[2] = r0.z; rw[3] = r0.w;
+  rw[4] = r1.x; rw[5] = r1.y; rw[6] = r1.z; rw[7] = r1.w;
+}
+
+// W[l, j0 .. j0+15] = SR(W - lrs * acc) for one label row: old weights from the
+// 128B-swizzled W tile in shared memory (row `row`, tile column jl), draws rw
+// from sr_draws16.
+//
+// v = fl(w - fl(lrs dW)) (two roundings, denormals kept); a probe (the sum of
+// 2^120 v for E4M3, of 2 v for bf16) is not finite when some v is NaN or
+// infinite or too large for the fast rounding (E4M3: |v| >= 2^8; bf16:
+// |v| >= 2^127, where rounding could pass the largest finite value), and such
+// groups take the exact per-element path.
+//
+// Fast rounding, both grids: add-and-truncate.  If the bits of v below the
+// target precision hold the fraction F (in units of 2^-n of a grid step),
+// u < f  <=>  2^(n-16) k < F  <=>  adding 2^n - 1 - 2^(n-16) k carries into the
+// first kept bit.
+// bf16 (n = 16): the hardware's stochastic conversion cvt.rs.bf16x2.f32 adds
+// its 16 random bits to the 16 discarded bits of each value and truncates, so
+// passing 2^16 - 1 - k (the complemented draw) gives exactly this rounding.
+// E4M3 (n = 20): |v| 2^-120 is fp32's own grid cut to 3 mantissa bits (E4M3's
+// subnormal spacing 2^-9 becomes 2^-129, 2^20 units of fp32's denormal spacing,
+// and its normal range starts at 2^-126, fp32's); the product is rounded toward
+// +infinity, which keeps ceil(F) and, k being an integer, the decision
+// 16 k < F exactly, also below 2^-6 where the product is denormal.  The
+// pattern is shifted up by 4 so that the code lands in its top byte: byte 3 of
+// 16 |pattern| + 2^24 - 1 - 2^8 k is the rounded magnitude code (|v| < 2^8
+// keeps it below 0x78), and the sign is merged from v.
+template <int kFp8>
+__device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t (&rw)[8],
+                                         const uint8_t* __restrict__ wtile, int row, int jl, int64_t l, int32_t d,
+                                         int j0, float lrs, void* __restrict__ Wglob) {
+  float wv[16];
+  if (kFp8) {
+    const uint4 x = *reinterpret_cast<const uint4*>(wtile + row * 128 + (((jl >> 4) ^ (row & 7)) << 4));
+    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float f4[4];
+      e4m3x4_to_f32(xw[e], f4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) wv[4 * e + i] = f4[i];
+    }
+  } else {
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int c16 = ((jl & 63) >> 3) + v;
+      const uint4 x = *reinterpret_cast<const uint4*>(wtile + (jl >> 6) * kBox + row * 128 + ((c16 ^ (row & 7)) << 4));
+      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        wv[8 * v + 2 * e] = __uint_as_float(xw[e] << 16);
+        wv[8 * v + 2 * e + 1] = __uint_as_float(xw[e] & 0xFFFF0000u);
+      }
+    }
+  }
+  float vv[16];
+  float probe = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
+    probe = __fmaf_rn(vv[i], kFp8 ? 0x1p120f : 2.0f, probe);
+  }
+  const bool fast = fabsf(probe) < INFINITY;
+  uint32_t wnew[8];
+  if (fast) {
+    if (kFp8) {
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        // 2^24 - 1 - 2^8 k for the four draws: bytes (0xFF, ~k lo, ~k hi, 0)
+        const uint32_t a0 = ~rw[2 * q4], a1 = ~rw[2 * q4 + 1];
+        const uint32_t radd[4] = {__byte_perm(a0, 0xFFu, 0x5104), __byte_perm(a0, 0xFFu, 0x5324),
+                                  __byte_perm(a1, 0xFFu, 0x5104), __byte_perm(a1, 0xFFu, 0x5324)};
+        uint32_t t[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float s = mul_rp(fabsf(vv[4 * q4 + e]), 0x1p-120f);
+          const uint32_t m = __float_as_uint(s) * 16u + radd[e];
+          t[e] = (m & 0x7FFFFFFFu) | (__float_as_uint(vv[4 * q4 + e]) & 0x80000000u);
+        }
+        wnew[q4] = __byte_perm(__byte_perm(t[0], t[1], 0x0073), __byte_perm(t[2], t[3], 0x0073), 0x5410);
+      }
+    } else {
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        uint32_t o;   // element 2p (low half) takes the low 16 random bits, 2p + 1 the high
+        asm("cvt.rs.bf16x2.f32 %0, %1, %2, %3;" : "=r"(o) : "f"(vv[2 * p + 1]), "f"(vv[2 * p]), "r"(~rw[p]));
+        wnew[p] = o;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      if (kFp8) {
+        if (p < 4) {
+          const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
+          const float o0 = sr_e4m3_value(vv[4 * p], w0 & 0xFFFFu), o1 = sr_e4m3_value(vv[4 * p + 1], w0 >> 16);
+          const float o2 = sr_e4m3_value(vv[4 * p + 2], w1 & 0xFFFFu), o3 = sr_e4m3_value(vv[4 * p + 3], w1 >> 16);
+          wnew[p] = pack_e4m3x2(o1, o0) | (pack_e4m3x2(o3, o2) << 16);
+        }
+      } else {
+        wnew[p] = (uint32_t)sr_bf16(vv[2 * p], rw[p] & 0xFFFFu) | ((uint32_t)sr_bf16(vv[2 * p + 1], rw[p] >> 16) << 16);
+      }
+    }
+  }
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(Wglob) + ((size_t)l * d + j0) * (kFp8 ? 1 : 2));
+  dst[0] = make_uint4(wnew[0], wnew[1], wnew[2], wnew[3]);
+  if (!kFp8) dst[1] = make_uint4(wnew[4], wnew[5], wnew[6], wnew[7]);
+}
+
+}  // namespace
+}  // namespace elmo

@@ -1,0 +1,598 @@
+// step_fused.cu -- the whole training step of a head in one persistent launch.
+//
+// "ELMO: Efficiency via Low-precision and Peak Memory Optimization in Large
+// Output Spaces", atlas summary "Approach": per label chunk the classifier
+// gradient is computed inside the momentum-free SGD update, applied with
+// stochastic rounding, and the label axis is processed chunk by chunk so that
+// the transient memory stays small.
+//
+// One CTA per SM, launched cooperatively so that every CTA is resident.  The
+// CTAs split into two roles that run at the same time on different SMs:
+//
+//   role A (the first nA CTAs): Z = X W_tile^T and G = sigmoid(Z) - Y for
+//     128-label tiles t = a, a + nA, ...: X stays in TMEM as the MMA's A
+//     operand, 64-label W k-blocks stream through a 16-stage TMA ring, and the
+//     16 epilogue warps write G (the next contractions' operand, sample-major)
+//     into slot t % R of a ring of R tiles in global memory, then publish
+//     ready[slot] = t / R + 1;
+//   role B (the other CTAs, nG groups x nD d-slices): the CTA of group g and
+//     slice s runs the units (t, s) for t = g, g + nG, ...: it waits for
+//     ready, copies G_t into shared memory (and counts itself in consumed[slot],
+//     which role A waits on before it reuses the slot), and issues
+//       dX^T[slice] += W_t[:, slice]^T G_t^T   (old W; TMEM-resident for the
+//                                              whole launch, one flush at the end)
+//       dW = G_t^T X[:, slice]                 (TMEM, never stored)
+//     while its 16 epilogue warps apply W = SR(W - lr dW) in place.
+//
+// Role A's tensor work and W stream overlap role B's SR epilogue (issue-bound)
+// across the GPU; W is read from HBM once, by role A, and role B finds its
+// slice in L2 shortly after (the ring keeps role A at most R tiles ahead); G
+// lives only in the R-tile ring.  The split nA : nB follows the two roles'
+// work per tile.  Every wait is bounded; a wait that runs out records
+// ELMO_ETIMEOUT in the status word, and the other CTAs stop at their next wait.
+//
+// Used for E4M3 heads with B <= 256 and bf16 heads with B <= 128, d <= 768,
+// d a multiple of 64 (X fits the 384 TMEM columns below role A's
+// accumulators); other shapes run the range-by-range kernels of step_tc.cu.
+#include <stdlib.h>
+
+#include <utility>
+
+#include "step_common.cuh"
+
+namespace elmo {
+namespace {
+
+constexpr int kFThreads = 576;              // warp 0 TMA, warp 1 MMA + TMEM, warps 2-17 epilogue
+constexpr int kFEpi = 16;
+constexpr int kFStagesA = 16;               // role A: W k-block ring
+constexpr int kFN = 64;                     // role A: labels per MMA tile
+constexpr uint32_t kFBoxA = kFN * 128;      // one W k-block: 64 labels x 128 bytes
+constexpr uint32_t kFAcc = 384;             // role A: first accumulator column (X below it)
+constexpr int kFGSlots = 3;                 // role B: G tiles in shared memory
+constexpr uint32_t kFGSlotBytes = 2 * kBox; // one G tile: 128 labels x up to 256 samples (E4M3) or 128 (bf16)
+constexpr uint32_t kFXBytes = 2 * 32768;    // role B: X[:, slice]
+constexpr uint32_t kFWBytes = 4 * kBox;     // role B: W slots (E4M3 4 x 16 KB, bf16 2 x 32 KB)
+
+struct SmemFA {
+  uint64_t wfull[kFStagesA], wempty[kFStagesA], tfull[2], tempty[2];
+  uint64_t xready;
+  uint64_t pmask[kFEpi][32];   // per epilogue warp: its 32 samples' positives among its labels
+  int arrivals[4];             // epilogue warps done with a tile's G (by local tile index mod 4)
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct SmemFB {
+  uint64_t xfull, dxfull;
+  uint64_t wfull[4], wempty[4];
+  uint64_t gfull[kFGSlots], gempty[kFGSlots];
+  uint64_t dwfull[2], dwempty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemF = 1024 + kFXBytes + kFWBytes + kFGSlots * kFGSlotBytes + 1024;
+static_assert(kSmemF <= 232448, "fused step shared memory");
+static_assert(kFStagesA * kFBoxA + sizeof(SmemFA) + 1024 <= kSmemF, "role A layout");
+static_assert(sizeof(SmemFB) <= 1024, "role B barriers");
+
+__device__ __forceinline__ int32_t ld_acquire(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int32_t* p, int32_t v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_release_add(int32_t* p, int32_t v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// orders this thread's generic-proxy accesses of global memory with later
+// async-proxy (TMA, bulk copy) accesses, and the other way round
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *flag >= target (acquire).  Gives up when `abort` is set,
+// when another CTA has recorded a timeout, or after `limit` clock cycles.
+__device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t target, volatile int* abort,
+                                          const int32_t* status, long long limit) {
+  if (ld_acquire(flag) >= target) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire(flag) >= target) return true;
+    if (*abort || *reinterpret_cast<const volatile int32_t*>(status) == (int32_t)ELMO_ETIMEOUT) return false;
+    if (clock64() - t0 > limit) return false;
+  }
+}
+
+template <int kFp8, int kG5>
+__global__ void __launch_bounds__(kFThreads, 1)
+    step_fused(const __grid_constant__ CUtensorMap tmWa, const __grid_constant__ CUtensorMap tmWb,
+               const __grid_constant__ CUtensorMap tmX, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
+               int32_t Bp, const uint8_t* __restrict__ xop, const uint32_t* __restrict__ keys,
+               const int32_t* __restrict__ tile_ptr, const float* __restrict__ xscale, uint8_t* __restrict__ gring,
+               int32_t R, int32_t* __restrict__ ready, int32_t* __restrict__ consumed, int32_t nA, int32_t nG,
+               float lr, uint64_t seed, uint64_t step, uint64_t blk_base, float* __restrict__ dX,
+               int32_t* __restrict__ status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = (int)((L + 127) / 128);                       // 128-label tiles of the head
+  const int nD = (d + 127) / 128;                             // 128-column d-slices
+  constexpr int kEl = kFp8 ? 1 : 2;
+  const size_t tile_bytes = (size_t)128 * Bp * kEl;           // one G tile in the ring
+
+  if ((int)blockIdx.x < nA) {
+    // ======================================================== role A
+    uint8_t* ring = base;
+    SmemFA* S = reinterpret_cast<SmemFA*>(base + kFStagesA * kFBoxA);
+    volatile int* abort = &S->abort;
+    const int a = blockIdx.x;
+    const int kbe = kFp8 ? 128 : 64;                          // elements of one 128-byte k-block
+    const int nkb = (d + kbe - 1) / kbe;
+    const uint32_t opcols = (uint32_t)nkb * 32;               // TMEM columns of one M-block of X
+    const int nmb = (Bp + 127) / 128;                         // M-blocks of samples: 1 or 2
+    if (threadIdx.x == 0) {
+      for (int s = 0; s < kFStagesA; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
+      for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], nmb == 2 ? 8 : kFEpi); }
+      mbar_init(&S->xready, kFEpi);
+      for (int i = 0; i < 4; ++i) S->arrivals[i] = 0;
+      S->abort = 0;
+      fence_barrier_init();
+    }
+    if (warp == 1) { tmem_alloc(&S->tmem_base, 512); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S->tmem_base;
+
+    if (warp >= 2) {
+      // X into TMEM: sample h*128 + r of M-block h in lane r, columns h*opcols ...
+      const int q = warp & 3, h = (warp - 2) >> 2;
+      if (h < nmb) {
+        const int b = h * 128 + q * 32 + lane;
+        const size_t rowbytes = (size_t)d * kEl;
+        // E4M3: xop holds the codes by 16-byte column chunk (chunk c of row b at
+        // (c * 256 + b) * 16); bf16: xop is X itself, row-major
+        const uint8_t* src = kFp8 ? xop + (size_t)b * 16 : xop + (size_t)b * rowbytes;
+        for (uint32_t c0 = 0; c0 < opcols; c0 += 64) {
+          uint32_t v[2][32];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const size_t off = (size_t)(c0 + 4 * u) * 4;
+            uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
+            if (b < B && off < rowbytes)
+              w4 = *reinterpret_cast<const uint4*>(kFp8 ? src + (off >> 4) * (ELMO_MAX_BATCH * 16) : src + off);
+            v[u >> 3][4 * (u & 7)] = w4.x; v[u >> 3][4 * (u & 7) + 1] = w4.y;
+            v[u >> 3][4 * (u & 7) + 2] = w4.z; v[u >> 3][4 * (u & 7) + 3] = w4.w;
+          }
+          tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)h * opcols + c0, v[0]);
+          if (c0 + 32 < opcols) tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)h * opcols + c0 + 32, v[1]);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S->xready);
+    }
+
+    if (warp == 0) {
+      if (elect_one()) {
+        tma_prefetch_desc(&tmWa);
+        uint32_t it = 0;
+        for (int t = a; t < T && !*abort; t += nA) {
+          for (int hf = 0; hf < 2; ++hf) {
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+              const int s = (int)(it % kFStagesA);
+              const uint32_t ph = (it / kFStagesA) & 1;
+              if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 81); break; }
+              mbar_arrive_expect_tx(&S->wfull[s], kFBoxA);
+              tma_load_2d(ring + s * kFBoxA, &tmWa, &S->wfull[s], kb * kbe, t * 128 + hf * kFN);
+            }
+          }
+        }
+      }
+    } else if (warp == 1) {
+      if (elect_one()) {
+        const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, kFN) : make_idesc(1, 1, 0, 0, 128, kFN);
+        uint32_t it = 0, u = 0;
+        if (!mbar_wait(&S->xready, 0, abort, kWaitCycles)) record_timeout(status, abort, 82);
+        tc_fence_after();
+        for (int t = a; t < T && !*abort; t += nA) {
+          for (int hf = 0; hf < 2 && !*abort; ++hf) {
+            for (int mb = 0; mb < nmb && !*abort; ++mb, ++u) {
+              const uint32_t slot = u & 1, ph = (u >> 1) & 1;
+              if (!mbar_wait(&S->tempty[slot], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 83); break; }
+              tc_fence_after();
+              const uint32_t dcol = tmem + kFAcc + slot * kFN;
+              for (int kb = 0; kb < nkb; ++kb) {
+                const uint32_t its = it + (uint32_t)kb;
+                const int s = (int)(its % kFStagesA);
+                if (mb == 0) {
+                  if (!mbar_wait(&S->wfull[s], (its / kFStagesA) & 1, abort, kWaitCycles)) {
+                    record_timeout(status, abort, 84);
+                    break;
+                  }
+                  tc_fence_after();
+                }
+                const uint32_t bsm = smem_u32(ring + s * kFBoxA);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const uint32_t aa = tmem + (uint32_t)mb * opcols + (uint32_t)kb * 32 + (uint32_t)k * 8;
+                  const uint64_t bd = sw128_desc(bsm + k * 32, 16, 1024);
+                  if (kFp8) mma_e4m3_ts(dcol, aa, bd, idesc, (kb | k) != 0);
+                  else mma_bf16_ts(dcol, aa, bd, idesc, (kb | k) != 0);
+                }
+                if (mb == nmb - 1) mma_commit(&S->wempty[s]);
+              }
+              mma_commit(&S->tfull[slot]);
+            }
+            it += (uint32_t)nkb;
+          }
+        }
+      }
+    } else {
+      // Epilogue: warp (q = warp % 4, h = (warp - 2) / 4).  Two M-blocks: warp
+      // h takes M-block h / 2, label columns 32 (h % 2) .. +31 of each 64-label
+      // half-tile; one M-block: label columns 16 h .. 16 h + 15.
+      const int q = warp & 3, h = (warp - 2) >> 2;
+      const int mb = nmb == 2 ? h >> 1 : 0;
+      const int c_lo = nmb == 2 ? 32 * (h & 1) : 16 * h;
+      const int ncol = nmb == 2 ? 32 : 16;
+      const int b = mb * 128 + q * 32 + lane;                // sample
+      const bool bvalid = b < B;
+      const bool bstore = b < Bp;
+      const float inv_sx = kFp8 ? xscale[1] : 1.0f;
+      constexpr int kG = kFp8 ? (kG5 ? 2 : 1) : 0;
+      constexpr int kChunk = 16 / kEl;                        // labels per 16-byte chunk
+      constexpr int kNlc = 128 / kChunk;                      // chunks per 128-label tile
+      unsigned long long* wm = reinterpret_cast<unsigned long long*>(S->pmask[warp - 2]);
+      uint32_t use = 0;
+      int lt = 0;
+      for (int t = a; t < T && !*abort; t += nA, ++lt) {
+        const int slot = t % R, round = t / R;
+        uint8_t* gtile = gring + (size_t)slot * tile_bytes;
+        // the slot is free once every d-slice's CTA has copied the tile it held
+        if (round > 0) {
+          bool ok = true;
+          if (lane == 0) ok = wait_flag(consumed + slot, nD * round, abort, status, kWaitCycles);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) { if (lane == 0) record_timeout(status, abort, 85); break; }
+        }
+        bool stop = false;
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t uu = nmb == 2 ? 2 * use + (uint32_t)mb : use;   // this thread's use of the slots
+          ++use;
+          const uint32_t buf = uu & 1;
+          if (!mbar_wait(&S->tfull[buf], (uu >> 1) & 1, abort, kWaitCycles)) {
+            record_timeout(status, abort, 86);
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          uint32_t v[32];
+          const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + kFAcc + buf * kFN + (uint32_t)c_lo;
+          if (ncol == 32) tmem_ld32(taddr, v);
+          else tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(v));
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S->tempty[buf]);
+          // positives of sample b among labels lc0 .. lc0 + ncol - 1, from the
+          // keys of their 128-label tile: the warp reads the keys together (a
+          // frequent label's tile holds hundreds) and scatters each into the
+          // mask of its sample when that sample is one of the warp's
+          const int64_t lc0 = (int64_t)t * 128 + hf * kFN + c_lo;
+          uint64_t pm;
+          {
+            const int k0 = __ldg(tile_ptr + t);
+            const int k1 = __ldg(tile_ptr + t + 1);
+            wm[lane] = 0;
+            __syncwarp();
+            const int wb = b - lane;
+            for (int i = k0 + lane; i < k1; i += 32) {
+              const uint32_t key = __ldg(keys + i);
+              const int sb = (int)(key & 0xFFu) - wb;
+              const int64_t dl = (int64_t)(key >> 8) - lc0;
+              if (sb >= 0 && sb < 32 && dl >= 0 && dl < ncol) atomicOr(wm + sb, 1ull << dl);
+            }
+            __syncwarp();
+            pm = wm[lane];
+            __syncwarp();
+          }
+          const int lt0 = hf * kFN + c_lo;                      // first label column within the tile
+#pragma unroll
+          for (int j = 0; j < 32; j += 16) {
+            if (j >= ncol) break;
+            const int64_t nv = L - (lc0 + j);
+            const uint32_t vbits = !bvalid || nv <= 0 ? 0u : (nv >= 16 ? 0xFFFFu : (1u << nv) - 1u);
+            uint32_t pk[8];
+            grad_codes16<kG>(v + j, inv_sx, (uint32_t)(pm >> j) & 0xFFFFu, vbits, pk);
+            if (bstore) {
+              const int lc = (lt0 + j) / kChunk;
+              *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =
+                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              if (!kFp8)
+                *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc + 1) * 128 + (b & 7) * 16) =
+                    make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+        }
+        if (stop) break;
+        // publish the tile once all 16 epilogue warps have stored their parts:
+        // each thread orders its stores (and, for the bulk copies that read
+        // them, the async proxy) before its warp's arrival; the last warp to
+        // arrive releases the flag
+        fence_proxy_async_global();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+          const int old = atomicAdd(&S->arrivals[lt & 3], 1);
+          if (old == kFEpi - 1) {
+            S->arrivals[lt & 3] = 0;
+            __threadfence();
+            st_release(ready + slot, round + 1);
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (*abort) __nanosleep(20000);   // let copies in flight land before the shared memory goes away
+    if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+    return;
+  }
+
+  // ========================================================== role B
+  const int bid = (int)blockIdx.x - nA;
+  const int g = bid / nD, sl = bid % nD;
+  if (g >= nG) return;                                        // spare CTA
+  constexpr int kWS = kFp8 ? 4 : 2;
+  constexpr uint32_t kWSB = kFp8 ? kBox : 2 * kBox;
+  constexpr int kBoxCols = 128 / kEl;                         // elements per 128-byte box row
+  constexpr int kK = kFp8 ? 32 : 16;                          // MMA K
+  uint8_t* xs = base;
+  uint8_t* ws = xs + kFXBytes;
+  uint8_t* gs = ws + kFWBytes;
+  SmemFB* S = reinterpret_cast<SmemFB*>(gs + kFGSlots * kFGSlotBytes);
+  volatile int* abort = &S->abort;
+  const int D0 = sl * 128;
+  if (threadIdx.x == 0) {
+    mbar_init(&S->xfull, 1);
+    mbar_init(&S->dxfull, 1);
+    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kFEpi); }
+    for (int s = 0; s < kFGSlots; ++s) { mbar_init(&S->gfull[s], 1); mbar_init(&S->gempty[s], 1); }
+    for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->dwfull[b2], 1); mbar_init(&S->dwempty[b2], kFEpi); }
+    S->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(&S->tmem_base, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S->tmem_base;
+  int nb = 0;                                                 // 128-byte boxes in this slice
+  for (int qq = 0; qq < 128 / kBoxCols; ++qq) nb += (D0 + qq * kBoxCols < d);
+
+  if (warp == 0) {
+    if (elect_one()) {
+      tma_prefetch_desc(&tmWb);
+      tma_prefetch_desc(&tmX);
+      mbar_arrive_expect_tx(&S->xfull, (uint32_t)nb * (uint32_t)Bp * 128u);
+      for (int qq = 0; qq < 128 / kBoxCols; ++qq)
+        if (D0 + qq * kBoxCols < d) tma_load_2d(xs + qq * 32768, &tmX, &S->xfull, D0 + qq * kBoxCols, 0);
+      uint32_t wit = 0, git = 0;
+      for (int t = g; t < T && !*abort; t += nG) {
+        {
+          const int s = wit % kWS;
+          const uint32_t ph = (wit / kWS) & 1;
+          ++wit;
+          if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 91); break; }
+          mbar_arrive_expect_tx(&S->wfull[s], (uint32_t)nb * kBox);
+          for (int qq = 0; qq < 128 / kBoxCols; ++qq)
+            if (D0 + qq * kBoxCols < d) tma_load_2d(ws + s * kWSB + qq * kBox, &tmWb, &S->wfull[s], D0 + qq * kBoxCols, t * 128);
+        }
+        {
+          const int s = git % kFGSlots;
+          const uint32_t ph = (git / kFGSlots) & 1;
+          ++git;
+          if (!mbar_wait(&S->gempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 92); break; }
+          const int slot = t % R, round = t / R;
+          if (!wait_flag(ready + slot, round + 1, abort, status, kWaitCycles)) { record_timeout(status, abort, 93); break; }
+          fence_proxy_async_global();
+          const uint32_t bytes = (uint32_t)Bp * kEl * 128u;
+          mbar_arrive_expect_tx(&S->gfull[s], bytes);
+          bulk_load(gs + s * kFGSlotBytes, gring + (size_t)slot * tile_bytes, bytes, &S->gfull[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      const uint32_t gfmt = kG5 ? 1u : 0u;
+      // G is stored sample-major: K-major as dX^T's B operand, MN-major as dW's A operand
+      const uint32_t idesc_dw = kFp8 ? make_idesc(gfmt, 0, 1, 1, 128, 128) : make_idesc(1, 1, 1, 1, 128, 128);
+      const uint32_t idesc_dx = kFp8 ? make_idesc(0, gfmt, 1, 0, 128, (uint32_t)Bp) : make_idesc(1, 1, 1, 0, 128, (uint32_t)Bp);
+      const uint32_t gstride = (uint32_t)(kFp8 ? 8 : 16) * 128u;   // bytes between 8-sample groups
+      uint32_t wit = 0, git = 0, dwit = 0;
+      bool first = true;
+      if (!mbar_wait(&S->xfull, 0, abort, kWaitCycles)) record_timeout(status, abort, 94);
+      tc_fence_after();
+      const uint32_t xa = smem_u32(xs);
+      for (int t = g; t < T && !*abort; t += nG) {
+        const int sw = wit % kWS;
+        const uint32_t phw = (wit / kWS) & 1;
+        ++wit;
+        const uint32_t db = dwit & 1, duse = dwit >> 1;
+        ++dwit;
+        const int sg = git % kFGSlots;
+        const uint32_t phg = (git / kFGSlots) & 1;
+        ++git;
+        if (!mbar_wait(&S->wfull[sw], phw, abort, kWaitCycles)) { record_timeout(status, abort, 95); break; }
+        if (!mbar_wait(&S->dwempty[db], (duse & 1) ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 96); break; }
+        if (!mbar_wait(&S->gfull[sg], phg, abort, kWaitCycles)) { record_timeout(status, abort, 97); break; }
+        tc_fence_after();
+        // G_t is in shared memory: its ring slot may be reused
+        red_release_add(consumed + t % R, 1);
+        const uint32_t wa = smem_u32(ws + sw * kWSB);
+        const uint32_t ga = smem_u32(gs + sg * kFGSlotBytes);
+        // dX^T[slice] += W^T G^T : M = 128 (columns of d), N = Bp, K = 128 labels
+#pragma unroll 1
+        for (int k = 0; k < 128 / kK; ++k) {
+          const uint64_t ad = sw128_desc(wa + k * kK * 128, kBox, 1024);
+          const uint64_t bd = nosw_desc(ga + k * 2 * 128, 128, gstride);
+          if (kFp8) mma_e4m3(tmem, ad, bd, idesc_dx, !(first && k == 0));
+          else mma_bf16(tmem, ad, bd, idesc_dx, !(first && k == 0));
+        }
+        // dW[tile, slice] = G^T X[:, slice] : M = 128 labels, N = 128, K = Bp samples
+        const uint32_t dwcol = tmem + 256 + db * 128;
+#pragma unroll 1
+        for (int k = 0; k < Bp / kK; ++k) {
+          const uint64_t ad = nosw_desc(ga + k * (kK / 8) * gstride, gstride, 128);
+          const uint64_t bd = sw128_desc(xa + k * kK * 128, 32768, 1024);
+          if (kFp8) mma_e4m3(dwcol, ad, bd, idesc_dw, k != 0);
+          else mma_bf16(dwcol, ad, bd, idesc_dw, k != 0);
+        }
+        mma_commit(&S->gempty[sg]);
+        mma_commit(&S->dwfull[db]);
+        first = false;
+      }
+      mma_commit(&S->dxfull);
+    }
+  } else {
+    const int q = warp & 3;
+    const int sub = (warp - 2) >> 2;                // columns sub * 32 .. +31 of the slice
+    const int row = q * 32 + lane;                  // label row of dW; column of d for dX^T
+    const float lrs = kFp8 ? lr * (0.00390625f * xscale[1]) : lr;
+    const float dx_scale = kFp8 ? 0.00390625f : 1.0f;
+    uint32_t wit = 0, dwit = 0;
+    bool any = false;
+    for (int t = g; t < T && !*abort; t += nG) {
+      any = true;
+      const int sw = wit % kWS;
+      ++wit;
+      const uint32_t db = dwit & 1, duse = dwit >> 1;
+      ++dwit;
+      const int64_t l = (int64_t)t * 128 + row;
+      const int jl = sub * 32;                      // columns jl .. jl + 31 of the 128-column slice
+      const int j0 = D0 + jl;
+      const bool valid = l < L && j0 < d;           // d is a multiple of 64: both groups or none
+      // the draws do not depend on the gradient: form them while the MMAs run
+      uint32_t rw0[8], rw1[8];
+      if (valid) {
+        sr_draws16(seed, step, blk_base, l, d, j0, rw0);
+        sr_draws16(seed, step, blk_base, l, d, j0 + 16, rw1);
+      }
+      if (!mbar_wait(&S->dwfull[db], duse & 1, abort, kWaitCycles)) { record_timeout(status, abort, 98); break; }
+      tc_fence_after();
+      const uint8_t* wrow = ws + sw * kWSB;
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + 256 + db * 128 + jl;
+      uint32_t r0[16], r1[16];
+      tmem_ld16(taddr, r0);
+      tmem_wait_ld();
+      tmem_ld16(taddr + 16, r1);
+      if (valid) update16<kFp8>(r0, rw0, wrow, row, jl, l, d, j0, lrs, Wglob);
+      tmem_wait_ld();
+      if (valid) update16<kFp8>(r1, rw1, wrow, row, jl + 16, l, d, j0 + 16, lrs, Wglob);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) { mbar_arrive(&S->dwempty[db]); mbar_arrive(&S->wempty[sw]); }
+    }
+    if (any && !*abort) {
+      // flush dX^T of this CTA: lane = column j of the slice, TMEM columns = samples
+      if (!mbar_wait(&S->dxfull, 0, abort, kWaitCycles)) {
+        record_timeout(status, abort, 99);
+      } else {
+        tc_fence_after();
+        const int j = D0 + row;
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
+        for (int c = sub; c < Bp / 32; c += 4) {
+          uint32_t ra[32];
+          tmem_ld32(taddr + c * 32, ra);
+          tmem_wait_ld();
+          if (j < d) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int bb = c * 32 + i;
+              if (bb < B) atomicAdd(dX + (size_t)bb * d + j, __uint_as_float(ra[i]) * dx_scale);
+            }
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (*abort) __nanosleep(20000);
+  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+}
+
+}  // namespace
+
+bool fused_step_supported(const elmo_head* h, int32_t B) {
+  const char* v = getenv("ELMO_STEP_FUSED");
+  if (v && v[0] == '0') return false;
+  const bool fp8 = h->dt == ELMO_FP8_E4M3;
+  const int32_t Bp = padded_batch(B, fp8);
+  return h->d % 64 == 0 && h->d <= 768 && (fp8 ? Bp <= 256 : Bp <= 128);
+}
+
+// Work of one 128-label tile in each role, in the units of the split: role A
+// (Z for the tile, G) against role B (dX^T and dW for every d-slice, and the
+// SR update of every weight, which the epilogue's instruction issue bounds).
+// Measured on B200 for the workloads' shapes; ELMO_FUSED_A overrides nA.
+void fused_split(int grid, int nD, int T, int* nA, int* nG) {
+  int a = (grid * 27 + 50) / 100;                   // about 27 % of the SMs form G
+  const char* v = getenv("ELMO_FUSED_A");
+  if (v && atoi(v) > 0) a = atoi(v);
+  if (a > grid - nD) a = grid - nD;
+  if (a < 1) a = 1;
+  int gg = (grid - a) / nD;
+  if (gg > T) gg = T;
+  if (a > T) a = T;
+  *nA = a;
+  *nG = gg;
+}
+
+cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float lr, uint64_t seed, uint64_t step,
+                              float* dX, cudaStream_t s) {
+  const bool fp8 = h->dt == ELMO_FP8_E4M3;
+  const int eb = fp8 ? 1 : 2;
+  const int32_t Bp = padded_batch(B, fp8);
+  const int T = (int)((h->L + 127) / 128);
+  const int nD = (h->d + 127) / 128;
+  int nA = 0, nG = 0;
+  fused_split(h->num_sms, nD, T, &nA, &nG);
+  const int grid = nA + nG * nD;
+  CUtensorMap tmWa, tmWb, tmX;
+  cudaError_t e = make_tma_map_2d(&tmWa, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, kFN);
+  if (e != cudaSuccess) return e;
+  e = make_tma_map_2d(&tmWb, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, 128);
+  if (e != cudaSuccess) return e;
+  e = make_tma_map_2d(&tmX, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
+                      (uint64_t)B, (uint64_t)h->d, (uint32_t)Bp);
+  if (e != cudaSuccess) return e;
+  auto kern = fp8 ? (h->g_e5m2 ? step_fused<1, 1> : step_fused<1, 0>) : step_fused<0, 0>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemF);
+  if (e != cudaSuccess) return e;
+  // the ring's flags start at zero every step
+  e = cudaMemsetAsync(h->ring_flags, 0, sizeof(int32_t) * 2 * (size_t)h->ring_tiles, s);
+  if (e != cudaSuccess) return e;
+  const uint8_t* xop = fp8 ? h->xqt : reinterpret_cast<const uint8_t*>(X);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)kFThreads);
+  cfg.dynamicSmemBytes = kSmemF;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: the roles wait on one another
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmWa, tmWb, tmX, h->W, h->L, h->d, B, Bp, xop, (const uint32_t*)h->keys,
+                            (const int32_t*)h->tile_ptr, (const float*)h->xscale, static_cast<uint8_t*>(h->ring),
+                            h->ring_tiles, h->ring_flags, h->ring_flags + h->ring_tiles, nA, nG, lr, seed, step,
+                            (uint64_t)h->label_base * (uint64_t)h->d / 8, dX, h->status);
+}
+
+}  // namespace elmo

@@ -42,247 +42,10 @@
 
 #include <utility>
 
-#include "elmo_common.cuh"
-#include "elmo_internal.h"
-#include "tc_ptx.cuh"
+#include "step_common.cuh"
 
 namespace elmo {
 namespace {
-
-using namespace tc;
-
-constexpr int kThreads = 576;                    // 18 warps: TMA, MMA, 16 epilogue
-constexpr int kEpiWarps = 16;
-constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 2 GHz: only a broken pipeline waits this long
-constexpr uint32_t kBox = 16384;                  // one 128-row x 128-byte TMA box
-
-__device__ __forceinline__ void record_timeout(int32_t* status, volatile int* abort, int site) {
-  *abort = 1;
-  if (atomicCAS(status, 0, (int)ELMO_ETIMEOUT) == 0) status[1] = site;
-}
-
-// Positives of label `l` among the sorted keys (label << 8 | sample) in
-// [k0, k1): a 256-bit sample mask.
-__device__ __forceinline__ void label_mask(const uint32_t* __restrict__ keys, int k0, int k1, int64_t l,
-                                           uint32_t (&m)[8]) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = 0;
-  for (int i = k0; i < k1; ++i) {
-    const uint32_t key = __ldg(keys + i);
-    if ((int64_t)(key >> 8) == l) {
-      const uint32_t b = key & 0xFFu;
-#pragma unroll
-      for (int w = 0; w < 8; ++w)
-        if ((b >> 5) == (uint32_t)w) m[w] |= 1u << (b & 31);
-    }
-  }
-}
-
-
-__device__ __forceinline__ float exp2f_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float rcpf_approx(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-// fp32 multiply that keeps denormal inputs and results whatever -ftz says
-__device__ __forceinline__ float mul_rn_denorm(float a, float b) {
-  float y;
-  asm("mul.rn.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
-  return y;
-}
-__device__ __forceinline__ float tanhf_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// ---------------------------------------------------------------- epilogue pieces
-// G = sigmoid(Z) - Y for 16 samples b0 .. b0+15 of one label row, written as
-// the next contraction's operand (bf16, or E4M3 of 2^8 G); padded samples get 0.
-// z = acc / s_X.  The special-function unit (16 results per clock per SM) is
-// the epilogue's narrowest pipe, so each form uses as few of its ops as its
-// operand precision allows:
-//   bf16: sigmoid(z) = 1 / (1 + 2^(-z log2 e)), an ex2 and a rcp, both to
-//         about 2^-22 relative, far below the bf16 rounding of G;
-//   E4M3: 2^8 sigmoid(z) = 2^7 + 2^7 tanh(z / 2), a single tanh.  Its
-//         relative error of about 2^-11 is an absolute error of at most 2^-4
-//         in units of 2^8 G, below half the E4M3 spacing (2^-3 or more)
-//         wherever 2^8 |G| >= 1; only the codes of negatives with
-//         sigmoid(z) < 2^-8 (z < -5.5) can move by more than one step.
-// `zmul` is -log2(e) / s_X (bf16) or 1 / (2 s_X) (E4M3).
-template <int kFp8, int kG5 = 0>
-__device__ __forceinline__ void grad16(const uint32_t* r, float zmul, float inv_sx, uint32_t ybits,
-                                       int b0, int B, uint8_t* __restrict__ gtile, int row, bool row_invalid,
-                                       float* __restrict__ Zrow, float* __restrict__ Grow) {
-  constexpr float gscale = kFp8 ? 256.0f : 1.0f;
-  float g[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if (kFp8) {
-      g[i] = __fmaf_rn(tanhf_approx(__fmul_rn(__uint_as_float(r[i]), zmul)), 128.0f, 128.0f);
-    } else {
-      const float e = exp2f_approx(__fmul_rn(__uint_as_float(r[i]), zmul));
-      g[i] = rcpf_approx(__fadd_rn(e, 1.0f));
-    }
-  }
-  if (ybits) {                        // positives are rare: subtract y where set
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if ((ybits >> i) & 1u) g[i] -= gscale;
-  }
-  if (b0 + 16 > B || row_invalid) {  // batch padding, and label rows past the range (their G
-#pragma unroll                        // must be 0: kernel B reads whole tiles)
-    for (int i = 0; i < 16; ++i)
-      if (b0 + i >= B || row_invalid) g[i] = 0.0f;
-  }
-  uint32_t packed[8];
-  if (kFp8) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      packed[i] = kG5 ? pack_e5m2x2(g[4 * i + 1], g[4 * i]) | (pack_e5m2x2(g[4 * i + 3], g[4 * i + 2]) << 16)
-                      : pack_e4m3x2(g[4 * i + 1], g[4 * i]) | (pack_e4m3x2(g[4 * i + 3], g[4 * i + 2]) << 16);
-    const int j = b0 >> 4;                                   // 16-byte chunk of samples
-    *reinterpret_cast<uint4*>(gtile + ((j * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
-        make_uint4(packed[0], packed[1], packed[2], packed[3]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(g[2 * i + 1], g[2 * i]);
-    const int j = b0 >> 3;                                   // first of two 16-byte chunks
-    *reinterpret_cast<uint4*>(gtile + ((j * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
-        make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    *reinterpret_cast<uint4*>(gtile + (((j + 1) * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
-        make_uint4(packed[4], packed[5], packed[6], packed[7]);
-  }
-  if (Grow && !row_invalid) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (b0 + i < B)
-        Grow[i] = kFp8 ? (kG5 ? e5m2_to_f32((uint8_t)(packed[i >> 2] >> (8 * (i & 3))))
-                              : e4m3_to_f32((uint8_t)(packed[i >> 2] >> (8 * (i & 3))))) * 0.00390625f
-                       : bf16_to_f32((uint16_t)(packed[i >> 1] >> (16 * (i & 1))));
-  }
-  if (Zrow && !row_invalid) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (b0 + i < B) Zrow[i] = __fmul_rn(__uint_as_float(r[i]), inv_sx);
-  }
-}
-
-// Positive-label bits of samples b0 .. b0+15 from the 256-bit mask.
-__device__ __forceinline__ uint32_t mask16(const uint32_t (&m)[8], int b0) {
-  uint32_t w = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) w = ((b0 >> 5) == i) ? m[i] : w;
-  return (w >> (b0 & 16)) & 0xFFFFu;
-}
-
-// W[l, j0 .. j0+15] = SR(W - lrs * acc) for one label row: old weights from the
-// 128B-swizzled W tile in shared memory (row `row`, tile column jl), draws from
-// the two Philox blocks of elements l*d + j0 .. +15 (blk_base more blocks in
-// when this head holds the rows of a larger head from label_base on:
-// blk_base = label_base * d / 8).
-template <int kFp8>
-__device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint8_t* __restrict__ wtile, int row, int jl,
-                                         int64_t l, int32_t d, int j0, float lrs, uint64_t seed, uint64_t step,
-                                         uint64_t blk_base, void* __restrict__ Wglob) {
-  float wv[16];
-  if (kFp8) {
-    const uint4 x = *reinterpret_cast<const uint4*>(wtile + row * 128 + (((jl >> 4) ^ (row & 7)) << 4));
-    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float f4[4];
-      e4m3x4_to_f32(xw[e], f4);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) wv[4 * e + i] = f4[i];
-    }
-  } else {
-#pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const int c16 = ((jl & 63) >> 3) + v;
-      const uint4 x = *reinterpret_cast<const uint4*>(wtile + (jl >> 6) * kBox + row * 128 + ((c16 ^ (row & 7)) << 4));
-      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        wv[8 * v + 2 * e] = __uint_as_float(xw[e] << 16);
-        wv[8 * v + 2 * e + 1] = __uint_as_float(xw[e] & 0xFFFF0000u);
-      }
-    }
-  }
-  // v = w - lr dW, and a probe that is not finite when some v is NaN or
-  // infinite (E4M3: the sum of 0 v; bf16: the sum of 2 v, which also overflows
-  // when some |v| >= 2^127, where rounding could pass the largest finite
-  // value); such groups take the exact per-element path
-  float vv[16];
-  float probe = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
-    probe = __fmaf_rn(vv[i], kFp8 ? 0.0f : 2.0f, probe);
-  }
-  const uint64_t blk = blk_base + (((uint64_t)l * (uint64_t)d + (uint64_t)j0) >> 3);
-  const u32x4 r0 = sr_block(seed, step, blk), r1 = sr_block(seed, step, blk + 1);
-  const uint32_t rw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-  uint32_t wnew[8];
-  if (fabsf(probe) < INFINITY) {
-    if (kFp8) {
-      // Scaled by 2^-120, the E4M3 grid is fp32's own grid cut to 3 mantissa
-      // bits: E4M3's subnormal spacing 2^-9 becomes 2^-129 = 2^20 units of
-      // fp32's denormal spacing 2^-149, and its normal range starts at 2^-126,
-      // fp32's.  So one add-and-truncate at 20 bits on the signed pattern rounds
-      // every magnitude (the carry runs into the exponent where it should).
-      // The scaling is exact for |v| >= 2^-6; below, it rounds v to a multiple
-      // of 2^-29, which changes the decision u < f only when f 2^16 lies less
-      // than 2^-5 above an integer equal to the draw (about 2^-21 of the
-      // elements there).  The elmo_sr_round kernel keeps the exact form.
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        float o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t word = rw[2 * q4 + (e >> 1)];
-          const uint32_t k16 = (e & 1) ? __umulhi(word, 0x10000u) : (word & 0xFFFFu);
-          const uint32_t radd = 0xFFFFFu - k16 * 16u;          // 2^20 - 1 - 16 k
-          const float vs = mul_rn_denorm(vv[4 * q4 + e], 0x1p-120f);
-          const uint32_t t = (__float_as_uint(vs) + radd) & 0xFFF00000u;
-          o[e] = mul_rn_denorm(__uint_as_float(t), 0x1p120f);
-        }
-        wnew[q4] = pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16);
-      }
-    } else {
-      // add-and-truncate at 16 bits directly on the signed patterns
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const uint32_t word = rw[p];
-        const uint32_t t0 = __float_as_uint(vv[2 * p]) + (0xFFFFu - (word & 0xFFFFu));
-        const uint32_t t1 = __float_as_uint(vv[2 * p + 1]) + (0xFFFFu - (word >> 16));
-        wnew[p] = __byte_perm(t0, t1, 0x7632);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      if (kFp8) {
-        if (p < 4) {
-          const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
-          const float o0 = sr_e4m3_value(vv[4 * p], w0 & 0xFFFFu), o1 = sr_e4m3_value(vv[4 * p + 1], w0 >> 16);
-          const float o2 = sr_e4m3_value(vv[4 * p + 2], w1 & 0xFFFFu), o3 = sr_e4m3_value(vv[4 * p + 3], w1 >> 16);
-          wnew[p] = pack_e4m3x2(o1, o0) | (pack_e4m3x2(o3, o2) << 16);
-        }
-      } else {
-        wnew[p] = (uint32_t)sr_bf16(vv[2 * p], rw[p] & 0xFFFFu) | ((uint32_t)sr_bf16(vv[2 * p + 1], rw[p] >> 16) << 16);
-      }
-    }
-  }
-  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(Wglob) + ((size_t)l * d + j0) * (kFp8 ? 1 : 2));
-  dst[0] = make_uint4(wnew[0], wnew[1], wnew[2], wnew[3]);
-  if (!kFp8) dst[1] = make_uint4(wnew[4], wnew[5], wnew[6], wnew[7]);
-}
 
 // ============================================================================
 // Kernel A: logits and gradient operand of a label range.
@@ -378,7 +141,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const float inv_sx = kFp8 ? xscale[1] : 1.0f;
-    const float zmul = kFp8 ? 0.5f * inv_sx : -1.4426950408889634f;   // see grad16
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
       const uint32_t buf = tc & 1, use = tc >> 1;
@@ -402,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int b0 = c * 32 + k * 16;
-          grad16<kFp8, kG5>(ra + k * 16, zmul, inv_sx, mask16(mask, b0), b0, B,
+          grad16<kFp8, kG5>(ra + k * 16, inv_sx, mask16(mask, b0), b0, B,
                        static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                        Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
         }
@@ -536,7 +298,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const float inv_sx = kFp8 ? xscale[1] : 1.0f;
-    const float zmul = kFp8 ? 0.5f * inv_sx : -1.4426950408889634f;   // see grad16
     uint32_t tc = 0;
     for (int p = 0; p < npanels && !*abort; ++p) {
       for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
@@ -561,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 2; ++k) {
             const int cb = c * 32 + k * 16;             // panel column
             const int b0 = p * PN + cb;                 // sample
-            grad16<kFp8, kG5>(ra + k * 16, zmul, inv_sx, mask16(mask, b0), b0, B,
+            grad16<kFp8, kG5>(ra + k * 16, inv_sx, mask16(mask, b0), b0, B,
                          static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                          Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
           }
@@ -737,7 +498,7 @@ __global__ void __launch_bounds__(kXtThreads, 1)
     const bool bvalid = b < B;
     const bool bstore = b < Bp;
     const float inv_sx = kFp8 ? xscale[1] : 1.0f;
-    const float zmul = kFp8 ? 0.5f * inv_sx : -1.4426950408889634f;   // see grad16
+    constexpr int kG = kFp8 ? (kG5 ? 2 : 1) : 0;                 // operand format of G
     constexpr int kEl = kFp8 ? 1 : 2;
     constexpr int kChunk = 16 / kEl;                          // labels per 16-byte chunk
     constexpr int kNlc = 128 / kChunk;                        // chunks per 128-label tile
@@ -785,35 +546,18 @@ __global__ void __launch_bounds__(kXtThreads, 1)
       uint8_t* gtile = static_cast<uint8_t*>(gbuf) + (size_t)(t >> 1) * 128 * Bp * kEl;
       const int lt = (t & 1) * kXtN + c_lo;                   // first label column within the 128-label tile
       for (int j = 0; j < ncol; j += 16) {
-        float g[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float z = __uint_as_float(v[j + i]);
-          float gv;
-          if (kFp8) {
-            gv = __fmaf_rn(tanhf_approx(__fmul_rn(z, zmul)), 128.0f, 128.0f);
-            if ((pm >> (j + i)) & 1) gv -= 256.0f;
-          } else {
-            gv = rcpf_approx(__fadd_rn(exp2f_approx(__fmul_rn(z, zmul)), 1.0f));
-            if ((pm >> (j + i)) & 1) gv -= 1.0f;
-          }
-          const int64_t l = lc0 + j + i;
-          g[i] = (bvalid && l < l1) ? gv : 0.0f;
-        }
+        // valid labels of this group: those below the range end, for a real sample
+        const int64_t nv = l1 - (lc0 + j);
+        const uint32_t vbits = !bvalid || nv <= 0 ? 0u : (nv >= 16 ? 0xFFFFu : (1u << nv) - 1u);
         uint32_t pk[8];
+        grad_codes16<kG>(v + j, inv_sx, (uint32_t)(pm >> j) & 0xFFFFu, vbits, pk);
         if (kFp8) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            pk[i] = kG5 ? pack_e5m2x2(g[4 * i + 1], g[4 * i]) | (pack_e5m2x2(g[4 * i + 3], g[4 * i + 2]) << 16)
-                        : pack_e4m3x2(g[4 * i + 1], g[4 * i]) | (pack_e4m3x2(g[4 * i + 3], g[4 * i + 2]) << 16);
           if (bstore) {
             const int lc = (lt + j) / kChunk;
             *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =
                 make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(g[2 * i + 1], g[2 * i]);
           if (bstore) {
             const int lc = (lt + j) / kChunk;
             *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =
@@ -830,9 +574,8 @@ __global__ void __launch_bounds__(kXtThreads, 1)
             const size_t o = (size_t)(l - l0) * B + b;
             if (Zout) Zout[o] = __fmul_rn(__uint_as_float(v[j + i]), inv_sx);
             if (Gout)
-              Gout[o] = kFp8 ? (kG5 ? e5m2_to_f32((uint8_t)(pk[i >> 2] >> (8 * (i & 3))))
-                                    : e4m3_to_f32((uint8_t)(pk[i >> 2] >> (8 * (i & 3))))) * 0.00390625f
-                             : bf16_to_f32((uint16_t)(pk[i >> 1] >> (16 * (i & 1))));
+              Gout[o] = grad_value<kG>(kFp8 ? (pk[i >> 2] >> (8 * (i & 3))) & 0xFFu
+                                            : (pk[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
           }
         }
       }
@@ -1081,8 +824,11 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
           const int j0 = D0 + jl;
           if (!valid || j0 >= d) continue;
 #pragma unroll
-          for (int g = 0; g < kGrp; ++g)
-            update16<kFp8>(r[g], wrow, row, jl + 16 * g, l, d, j0 + 16 * g, lrs, seed, step, blk_base, Wglob);
+          for (int g = 0; g < kGrp; ++g) {
+            uint32_t rw[8];
+            sr_draws16(seed, step, blk_base, l, d, j0 + 16 * g, rw);
+            update16<kFp8>(r[g], rw, wrow, row, jl + 16 * g, l, d, j0 + 16 * g, lrs, Wglob);
+          }
         }
         tc_fence_before();
         __syncwarp();

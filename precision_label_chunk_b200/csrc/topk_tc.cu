@@ -253,10 +253,11 @@ __device__ __forceinline__ float ord_value(uint32_t k) {
 // operands take 384 of the 512 TMEM columns.
 template <int kFp8>
 __global__ void __launch_bounds__(kSThreads, 1)
-    topk_screen_tc(const __grid_constant__ CUtensorMap tmW, int64_t L, int32_t d, int32_t B, int32_t kp,
+    topk_screen_tc(const __grid_constant__ CUtensorMap tmW, int64_t lbase, int64_t L, int32_t d, int32_t B, int32_t kp,
                    int32_t ngroups, const uint8_t* __restrict__ xa, const uint8_t* __restrict__ xb,
                    const float* __restrict__ xinv, float* __restrict__ cand_s, int32_t* __restrict__ cand_i,
-                   float* __restrict__ thr, uint32_t* __restrict__ tshare, int32_t* __restrict__ status) {
+                   float* __restrict__ thr, uint32_t* __restrict__ tshare, float* __restrict__ dump,
+                   int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = base;                                                   // kSStages W k-blocks
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
           const uint32_t ph = (it / kSStages) & 1;
           if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kSWait)) { record_timeout(status, abort, 61); break; }
           mbar_arrive_expect_tx(&S->wfull[s], kSBox);
-          tma_load_2d(ring + s * kSBox, &tmW, &S->wfull[s], kb * kbe, (int32_t)(t * kN));
+          tma_load_2d(ring + s * kSBox, &tmW, &S->wfull[s], kb * kbe, (int32_t)(lbase + t * kN));
         }
       }
     }
@@ -379,6 +380,13 @@ __global__ void __launch_bounds__(kSThreads, 1)
       if (lane == 0) mbar_arrive(&S->tempty[buf]);
       if (!live) continue;
       const int64_t lb = t * kN;
+      if (dump) {   // inspection: every screening score of the range, unscaled, no selection
+        const float inv = xinv[row];
+#pragma unroll
+        for (int c = 0; c < kN; ++c)
+          if (lb + c < L) dump[(size_t)row * L + lb + c] = __fmul_rn(__uint_as_float(v[c >> 5][c & 31]), inv);
+        continue;
+      }
       float teff = fmaxf(tau, ord_value(__ldcg(tshare + row)));
       // scores above the threshold, as a bit mask (the selection code below is
       // kept out of the unrolled scan so that it exists once in the binary)
@@ -406,7 +414,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
       }
       tused = fmaxf(tused, teff);
     }
-    if (live) {
+    if (live && !dump) {
       const float inv = xinv[row];
       const size_t o = ((size_t)row * ngroups + g) * kp;
       for (int i = 0; i < kp; ++i) {
@@ -426,6 +434,30 @@ __global__ void __launch_bounds__(kSThreads, 1)
 __device__ __forceinline__ float w_at(const void* W, int dt, int64_t i) {
   return dt == ELMO_BF16 ? bf16_to_f32(static_cast<const uint16_t*>(W)[i])
                          : e4m3_to_f32(static_cast<const uint8_t*>(W)[i]);
+}
+
+// The certificate's bound on |exact chain score - screening score| of a query
+// row (any label): (gamma (n1 + r1) + r1) max|W|, rounded up, plus 2^-126 for
+// the rescaling of subnormal partial results.
+__device__ __forceinline__ float screen_bound(float gamma, float n1, float r1, float maxw) {
+  float dl = __fmul_ru(gamma, __fadd_ru(n1, r1));
+  dl = __fmul_ru(__fadd_ru(dl, r1), maxw);
+  return __fadd_ru(dl, 0x1p-126f);
+}
+
+__device__ __forceinline__ float maxw_value(uint32_t wc, int dt) {
+  return dt == ELMO_FP8_E4M3 ? (wc >= 0x7Fu ? NAN : e4m3_to_f32((uint8_t)wc))
+                             : (wc >= 0x7F80u ? NAN : bf16_to_f32((uint16_t)wc));
+}
+
+// Inspection: the bound of every query row (NaN where the row or the head
+// holds non-finite values).
+__global__ void topk_bound_kernel(int32_t B, float gamma, const float* __restrict__ n1, const float* __restrict__ r1,
+                                  const int32_t* __restrict__ rflag, const uint32_t* __restrict__ wmax, int dt,
+                                  float* __restrict__ out) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  out[b] = rflag[b] ? NAN : screen_bound(gamma, n1[b], r1[b], maxw_value(*wmax, dt));
 }
 
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(
@@ -519,17 +551,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(
   }
   __syncthreads();
   if (tid == 0) {
-    const uint32_t wc = *wmax;
-    const float maxw = dt == ELMO_FP8_E4M3 ? (wc >= 0x7Fu ? NAN : e4m3_to_f32((uint8_t)wc))
-                                           : (wc >= 0x7F80u ? NAN : bf16_to_f32((uint16_t)wc));
+    const float maxw = maxw_value(*wmax, dt);
     bool ok = rflag[b] == 0 && m >= k && !isnan(maxw);
     if (ok) ok = !isnan(rs[k - 1]);
-    if (ok && u != -INFINITY) {
-      float dl = __fmul_ru(gamma, __fadd_ru(n1[b], r1[b]));
-      dl = __fmul_ru(__fadd_ru(dl, r1[b]), maxw);
-      dl = __fadd_ru(dl, 0x1p-126f);                     // rescaling of subnormal partial results
-      ok = rs[k - 1] > __fadd_ru(u, dl);
-    }
+    if (ok && u != -INFINITY) ok = rs[k - 1] > __fadd_ru(u, screen_bound(gamma, n1[b], r1[b], maxw));
     if (ok) {
       for (int q = 0; q < k; ++q) {
         idx[(size_t)b * k + q] = ri[q];
@@ -654,9 +679,9 @@ cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k
   if (e != cudaSuccess) return e;
   {
     KernelScope sc(h, ELMO_K_TOPK_SCORE, s, 1);
-    ks<<<o.P * o.G, kSThreads, smem, s>>>(tmW, h->L, h->d, B, o.kp, o.G,
+    ks<<<o.P * o.G, kSThreads, smem, s>>>(tmW, (int64_t)0, h->L, h->d, B, o.kp, o.G,
                                           fp8 ? xa : reinterpret_cast<const uint8_t*>(X), xb, xinv, cs, ci, thr, tshare,
-                                          h->status);
+                                          nullptr, h->status);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
@@ -675,6 +700,61 @@ cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k
 
   // stage 3: the rows the certificate did not clear (a device-side list; usually empty)
   return launch_topk_simt_rows(h, X, B, k, fail, nfail, ws + o.simt, idx, score, s);
+}
+
+cudaError_t topk_uncertified_rows(elmo_head* h, int32_t B, int32_t k, int32_t* rows, cudaStream_t s) {
+  const TopkLayout o = topk_layout(h, B, k);
+  cudaError_t e = cudaMemcpyAsync(rows, static_cast<uint8_t*>(h->cand) + o.nfail, sizeof(int32_t),
+                                  cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(s);
+}
+
+cudaError_t launch_topk_screen_dump(elmo_head* h, const uint16_t* X, int32_t B, int64_t l0, int64_t l1, float* S,
+                                    float* bound, cudaStream_t s) {
+  const bool fp8 = h->dt == ELMO_FP8_E4M3;
+  const TopkLayout o = topk_layout(h, B, 1);
+  uint8_t* ws = static_cast<uint8_t*>(h->cand);
+  uint8_t* xa = ws + o.xa;
+  uint8_t* xb = ws + o.xb;
+  float* xinv = reinterpret_cast<float*>(ws + o.xinv);
+  float* n1 = reinterpret_cast<float*>(ws + o.n1);
+  float* r1 = reinterpret_cast<float*>(ws + o.r1);
+  int32_t* rflag = reinterpret_cast<int32_t*>(ws + o.rflag);
+  uint32_t* wmax = reinterpret_cast<uint32_t*>(ws + o.wmax);
+  int32_t* nfail = reinterpret_cast<int32_t*>(ws + o.nfail);
+  uint32_t* tshare = reinterpret_cast<uint32_t*>(ws + o.tshare);
+  h->launches += 4;
+  if (fp8) topk_xprep_kernel<1><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail, tshare);
+  else topk_xprep_kernel<0><<<B, kPrepT, 0, s>>>(X, h->d, xa, xb, xinv, n1, r1, rflag, wmax, nfail, tshare);
+  const int64_t n16 = h->L * (int64_t)h->d * (fp8 ? 1 : 2) / 16;
+  if (fp8) topk_wmax_kernel<1><<<h->num_sms * 4, 256, 0, s>>>(static_cast<const uint4*>(h->W), n16, wmax);
+  else topk_wmax_kernel<0><<<h->num_sms * 4, 256, 0, s>>>(static_cast<const uint4*>(h->W), n16, wmax);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap tmW;
+  const int eb = fp8 ? 1 : 2;
+  e = make_tma_map_2d(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, (uint32_t)o.N);
+  if (e != cudaSuccess) return e;
+  auto ks = fp8 ? topk_screen_tc<1> : topk_screen_tc<0>;
+  e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScreenSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t nl = l1 - l0;
+  int64_t G = h->num_sms / o.P;
+  const int64_t T = (nl + kN - 1) / kN;
+  if (G > T) G = T;
+  if (G < 1) G = 1;
+  const size_t smem = 1024 + kSStages * kSBox + sizeof(float) * kN * 128 + 2 * sizeof(float) * 16 * 128 +
+                      sizeof(SmemS);
+  ks<<<o.P * (int)G, kSThreads, smem, s>>>(tmW, l0, nl, h->d, B, 16, (int32_t)G,
+                                           fp8 ? xa : reinterpret_cast<const uint8_t*>(X), xb, xinv, nullptr, nullptr,
+                                           nullptr, tshare, S, h->status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int nkb = (h->d * eb + 127) / 128;
+  const int nsteps = (fp8 ? 2 : 1) * nkb * 4;
+  const float gamma = (float)((double)nsteps * 0x1p-20 + 1.01 * (double)h->d * 0x1p-24);
+  topk_bound_kernel<<<(B + 127) / 128, 128, 0, s>>>(B, gamma, n1, r1, rflag, wmax, (int)h->dt, bound);
+  return cudaGetLastError();
 }
 
 }  // namespace elmo

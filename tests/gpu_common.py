@@ -42,3 +42,27 @@ def run_step(elmo, W, X, rowptr, cols, lr, chunk, seed, step, dtype, head=None):
     out = w_to_host(Wd, dtype), dX.cpu().numpy()
     h.close()
     return out
+
+
+def run_step_with_operands(elmo, W, X, rowptr, cols, lr, chunk, seed, step, dtype, span=1 << 16):
+    """The logits and gradient operands of every label (forward_chunk, over
+    ranges of `span` labels; W untouched), then one step on the same head.
+    Returns (new W codes, dX, Z [L, B], G [L, B])."""
+    Wd = w_to_dev(W, "bf16" if dtype == "bf16" else "fp8")
+    h = elmo.elmo_init_head(Wd, dtype)
+    Xd, rp, cl = to_dev_u16(X), to_dev_i32(rowptr), to_dev_i32(cols)
+    L, B = W.shape[0], X.shape[0]
+    Z = np.empty((L, B), np.float32)
+    G = np.empty((L, B), np.float32)
+    for a in range(0, L, span):
+        e = min(L, a + span)
+        Zd = torch.empty(e - a, B, device="cuda")
+        Gd = torch.empty(e - a, B, device="cuda")
+        elmo.elmo_forward_chunk(h, Xd, rp, cl, a, e, Zd, Gd)
+        Z[a:e], G[a:e] = Zd.cpu().numpy(), Gd.cpu().numpy()
+    dX = torch.empty(B, X.shape[1], dtype=torch.float32, device="cuda")
+    elmo.elmo_train_step_chunked(h, Xd, rp, cl, lr, chunk, seed, step, dX)
+    elmo.elmo_sync_status(h)
+    out = w_to_host(Wd, "bf16" if dtype == "bf16" else "fp8"), dX.cpu().numpy(), Z, G
+    h.close()
+    return out

@@ -67,3 +67,15 @@ def test_binding_rejects_unknown_dtypes():
     assert elmo._dt("e5m2") == elmo.FP8_E5M2 == 3
     with pytest.raises(ValueError):
         elmo._dt("e4m3fnuz")
+
+
+def test_library_carries_nvtx_ranges():
+    """Every entry point of the library opens an NVTX range named after itself
+    (header-only NVTX 3: the ranges cost nothing unless a profiler injects
+    itself through NVTX_INJECTION64_PATH)."""
+    import precision_label_chunk_b200 as elmo
+    with open(elmo.library_path(), "rb") as f:
+        blob = f.read()
+    assert b"NVTX_INJECTION64_PATH" in blob
+    for name in (b"elmo_train_step_chunked", b"elmo_topk_predict", b"elmo_sr_round"):
+        assert name in blob

@@ -8,7 +8,7 @@ import torch
 
 from synthetic import make_labels, make_X, workload
 from tests.gpu_common import need_gpu, to_dev_i32, to_dev_u16, w_to_host
-from tests.parity import assert_rel_close, assert_weights_close
+from tests.parity import assert_operands_of_logits, assert_rel_close, assert_weights_close, flip_corrected_dx
 
 pytestmark = pytest.mark.gpu
 
@@ -37,15 +37,35 @@ def test_step_full_size_sampled(orc, name):
     X = make_X(w, 0)
     rowptr, cols = make_labels(w, 0)
     dX = torch.empty(w.B, w.d, device="cuda")
-    elmo.elmo_train_step_chunked(h, to_dev_u16(X), to_dev_i32(rowptr), to_dev_i32(cols), w.lr, w.chunk, 0, 0, dX)
+    samples = [0, w.B // 2, w.B - 1]
+    Xd, rp, cl = to_dev_u16(X), to_dev_i32(rowptr), to_dev_i32(cols)
+    if w.L <= 3_000_000:          # dX rows need every label; the 8.6M head checks weights only
+        # logits and operands of the sampled samples over all labels, before the step
+        Zs = np.empty((len(samples), w.L), np.float32)
+        Gs = np.empty((len(samples), w.L), np.float32)
+        for a in range(0, w.L, w.chunk):
+            e = min(w.L, a + w.chunk)
+            Zd = torch.empty(e - a, w.B, device="cuda")
+            Gd = torch.empty(e - a, w.B, device="cuda")
+            elmo.elmo_forward_chunk(h, Xd, rp, cl, a, e, Zd, Gd)
+            Zs[:, a:e] = Zd[:, samples].T.cpu().numpy()
+            Gs[:, a:e] = Gd[:, samples].T.cpu().numpy()
+            del Zd, Gd
+    elmo.elmo_train_step_chunked(h, Xd, rp, cl, w.lr, w.chunk, 0, 0, dX)
     elmo.elmo_sync_status(h)
     for l0, l1 in _label_ranges(w.L, w.chunk):
         r = orc.train_step(W0[:l1], X, rowptr, cols, w.lr, 0, 0, w.dtype, l0=l0, l1=l1, want_dx=False, L=w.L)
         assert_weights_close(w_to_host(Wd[l0:l1], w.dtype), r["W"], w.dtype)
-    if w.L <= 3_000_000:          # dX rows need every label; the 8.6M head checks weights only
-        samples = [0, w.B // 2, w.B - 1]
-        ref = orc.dx_rows(W0, X, rowptr, cols, samples, w.dtype)
-        assert_rel_close(dX.cpu().numpy()[samples], ref, w.dtype, what="dX rows")
+    if w.L <= 3_000_000:
+        ref, Zo, Go = orc.dx_rows(W0, X, rowptr, cols, samples, w.dtype, want_zg=True)
+        Y = np.zeros((len(samples), w.L), np.float32)
+        for i, b in enumerate(samples):
+            Y[i, cols[rowptr[b]:rowptr[b + 1]]] = 1.0
+        assert_rel_close(Zs, Zo, w.dtype, axis=None, what="Z rows")
+        assert_operands_of_logits(Gs, Zs, Y, w.dtype, what="G rows (GPU)")
+        assert_operands_of_logits(Go, Zo, Y, w.dtype, what="G rows (oracle)")
+        dx_ref, _ = flip_corrected_dx(ref, Gs.T, Go.T, W0, w.dtype)
+        assert_rel_close(dX.cpu().numpy()[samples], dx_ref, w.dtype, what="dX rows")
     h.close()
 
 

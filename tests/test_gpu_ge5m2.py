@@ -6,8 +6,8 @@ import pytest
 import torch
 
 from synthetic import make_labels, make_W_f32, make_X, workload
-from tests.gpu_common import need_gpu, run_step, to_dev_i32, to_dev_u16, w_to_dev, w_to_host
-from tests.parity import assert_rel_close, assert_weights_close
+from tests.gpu_common import need_gpu, run_step_with_operands, to_dev_i32, to_dev_u16, w_to_dev, w_to_host
+from tests.parity import assert_operands_of_logits, assert_rel_close, assert_weights_close, check_step, positives
 
 pytestmark = pytest.mark.gpu
 DT = "fp8_ge5m2"
@@ -35,10 +35,8 @@ def test_ge5m2_step_matches_oracle(orc, name, over):
     w = workload(name, dtype="fp8", **over)
     W, X, rowptr, cols = _inputs(orc, w)
     chunk = 512
-    Wg, dXg = run_step(elmo, W, X, rowptr, cols, w.lr, chunk, 0, 0, DT)
-    r = orc.train_step(W, X, rowptr, cols, w.lr, 0, 0, DT)
-    assert_weights_close(Wg, r["W"], "fp8", chunk_rows=chunk)
-    assert_rel_close(dXg, r["dX"], DT, what="dX")
+    Wg, dXg, Zg, Gg = run_step_with_operands(elmo, W, X, rowptr, cols, w.lr, chunk, 0, 0, DT)
+    r, _ = check_step(orc, W, X, rowptr, cols, w.lr, 0, 0, DT, Wg, dXg, Zg, Gg, chunk_rows=chunk)
     # and it is not the E4M3-gradient step: the operand grids differ
     r4 = orc.train_step(W, X, rowptr, cols, w.lr, 0, 0, "fp8")
     assert not np.array_equal(r["W"], r4["W"])
@@ -58,12 +56,14 @@ def test_ge5m2_forward_chunk_gradient_operand(orc):
     elmo.elmo_sync_status(h)
     r = orc.train_step(W, X, rowptr, cols, 0.0, 0, 0, DT, l0=l0, l1=l1, want_zg=True)
     assert_rel_close(Z.cpu().numpy(), r["Z"], "fp8", axis=None, what="Z")
-    g, go = G.cpu().numpy(), r["G"]
-    # values on the E5M2 grid of 2^8 G; equal where the logits agree, else one step apart
+    g, go, z = G.cpu().numpy(), r["G"], Z.cpu().numpy()
+    # values on the E5M2 grid of 2^8 G, each the correctly rounded operand of its
+    # own logit; equal to the oracle's where the logits agree
     codes = orc.rne_e5m2(g * 256.0)
     assert np.array_equal(orc.e5m2_value(codes) / 256.0, g)
-    assert np.all(np.abs(g - go) <= 2.0 ** -2 * np.maximum(np.abs(go), 2.0 ** -10) + 1e-7)
-    assert np.mean(g == go) > 0.99
+    assert_operands_of_logits(g, z, positives(rowptr, cols, w.L, w.B, l0, l1), DT)
+    same = z == r["Z"]
+    assert np.array_equal(g[same], go[same])
     assert np.array_equal(w_to_host(Wd, "fp8"), W)
     h.close()
 

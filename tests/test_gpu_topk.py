@@ -141,3 +141,48 @@ def test_precision_at_k_matches_oracle(orc, B, k, L):
                              torch.from_numpy(cols).cuda(), p)
     want = orc.precision_at_k(idx, rowptr, cols).astype(np.float32)
     assert np.array_equal(p.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("dtype,L", [("fp8", 3_000_000), ("bf16", 500_000)])
+def test_screening_error_within_a_quarter_of_the_bound(orc, dtype, L):
+    """The certificate assumes every accumulating MMA is off by at most 2^-20 of
+    the sum of its products' magnitudes.  Measured on a full 131,072-label
+    range of a workload-sized head: the screening scores stay within a quarter
+    of each row's bound of the exact chain scores, and within a quarter of the
+    per-element form of the same model (each label's own sum of |x w|)."""
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("topk5_3m_fp8", L=L, dtype=dtype)
+    Wd = torch.empty(w.L, w.d, dtype=torch.uint8 if dtype == "fp8" else torch.int16, device="cuda")
+    h = elmo.elmo_init_head(Wd, dtype, fill=True, init_std=0.02, seed=0)
+    X = make_X(w, 0)
+    l0 = (w.L // 2) // 128 * 128
+    l1 = l0 + 131072
+    rows = [0, 1, 255, 511, 1023]
+    Xs = X[rows]
+    S = torch.empty(len(rows), l1 - l0, device="cuda")
+    bound = torch.empty(len(rows), device="cuda")
+    elmo.elmo_topk_screen_scores(h, to_dev_u16(Xs), l0, l1, S, bound)
+    torch.cuda.synchronize()
+    Wh = Wd.cpu().numpy().view(np.uint8 if dtype == "fp8" else np.uint16)
+    exact = orc.scores(Wh, Xs, np.arange(len(rows)), l0, l1, dtype)
+    err = np.abs(S.cpu().numpy().astype(np.float64) - exact.astype(np.float64))
+    bnd = bound.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(bnd)) and np.all(bnd > 0)
+    worst = (err.max(axis=1) / bnd)
+    assert worst.max() <= 0.25, f"screening error reaches {worst.max():.3f} of the certificate's bound"
+    # per element: nsteps 2^-20 sum|q w| (+ the E4M3 split's residual, + the chain's own error)
+    xv = (Xs.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    wv = (Wh[l0:l1].view(ml_dtypes.float8_e4m3fn) if dtype == "fp8" else Wh[l0:l1].view(ml_dtypes.bfloat16))
+    absw = np.abs(wv.astype(np.float32))
+    mag = (np.abs(xv).astype(np.float32) @ absw.T).astype(np.float64) * (1 + 2.0 ** -16)   # sum_j |x_j w_lj|
+    nsteps = (2 if dtype == "fp8" else 1) * (w.d * (1 if dtype == "fp8" else 2) // 128) * 4
+    model = (nsteps * 2.0 ** -20 + 1.01 * w.d * 2.0 ** -24) * mag
+    if dtype == "fp8":
+        # the lo part of the E4M3 split is exact unless below 2^-9 (in scaled units):
+        # residual at most 2^-10 / s_b per element
+        s_b = np.array([2.0 ** np.floor(np.log2(448.0 / np.abs(x).max())) for x in xv])
+        model += (2.0 ** -10 / s_b)[:, None] * absw.sum(axis=1)[None, :]
+    ratio = err / np.maximum(model, 1e-30)
+    assert ratio.max() <= 0.25, f"screening error reaches {ratio.max():.3f} of the per-element model"
+    h.close()

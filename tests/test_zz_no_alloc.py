@@ -12,7 +12,7 @@ import torch
 
 from synthetic import make_labels, make_W_f32, make_W_bf16, make_X, workload
 from tests.gpu_common import need_gpu, to_dev_i32, to_dev_u16, w_to_dev, w_to_host
-from tests.parity import assert_rel_close, assert_weights_close
+from tests.parity import assert_rel_close
 
 pytestmark = pytest.mark.gpu
 
@@ -43,7 +43,9 @@ def test_noalloc_step_matches_head_step_twice(orc, name, over):
         elmo.elmo_sync_status(head)
         torch.cuda.synchronize()
         assert status.cpu().tolist() == [0, 0]
-        assert_weights_close(w_to_host(W_free, w.dtype), w_to_host(W_head, w.dtype), w.dtype, chunk_rows=w.chunk)
+        # the same kernels and the same index-keyed draws: the weights agree bit for bit,
+        # even though this path splits a chunk into shorter passes to fit its fixed scratch
+        assert torch.equal(W_free, W_head), f"step {step}: weights differ from the head-based step"
         assert_rel_close(dX_free.cpu().numpy(), dX_head.cpu().numpy(), w.dtype, what=f"dX step {step}")
     head.close()
 
