@@ -43,7 +43,9 @@ typedef enum {
   ELMO_FP8_E4M3 = 1,       /* OCP E4M3FN weights: max 448, no infinities, saturating */
   ELMO_FP8_E4M3_GE5M2 = 2, /* E4M3 weights (and X) as above; the training step's gradient
                               operand is OCP E5M2 of 2^8 G instead of E4M3 (heads only) */
-  ELMO_FP8_E5M2 = 3        /* OCP E5M2 values (max 57344, with infinities): elmo_sr_round only */
+  ELMO_FP8_E5M2 = 3        /* OCP E5M2 values (max 57344, with infinities): an SR output grid of
+                              elmo_sr_round, and as a head E5M2 weights with X and the
+                              gradient operand in E4M3 (the adjacent 8-bit format) */
 } elmo_dtype;
 
 typedef enum {
@@ -75,9 +77,13 @@ typedef struct elmo_head elmo_head;
  * unscaled E4M3 (abstract; atlas summary "Approach", "Surprising findings").
  *
  *   out      : receives the new handle (host pointer).
- *   W_dev    : device pointer to W [L x d], bf16 bits (dt = ELMO_BF16) or E4M3
- *              codes (dt = ELMO_FP8_E4M3); row-major, label-major.  Borrowed
- *              for the life of the head; updated in place by training steps.
+ *   W_dev    : device pointer to W [L x d], bf16 bits (dt = ELMO_BF16), E4M3
+ *              codes (ELMO_FP8_E4M3, ELMO_FP8_E4M3_GE5M2) or E5M2 codes
+ *              (ELMO_FP8_E5M2: the weights are stored and stochastically rounded
+ *              on the E5M2 grid, +-inf kept, finite values saturating at 57344;
+ *              X and the gradient operand are E4M3 as for ELMO_FP8_E4M3);
+ *              row-major, label-major.  Borrowed for the life of the head;
+ *              updated in place by training steps.
  *   L        : number of labels, 1 <= L < ELMO_MAX_LABELS.
  *   d        : width, a multiple of 64 in [64, 4096].
  *   fill     : 0 = keep W as is; 1 = overwrite W with SR(init_std * N(0,1)),

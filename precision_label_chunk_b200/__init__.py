@@ -36,7 +36,7 @@ __all__ = [
 BF16 = 0
 FP8_E4M3 = 1
 FP8_E4M3_GE5M2 = 2    # E4M3 weights, E5M2 gradient operand in the training step
-FP8_E5M2 = 3          # E5M2 values (elmo_sr_round only)
+FP8_E5M2 = 3          # E5M2 values: an SR output grid, and heads with E5M2 weights (E4M3 X and G)
 WAIT_CHECK_SITE = 99
 MAX_BATCH = 256
 MAX_NNZ = 32768

@@ -84,10 +84,10 @@ elmo_status ensure_gbuf(elmo_head* h, size_t bytes) {
 }
 
 // The persistent step's ring: kRingTiles gradient-operand tiles of up to
-// 128 labels x 256 E4M3 (or 128 bf16) samples, and its two flag arrays.
+// 128 labels x 256 samples (64 KB in bf16), and its two flag arrays.
 elmo_status ensure_ring(elmo_head* h) {
   const size_t tiles = elmo::kRingTiles;
-  const size_t bytes = tiles * 32768 + 2 * sizeof(int32_t) * tiles;
+  const size_t bytes = tiles * 65536 + 2 * sizeof(int32_t) * tiles;
   if (h->ring_bytes >= bytes) return ELMO_OK;
   if (h->ring) cudaFree(h->ring);
   h->ring = nullptr;
@@ -98,7 +98,7 @@ elmo_status ensure_ring(elmo_head* h) {
   }
   h->ring_bytes = bytes;
   h->ring_tiles = (int32_t)tiles;
-  h->ring_flags = reinterpret_cast<int32_t*>(static_cast<char*>(h->ring) + tiles * 32768);
+  h->ring_flags = reinterpret_cast<int32_t*>(static_cast<char*>(h->ring) + tiles * 65536);
   return ELMO_OK;
 }
 
@@ -214,11 +214,12 @@ elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_
   g_last_error.clear();
   if (!out || !W_dev) return fail(ELMO_EINVAL, "null out or W");
   *out = nullptr;
-  if (dt == ELMO_FP8_E5M2) return fail(ELMO_EUNSUPPORTED, "E5M2 weights: ELMO_FP8_E5M2 is an SR output grid only");
-  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3 && dt != ELMO_FP8_E4M3_GE5M2)
+  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3 && dt != ELMO_FP8_E4M3_GE5M2 && dt != ELMO_FP8_E5M2)
     return fail(ELMO_EINVAL, "unknown dtype %d", (int)dt);
+  const elmo_dtype fill_dt = dt == ELMO_FP8_E4M3_GE5M2 ? ELMO_FP8_E4M3 : dt;   // the weights' own grid
   const bool g_e5m2 = dt == ELMO_FP8_E4M3_GE5M2;
-  if (g_e5m2) dt = ELMO_FP8_E4M3;                    // the weights are E4M3
+  const bool w_e5m2 = dt == ELMO_FP8_E5M2;
+  if (g_e5m2 || w_e5m2) dt = ELMO_FP8_E4M3;          // the tensor-core operand path: X and G in E4M3 (or E5M2 G)
   if (L < 1 || L >= ELMO_MAX_LABELS) return fail(ELMO_EINVAL, "L = %lld outside [1, 2^24)", (long long)L);
   if (label_base < 0 || labels_total > ELMO_MAX_TOTAL_LABELS || label_base > labels_total - L)
     return fail(ELMO_EINVAL, "label rows [%lld, %lld) outside a head of %lld labels (at most %lld)",
@@ -239,6 +240,7 @@ elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_
   h->label_base = label_base;
   h->labels_total = labels_total;
   h->g_e5m2 = g_e5m2;
+  h->w_e5m2 = w_e5m2;
   h->d = d;
   h->dt = dt;
   h->device = dev;
@@ -264,7 +266,7 @@ elmo_status elmo_init_head_shard(elmo_head** out, void* W_dev, int64_t L, int32_
   cudaError_t e = cudaMemsetAsync(base, 0, 64, s);
   if (e == cudaSuccess && fill) {
     h->launches += 1;
-    e = elmo::launch_fill(W_dev, L * (int64_t)d, dt, init_std, seed, (uint64_t)label_base * (uint64_t)d, s);
+    e = elmo::launch_fill(W_dev, L * (int64_t)d, fill_dt, init_std, seed, (uint64_t)label_base * (uint64_t)d, s);
   }
   if (e != cudaSuccess) {
     cudaFree(base);

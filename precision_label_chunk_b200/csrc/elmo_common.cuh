@@ -211,6 +211,45 @@ __device__ __forceinline__ uint2 sr8_e4m3(const float (&v)[8], const u32x4& r) {
                     pack_e4m3x2(o[5], o[4]) | (pack_e4m3x2(o[7], o[6]) << 16));
 }
 
+// Stochastic rounding of v onto the OCP E5M2 grid with a 16-bit draw k, as
+// an E5M2 code: NaN -> 0x7F, +-inf kept, magnitudes at or above the largest
+// finite 57344 saturate to it.  From 2^-14 up E5M2 keeps 2 of fp32's 23
+// mantissa bits (add-and-truncate at 21 bits); below, its subnormal grid is
+// the multiples of 2^-16, and with t = |v| 2^16 (exact) and q = floor(t),
+// t - q are exact in fp32, and the result is (q + [k < 2^16 (t - q)]) 2^-16.
+__device__ __forceinline__ uint32_t sr_e5m2_code(float v, uint32_t k) {
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t sign = (b >> 24) & 0x80u;
+  const uint32_t mag = b & 0x7FFFFFFFu;
+  if (mag > 0x7F800000u) return 0x7Fu;                    // NaN
+  if (mag == 0x7F800000u) return sign | 0x7Cu;            // +-inf
+  if (mag >= 0x47600000u) return sign | 0x7Bu;            // |v| >= 57344: the largest finite value
+  float o;
+  if (mag >= 0x38800000u) {                               // |v| >= 2^-14
+    o = __uint_as_float((mag + (0x1FFFFFu - 32u * k)) & ~0x1FFFFFu);
+  } else {
+    const float t = __fmul_rn(__uint_as_float(mag), 65536.0f);
+    const float q = floorf(t);
+    const float up = (float)k < __fmul_rn(__fsub_rn(t, q), 65536.0f) ? 1.0f : 0.0f;
+    o = __fmul_rn(__fadd_rn(q, up), 0x1p-16f);
+  }
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(o));
+  return sign | (r & 0x7Fu);                              // o is on the grid: the conversion is exact
+}
+
+// Four E5M2 codes (byte i = element i) -> fp32 values, exact (an E5M2 code is
+// the upper byte of the binary16 value).
+__device__ __forceinline__ void e5m2x4_to_f32(uint32_t w, float (&o)[4]) {
+  uint32_t h01, h23;
+  asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h01) : "h"((uint16_t)(w & 0xFFFF)));
+  asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h23) : "h"((uint16_t)(w >> 16)));
+  o[0] = __half2float(__ushort_as_half((unsigned short)(h01 & 0xFFFF)));
+  o[1] = __half2float(__ushort_as_half((unsigned short)(h01 >> 16)));
+  o[2] = __half2float(__ushort_as_half((unsigned short)(h23 & 0xFFFF)));
+  o[3] = __half2float(__ushort_as_half((unsigned short)(h23 >> 16)));
+}
+
 // Four E4M3 codes (byte i = element i) -> fp32 values, exact.
 __device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&o)[4]) {
   uint32_t h01, h23;

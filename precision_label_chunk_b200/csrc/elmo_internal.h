@@ -24,6 +24,7 @@ struct elmo_head {
   int32_t d = 0;
   elmo_dtype dt = ELMO_BF16;    // format of W (and of X and G in the tensor cores): BF16 or E4M3
   bool g_e5m2 = false;         // E4M3 step whose gradient operand G is E5M2 (ELMO_FP8_E4M3_GE5M2)
+  bool w_e5m2 = false;         // E5M2 weights (ELMO_FP8_E5M2 head): X and G stay E4M3
   int device = 0;
   int num_sms = 0;
   // workspace owned by the head
@@ -66,6 +67,9 @@ struct KernelScope {
 }  // namespace elmo
 
 namespace elmo {
+
+// The stored weights' grid: ELMO_BF16, ELMO_FP8_E4M3 or ELMO_FP8_E5M2.
+inline int w_format(const elmo_head* h) { return h->w_e5m2 ? (int)ELMO_FP8_E5M2 : (int)h->dt; }
 
 constexpr int kTileLabels = 128;        // labels per tensor-core tile
 

@@ -57,10 +57,11 @@ extern "C" elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d
   // ---- arguments (the same limits as the head-based step; the scratch is sized for them)
   if (!W_dev || !X_dev || !rowptr_dev || !dX_dev || !status_dev) return fail(ELMO_EINVAL, "null pointer argument");
   if (nnz > 0 && !cols_dev) return fail(ELMO_EINVAL, "null cols with nnz > 0");
-  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3 && dt != ELMO_FP8_E4M3_GE5M2)
+  if (dt != ELMO_BF16 && dt != ELMO_FP8_E4M3 && dt != ELMO_FP8_E4M3_GE5M2 && dt != ELMO_FP8_E5M2)
     return fail(ELMO_EINVAL, "unknown dtype %d", (int)dt);
   const bool g_e5m2 = dt == ELMO_FP8_E4M3_GE5M2;
-  if (g_e5m2) dt = ELMO_FP8_E4M3;                    // the weights are E4M3
+  const bool w_e5m2 = dt == ELMO_FP8_E5M2;
+  if (g_e5m2 || w_e5m2) dt = ELMO_FP8_E4M3;          // X and G in E4M3 (or E5M2 G)
   if (L < 1 || L >= ELMO_MAX_LABELS)
     return fail(ELMO_EUNSUPPORTED, "L = %lld: the no-allocation step supports 1 <= L < 2^24", (long long)L);
   if (d < 64 || d > 4096 || d % 64 != 0)
@@ -106,6 +107,7 @@ extern "C" elmo_status elmo_train_step_noalloc(void* W_dev, int64_t L, int32_t d
   h.d = d;
   h.dt = dt;
   h.g_e5m2 = g_e5m2;
+  h.w_e5m2 = w_e5m2;
   h.device = dev;
   h.num_sms = nsm;
   h.status = status_dev;

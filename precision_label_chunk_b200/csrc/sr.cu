@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(256) fill_kernel(void* __restrict__ W, int64_t
       const uint32_t k = (e & 1) ? (word >> 16) : (word & 0xFFFFu);
       const float v = std * nv[e];
       if (dt == ELMO_BF16) static_cast<uint16_t*>(W)[i] = sr_bf16(v, k);
+      else if (dt == ELMO_FP8_E5M2) static_cast<uint8_t*>(W)[i] = (uint8_t)sr_e5m2_code(v, k);
       else static_cast<uint8_t*>(W)[i] = sr_e4m3(v, k);
     }
   }

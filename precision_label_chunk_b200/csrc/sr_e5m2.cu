@@ -19,25 +19,6 @@
 namespace elmo {
 namespace {
 
-__device__ __forceinline__ uint32_t sr_e5m2_code(float v, uint32_t k) {
-  const uint32_t b = __float_as_uint(v);
-  const uint32_t sign = (b >> 24) & 0x80u;
-  const uint32_t mag = b & 0x7FFFFFFFu;
-  if (mag > 0x7F800000u) return 0x7Fu;                    // NaN
-  if (mag == 0x7F800000u) return sign | 0x7Cu;            // +-inf
-  if (mag >= 0x47600000u) return sign | 0x7Bu;            // |v| >= 57344: the largest finite value
-  float o;
-  if (mag >= 0x38800000u) {                               // |v| >= 2^-14
-    o = __uint_as_float((mag + (0x1FFFFFu - 32u * k)) & ~0x1FFFFFu);
-  } else {
-    const float t = __fmul_rn(__uint_as_float(mag), 65536.0f);
-    const float q = floorf(t);
-    const float up = (float)k < __fmul_rn(__fsub_rn(t, q), 65536.0f) ? 1.0f : 0.0f;
-    o = __fmul_rn(__fadd_rn(q, up), 0x1p-16f);
-  }
-  return sign | (pack_e5m2x2(0.0f, o) & 0x7Fu);           // o is on the grid: the conversion is exact
-}
-
 __global__ void __launch_bounds__(256) sr_e5m2_kernel(const float* __restrict__ in, uint8_t* __restrict__ out,
                                                       int64_t n, uint64_t seed, uint64_t step, uint64_t base) {
   const uint64_t first_blk = base >> 3;

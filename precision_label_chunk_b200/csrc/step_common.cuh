@@ -58,6 +58,11 @@ __device__ __forceinline__ float rcpf_approx(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float tanhf_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 // fp32 multiply that keeps denormal inputs and results whatever -ftz says
 __device__ __forceinline__ float mul_rn_denorm(float a, float b) {
   float y;
@@ -70,8 +75,9 @@ __device__ __forceinline__ float mul_rn_denorm(float a, float b) {
 // G = sigmoid(z) - y rounded to nearest even onto bf16 (kG = 0), or 2^8 G onto
 // E4M3 (kG = 1) or E5M2 (kG = 2), z = acc * inv_sx; y = 1 at the positives.
 // The code is the one that sigmoid(z) = 1 / (1 + e^-z) correctly rounded to
-// fp32 gives.  sigmoid comes from one ex2 and one rcp of the special-function
-// unit, within 2^-21 relative plus |z| 2^-23 from the rounded argument of ex2;
+// fp32 gives.  8-bit grids try a one-tanh pass first (below).  Otherwise
+// sigmoid comes from one ex2 and one rcp of the special-function unit, within
+// 2^-21 relative plus |z| 2^-23 from the rounded argument of ex2;
 // each element is rounded from both ends of an interval around its value that
 // is wider than that error, and where the two ends land on different codes
 // (the value lies within that error of a midpoint of the operand grid, about
@@ -99,6 +105,32 @@ __device__ __forceinline__ void grad_codes16(const uint32_t* acc, float inv_sx, 
   constexpr float sc = kG ? 256.0f : 1.0f;
   constexpr int kPer = kG ? 4 : 2;                 // codes per 32-bit word
   constexpr int kBits = 32 / kPer;
+  if (kG) {
+    // 8-bit grids: first 2^8 sigmoid(z) = 128 + 128 tanh(z/2) with a single
+    // tanh of the special-function unit (relative error below 2^-10, so below
+    // 2^-3 in units of 2^8 G); each element is rounded from both ends of a
+    // window of +-0.13 around that value, and the group is done when all the
+    // ends agree.  That holds unless some value lies near a midpoint of the
+    // grid, or is small (2^8 G below a few units, where the grid is finer than
+    // the window): then the group takes the path below.
+    float lo[16], hi[16];
+    const float zh = 0.5f * inv_sx;                 // exact: a power of two
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float x = __fmaf_rn(tanhf_approx(__fmul_rn(__uint_as_float(acc[i]), zh)), 128.0f, 128.0f) -
+                      (((ybits >> i) & 1u) ? 256.0f : 0.0f);
+      const bool v = (vbits >> i) & 1u;
+      lo[i] = v ? x - 0.13f : 0.0f;
+      hi[i] = v ? x + 0.13f : 0.0f;
+    }
+    uint32_t diff = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      out[q] = grad_pack2<kG>(lo[4 * q + 1], lo[4 * q]) | (grad_pack2<kG>(lo[4 * q + 3], lo[4 * q + 2]) << 16);
+      diff |= out[q] ^ (grad_pack2<kG>(hi[4 * q + 1], hi[4 * q]) | (grad_pack2<kG>(hi[4 * q + 3], hi[4 * q + 2]) << 16));
+    }
+    if (!diff) return;
+  }
   const float zmul = -1.4426950408889634f * inv_sx;
   float lo[16], hi[16];
 #pragma unroll
@@ -108,8 +140,11 @@ __device__ __forceinline__ void grad_codes16(const uint32_t* acc, float inv_sx, 
     const float s = rcpf_approx(__fadd_rn(e, 1.0f));
     const float as = s * sc;
     const float xc = as - (((ybits >> i) & 1u) ? sc : 0.0f);
-    const float eps = __fmaf_rn(fabsf(__fmul_rn(a, inv_sx)), 0x1p-22f, 0x1p-20f);
-    const float w = __fmaf_rn(fabsf(xc), 0x1p-22f, as * eps);
+    // |z| is clamped: beyond 128 sigmoid is 0 or 1 to within fp32's smallest
+    // normal, which the absolute term sc 2^-126 covers (the approximations
+    // flush denormal results to zero); the clamp also keeps 0 * inf out of w
+    const float eps = __fmaf_rn(fminf(fabsf(__fmul_rn(a, inv_sx)), 128.0f), 0x1p-22f, 0x1p-20f);
+    const float w = __fmaf_rn(fabsf(xc), 0x1p-22f, __fmaf_rn(as, eps, sc * 0x1p-126f));
     const bool v = (vbits >> i) & 1u;
     lo[i] = v ? xc - w : 0.0f;
     hi[i] = v ? xc + w : 0.0f;
@@ -193,13 +228,6 @@ __device__ __forceinline__ uint32_t mask16(const uint32_t (&m)[8], int b0) {
 }
 
 // ---------------------------------------------------------------- the SR update
-// fp32 product rounded toward +infinity, denormal inputs and results kept
-__device__ __forceinline__ float mul_rp(float a, float b) {
-  float y;
-  asm("mul.rp.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
-  return y;
-}
-
 // The 16 draws of elements l*d + j0 .. +15 (two Philox blocks; blk_base more
 // blocks in when this head holds the rows of a larger head from label_base on:
 // blk_base = label_base * d / 8).  Independent of the gradient, so the update
@@ -216,11 +244,10 @@ __device__ __forceinline__ void sr_draws16(uint64_t seed, uint64_t step, uint64_
 // 128B-swizzled W tile in shared memory (row `row`, tile column jl), draws rw
 // from sr_draws16.
 //
-// v = fl(w - fl(lrs dW)) (two roundings, denormals kept); a probe (the sum of
-// 2^120 v for E4M3, of 2 v for bf16) is not finite when some v is NaN or
-// infinite or too large for the fast rounding (E4M3: |v| >= 2^8; bf16:
-// |v| >= 2^127, where rounding could pass the largest finite value), and such
-// groups take the exact per-element path.
+// v = fl(w - fl(lrs dW)) (two roundings, denormals kept); a probe that is not
+// finite when some v is NaN or infinite (E4M3: the sum of 0 v; bf16: the sum
+// of 2 v, which also overflows once some |v| >= 2^127, where rounding could
+// pass the largest finite value) sends the group to the exact per-element path.
 //
 // Fast rounding, both grids: add-and-truncate.  If the bits of v below the
 // target precision hold the fraction F (in units of 2^-n of a grid step),
@@ -229,26 +256,29 @@ __device__ __forceinline__ void sr_draws16(uint64_t seed, uint64_t step, uint64_
 // bf16 (n = 16): the hardware's stochastic conversion cvt.rs.bf16x2.f32 adds
 // its 16 random bits to the 16 discarded bits of each value and truncates, so
 // passing 2^16 - 1 - k (the complemented draw) gives exactly this rounding.
-// E4M3 (n = 20): |v| 2^-120 is fp32's own grid cut to 3 mantissa bits (E4M3's
-// subnormal spacing 2^-9 becomes 2^-129, 2^20 units of fp32's denormal spacing,
-// and its normal range starts at 2^-126, fp32's); the product is rounded toward
-// +infinity, which keeps ceil(F) and, k being an integer, the decision
-// 16 k < F exactly, also below 2^-6 where the product is denormal.  The
-// pattern is shifted up by 4 so that the code lands in its top byte: byte 3 of
-// 16 |pattern| + 2^24 - 1 - 2^8 k is the rounded magnitude code (|v| < 2^8
-// keeps it below 0x78), and the sign is merged from v.
-template <int kFp8>
+// E4M3 (n = 20): from 2^-6 up, E4M3 keeps 3 of fp32's 23 mantissa bits; below
+// 2^-6 (its subnormal range, spacing 2^-9) |v| is first moved into
+// [2^-6, 2^-5), whose spacing is also 2^-9, by adding 2^-6 rounded toward
+// +infinity (that keeps ceil(F), and for an integer k, 16 k < F <=> 16 k <
+// ceil(F), so the decision stays exact), truncated there and moved back
+// exactly; the sign is restored and the saturating conversion maps magnitudes
+// at or above 448 to 448.
+// kW: the weight grid, 0 bf16, 1 E4M3, 2 E5M2 (E5M2 as E4M3 with 2 mantissa
+// bits kept, n = 21, subnormal range below 2^-14 with spacing 2^-16; +-inf is
+// an E5M2 value and stays, so groups holding one take the per-element path).
+template <int kW>
 __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t (&rw)[8],
                                          const uint8_t* __restrict__ wtile, int row, int jl, int64_t l, int32_t d,
                                          int j0, float lrs, void* __restrict__ Wglob) {
   float wv[16];
-  if (kFp8) {
+  if (kW) {
     const uint4 x = *reinterpret_cast<const uint4*>(wtile + row * 128 + (((jl >> 4) ^ (row & 7)) << 4));
     const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       float f4[4];
-      e4m3x4_to_f32(xw[e], f4);
+      if (kW == 1) e4m3x4_to_f32(xw[e], f4);
+      else e5m2x4_to_f32(xw[e], f4);
 #pragma unroll
       for (int i = 0; i < 4; ++i) wv[4 * e + i] = f4[i];
     }
@@ -270,26 +300,34 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
-    probe = __fmaf_rn(vv[i], kFp8 ? 0x1p120f : 2.0f, probe);
+    probe = __fmaf_rn(vv[i], kW ? 0.0f : 2.0f, probe);
   }
   const bool fast = fabsf(probe) < INFINITY;
   uint32_t wnew[8];
   if (fast) {
-    if (kFp8) {
+    if (kW) {
+      // the subnormal range is moved up one binade: [2^-6, 2^-5) for E4M3,
+      // [2^-14, 2^-13) for E5M2, whose spacing equals the subnormal spacing
+      constexpr float kLow = kW == 1 ? 0x1p-6f : 0x1p-14f;
+      constexpr float kSel = kW == 1 ? 0x1p94f : 0x1p86f;   // (kLow - |v|) 2^100 >= 1 exactly when |v| < kLow
+      constexpr uint32_t kMask = kW == 1 ? 0xFFF00000u : 0xFFE00000u;
+      constexpr uint32_t kOne = kW == 1 ? 0xFFFFFu : 0x1FFFFFu;
+      constexpr int kShift = kW == 1 ? 4 : 5;
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        // 2^24 - 1 - 2^8 k for the four draws: bytes (0xFF, ~k lo, ~k hi, 0)
-        const uint32_t a0 = ~rw[2 * q4], a1 = ~rw[2 * q4 + 1];
-        const uint32_t radd[4] = {__byte_perm(a0, 0xFFu, 0x5104), __byte_perm(a0, 0xFFu, 0x5324),
-                                  __byte_perm(a1, 0xFFu, 0x5104), __byte_perm(a1, 0xFFu, 0x5324)};
-        uint32_t t[4];
+        float o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float s = mul_rp(fabsf(vv[4 * q4 + e]), 0x1p-120f);
-          const uint32_t m = __float_as_uint(s) * 16u + radd[e];
-          t[e] = (m & 0x7FFFFFFFu) | (__float_as_uint(vv[4 * q4 + e]) & 0x80000000u);
+          const uint32_t word = rw[2 * q4 + (e >> 1)];
+          const uint32_t k16 = (e & 1) ? (word >> 16) : (word & 0xFFFFu);
+          const float a = fabsf(vv[4 * q4 + e]);
+          const float sat = __saturatef(__fmaf_rn(-a, 0x1p100f, kSel));
+          const float sh = __fmaf_ru(sat, kLow, a);
+          const uint32_t t = (__float_as_uint(sh) + (kOne - (k16 << kShift))) & kMask;
+          o[e] = copysignf(__fmaf_rn(sat, -kLow, __uint_as_float(t)), vv[4 * q4 + e]);
         }
-        wnew[q4] = __byte_perm(__byte_perm(t[0], t[1], 0x0073), __byte_perm(t[2], t[3], 0x0073), 0x5410);
+        wnew[q4] = kW == 1 ? pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16)
+                           : pack_e5m2x2(o[1], o[0]) | (pack_e5m2x2(o[3], o[2]) << 16);
       }
     } else {
 #pragma unroll
@@ -302,21 +340,27 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t
   } else {
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
-      if (kFp8) {
+      if (kW == 1) {
         if (p < 4) {
           const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
           const float o0 = sr_e4m3_value(vv[4 * p], w0 & 0xFFFFu), o1 = sr_e4m3_value(vv[4 * p + 1], w0 >> 16);
           const float o2 = sr_e4m3_value(vv[4 * p + 2], w1 & 0xFFFFu), o3 = sr_e4m3_value(vv[4 * p + 3], w1 >> 16);
           wnew[p] = pack_e4m3x2(o1, o0) | (pack_e4m3x2(o3, o2) << 16);
         }
+      } else if (kW == 2) {
+        if (p < 4) {
+          const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
+          wnew[p] = sr_e5m2_code(vv[4 * p], w0 & 0xFFFFu) | (sr_e5m2_code(vv[4 * p + 1], w0 >> 16) << 8) |
+                    (sr_e5m2_code(vv[4 * p + 2], w1 & 0xFFFFu) << 16) | (sr_e5m2_code(vv[4 * p + 3], w1 >> 16) << 24);
+        }
       } else {
         wnew[p] = (uint32_t)sr_bf16(vv[2 * p], rw[p] & 0xFFFFu) | ((uint32_t)sr_bf16(vv[2 * p + 1], rw[p] >> 16) << 16);
       }
     }
   }
-  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(Wglob) + ((size_t)l * d + j0) * (kFp8 ? 1 : 2));
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(Wglob) + ((size_t)l * d + j0) * (kW ? 1 : 2));
   dst[0] = make_uint4(wnew[0], wnew[1], wnew[2], wnew[3]);
-  if (!kFp8) dst[1] = make_uint4(wnew[4], wnew[5], wnew[6], wnew[7]);
+  if (!kW) dst[1] = make_uint4(wnew[4], wnew[5], wnew[6], wnew[7]);
 }
 
 }  // namespace

@@ -13,8 +13,9 @@
 //     128-label tiles t = a, a + nA, ...: X stays in TMEM as the MMA's A
 //     operand, 64-label W k-blocks stream through a 16-stage TMA ring, and the
 //     16 epilogue warps write G (the next contractions' operand, sample-major)
-//     into slot t % R of a ring of R tiles in global memory, then publish
-//     ready[slot] = t / R + 1;
+////     into slot t % R of a ring of R tiles in global memory, then count
+//     themselves in ready[slot] (bf16 with more than 128 samples: two CTAs,
+//     one M-block of X each, write the two halves of a tile);
 //   role B (the other CTAs, nG groups x nD d-slices): the CTA of group g and
 //     slice s runs the units (t, s) for t = g, g + nG, ...: it waits for
 //     ready, copies G_t into shared memory (and counts itself in consumed[slot],
@@ -31,9 +32,9 @@
 // work per tile.  Every wait is bounded; a wait that runs out records
 // ELMO_ETIMEOUT in the status word, and the other CTAs stop at their next wait.
 //
-// Used for E4M3 heads with B <= 256 and bf16 heads with B <= 128, d <= 768,
-// d a multiple of 64 (X fits the 384 TMEM columns below role A's
-// accumulators); other shapes run the range-by-range kernels of step_tc.cu.
+// Used for B <= 256, d <= 768, d a multiple of 64 (one M-block of X fits the
+// 384 TMEM columns below role A's accumulators); other shapes run the
+// range-by-range kernels of step_tc.cu.
 #include <stdlib.h>
 
 #include <utility>
@@ -108,7 +109,7 @@ __device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t target, v
   }
 }
 
-template <int kFp8, int kG5>
+template <int kFp8, int kG5, int kW5 = 0>
 __global__ void __launch_bounds__(kFThreads, 1)
     step_fused(const __grid_constant__ CUtensorMap tmWa, const __grid_constant__ CUtensorMap tmWb,
                const __grid_constant__ CUtensorMap tmX, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
@@ -130,11 +131,17 @@ __global__ void __launch_bounds__(kFThreads, 1)
     uint8_t* ring = base;
     SmemFA* S = reinterpret_cast<SmemFA*>(base + kFStagesA * kFBoxA);
     volatile int* abort = &S->abort;
-    const int a = blockIdx.x;
     const int kbe = kFp8 ? 128 : 64;                          // elements of one 128-byte k-block
     const int nkb = (d + kbe - 1) / kbe;
     const uint32_t opcols = (uint32_t)nkb * 32;               // TMEM columns of one M-block of X
-    const int nmb = (Bp + 127) / 128;                         // M-blocks of samples: 1 or 2
+    // Producers of a tile: one CTA holds every M-block of X (E4M3 up to 256
+    // samples, bf16 up to 128), or, for bf16 with more than 128 samples, two
+    // neighbouring CTAs hold one M-block each and write their halves of G.
+    const int nprod = (!kFp8 && Bp > 128) ? 2 : 1;
+    const int amb = nprod == 2 ? (int)(blockIdx.x & 1) : 0;   // first M-block held here
+    const int a = nprod == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int aN = nprod == 2 ? (nA >> 1) : nA;               // tile stride of the producers
+    const int nmb = nprod == 2 ? 1 : (Bp + 127) / 128;        // M-blocks computed here: 1 or 2
     if (threadIdx.x == 0) {
       for (int s = 0; s < kFStagesA; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
       for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], nmb == 2 ? 8 : kFEpi); }
@@ -153,7 +160,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       // X into TMEM: sample h*128 + r of M-block h in lane r, columns h*opcols ...
       const int q = warp & 3, h = (warp - 2) >> 2;
       if (h < nmb) {
-        const int b = h * 128 + q * 32 + lane;
+        const int b = (amb + h) * 128 + q * 32 + lane;
         const size_t rowbytes = (size_t)d * kEl;
         // E4M3: xop holds the codes by 16-byte column chunk (chunk c of row b at
         // (c * 256 + b) * 16); bf16: xop is X itself, row-major
@@ -183,7 +190,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       if (elect_one()) {
         tma_prefetch_desc(&tmWa);
         uint32_t it = 0;
-        for (int t = a; t < T && !*abort; t += nA) {
+        for (int t = a; t < T && !*abort; t += aN) {
           for (int hf = 0; hf < 2; ++hf) {
             for (int kb = 0; kb < nkb; ++kb, ++it) {
               const int s = (int)(it % kFStagesA);
@@ -197,11 +204,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
       }
     } else if (warp == 1) {
       if (elect_one()) {
-        const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, kFN) : make_idesc(1, 1, 0, 0, 128, kFN);
+        const uint32_t idesc = kFp8 ? make_idesc(0, kW5, 0, 0, 128, kFN) : make_idesc(1, 1, 0, 0, 128, kFN);
         uint32_t it = 0, u = 0;
         if (!mbar_wait(&S->xready, 0, abort, kWaitCycles)) record_timeout(status, abort, 82);
         tc_fence_after();
-        for (int t = a; t < T && !*abort; t += nA) {
+        for (int t = a; t < T && !*abort; t += aN) {
           for (int hf = 0; hf < 2 && !*abort; ++hf) {
             for (int mb = 0; mb < nmb && !*abort; ++mb, ++u) {
               const uint32_t slot = u & 1, ph = (u >> 1) & 1;
@@ -242,7 +249,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       const int mb = nmb == 2 ? h >> 1 : 0;
       const int c_lo = nmb == 2 ? 32 * (h & 1) : 16 * h;
       const int ncol = nmb == 2 ? 32 : 16;
-      const int b = mb * 128 + q * 32 + lane;                // sample
+      const int b = (amb + mb) * 128 + q * 32 + lane;        // sample
       const bool bvalid = b < B;
       const bool bstore = b < Bp;
       const float inv_sx = kFp8 ? xscale[1] : 1.0f;
@@ -252,7 +259,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       unsigned long long* wm = reinterpret_cast<unsigned long long*>(S->pmask[warp - 2]);
       uint32_t use = 0;
       int lt = 0;
-      for (int t = a; t < T && !*abort; t += nA, ++lt) {
+      for (int t = a; t < T && !*abort; t += aN, ++lt) {
         const int slot = t % R, round = t / R;
         uint8_t* gtile = gring + (size_t)slot * tile_bytes;
         // the slot is free once every d-slice's CTA has copied the tile it held
@@ -334,7 +341,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
           if (old == kFEpi - 1) {
             S->arrivals[lt & 3] = 0;
             __threadfence();
-            st_release(ready + slot, round + 1);
+            red_release_add(ready + slot, 1);      // nprod arrivals per round make the tile ready
           }
         }
       }
@@ -353,6 +360,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
   constexpr uint32_t kWSB = kFp8 ? kBox : 2 * kBox;
   constexpr int kBoxCols = 128 / kEl;                         // elements per 128-byte box row
   constexpr int kK = kFp8 ? 32 : 16;                          // MMA K
+  constexpr int kPart = kFp8 ? 256 : 128;                     // samples per G part (one 32 KB slot)
+  const int nparts = (Bp + kPart - 1) / kPart;
+  const int nprod = (!kFp8 && Bp > 128) ? 2 : 1;
   uint8_t* xs = base;
   uint8_t* ws = xs + kFXBytes;
   uint8_t* gs = ws + kFWBytes;
@@ -394,18 +404,26 @@ __global__ void __launch_bounds__(kFThreads, 1)
           for (int qq = 0; qq < 128 / kBoxCols; ++qq)
             if (D0 + qq * kBoxCols < d) tma_load_2d(ws + s * kWSB + qq * kBox, &tmWb, &S->wfull[s], D0 + qq * kBoxCols, t * 128);
         }
-        {
+        const int slot = t % R, round = t / R;
+        if (!wait_flag(ready + slot, nprod * (round + 1), abort, status, kWaitCycles)) {
+          record_timeout(status, abort, 93);
+          break;
+        }
+        fence_proxy_async_global();
+        bool stop = false;
+        for (int p = 0; p < nparts; ++p) {
           const int s = git % kFGSlots;
           const uint32_t ph = (git / kFGSlots) & 1;
           ++git;
-          if (!mbar_wait(&S->gempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 92); break; }
-          const int slot = t % R, round = t / R;
-          if (!wait_flag(ready + slot, round + 1, abort, status, kWaitCycles)) { record_timeout(status, abort, 93); break; }
-          fence_proxy_async_global();
-          const uint32_t bytes = (uint32_t)Bp * kEl * 128u;
+          if (!mbar_wait(&S->gempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 92); stop = true; break; }
+          // samples [p kPart, p kPart + np): a contiguous run of 16-byte chunks
+          const int np = min(kPart, Bp - p * kPart);
+          const uint32_t bytes = (uint32_t)np * kEl * 128u;
           mbar_arrive_expect_tx(&S->gfull[s], bytes);
-          bulk_load(gs + s * kFGSlotBytes, gring + (size_t)slot * tile_bytes, bytes, &S->gfull[s]);
+          bulk_load(gs + s * kFGSlotBytes, gring + (size_t)slot * tile_bytes + (size_t)p * kPart * kEl * 128u, bytes,
+                    &S->gfull[s]);
         }
+        if (stop) break;
       }
     }
   } else if (warp == 1) {
@@ -413,7 +431,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
       const uint32_t gfmt = kG5 ? 1u : 0u;
       // G is stored sample-major: K-major as dX^T's B operand, MN-major as dW's A operand
       const uint32_t idesc_dw = kFp8 ? make_idesc(gfmt, 0, 1, 1, 128, 128) : make_idesc(1, 1, 1, 1, 128, 128);
-      const uint32_t idesc_dx = kFp8 ? make_idesc(0, gfmt, 1, 0, 128, (uint32_t)Bp) : make_idesc(1, 1, 1, 0, 128, (uint32_t)Bp);
       const uint32_t gstride = (uint32_t)(kFp8 ? 8 : 16) * 128u;   // bytes between 8-sample groups
       uint32_t wit = 0, git = 0, dwit = 0;
       bool first = true;
@@ -426,35 +443,43 @@ __global__ void __launch_bounds__(kFThreads, 1)
         ++wit;
         const uint32_t db = dwit & 1, duse = dwit >> 1;
         ++dwit;
-        const int sg = git % kFGSlots;
-        const uint32_t phg = (git / kFGSlots) & 1;
-        ++git;
         if (!mbar_wait(&S->wfull[sw], phw, abort, kWaitCycles)) { record_timeout(status, abort, 95); break; }
         if (!mbar_wait(&S->dwempty[db], (duse & 1) ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 96); break; }
-        if (!mbar_wait(&S->gfull[sg], phg, abort, kWaitCycles)) { record_timeout(status, abort, 97); break; }
         tc_fence_after();
-        // G_t is in shared memory: its ring slot may be reused
-        red_release_add(consumed + t % R, 1);
         const uint32_t wa = smem_u32(ws + sw * kWSB);
-        const uint32_t ga = smem_u32(gs + sg * kFGSlotBytes);
-        // dX^T[slice] += W^T G^T : M = 128 (columns of d), N = Bp, K = 128 labels
-#pragma unroll 1
-        for (int k = 0; k < 128 / kK; ++k) {
-          const uint64_t ad = sw128_desc(wa + k * kK * 128, kBox, 1024);
-          const uint64_t bd = nosw_desc(ga + k * 2 * 128, 128, gstride);
-          if (kFp8) mma_e4m3(tmem, ad, bd, idesc_dx, !(first && k == 0));
-          else mma_bf16(tmem, ad, bd, idesc_dx, !(first && k == 0));
-        }
-        // dW[tile, slice] = G^T X[:, slice] : M = 128 labels, N = 128, K = Bp samples
         const uint32_t dwcol = tmem + 256 + db * 128;
+        bool stop = false;
+        for (int p = 0; p < nparts; ++p) {
+          const int sg = git % kFGSlots;
+          const uint32_t phg = (git / kFGSlots) & 1;
+          ++git;
+          if (!mbar_wait(&S->gfull[sg], phg, abort, kWaitCycles)) { record_timeout(status, abort, 97); stop = true; break; }
+          tc_fence_after();
+          // G_t is in shared memory once its last part is: the ring slot may be reused
+          if (p == nparts - 1) red_release_add(consumed + t % R, 1);
+          const uint32_t ga = smem_u32(gs + sg * kFGSlotBytes);
+          const int np = min(kPart, Bp - p * kPart);
+          const uint32_t idesc_dx =
+              kFp8 ? make_idesc(kW5, gfmt, 1, 0, 128, (uint32_t)np) : make_idesc(1, 1, 1, 0, 128, (uint32_t)np);
+          // dX^T[slice, part] += W^T G_part^T : M = 128 (columns of d), N = np, K = 128 labels
 #pragma unroll 1
-        for (int k = 0; k < Bp / kK; ++k) {
-          const uint64_t ad = nosw_desc(ga + k * (kK / 8) * gstride, gstride, 128);
-          const uint64_t bd = sw128_desc(xa + k * kK * 128, 32768, 1024);
-          if (kFp8) mma_e4m3(dwcol, ad, bd, idesc_dw, k != 0);
-          else mma_bf16(dwcol, ad, bd, idesc_dw, k != 0);
+          for (int k = 0; k < 128 / kK; ++k) {
+            const uint64_t ad = sw128_desc(wa + k * kK * 128, kBox, 1024);
+            const uint64_t bd = nosw_desc(ga + k * 2 * 128, 128, gstride);
+            if (kFp8) mma_e4m3(tmem + (uint32_t)(p * kPart), ad, bd, idesc_dx, !(first && k == 0));
+            else mma_bf16(tmem + (uint32_t)(p * kPart), ad, bd, idesc_dx, !(first && k == 0));
+          }
+          // dW[tile, slice] += G_part^T X[part, slice] : M = 128 labels, N = 128, K = np samples
+#pragma unroll 1
+          for (int k = 0; k < np / kK; ++k) {
+            const uint64_t ad = nosw_desc(ga + k * (kK / 8) * gstride, gstride, 128);
+            const uint64_t bd = sw128_desc(xa + (p * kPart + k * kK) * 128, 32768, 1024);
+            if (kFp8) mma_e4m3(dwcol, ad, bd, idesc_dw, (p | k) != 0);
+            else mma_bf16(dwcol, ad, bd, idesc_dw, (p | k) != 0);
+          }
+          mma_commit(&S->gempty[sg]);
         }
-        mma_commit(&S->gempty[sg]);
+        if (stop) break;
         mma_commit(&S->dwfull[db]);
         first = false;
       }
@@ -492,9 +517,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
       tmem_ld16(taddr, r0);
       tmem_wait_ld();
       tmem_ld16(taddr + 16, r1);
-      if (valid) update16<kFp8>(r0, rw0, wrow, row, jl, l, d, j0, lrs, Wglob);
+      constexpr int kWf = kFp8 ? (kW5 ? 2 : 1) : 0;
+      if (valid) update16<kWf>(r0, rw0, wrow, row, jl, l, d, j0, lrs, Wglob);
       tmem_wait_ld();
-      if (valid) update16<kFp8>(r1, rw1, wrow, row, jl + 16, l, d, j0 + 16, lrs, Wglob);
+      if (valid) update16<kWf>(r1, rw1, wrow, row, jl + 16, l, d, j0 + 16, lrs, Wglob);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) { mbar_arrive(&S->dwempty[db]); mbar_arrive(&S->wempty[sw]); }
@@ -534,22 +560,23 @@ bool fused_step_supported(const elmo_head* h, int32_t B) {
   if (v && v[0] == '0') return false;
   const bool fp8 = h->dt == ELMO_FP8_E4M3;
   const int32_t Bp = padded_batch(B, fp8);
-  return h->d % 64 == 0 && h->d <= 768 && (fp8 ? Bp <= 256 : Bp <= 128);
+  return h->d % 64 == 0 && h->d <= 768 && Bp <= 256;
 }
 
 // Work of one 128-label tile in each role, in the units of the split: role A
 // (Z for the tile, G) against role B (dX^T and dW for every d-slice, and the
 // SR update of every weight, which the epilogue's instruction issue bounds).
 // Measured on B200 for the workloads' shapes; ELMO_FUSED_A overrides nA.
-void fused_split(int grid, int nD, int T, int* nA, int* nG) {
+void fused_split(int grid, int nD, int T, int nprod, int* nA, int* nG) {
   int a = (grid * 27 + 50) / 100;                   // about 27 % of the SMs form G
   const char* v = getenv("ELMO_FUSED_A");
   if (v && atoi(v) > 0) a = atoi(v);
   if (a > grid - nD) a = grid - nD;
-  if (a < 1) a = 1;
+  if (a > nprod * T) a = nprod * T;
+  a = a / nprod * nprod;                            // whole groups of producers
+  if (a < nprod) a = nprod;
   int gg = (grid - a) / nD;
   if (gg > T) gg = T;
-  if (a > T) a = T;
   *nA = a;
   *nG = gg;
 }
@@ -562,7 +589,7 @@ cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float 
   const int T = (int)((h->L + 127) / 128);
   const int nD = (h->d + 127) / 128;
   int nA = 0, nG = 0;
-  fused_split(h->num_sms, nD, T, &nA, &nG);
+  fused_split(h->num_sms, nD, T, (!fp8 && Bp > 128) ? 2 : 1, &nA, &nG);
   const int grid = nA + nG * nD;
   CUtensorMap tmWa, tmWb, tmX;
   cudaError_t e = make_tma_map_2d(&tmWa, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, kFN);
@@ -572,7 +599,8 @@ cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float 
   e = make_tma_map_2d(&tmX, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
                       (uint64_t)B, (uint64_t)h->d, (uint32_t)Bp);
   if (e != cudaSuccess) return e;
-  auto kern = fp8 ? (h->g_e5m2 ? step_fused<1, 1> : step_fused<1, 0>) : step_fused<0, 0>;
+  auto kern = fp8 ? (h->g_e5m2 ? step_fused<1, 1> : h->w_e5m2 ? step_fused<1, 0, 1> : step_fused<1, 0>)
+                  : step_fused<0, 0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemF);
   if (e != cudaSuccess) return e;
   // the ring's flags start at zero every step

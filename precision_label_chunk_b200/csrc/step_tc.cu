@@ -59,7 +59,7 @@ struct SmemA {
   int abort;
 };
 
-template <int kFp8, int kG5 = 0>
+template <int kFp8, int kG5 = 0, int kW5 = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     logits_grad_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int64_t L,
                    int32_t d, int32_t B, int32_t Bp, int64_t l0, int64_t l1, const uint32_t* __restrict__ keys,
@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, (uint32_t)Bp) : make_idesc(1, 1, 0, 0, 128, (uint32_t)Bp);
+      const uint32_t idesc = kFp8 ? make_idesc(kW5, 0, 0, 0, 128, (uint32_t)Bp) : make_idesc(1, 1, 0, 0, 128, (uint32_t)Bp);
       uint32_t it = 0, tc = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
         const uint32_t buf = tc & 1, use = tc >> 1;
@@ -194,7 +194,7 @@ struct SmemP {
   int abort;
 };
 
-template <int kFp8, int kG5 = 0>
+template <int kFp8, int kG5 = 0, int kW5 = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     logits_grad_panel_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                          int64_t L, int32_t d, int32_t B, int32_t Bp, int32_t PN, int32_t nstages, int64_t l0,
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, (uint32_t)PN) : make_idesc(1, 1, 0, 0, 128, (uint32_t)PN);
+      const uint32_t idesc = kFp8 ? make_idesc(kW5, 0, 0, 0, 128, (uint32_t)PN) : make_idesc(1, 1, 0, 0, 128, (uint32_t)PN);
       uint32_t it = 0, tc = 0;
       for (int p = 0; p < npanels && !*abort; ++p) {
         if (!mbar_wait(&S->xfull, p & 1, abort, kWaitCycles)) { record_timeout(status, abort, 43); break; }
@@ -365,7 +365,7 @@ struct SmemXt {
   int abort;
 };
 
-template <int kFp8, int kG5 = 0>
+template <int kFp8, int kG5 = 0, int kW5 = 0>
 __global__ void __launch_bounds__(kXtThreads, 1)
     logits_grad_xt(const __grid_constant__ CUtensorMap tmW, int64_t L, int32_t d, int32_t B, int32_t Bp, int64_t l0,
                    int64_t l1, const uint8_t* __restrict__ xop, const uint32_t* __restrict__ keys,
@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(kXtThreads, 1)
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, kXtN) : make_idesc(1, 1, 0, 0, 128, kXtN);
+      const uint32_t idesc = kFp8 ? make_idesc(0, kW5, 0, 0, 128, kXtN) : make_idesc(1, 1, 0, 0, 128, kXtN);
       uint32_t it = 0, u = 0;
       if (!mbar_wait(&S->xready, 0, abort, kWaitCycles)) record_timeout(status, abort, 75);
       tc_fence_after();
@@ -608,7 +608,7 @@ struct UnitRange {
   int u0, u1;  // [u0, u1) of units ordered (slice-major, tile-minor)
 };
 
-template <int kFp8>
+template <int kFp8, int kW5 = 0>
 __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
     update_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
               const uint8_t* __restrict__ gbuf, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
@@ -750,7 +750,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
             const uint32_t ga = smem_u32(gs + sg * kGSlotBytes);
             const int np = min(kPart, Bp - p * kPart);   // samples in this part (multiple of 32)
             // dX^T[slice, part] += W^T G^T : M = 128 (columns of d), N = np, K = 128 labels
-            const uint32_t idesc_dx = kFp8 ? make_idesc(0, gfmt, 1, gmn ^ 1u, 128, (uint32_t)np)
+            const uint32_t idesc_dx = kFp8 ? make_idesc(kW5, gfmt, 1, gmn ^ 1u, 128, (uint32_t)np)
                                            : make_idesc(1, 1, 1, gmn ^ 1u, 128, (uint32_t)np);
             const uint32_t dxcol = tmem + (uint32_t)(p * kPart);
 #pragma unroll 1
@@ -827,7 +827,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
           for (int g = 0; g < kGrp; ++g) {
             uint32_t rw[8];
             sr_draws16(seed, step, blk_base, l, d, j0 + 16 * g, rw);
-            update16<kFp8>(r[g], rw, wrow, row, jl + 16 * g, l, d, j0 + 16 * g, lrs, Wglob);
+            update16<kFp8 ? (kW5 ? 2 : 1) : 0>(r[g], rw, wrow, row, jl + 16 * g, l, d, j0 + 16 * g, lrs, Wglob);
           }
         }
         tc_fence_before();
@@ -959,7 +959,8 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
     if (e != cudaSuccess) return e;
     const int T = 2 * (int)((l1 - l0 + 127) / 128);
     const int grid = T < h->num_sms ? T : h->num_sms;
-    auto kx = fp8 ? (h->g_e5m2 ? logits_grad_xt<1, 1> : logits_grad_xt<1>) : logits_grad_xt<0>;
+    auto kx = fp8 ? (h->g_e5m2 ? logits_grad_xt<1, 1> : h->w_e5m2 ? logits_grad_xt<1, 0, 1> : logits_grad_xt<1>)
+                  : logits_grad_xt<0>;
     e = cudaFuncSetAttribute(kx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemXt);
     if (e != cudaSuccess) return e;
     const uint8_t* xop = fp8 ? h->xqt : reinterpret_cast<const uint8_t*>(X);
@@ -992,14 +993,17 @@ cudaError_t launch_logits_grad_tc(const elmo_head* h, const uint16_t* X, int32_t
     e = make_tma_map_2d(&tmXp, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
                  (uint64_t)B, (uint64_t)h->d, (uint32_t)PN);
     if (e != cudaSuccess) return e;
-    auto kp = fp8 ? (h->g_e5m2 ? logits_grad_panel_tc<1, 1> : logits_grad_panel_tc<1>) : logits_grad_panel_tc<0>;
+    auto kp = fp8 ? (h->g_e5m2 ? logits_grad_panel_tc<1, 1>
+                               : h->w_e5m2 ? logits_grad_panel_tc<1, 0, 1> : logits_grad_panel_tc<1>)
+                  : logits_grad_panel_tc<0>;
     e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemP);
     if (e != cudaSuccess) return e;
     return launch_k(kp, grid, kThreads, kSmemP, s, pdl, tmW, tmXp, h->L, h->d, B, Bp, PN, nst, l0, l1,
                     (const uint32_t*)h->keys, (const int32_t*)h->tile_ptr, (const float*)h->xscale, gbuf, Zout, Gout,
                     h->status);
   }
-  auto kern = fp8 ? (h->g_e5m2 ? logits_grad_tc<1, 1> : logits_grad_tc<1>) : logits_grad_tc<0>;
+  auto kern = fp8 ? (h->g_e5m2 ? logits_grad_tc<1, 1> : h->w_e5m2 ? logits_grad_tc<1, 0, 1> : logits_grad_tc<1>)
+                  : logits_grad_tc<0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemA);
   if (e != cudaSuccess) return e;
   return launch_k(kern, grid, kThreads, kSmemA, s, pdl, tmW, tmX, h->L, h->d, B, Bp, l0, l1, (const uint32_t*)h->keys,
@@ -1022,7 +1026,7 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
   const int T = (int)((l1 - l0 + 127) / 128);
   const int units = T * ((h->d + 127) / 128);
   const int grid = units < h->num_sms ? units : h->num_sms;
-  auto kern = fp8 ? update_tc<1> : update_tc<0>;
+  auto kern = fp8 ? (h->w_e5m2 ? update_tc<1, 1> : update_tc<1>) : update_tc<0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB);
   if (e != cudaSuccess) return e;
   return launch_k(kern, grid, fp8 ? kThreads : 320, kSmemB, s, pdl, tmW, tmX, static_cast<const uint8_t*>(gbuf), h->W,

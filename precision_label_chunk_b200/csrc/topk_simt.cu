@@ -31,7 +31,8 @@ __device__ __forceinline__ bool before(float sa, int32_t ia, float sb, int32_t i
 
 __device__ __forceinline__ float w_at(const void* W, int dt, int64_t i) {
   return dt == ELMO_BF16 ? bf16_to_f32(static_cast<const uint16_t*>(W)[i])
-                         : e4m3_to_f32(static_cast<const uint8_t*>(W)[i]);
+         : dt == ELMO_FP8_E5M2 ? e5m2_to_f32(static_cast<const uint8_t*>(W)[i])
+                               : e4m3_to_f32(static_cast<const uint8_t*>(W)[i]);
 }
 
 // Work item w = (row r, segment seg) with r = w / nseg: the segment's top-k of
@@ -175,7 +176,7 @@ cudaError_t launch_topk_simt_rows(const elmo_head* h, const uint16_t* X, int32_t
   const int64_t items = (int64_t)B * nseg;
   const int64_t cap = (int64_t)h->num_sms * 8;
   const int grid = (int)(rows ? cap : (items < cap ? items : cap));
-  topk_segment_kernel<<<grid, kTopkThreads, smem, s>>>(h->W, (int)h->dt, h->L, h->d, X, k, nseg, B, rows, nrows, cs,
+  topk_segment_kernel<<<grid, kTopkThreads, smem, s>>>(h->W, w_format(h), h->L, h->d, X, k, nseg, B, rows, nrows, cs,
                                                        ci);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

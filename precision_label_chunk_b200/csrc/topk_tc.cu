@@ -251,7 +251,7 @@ __device__ __forceinline__ float ord_value(uint32_t k) {
 // thr of a range is the largest threshold it used.
 // Tiles of 64 labels (the MMA's N) with two accumulator buffers: the A
 // operands take 384 of the 512 TMEM columns.
-template <int kFp8>
+template <int kFp8, int kW5 = 0>
 __global__ void __launch_bounds__(kSThreads, 1)
     topk_screen_tc(const __grid_constant__ CUtensorMap tmW, int64_t lbase, int64_t L, int32_t d, int32_t B, int32_t kp,
                    int32_t ngroups, const uint8_t* __restrict__ xa, const uint8_t* __restrict__ xb,
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const uint32_t idesc = kFp8 ? make_idesc(0, 0, 0, 0, 128, kN) : make_idesc(1, 1, 0, 0, 128, kN);
+      const uint32_t idesc = kFp8 ? make_idesc(0, kW5, 0, 0, 128, kN) : make_idesc(1, 1, 0, 0, 128, kN);
       uint32_t it = 0, tc = 0;
       for (int64_t t = t0; t < t1 && !*abort; ++t, ++tc) {
         const uint32_t buf = tc % kNBuf, use = tc / kNBuf;
@@ -433,7 +433,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
 // ---------------------------------------------------------------- stage 2: selection, exact rescoring, certificate
 __device__ __forceinline__ float w_at(const void* W, int dt, int64_t i) {
   return dt == ELMO_BF16 ? bf16_to_f32(static_cast<const uint16_t*>(W)[i])
-                         : e4m3_to_f32(static_cast<const uint8_t*>(W)[i]);
+         : dt == ELMO_FP8_E5M2 ? e5m2_to_f32(static_cast<const uint8_t*>(W)[i])
+                               : e4m3_to_f32(static_cast<const uint8_t*>(W)[i]);
 }
 
 // The certificate's bound on |exact chain score - screening score| of a query
@@ -446,6 +447,7 @@ __device__ __forceinline__ float screen_bound(float gamma, float n1, float r1, f
 }
 
 __device__ __forceinline__ float maxw_value(uint32_t wc, int dt) {
+  if (dt == ELMO_FP8_E5M2) return wc >= 0x7Cu ? NAN : e5m2_to_f32((uint8_t)wc);   // 0x7C inf, above NaN
   return dt == ELMO_FP8_E4M3 ? (wc >= 0x7Fu ? NAN : e4m3_to_f32((uint8_t)wc))
                              : (wc >= 0x7F80u ? NAN : bf16_to_f32((uint16_t)wc));
 }
@@ -523,7 +525,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(
   if (tid < m) {
     const int64_t l = si[tid];
     float acc = 0.0f;
-    if (dt == ELMO_FP8_E4M3) {
+    if (dt == ELMO_FP8_E4M3 || dt == ELMO_FP8_E5M2) {
       const uint4* wr = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(W) + l * d);
       for (int j0 = 0; j0 < d; j0 += 16) {
         const uint4 q4 = wr[j0 >> 4];
@@ -531,7 +533,8 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float f4[4];
-          e4m3x4_to_f32(wq[e], f4);
+          if (dt == ELMO_FP8_E5M2) e5m2x4_to_f32(wq[e], f4);
+          else e4m3x4_to_f32(wq[e], f4);
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc = __fmaf_rn(xs[j0 + 4 * e + i], f4[i], acc);
         }
@@ -674,7 +677,7 @@ cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k
   if (e != cudaSuccess) return e;
   const size_t smem = 1024 + kSStages * kSBox + sizeof(float) * kN * 128 + 2 * sizeof(float) * (size_t)o.kp * 128 +
                       sizeof(SmemS);
-  auto ks = fp8 ? topk_screen_tc<1> : topk_screen_tc<0>;
+  auto ks = fp8 ? (h->w_e5m2 ? topk_screen_tc<1, 1> : topk_screen_tc<1>) : topk_screen_tc<0>;
   e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScreenSmem);
   if (e != cudaSuccess) return e;
   {
@@ -694,7 +697,7 @@ cudaError_t launch_topk_tc(elmo_head* h, const uint16_t* X, int32_t B, int32_t k
   if (e != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(s, h->join, 0)) != cudaSuccess) return e;
   KernelScope sc(h, ELMO_K_TOPK_MERGE, s, 3);
-  topk_select_kernel<<<B, kSelThreads, ssmem, s>>>(cs, ci, thr, o.G, o.kp, k, o.npow2, X, h->W, (int)h->dt, h->d,
+  topk_select_kernel<<<B, kSelThreads, ssmem, s>>>(cs, ci, thr, o.G, o.kp, k, o.npow2, X, h->W, w_format(h), h->d,
                                                    gamma, n1, r1, rflag, wmax, idx, score, fail, nfail);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
@@ -736,7 +739,7 @@ cudaError_t launch_topk_screen_dump(elmo_head* h, const uint16_t* X, int32_t B, 
   const int eb = fp8 ? 1 : 2;
   e = make_tma_map_2d(&tmW, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, (uint32_t)o.N);
   if (e != cudaSuccess) return e;
-  auto ks = fp8 ? topk_screen_tc<1> : topk_screen_tc<0>;
+  auto ks = fp8 ? (h->w_e5m2 ? topk_screen_tc<1, 1> : topk_screen_tc<1>) : topk_screen_tc<0>;
   e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScreenSmem);
   if (e != cudaSuccess) return e;
   const int64_t nl = l1 - l0;
@@ -753,7 +756,7 @@ cudaError_t launch_topk_screen_dump(elmo_head* h, const uint16_t* X, int32_t B, 
   const int nkb = (h->d * eb + 127) / 128;
   const int nsteps = (fp8 ? 2 : 1) * nkb * 4;
   const float gamma = (float)((double)nsteps * 0x1p-20 + 1.01 * (double)h->d * 0x1p-24);
-  topk_bound_kernel<<<(B + 127) / 128, 128, 0, s>>>(B, gamma, n1, r1, rflag, wmax, (int)h->dt, bound);
+  topk_bound_kernel<<<(B + 127) / 128, 128, 0, s>>>(B, gamma, n1, r1, rflag, wmax, w_format(h), bound);
   return cudaGetLastError();
 }
 

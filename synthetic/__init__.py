@@ -40,7 +40,8 @@ class Workload:
     B: int                # samples per step
     d: int                # embedding width
     L: int                # number of labels
-    dtype: str            # "bf16" or "fp8" (storage type of W); "fp8_ge5m2": E4M3 W, E5M2 gradient operand
+    dtype: str            # "bf16" or "fp8" (storage type of W); "fp8_ge5m2": E4M3 W, E5M2 gradient operand;
+                          # "e5m2": E5M2 W (E4M3 X and gradient operand)
     lam: float            # positives per sample: 1 + Poisson(lam)
     zipf_s: float         # Zipf exponent of the label law
     lr: float
@@ -64,6 +65,9 @@ WORKLOADS = {
                  zipf_s=1.0, lr=0.0, chunk=131_072, steps=1, topk=5),
         # the 3M-label head with an E5M2 gradient operand (same inputs as product3m_fp8)
         Workload("product3m_fp8_ge5m2", 2, B=256, d=768, L=3_000_000, dtype="fp8_ge5m2", lam=35,
+                 zipf_s=1.0, lr=0.1, chunk=131_072, steps=20),
+        # the 3M-label head with E5M2 weights (same inputs as product3m_fp8)
+        Workload("product3m_e5m2", 2, B=256, d=768, L=3_000_000, dtype="e5m2", lam=35,
                  zipf_s=1.0, lr=0.1, chunk=131_072, steps=20),
     ]
 }

@@ -48,7 +48,7 @@ def run_step_with_operands(elmo, W, X, rowptr, cols, lr, chunk, seed, step, dtyp
     """The logits and gradient operands of every label (forward_chunk, over
     ranges of `span` labels; W untouched), then one step on the same head.
     Returns (new W codes, dX, Z [L, B], G [L, B])."""
-    Wd = w_to_dev(W, "bf16" if dtype == "bf16" else "fp8")
+    Wd = w_to_dev(W, "bf16" if dtype == "bf16" else "fp8")     # one byte per code for every 8-bit grid
     h = elmo.elmo_init_head(Wd, dtype)
     Xd, rp, cl = to_dev_u16(X), to_dev_i32(rowptr), to_dev_i32(cols)
     L, B = W.shape[0], X.shape[0]

@@ -23,7 +23,12 @@ import os
 
 import numpy as np
 
-REL_TOL = {"bf16": 2e-2, "fp8": 6e-2, "fp8_ge5m2": 1.2e-1}
+REL_TOL = {"bf16": 2e-2, "fp8": 6e-2, "fp8_ge5m2": 1.2e-1, "e5m2": 6e-2}
+
+
+def weight_dtype(dtype):
+    """The grid the weights of a head of `dtype` are stored on."""
+    return {"bf16": "bf16", "fp8": "fp8", "fp8_ge5m2": "fp8", "e5m2": "e5m2"}[dtype]
 
 FLOOR = 1e-2
 
@@ -79,11 +84,21 @@ def weight_parity(gpu_codes, orc_codes, dtype, chunk_rows=None):
     return within, worst
 
 
+def _worst_weights(gpu_codes, orc_codes, dtype, n=6):
+    d = np.abs(ordinal(gpu_codes, dtype) - ordinal(orc_codes, dtype)).reshape(np.shape(gpu_codes)[0], -1)
+    idx = np.argsort(d, axis=None)[::-1][:n]
+    g = np.asarray(gpu_codes).reshape(d.shape)
+    o = np.asarray(orc_codes).reshape(d.shape)
+    return [(int(i // d.shape[1]), int(i % d.shape[1]), hex(int(g.flat[i])), hex(int(o.flat[i]))) for i in idx]
+
+
 def assert_weights_close(gpu_codes, orc_codes, dtype, chunk_rows=None):
     within, worst = weight_parity(gpu_codes, orc_codes, dtype, chunk_rows)
     _record({"what": "weights", "within_1ulp": within, "mean_signed_err_ulp": worst})
-    assert within >= 0.999, f"only {within:.5%} of weights within 1 ulp"
-    assert worst <= 0.05, f"mean signed error {worst:.4f} ulp over a chunk"
+    assert within >= 0.999, (f"only {within:.5%} of weights within 1 ulp; largest differences "
+                             f"(row, col, gpu, oracle) {_worst_weights(gpu_codes, orc_codes, dtype)}")
+    assert worst <= 0.05, (f"mean signed error {worst:.4f} ulp over a chunk; largest differences "
+                           f"(row, col, gpu, oracle) {_worst_weights(gpu_codes, orc_codes, dtype)}")
 
 
 def assert_rel_close(a, b, dtype, axis=-1, what="values"):
@@ -97,7 +112,7 @@ def assert_rel_close(a, b, dtype, axis=-1, what="values"):
 
 # ---------------------------------------------------------------- gradient operands
 def operand_format(dtype):
-    return {"bf16": "bf16", "fp8": "e4m3", "fp8_ge5m2": "e5m2"}[dtype]
+    return {"bf16": "bf16", "fp8": "e4m3", "fp8_ge5m2": "e5m2", "e5m2": "e4m3"}[dtype]
 
 
 def sigmoid_f32(z):
@@ -134,6 +149,8 @@ def weight_values(W, dtype):
     import ml_dtypes
     if dtype == "bf16":
         return np.asarray(W).view(ml_dtypes.bfloat16).astype(np.float64)
+    if dtype == "e5m2":
+        return np.asarray(W).view(ml_dtypes.float8_e5m2).astype(np.float64)
     return np.asarray(W).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
 
 
@@ -175,8 +192,8 @@ def check_step(orc, W, X, rowptr, cols, lr, seed, step, dtype, Wg, dXg, Zg, Gg, 
         assert_rel_close(Zg, r["Z"], "bf16" if dtype == "bf16" else "fp8", axis=None, what="Z")
     assert_operands_of_logits(Gg, Zg, Y, dtype, what="G (GPU)")
     assert_operands_of_logits(r["G"], r["Z"], Y, dtype, what="G (oracle)")
-    dx_ref, flips = flip_corrected_dx(r["dX"], Gg, r["G"], W, "bf16" if dtype == "bf16" else "fp8")
+    dx_ref, flips = flip_corrected_dx(r["dX"], Gg, r["G"], W, weight_dtype(dtype))
     _record({"what": "G flips", "dtype": dtype, "elements": int(np.size(Gg)), "flips": flips})
     assert_rel_close(dXg, dx_ref, dtype, what="dX")
-    assert_weights_close(Wg, r["W"], "bf16" if dtype == "bf16" else "fp8", chunk_rows=chunk_rows)
+    assert_weights_close(Wg, r["W"], weight_dtype(dtype), chunk_rows=chunk_rows)
     return r, flips

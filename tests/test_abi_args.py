@@ -28,8 +28,8 @@ def test_init_head_shard_arguments(lib):
         return lib.elmo_init_head_shard(ctypes.byref(out), W, L, d, dt, base, total, fill, std, 0, None)
 
     assert init(W=None) == EINVAL
-    assert init(dt=3) == EUNSUPPORTED and "E5M2" in _err(lib)        # an SR output grid, not a weight format
-    assert init(dt=9) == EINVAL
+    assert init(dt=9) == EINVAL and "dtype" in _err(lib)
+    assert init(dt=3, L=0) == EINVAL                                   # E5M2 heads take the same checks
     assert init(L=0) == EINVAL and init(L=1 << 24, total=1 << 24) == EINVAL
     assert init(base=-1) == EINVAL
     assert init(base=500, L=600, total=1000) == EINVAL and "outside a head" in _err(lib)
