@@ -122,6 +122,19 @@ __device__ __forceinline__ float sr_e4m3_value(float v, uint32_t k) {
   return (mag > 0x7F800000u) ? __uint_as_float(0x7FC00000u) : out;
 }
 
+// The SR result of a finite v as an fp32 value on the E5M2 grid (magnitudes
+// above 57344 are left there for the saturating conversion).  As for E4M3,
+// with the subnormal range below 2^-14 (spacing 2^-16) moved up one binade.
+__device__ __forceinline__ float sr_e5m2_finite_value(float v, uint32_t k) {
+  const uint32_t b = __float_as_uint(v);
+  const float a = __uint_as_float(b & 0x7FFFFFFFu);
+  const float c = (a < 0x1p-14f) ? 0x1p-14f : 0.0f;
+  const float s = __fadd_ru(a, c);
+  const uint32_t t = (__float_as_uint(s) + 0x1FFFFFu - (k << 5)) & 0xFFE00000u;
+  const float r = __fsub_rn(__uint_as_float(t), c);
+  return __uint_as_float(__float_as_uint(r) | (b & 0x80000000u));
+}
+
 // Two fp32 values -> two E4M3 codes (hi in the upper byte), RNE + saturating.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float hi, float lo) {
   uint16_t r;

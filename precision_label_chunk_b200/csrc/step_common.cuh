@@ -75,14 +75,23 @@ __device__ __forceinline__ float mul_rn_denorm(float a, float b) {
 // G = sigmoid(z) - y rounded to nearest even onto bf16 (kG = 0), or 2^8 G onto
 // E4M3 (kG = 1) or E5M2 (kG = 2), z = acc * inv_sx; y = 1 at the positives.
 // The code is the one that sigmoid(z) = 1 / (1 + e^-z) correctly rounded to
-// fp32 gives.  8-bit grids try a one-tanh pass first (below).  Otherwise
-// sigmoid comes from one ex2 and one rcp of the special-function unit, within
-// 2^-21 relative plus |z| 2^-23 from the rounded argument of ex2;
-// each element is rounded from both ends of an interval around its value that
-// is wider than that error, and where the two ends land on different codes
-// (the value lies within that error of a midpoint of the operand grid, about
-// 2^-15 of the elements at the workloads' logits) sigmoid is recomputed in
-// double precision and rounded to fp32 first.  ybits: positives; vbits: valid
+// fp32 gives.
+//
+// Fast path (y = 0): x = 2^8 sigmoid(z) (or sigmoid(z) for bf16) from one ex2
+// and one rcp of the special-function unit, x = 1 / (2^-8 (1 + 2^t)) with
+// t = acc * (-log2(e) inv_sx) (inv_sx is a power of two, so the one rounding
+// of t is relative 2^-24 and the fp32 log2(e) is within 2^-26 of log2(e)).
+// For z >= -kZlim the distance of x from 2^8 fl32(sigmoid(z)) is below kT
+// units in the last place of x: the rounding of t moves 2^t by at most
+// |z| 1.22 2^-24, ex2 and rcp add their own relative errors (measured on the
+// device: below 2^-22 and 2^-23 over the range used) and 1 + 2^t and sigmoid's
+// own fp32 rounding one ulp each.  Within one binade the grid's midpoints are
+// the fp32 values whose bits below the grid's last mantissa bit read
+// 100...0 (kMid), so x rounds like 2^8 fl32(sigmoid(z)) unless those bits lie
+// within kT of kMid.  Elements where they do (about 2 kT 2^-16 of them for
+// bf16, 2 kT 2^-20 for E4M3), positives, logits below -kZlim, NaN logits and
+// padding take the per-element exact path: sigmoid in double precision,
+// rounded to fp32, then the format's rounding.  ybits: positives; vbits: valid
 // elements (the others, batch padding and labels past the range, get code 0);
 // out: 4 words of 8-bit codes or 8 words of bf16, element 0 in the low bits.
 template <int kG>
@@ -100,80 +109,56 @@ __device__ __noinline__ uint32_t grad_code_exact(float acc, float inv_sx, bool p
 }
 
 template <int kG>
-__device__ __forceinline__ void grad_codes16(const uint32_t* acc, float inv_sx, uint32_t ybits, uint32_t vbits,
-                                             uint32_t* out) {
-  constexpr float sc = kG ? 256.0f : 1.0f;
-  constexpr int kPer = kG ? 4 : 2;                 // codes per 32-bit word
-  constexpr int kBits = 32 / kPer;
-  if (kG) {
-    // 8-bit grids: first 2^8 sigmoid(z) = 128 + 128 tanh(z/2) with a single
-    // tanh of the special-function unit (relative error below 2^-10, so below
-    // 2^-3 in units of 2^8 G); each element is rounded from both ends of a
-    // window of +-0.13 around that value, and the group is done when all the
-    // ends agree.  That holds unless some value lies near a midpoint of the
-    // grid, or is small (2^8 G below a few units, where the grid is finer than
-    // the window): then the group takes the path below.
-    float lo[16], hi[16];
-    const float zh = 0.5f * inv_sx;                 // exact: a power of two
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float x = __fmaf_rn(tanhf_approx(__fmul_rn(__uint_as_float(acc[i]), zh)), 128.0f, 128.0f) -
-                      (((ybits >> i) & 1u) ? 256.0f : 0.0f);
-      const bool v = (vbits >> i) & 1u;
-      lo[i] = v ? x - 0.13f : 0.0f;
-      hi[i] = v ? x + 0.13f : 0.0f;
-    }
-    uint32_t diff = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      out[q] = grad_pack2<kG>(lo[4 * q + 1], lo[4 * q]) | (grad_pack2<kG>(lo[4 * q + 3], lo[4 * q + 2]) << 16);
-      diff |= out[q] ^ (grad_pack2<kG>(hi[4 * q + 1], hi[4 * q]) | (grad_pack2<kG>(hi[4 * q + 3], hi[4 * q + 2]) << 16));
-    }
-    if (!diff) return;
-  }
+struct GradWindow {
+  // fp32 bits below the grid's last mantissa bit, the pattern of a midpoint,
+  // the half-width of the window in ulps of x, the lowest logit of the fast path
+  static constexpr uint32_t kMask = kG == 0 ? 0xFFFFu : (kG == 1 ? 0xFFFFFu : 0x1FFFFFu);
+  static constexpr uint32_t kMid = (kMask >> 1) + 1u;
+  static constexpr uint32_t kT = kG == 0 ? 14u : 24u;
+  static constexpr float kZlim = kG == 0 ? 4.0f : 8.0f;
+};
+
+// the lowest accumulator value of the fast path: -kZlim / inv_sx
+template <int kG>
+__device__ __forceinline__ float grad_acc_floor(float inv_sx) {
+  return __fdiv_rn(-GradWindow<kG>::kZlim, inv_sx);
+}
+
+template <int kG>
+__device__ __forceinline__ void grad_codes16(const uint32_t* acc, float inv_sx, float acc_lo, uint32_t ybits,
+                                             uint32_t vbits, uint32_t* out) {
+  using Wd = GradWindow<kG>;
+  constexpr float isc = kG ? 0.00390625f : 1.0f;
   const float zmul = -1.4426950408889634f * inv_sx;
-  float lo[16], hi[16];
+  float x[16];
+  bool slow = (ybits != 0u) | (vbits != 0xFFFFu);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float a = __uint_as_float(acc[i]);
-    const float e = exp2f_approx(__fmul_rn(a, zmul));
-    const float s = rcpf_approx(__fadd_rn(e, 1.0f));
-    const float as = s * sc;
-    const float xc = as - (((ybits >> i) & 1u) ? sc : 0.0f);
-    // |z| is clamped: beyond 128 sigmoid is 0 or 1 to within fp32's smallest
-    // normal, which the absolute term sc 2^-126 covers (the approximations
-    // flush denormal results to zero); the clamp also keeps 0 * inf out of w
-    const float eps = __fmaf_rn(fminf(fabsf(__fmul_rn(a, inv_sx)), 128.0f), 0x1p-22f, 0x1p-20f);
-    const float w = __fmaf_rn(fabsf(xc), 0x1p-22f, __fmaf_rn(as, eps, sc * 0x1p-126f));
-    const bool v = (vbits >> i) & 1u;
-    lo[i] = v ? xc - w : 0.0f;
-    hi[i] = v ? xc + w : 0.0f;
+    x[i] = rcpf_approx(__fmaf_rn(exp2f_approx(__fmul_rn(a, zmul)), isc, isc));
+    const uint32_t off = (__float_as_uint(x[i]) - (Wd::kMid - Wd::kT)) & Wd::kMask;
+    slow |= (off <= 2u * Wd::kT) | !(a >= acc_lo);
   }
-  uint32_t wlo[16 / kPer], whi[16 / kPer];
 #pragma unroll
-  for (int q = 0; q < 16 / kPer; ++q) {
-    if (kG) {
-      wlo[q] = grad_pack2<kG>(lo[4 * q + 1], lo[4 * q]) | (grad_pack2<kG>(lo[4 * q + 3], lo[4 * q + 2]) << 16);
-      whi[q] = grad_pack2<kG>(hi[4 * q + 1], hi[4 * q]) | (grad_pack2<kG>(hi[4 * q + 3], hi[4 * q + 2]) << 16);
-    } else {
-      wlo[q] = grad_pack2<kG>(lo[2 * q + 1], lo[2 * q]);
-      whi[q] = grad_pack2<kG>(hi[2 * q + 1], hi[2 * q]);
-    }
-  }
-  uint32_t diff = 0;
-#pragma unroll
-  for (int q = 0; q < 16 / kPer; ++q) diff |= wlo[q] ^ whi[q];
-  if (diff) {                                      // rare: a value near a midpoint of the grid
-#pragma unroll
+  for (int q = 0; q < (kG ? 4 : 8); ++q)
+    out[q] = kG ? grad_pack2<kG>(x[4 * q + 1], x[4 * q]) | (grad_pack2<kG>(x[4 * q + 3], x[4 * q + 2]) << 16)
+                : grad_pack2<kG>(x[2 * q + 1], x[2 * q]);
+  if (slow) {                                  // rare: positives, padding, near-midpoint or low logits
+    constexpr int kPer = kG ? 4 : 2;
+    constexpr int kBits = 32 / kPer;
+#pragma unroll 1
     for (int i = 0; i < 16; ++i) {
-      const int q = i / kPer, sh = (i % kPer) * kBits;
-      const uint32_t m = (kG ? 0xFFu : 0xFFFFu) << sh;
-      if ((wlo[q] ^ whi[q]) & m)
-        wlo[q] = (wlo[q] & ~m) | (grad_code_exact<kG>(__uint_as_float(acc[i]), inv_sx, (ybits >> i) & 1u) << sh);
+      const float a = __uint_as_float(acc[i]);
+      const uint32_t off = (__float_as_uint(x[i]) - (Wd::kMid - Wd::kT)) & Wd::kMask;
+      const bool v = (vbits >> i) & 1u, y = (ybits >> i) & 1u;
+      if (!v || y || off <= 2u * Wd::kT || !(a >= acc_lo)) {
+        const uint32_t c = v ? grad_code_exact<kG>(a, inv_sx, y) : 0u;
+        const int q = i / kPer, sh = (i % kPer) * kBits;
+        const uint32_t m = (kG ? 0xFFu : 0xFFFFu) << sh;
+        out[q] = (out[q] & ~m) | (c << sh);
+      }
     }
   }
-#pragma unroll
-  for (int q = 0; q < 16 / kPer; ++q) out[q] = wlo[q];
 }
 
 // The operand value of code `c` (G, with 2^-8 undone for the 8-bit formats).
@@ -186,14 +171,14 @@ __device__ __forceinline__ float grad_value(uint32_t c) {
 // G for 16 samples b0 .. b0+15 of one label row, stored label-major as the
 // next contraction's operand (the resident-X and streamed-X kernels A).
 template <int kFp8, int kG5 = 0>
-__device__ __forceinline__ void grad16(const uint32_t* r, float inv_sx, uint32_t ybits, int b0, int B,
+__device__ __forceinline__ void grad16(const uint32_t* r, float inv_sx, float acc_lo, uint32_t ybits, int b0, int B,
                                        uint8_t* __restrict__ gtile, int row, bool row_invalid,
                                        float* __restrict__ Zrow, float* __restrict__ Grow) {
   constexpr int kG = kFp8 ? (kG5 ? 2 : 1) : 0;
   uint32_t vbits = 0;
   if (!row_invalid) vbits = b0 + 16 <= B ? 0xFFFFu : (B > b0 ? (1u << (B - b0)) - 1u : 0u);
   uint32_t packed[8];
-  grad_codes16<kG>(r, inv_sx, ybits, vbits, packed);
+  grad_codes16<kG>(r, inv_sx, acc_lo, ybits, vbits, packed);
   if (kFp8) {
     const int j = b0 >> 4;                                   // 16-byte chunk of samples
     *reinterpret_cast<uint4*>(gtile + ((j * 16 + (row >> 3)) << 7) + ((row & 7) << 4)) =
@@ -244,28 +229,22 @@ __device__ __forceinline__ void sr_draws16(uint64_t seed, uint64_t step, uint64_
 // 128B-swizzled W tile in shared memory (row `row`, tile column jl), draws rw
 // from sr_draws16.
 //
-// v = fl(w - fl(lrs dW)) (two roundings, denormals kept); a probe that is not
-// finite when some v is NaN or infinite (E4M3: the sum of 0 v; bf16: the sum
-// of 2 v, which also overflows once some |v| >= 2^127, where rounding could
-// pass the largest finite value) sends the group to the exact per-element path.
-//
-// Fast rounding, both grids: add-and-truncate.  If the bits of v below the
-// target precision hold the fraction F (in units of 2^-n of a grid step),
-// u < f  <=>  2^(n-16) k < F  <=>  adding 2^n - 1 - 2^(n-16) k carries into the
-// first kept bit.
+// v = fl(w - fl(lrs dW)) (two roundings, denormals kept), then add-and-
+// truncate: if the bits of v below the target precision hold the fraction F
+// (in units of 2^-n of a grid step), u < f  <=>  2^(n-16) k < F  <=>  adding
+// 2^n - 1 - 2^(n-16) k carries into the first kept bit.
 // bf16 (n = 16): the hardware's stochastic conversion cvt.rs.bf16x2.f32 adds
 // its 16 random bits to the 16 discarded bits of each value and truncates, so
 // passing 2^16 - 1 - k (the complemented draw) gives exactly this rounding.
-// E4M3 (n = 20): from 2^-6 up, E4M3 keeps 3 of fp32's 23 mantissa bits; below
-// 2^-6 (its subnormal range, spacing 2^-9) |v| is first moved into
-// [2^-6, 2^-5), whose spacing is also 2^-9, by adding 2^-6 rounded toward
-// +infinity (that keeps ceil(F), and for an integer k, 16 k < F <=> 16 k <
+// E4M3 (n = 20) and E5M2 (n = 21): below the smallest normal value (2^-6,
+// 2^-14) the grid is uniform; |v| is first moved up one binade, whose spacing
+// equals the subnormal spacing, by an add rounded toward +infinity (that
+// keeps ceil(F), and for an integer k, 2^(n-16) k < F <=> 2^(n-16) k <
 // ceil(F), so the decision stays exact), truncated there and moved back
-// exactly; the sign is restored and the saturating conversion maps magnitudes
-// at or above 448 to 448.
-// kW: the weight grid, 0 bf16, 1 E4M3, 2 E5M2 (E5M2 as E4M3 with 2 mantissa
-// bits kept, n = 21, subnormal range below 2^-14 with spacing 2^-16; +-inf is
-// an E5M2 value and stays, so groups holding one take the per-element path).
+// exactly; the sign is restored and the saturating conversion maps
+// magnitudes at or above the largest finite value to it.
+// kW: the weight grid, 0 bf16, 1 E4M3, 2 E5M2 (+-inf is an E5M2 value and
+// stays, so E5M2 groups holding one take the per-element path).
 template <int kW>
 __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t (&rw)[8],
                                          const uint8_t* __restrict__ wtile, int row, int jl, int64_t l, int32_t d,
@@ -296,65 +275,63 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t
     }
   }
   float vv[16];
-  float probe = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
-    probe = __fmaf_rn(vv[i], kW ? 0.0f : 2.0f, probe);
-  }
-  const bool fast = fabsf(probe) < INFINITY;
+  for (int i = 0; i < 16; ++i) vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
   uint32_t wnew[8];
-  if (fast) {
-    if (kW) {
-      // the subnormal range is moved up one binade: [2^-6, 2^-5) for E4M3,
-      // [2^-14, 2^-13) for E5M2, whose spacing equals the subnormal spacing
-      constexpr float kLow = kW == 1 ? 0x1p-6f : 0x1p-14f;
-      constexpr float kSel = kW == 1 ? 0x1p94f : 0x1p86f;   // (kLow - |v|) 2^100 >= 1 exactly when |v| < kLow
-      constexpr uint32_t kMask = kW == 1 ? 0xFFF00000u : 0xFFE00000u;
-      constexpr uint32_t kOne = kW == 1 ? 0xFFFFFu : 0x1FFFFFu;
-      constexpr int kShift = kW == 1 ? 4 : 5;
+  if (kW == 1) {
+    // per element and branch-free, NaN and infinities included (the
+    // saturating conversion maps magnitudes at or above 448 to 448)
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        float o[4];
+    for (int q4 = 0; q4 < 4; ++q4) {
+      float o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t word = rw[2 * q4 + (e >> 1)];
-          const uint32_t k16 = (e & 1) ? (word >> 16) : (word & 0xFFFFu);
-          const float a = fabsf(vv[4 * q4 + e]);
-          const float sat = __saturatef(__fmaf_rn(-a, 0x1p100f, kSel));
-          const float sh = __fmaf_ru(sat, kLow, a);
-          const uint32_t t = (__float_as_uint(sh) + (kOne - (k16 << kShift))) & kMask;
-          o[e] = copysignf(__fmaf_rn(sat, -kLow, __uint_as_float(t)), vv[4 * q4 + e]);
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t word = rw[2 * q4 + (e >> 1)];
+        o[e] = sr_e4m3_value(vv[4 * q4 + e], (e & 1) ? (word >> 16) : (word & 0xFFFFu));
+      }
+      wnew[q4] = pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16);
+    }
+  } else {
+    // a probe that is not finite when some v is NaN or infinite (E5M2: the
+    // sum of 0 v; bf16: the sum of 2 v, which also overflows once some
+    // |v| >= 2^127, where rounding could pass the largest finite value) sends
+    // the group to the exact per-element path
+    float probe = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) probe = __fmaf_rn(vv[i], kW ? 0.0f : 2.0f, probe);
+    if (fabsf(probe) < INFINITY) {
+      if (kW) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t word = rw[2 * q4 + (e >> 1)];
+            o[e] = sr_e5m2_finite_value(vv[4 * q4 + e], (e & 1) ? (word >> 16) : (word & 0xFFFFu));
+          }
+          wnew[q4] = pack_e5m2x2(o[1], o[0]) | (pack_e5m2x2(o[3], o[2]) << 16);
         }
-        wnew[q4] = kW == 1 ? pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16)
-                           : pack_e5m2x2(o[1], o[0]) | (pack_e5m2x2(o[3], o[2]) << 16);
+      } else {
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          uint32_t o;   // element 2p (low half) takes the low 16 random bits, 2p + 1 the high
+          asm("cvt.rs.bf16x2.f32 %0, %1, %2, %3;" : "=r"(o) : "f"(vv[2 * p + 1]), "f"(vv[2 * p]), "r"(~rw[p]));
+          wnew[p] = o;
+        }
       }
     } else {
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        uint32_t o;   // element 2p (low half) takes the low 16 random bits, 2p + 1 the high
-        asm("cvt.rs.bf16x2.f32 %0, %1, %2, %3;" : "=r"(o) : "f"(vv[2 * p + 1]), "f"(vv[2 * p]), "r"(~rw[p]));
-        wnew[p] = o;
-      }
-    }
-  } else {
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      if (kW == 1) {
-        if (p < 4) {
-          const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
-          const float o0 = sr_e4m3_value(vv[4 * p], w0 & 0xFFFFu), o1 = sr_e4m3_value(vv[4 * p + 1], w0 >> 16);
-          const float o2 = sr_e4m3_value(vv[4 * p + 2], w1 & 0xFFFFu), o3 = sr_e4m3_value(vv[4 * p + 3], w1 >> 16);
-          wnew[p] = pack_e4m3x2(o1, o0) | (pack_e4m3x2(o3, o2) << 16);
+        if (kW == 2) {
+          if (p < 4) {
+            const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
+            wnew[p] = sr_e5m2_code(vv[4 * p], w0 & 0xFFFFu) | (sr_e5m2_code(vv[4 * p + 1], w0 >> 16) << 8) |
+                      (sr_e5m2_code(vv[4 * p + 2], w1 & 0xFFFFu) << 16) |
+                      (sr_e5m2_code(vv[4 * p + 3], w1 >> 16) << 24);
+          }
+        } else {
+          wnew[p] = (uint32_t)sr_bf16(vv[2 * p], rw[p] & 0xFFFFu) | ((uint32_t)sr_bf16(vv[2 * p + 1], rw[p] >> 16) << 16);
         }
-      } else if (kW == 2) {
-        if (p < 4) {
-          const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
-          wnew[p] = sr_e5m2_code(vv[4 * p], w0 & 0xFFFFu) | (sr_e5m2_code(vv[4 * p + 1], w0 >> 16) << 8) |
-                    (sr_e5m2_code(vv[4 * p + 2], w1 & 0xFFFFu) << 16) | (sr_e5m2_code(vv[4 * p + 3], w1 >> 16) << 24);
-        }
-      } else {
-        wnew[p] = (uint32_t)sr_bf16(vv[2 * p], rw[p] & 0xFFFFu) | ((uint32_t)sr_bf16(vv[2 * p + 1], rw[p] >> 16) << 16);
       }
     }
   }

@@ -253,6 +253,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       const bool bvalid = b < B;
       const bool bstore = b < Bp;
       const float inv_sx = kFp8 ? xscale[1] : 1.0f;
+      const float acc_lo = grad_acc_floor<kFp8 ? (kG5 ? 2 : 1) : 0>(inv_sx);
       constexpr int kG = kFp8 ? (kG5 ? 2 : 1) : 0;
       constexpr int kChunk = 16 / kEl;                        // labels per 16-byte chunk
       constexpr int kNlc = 128 / kChunk;                      // chunks per 128-label tile
@@ -317,7 +318,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
             const int64_t nv = L - (lc0 + j);
             const uint32_t vbits = !bvalid || nv <= 0 ? 0u : (nv >= 16 ? 0xFFFFu : (1u << nv) - 1u);
             uint32_t pk[8];
-            grad_codes16<kG>(v + j, inv_sx, (uint32_t)(pm >> j) & 0xFFFFu, vbits, pk);
+            grad_codes16<kG>(v + j, inv_sx, acc_lo, (uint32_t)(pm >> j) & 0xFFFFu, vbits, pk);
             if (bstore) {
               const int lc = (lt0 + j) / kChunk;
               *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =

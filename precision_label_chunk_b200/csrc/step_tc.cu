@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const float inv_sx = kFp8 ? xscale[1] : 1.0f;
+    const float acc_lo = grad_acc_floor<kFp8 ? (kG5 ? 2 : 1) : 0>(inv_sx);
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
       const uint32_t buf = tc & 1, use = tc >> 1;
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int b0 = c * 32 + k * 16;
-          grad16<kFp8, kG5>(ra + k * 16, inv_sx, mask16(mask, b0), b0, B,
+          grad16<kFp8, kG5>(ra + k * 16, inv_sx, acc_lo, mask16(mask, b0), b0, B,
                        static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                        Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
         }
@@ -298,6 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const float inv_sx = kFp8 ? xscale[1] : 1.0f;
+    const float acc_lo = grad_acc_floor<kFp8 ? (kG5 ? 2 : 1) : 0>(inv_sx);
     uint32_t tc = 0;
     for (int p = 0; p < npanels && !*abort; ++p) {
       for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tc) {
@@ -322,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 2; ++k) {
             const int cb = c * 32 + k * 16;             // panel column
             const int b0 = p * PN + cb;                 // sample
-            grad16<kFp8, kG5>(ra + k * 16, inv_sx, mask16(mask, b0), b0, B,
+            grad16<kFp8, kG5>(ra + k * 16, inv_sx, acc_lo, mask16(mask, b0), b0, B,
                          static_cast<uint8_t*>(gbuf) + (size_t)t * 128 * Bp * (kFp8 ? 1 : 2), row, !valid,
                          Zout ? Zout + rowoff * B + b0 : nullptr, Gout ? Gout + rowoff * B + b0 : nullptr);
           }
@@ -498,6 +500,7 @@ __global__ void __launch_bounds__(kXtThreads, 1)
     const bool bvalid = b < B;
     const bool bstore = b < Bp;
     const float inv_sx = kFp8 ? xscale[1] : 1.0f;
+    const float acc_lo = grad_acc_floor<kFp8 ? (kG5 ? 2 : 1) : 0>(inv_sx);
     constexpr int kG = kFp8 ? (kG5 ? 2 : 1) : 0;                 // operand format of G
     constexpr int kEl = kFp8 ? 1 : 2;
     constexpr int kChunk = 16 / kEl;                          // labels per 16-byte chunk
@@ -550,7 +553,7 @@ __global__ void __launch_bounds__(kXtThreads, 1)
         const int64_t nv = l1 - (lc0 + j);
         const uint32_t vbits = !bvalid || nv <= 0 ? 0u : (nv >= 16 ? 0xFFFFu : (1u << nv) - 1u);
         uint32_t pk[8];
-        grad_codes16<kG>(v + j, inv_sx, (uint32_t)(pm >> j) & 0xFFFFu, vbits, pk);
+        grad_codes16<kG>(v + j, inv_sx, acc_lo, (uint32_t)(pm >> j) & 0xFFFFu, vbits, pk);
         if (kFp8) {
           if (bstore) {
             const int lc = (lt + j) / kChunk;

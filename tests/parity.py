@@ -13,7 +13,10 @@ Tolerances (from the stated targets of the step):
                  to nearest even onto bf16, or 2^8 G onto E4M3 / E5M2), checked
                  element by element; where the two logits (fp32 sums in
                  different orders) round to different operand codes, the oracle's
-                 dX is corrected by exactly those terms before comparing;
+                 dX is corrected by exactly those terms before comparing, and
+                 the label rows holding them are re-stepped from the GPU's
+                 operands (the flip moves the whole row's update); operands
+                 of the two sides never differ by more than one grid step;
   weights:       at least 99.9 % of elements within 1 grid ulp of the oracle
                  and |mean signed error| <= 0.05 ulp over every chunk;
   SR, Philox draws and top-k indices: bit-exact.
@@ -177,6 +180,60 @@ def flip_corrected_dx(dx_orc, G_gpu, G_orc, W, w_dtype):
     return dx, int(ls.size)
 
 
+def operand_codes(G, dtype):
+    """Grid codes (as ordinals) of gradient operand values G (2^-8 undone)."""
+    import ml_dtypes
+    fmt = operand_format(dtype)
+    g = np.asarray(G, np.float32)
+    if fmt == "bf16":
+        return ordinal(g.astype(ml_dtypes.bfloat16).view(np.uint16), "bf16")
+    t = ml_dtypes.float8_e4m3fn if fmt == "e4m3" else ml_dtypes.float8_e5m2
+    return ordinal((g * np.float32(256.0)).astype(t).view(np.uint8), "fp8")
+
+
+def x_operand(orc, X, dtype):
+    """The X values the update's contraction uses: the bf16 inputs, or (8-bit
+    heads) their E4M3 codes under the per-step scale s_X, divided by s_X."""
+    Xf = orc.bf16_value(np.asarray(X, np.uint16))
+    if dtype == "bf16":
+        return Xf
+    sx = np.float32(orc.fp8_x_scale(X))
+    return orc.e4m3_value(orc.rne_e4m3((Xf * sx).astype(np.float32))) / sx
+
+
+def flip_corrected_weights(orc, W, X, G_gpu, G_orc, W_new, lr, seed, step, dtype):
+    """The oracle's new weights with every label row whose gradient operands
+    differ between the two sides re-stepped from the GPU's operands.  A
+    differing operand is one grid step of G (a logit within rounding of a
+    midpoint on one side); in an update W - lr G^T X that step moves the whole
+    row by lr ulp(G) x, which can be many ulps of small weights.  The re-step
+    follows the oracle's own arithmetic (fp32 products and sums in sample
+    order, v = w - lr dw, the same 16-bit draws), checked first by
+    re-stepping each such row from the oracle's operands and getting the
+    oracle's codes back.  Returns (weights, rows re-stepped)."""
+    dG = np.asarray(G_gpu, np.float64) - np.asarray(G_orc, np.float64)
+    rows = np.unique(np.nonzero(dG)[0])
+    if rows.size == 0:
+        return W_new, 0
+    wd = weight_dtype(dtype)
+    xv = x_operand(orc, X, dtype).astype(np.float32)
+    d = xv.shape[1]
+    out = np.array(W_new, copy=True)
+    lr32 = np.float32(lr)
+
+    def restep(l, g):
+        dw = np.zeros(d, np.float32)
+        for b in range(xv.shape[0]):
+            dw = (dw + (np.float32(g[b]) * xv[b]).astype(np.float32)).astype(np.float32)
+        v = (orc.w_value(W[l], wd).astype(np.float32) - (lr32 * dw).astype(np.float32)).astype(np.float32)
+        return orc.sr_with_draws(v, orc.draw16(seed, step, int(l) * d, d), wd)
+
+    for l in rows:
+        assert np.array_equal(restep(l, G_orc[l]), W_new[l]), f"re-stepping label {l} does not reproduce the oracle"
+        out[l] = restep(l, G_gpu[l])
+    return out, int(rows.size)
+
+
 def check_step(orc, W, X, rowptr, cols, lr, seed, step, dtype, Wg, dXg, Zg, Gg, chunk_rows=None,
                same_weights=True):
     """The GPU step (new weights Wg, dX dXg, logits Zg and operands Gg of the
@@ -193,7 +250,11 @@ def check_step(orc, W, X, rowptr, cols, lr, seed, step, dtype, Wg, dXg, Zg, Gg, 
     assert_operands_of_logits(Gg, Zg, Y, dtype, what="G (GPU)")
     assert_operands_of_logits(r["G"], r["Z"], Y, dtype, what="G (oracle)")
     dx_ref, flips = flip_corrected_dx(r["dX"], Gg, r["G"], W, weight_dtype(dtype))
-    _record({"what": "G flips", "dtype": dtype, "elements": int(np.size(Gg)), "flips": flips})
+    steps = np.abs(operand_codes(Gg, dtype) - operand_codes(r["G"], dtype))
+    w_ref, rows = flip_corrected_weights(orc, W, X, Gg, r["G"], r["W"], lr, seed, step, dtype)
+    _record({"what": "G flips", "dtype": dtype, "elements": int(np.size(Gg)), "flips": flips,
+             "largest_code_step": int(steps.max()) if steps.size else 0, "label_rows_restepped": rows})
+    assert steps.size == 0 or int(steps.max()) <= 1, "two sides' gradient operands differ by more than one grid step"
     assert_rel_close(dXg, dx_ref, dtype, what="dX")
-    assert_weights_close(Wg, r["W"], weight_dtype(dtype), chunk_rows=chunk_rows)
+    assert_weights_close(Wg, w_ref, weight_dtype(dtype), chunk_rows=chunk_rows)
     return r, flips
