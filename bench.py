@@ -405,6 +405,9 @@ def run_topk(args, w, rank, world, local):
     e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    # rows of the last call whose screening could not certify the top-k and
+    # that took the exact CUDA-core path
+    uncertified = elmo.elmo_topk_uncertified_rows(head, w.B, w.topk)
     # P@1, P@3, P@5 of the last predictions against the queries' synthetic labels
     # (random weights: near zero; the point is that the metric runs on the device)
     from synthetic import make_labels, workload
@@ -439,6 +442,7 @@ def run_topk(args, w, rank, world, local):
             "e2e": {"value": world * w.B * w.L / (ms_e2e / 1e3), "unit": "query-labels/s",
                     "h2d_bytes_per_step": w.B * w.d * 2, "d2h_bytes_per_step": w.B * w.topk * 8},
             "cpu_baseline": cpu, "clocks": clocks, "p_at_k": p_at_k,
+            "uncertified_rows": {"rows": uncertified, "of": w.B},
         }
         print(json.dumps(line), flush=True)
     head.close()

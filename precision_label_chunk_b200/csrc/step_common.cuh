@@ -146,8 +146,8 @@ __device__ __forceinline__ void grad_codes16(const uint32_t* acc, float inv_sx, 
   if (slow) {                                  // rare: positives, padding, near-midpoint or low logits
     constexpr int kPer = kG ? 4 : 2;
     constexpr int kBits = 32 / kPer;
-#pragma unroll 1
-    for (int i = 0; i < 16; ++i) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {             // unrolled: x and acc stay in registers
       const float a = __uint_as_float(acc[i]);
       const uint32_t off = (__float_as_uint(x[i]) - (Wd::kMid - Wd::kT)) & Wd::kMask;
       const bool v = (vbits >> i) & 1u, y = (ybits >> i) & 1u;
@@ -237,14 +237,11 @@ __device__ __forceinline__ void sr_draws16(uint64_t seed, uint64_t step, uint64_
 // its 16 random bits to the 16 discarded bits of each value and truncates, so
 // passing 2^16 - 1 - k (the complemented draw) gives exactly this rounding.
 // E4M3 (n = 20) and E5M2 (n = 21): below the smallest normal value (2^-6,
-// 2^-14) the grid is uniform; |v| is first moved up one binade, whose spacing
-// equals the subnormal spacing, by an add rounded toward +infinity (that
-// keeps ceil(F), and for an integer k, 2^(n-16) k < F <=> 2^(n-16) k <
-// ceil(F), so the decision stays exact), truncated there and moved back
-// exactly; the sign is restored and the saturating conversion maps
-// magnitudes at or above the largest finite value to it.
-// kW: the weight grid, 0 bf16, 1 E4M3, 2 E5M2 (+-inf is an E5M2 value and
-// stays, so E5M2 groups holding one take the per-element path).
+// 2^-14) the grid is uniform with the spacing of the lowest binade; |v| is
+// scaled so that fp32's denormals take the same structure (below), truncated
+// there and scaled back exactly; the sign is restored and the saturating
+// conversion maps magnitudes at or above the largest finite value to it.
+// kW: the weight grid, 0 bf16, 1 E4M3, 2 E5M2.
 template <int kW>
 __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t (&rw)[8],
                                          const uint8_t* __restrict__ wtile, int row, int jl, int64_t l, int32_t d,
@@ -278,60 +275,67 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t
 #pragma unroll
   for (int i = 0; i < 16; ++i) vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
   uint32_t wnew[8];
-  if (kW == 1) {
-    // per element and branch-free, NaN and infinities included (the
-    // saturating conversion maps magnitudes at or above 448 to 448)
+  // a probe that is not finite when some v is NaN or infinite (8-bit grids:
+  // the sum of 0 v; bf16: the sum of 2 v, which also overflows once some
+  // |v| >= 2^127, where rounding could pass the largest finite value) sends
+  // the group to the exact per-element path
+  float probe = 0.0f;
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      float o[4];
+  for (int i = 0; i < 16; ++i) probe = __fmaf_rn(vv[i], kW ? 0.0f : 2.0f, probe);
+  if (fabsf(probe) < INFINITY) {
+    if (kW) {
+      // |v| scaled by 2^-120 (E4M3) or 2^-112 (E5M2) puts the grid's smallest
+      // normal on fp32's (2^-126) and its subnormal spacing on 2^20 (2^21) of
+      // fp32's denormal steps, so one add-and-truncate covers both ranges; the
+      // scaling rounds up, which keeps ceil(F) of the fraction (for an integer
+      // k, 2^(n-16) k < F <=> 2^(n-16) k < ceil(F)), and scaling back is exact
+      constexpr float kDown = kW == 1 ? 0x1p-120f : 0x1p-112f;
+      constexpr float kUp = kW == 1 ? 0x1p120f : 0x1p112f;
+      constexpr uint32_t kMask = kW == 1 ? 0xFFF00000u : 0xFFE00000u;
+      constexpr uint32_t kOne = kW == 1 ? 0xFFFFFu : 0x1FFFFFu;
+      constexpr int kShift = kW == 1 ? 4 : 5;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t word = rw[2 * q4 + (e >> 1)];
-        o[e] = sr_e4m3_value(vv[4 * q4 + e], (e & 1) ? (word >> 16) : (word & 0xFFFFu));
-      }
-      wnew[q4] = pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16);
-    }
-  } else {
-    // a probe that is not finite when some v is NaN or infinite (E5M2: the
-    // sum of 0 v; bf16: the sum of 2 v, which also overflows once some
-    // |v| >= 2^127, where rounding could pass the largest finite value) sends
-    // the group to the exact per-element path
-    float probe = 0.0f;
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float o[4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) probe = __fmaf_rn(vv[i], kW ? 0.0f : 2.0f, probe);
-    if (fabsf(probe) < INFINITY) {
-      if (kW) {
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          float o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t word = rw[2 * q4 + (e >> 1)];
-            o[e] = sr_e5m2_finite_value(vv[4 * q4 + e], (e & 1) ? (word >> 16) : (word & 0xFFFFu));
-          }
-          wnew[q4] = pack_e5m2x2(o[1], o[0]) | (pack_e5m2x2(o[3], o[2]) << 16);
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t word = rw[2 * q4 + (e >> 1)];
+          const uint32_t k16 = (e & 1) ? (word >> 16) : (word & 0xFFFFu);
+          const float v = vv[4 * q4 + e];
+          const float sm = __fmul_ru(fabsf(v), kDown);
+          const uint32_t t = (__float_as_uint(sm) + (kOne - (k16 << kShift))) & kMask;
+          o[e] = __fmul_rn(__uint_as_float(t | (__float_as_uint(v) & 0x80000000u)), kUp);
         }
-      } else {
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          uint32_t o;   // element 2p (low half) takes the low 16 random bits, 2p + 1 the high
-          asm("cvt.rs.bf16x2.f32 %0, %1, %2, %3;" : "=r"(o) : "f"(vv[2 * p + 1]), "f"(vv[2 * p]), "r"(~rw[p]));
-          wnew[p] = o;
-        }
+        wnew[q4] = kW == 1 ? pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16)
+                           : pack_e5m2x2(o[1], o[0]) | (pack_e5m2x2(o[3], o[2]) << 16);
       }
     } else {
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        if (kW == 2) {
-          if (p < 4) {
-            const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
-            wnew[p] = sr_e5m2_code(vv[4 * p], w0 & 0xFFFFu) | (sr_e5m2_code(vv[4 * p + 1], w0 >> 16) << 8) |
-                      (sr_e5m2_code(vv[4 * p + 2], w1 & 0xFFFFu) << 16) |
-                      (sr_e5m2_code(vv[4 * p + 3], w1 >> 16) << 24);
-          }
-        } else {
-          wnew[p] = (uint32_t)sr_bf16(vv[2 * p], rw[p] & 0xFFFFu) | ((uint32_t)sr_bf16(vv[2 * p + 1], rw[p] >> 16) << 16);
+        uint32_t o;   // element 2p (low half) takes the low 16 random bits, 2p + 1 the high
+        asm("cvt.rs.bf16x2.f32 %0, %1, %2, %3;" : "=r"(o) : "f"(vv[2 * p + 1]), "f"(vv[2 * p]), "r"(~rw[p]));
+        wnew[p] = o;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      if (kW == 1) {
+        if (p < 4) {
+          const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
+          const float o0 = sr_e4m3_value(vv[4 * p], w0 & 0xFFFFu), o1 = sr_e4m3_value(vv[4 * p + 1], w0 >> 16);
+          const float o2 = sr_e4m3_value(vv[4 * p + 2], w1 & 0xFFFFu), o3 = sr_e4m3_value(vv[4 * p + 3], w1 >> 16);
+          wnew[p] = pack_e4m3x2(o1, o0) | (pack_e4m3x2(o3, o2) << 16);
         }
+      } else if (kW == 2) {
+        if (p < 4) {
+          const uint32_t w0 = rw[2 * p], w1 = rw[2 * p + 1];
+          wnew[p] = sr_e5m2_code(vv[4 * p], w0 & 0xFFFFu) | (sr_e5m2_code(vv[4 * p + 1], w0 >> 16) << 8) |
+                    (sr_e5m2_code(vv[4 * p + 2], w1 & 0xFFFFu) << 16) |
+                    (sr_e5m2_code(vv[4 * p + 3], w1 >> 16) << 24);
+        }
+      } else {
+        wnew[p] = (uint32_t)sr_bf16(vv[2 * p], rw[p] & 0xFFFFu) | ((uint32_t)sr_bf16(vv[2 * p + 1], rw[p] >> 16) << 16);
       }
     }
   }

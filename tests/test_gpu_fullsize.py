@@ -8,7 +8,8 @@ import torch
 
 from synthetic import make_labels, make_X, workload
 from tests.gpu_common import need_gpu, to_dev_i32, to_dev_u16, w_to_host
-from tests.parity import assert_operands_of_logits, assert_rel_close, assert_weights_close, flip_corrected_dx
+from tests.parity import (assert_operands_of_logits, assert_rel_close, assert_weights_close, flip_corrected_dx,
+                           flip_corrected_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -51,11 +52,23 @@ def test_step_full_size_sampled(orc, name):
             Zs[:, a:e] = Zd[:, samples].T.cpu().numpy()
             Gs[:, a:e] = Gd[:, samples].T.cpu().numpy()
             del Zd, Gd
+    # the operands of the checked label ranges before the step: where one of
+    # them lands on the other neighbour of the oracle's (logits within rounding
+    # of a midpoint), its label row is re-stepped from the GPU's operand
+    ranges = _label_ranges(w.L, w.chunk)
+    Granges = []
+    for l0, l1 in ranges:
+        Zd = torch.empty(l1 - l0, w.B, device="cuda")
+        Gd = torch.empty(l1 - l0, w.B, device="cuda")
+        elmo.elmo_forward_chunk(h, Xd, rp, cl, l0, l1, Zd, Gd)
+        Granges.append(Gd.cpu().numpy())
     elmo.elmo_train_step_chunked(h, Xd, rp, cl, w.lr, w.chunk, 0, 0, dX)
     elmo.elmo_sync_status(h)
-    for l0, l1 in _label_ranges(w.L, w.chunk):
-        r = orc.train_step(W0[:l1], X, rowptr, cols, w.lr, 0, 0, w.dtype, l0=l0, l1=l1, want_dx=False, L=w.L)
-        assert_weights_close(w_to_host(Wd[l0:l1], w.dtype), r["W"], w.dtype)
+    for (l0, l1), Gg in zip(ranges, Granges):
+        r = orc.train_step(W0[:l1], X, rowptr, cols, w.lr, 0, 0, w.dtype, l0=l0, l1=l1, want_dx=False, want_zg=True,
+                           L=w.L)
+        w_ref, _ = flip_corrected_weights(orc, W0, X, Gg, r["G"], r["W"], w.lr, 0, 0, w.dtype, l0=l0)
+        assert_weights_close(w_to_host(Wd[l0:l1], w.dtype), w_ref, w.dtype)
     if w.L <= 3_000_000:
         ref, Zo, Go = orc.dx_rows(W0, X, rowptr, cols, samples, w.dtype, want_zg=True)
         Y = np.zeros((len(samples), w.L), np.float32)

@@ -1,4 +1,6 @@
 """GPU stochastic rounding and its random draws are bit-exact with the oracle."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -103,8 +105,7 @@ def test_sr_round_empty_and_errors():
     assert lib.elmo_sr_round(None, None, -1, 0, 0, 0, 0, None) == 1     # n < 0: EINVAL
     xd = torch.zeros(4, device="cuda")
     assert lib.elmo_sr_round(xd.data_ptr(), out.data_ptr(), 4, 7, 0, 0, 0, None) == 1  # bad dtype
-    # E5M2 is an output grid of the standalone rounding, not a weight format
+    # a head takes bf16, E4M3 or E5M2 weights; another format code is refused
     W = torch.zeros(128, 64, dtype=torch.uint8, device="cuda")
-    with pytest.raises(elmo.ElmoError) as ei:
-        elmo.elmo_init_head(W, "e5m2")
-    assert ei.value.status == 5                                                     # ELMO_EUNSUPPORTED
+    h = ctypes.c_void_p()
+    assert lib.elmo_init_head(ctypes.byref(h), W.data_ptr(), 128, 64, 9, 0, 0.0, 0, None) == 1        # EINVAL
