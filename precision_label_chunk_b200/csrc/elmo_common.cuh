@@ -39,6 +39,41 @@ __device__ __forceinline__ u32x4 philox10(uint32_t c0, uint32_t c1, uint32_t c2,
   return {c0, c1, c2, c3};
 }
 
+// The round keys of one seed: round r uses (k0[r], k1[r]) = the seed's low
+// and high words plus r times the Weyl increments (mod 2^32), the schedule of
+// philox10 above.  Formed once on the host and passed by value as a kernel
+// parameter, so each round's XOR reads its key from the constant bank.
+struct PhiloxKeys { uint32_t k0[10], k1[10]; };
+
+inline PhiloxKeys philox_keys(uint64_t seed) {
+  PhiloxKeys K;
+  uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    K.k0[r] = a;
+    K.k1[r] = b;
+    a += 0x9E3779B9u;
+    b += 0xBB67AE85u;
+  }
+  return K;
+}
+
+__device__ __forceinline__ u32x4 philox10_rk(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                              const PhiloxKeys& K) {
+  constexpr uint32_t kMulA = 0xD2511F53u, kMulB = 0xCD9E8D57u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t hiA = __umulhi(kMulA, c0), loA = kMulA * c0;
+    const uint32_t hiB = __umulhi(kMulB, c2), loB = kMulB * c2;
+    const uint32_t n0 = hiB ^ c1 ^ K.k0[r], n2 = hiA ^ c3 ^ K.k1[r];
+    c0 = n0; c1 = loB; c2 = n2; c3 = loA;
+  }
+  return {c0, c1, c2, c3};
+}
+
+__device__ __forceinline__ u32x4 sr_block_rk(const PhiloxKeys& K, uint64_t step, uint64_t blk) {
+  return philox10_rk((uint32_t)blk, (uint32_t)(blk >> 32), (uint32_t)step, (uint32_t)(step >> 32), K);
+}
+
 // The Philox block that serves elements 8*blk .. 8*blk+7 of SR stream
 // (seed, step): counter (blk, step), key = seed.  Element idx takes the
 // 16-bit half (idx & 1) of word ((idx >> 1) & 3), low half first.

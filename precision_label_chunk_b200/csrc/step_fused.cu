@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
                int32_t Bp, const uint8_t* __restrict__ xop, const uint32_t* __restrict__ keys,
                const int32_t* __restrict__ tile_ptr, const float* __restrict__ xscale, uint8_t* __restrict__ gring,
                int32_t R, int32_t* __restrict__ ready, int32_t* __restrict__ consumed, int32_t nA, int32_t nG,
-               float lr, uint64_t seed, uint64_t step, uint64_t blk_base, float* __restrict__ dX,
+               float lr, const PhiloxKeys rk, uint64_t step, uint64_t blk_base, float* __restrict__ dX,
                int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -270,6 +270,30 @@ __global__ void __launch_bounds__(kFThreads, 1)
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) { if (lane == 0) record_timeout(status, abort, 85); break; }
         }
+        // positives of sample b among this warp's label columns of the tile
+        // (c_lo .. c_lo + ncol - 1 of each 64-label half; bit 32 hf + c of pm2
+        // for column c of half hf), from the tile's keys: the warp reads them
+        // together (a frequent label's tile holds hundreds) and scatters each
+        // into the mask of its sample when that sample is one of the warp's
+        uint64_t pm2;
+        {
+          const int k0 = __ldg(tile_ptr + t);
+          const int k1 = __ldg(tile_ptr + t + 1);
+          wm[lane] = 0;
+          __syncwarp();
+          const int wb = b - lane;
+          const int64_t lbase = (int64_t)t * 128 + c_lo;
+          for (int i = k0 + lane; i < k1; i += 32) {
+            const uint32_t key = __ldg(keys + i);
+            const int sb = (int)(key & 0xFFu) - wb;
+            const int64_t dl = (int64_t)(key >> 8) - lbase;      // column in the first half, or 64 + column
+            const int64_t c = dl >= kFN ? dl - kFN : dl;
+            if (sb >= 0 && sb < 32 && dl >= 0 && c < ncol) atomicOr(wm + sb, 1ull << (c + (dl >= kFN ? 32 : 0)));
+          }
+          __syncwarp();
+          pm2 = wm[lane];
+          __syncwarp();
+        }
         bool stop = false;
         for (int hf = 0; hf < 2; ++hf) {
           const uint32_t uu = nmb == 2 ? 2 * use + (uint32_t)mb : use;   // this thread's use of the slots
@@ -289,28 +313,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&S->tempty[buf]);
-          // positives of sample b among labels lc0 .. lc0 + ncol - 1, from the
-          // keys of their 128-label tile: the warp reads the keys together (a
-          // frequent label's tile holds hundreds) and scatters each into the
-          // mask of its sample when that sample is one of the warp's
           const int64_t lc0 = (int64_t)t * 128 + hf * kFN + c_lo;
-          uint64_t pm;
-          {
-            const int k0 = __ldg(tile_ptr + t);
-            const int k1 = __ldg(tile_ptr + t + 1);
-            wm[lane] = 0;
-            __syncwarp();
-            const int wb = b - lane;
-            for (int i = k0 + lane; i < k1; i += 32) {
-              const uint32_t key = __ldg(keys + i);
-              const int sb = (int)(key & 0xFFu) - wb;
-              const int64_t dl = (int64_t)(key >> 8) - lc0;
-              if (sb >= 0 && sb < 32 && dl >= 0 && dl < ncol) atomicOr(wm + sb, 1ull << dl);
-            }
-            __syncwarp();
-            pm = wm[lane];
-            __syncwarp();
-          }
+          const uint64_t pm = pm2 >> (32 * hf);
           const int lt0 = hf * kFN + c_lo;                      // first label column within the tile
 #pragma unroll
           for (int j = 0; j < 32; j += 16) {
@@ -507,8 +511,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
       // the draws do not depend on the gradient: form them while the MMAs run
       uint32_t rw0[8], rw1[8];
       if (valid) {
-        sr_draws16(seed, step, blk_base, l, d, j0, rw0);
-        sr_draws16(seed, step, blk_base, l, d, j0 + 16, rw1);
+        sr_draws16(rk, step, blk_base, l, d, j0, rw0);
+        sr_draws16(rk, step, blk_base, l, d, j0 + 16, rw1);
       }
       if (!mbar_wait(&S->dwfull[db], duse & 1, abort, kWaitCycles)) { record_timeout(status, abort, 98); break; }
       tc_fence_after();
@@ -620,7 +624,7 @@ cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float 
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, tmWa, tmWb, tmX, h->W, h->L, h->d, B, Bp, xop, (const uint32_t*)h->keys,
                             (const int32_t*)h->tile_ptr, (const float*)h->xscale, static_cast<uint8_t*>(h->ring),
-                            h->ring_tiles, h->ring_flags, h->ring_flags + h->ring_tiles, nA, nG, lr, seed, step,
+                            h->ring_tiles, h->ring_flags, h->ring_flags + h->ring_tiles, nA, nG, lr, philox_keys(seed), step,
                             (uint64_t)h->label_base * (uint64_t)h->d / 8, dX, h->status);
 }
 

@@ -615,7 +615,7 @@ template <int kFp8, int kW5 = 0>
 __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
     update_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
               const uint8_t* __restrict__ gbuf, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
-              int32_t Bp, int64_t l0, int64_t l1, const float* __restrict__ xscale, float lr, uint64_t seed,
+              int32_t Bp, int64_t l0, int64_t l1, const float* __restrict__ xscale, float lr, const PhiloxKeys rk,
               uint64_t step, uint64_t blk_base, float* __restrict__ dX, int gsm, uint32_t gfmt,
               int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -829,7 +829,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreads : 320, 1)
 #pragma unroll
           for (int g = 0; g < kGrp; ++g) {
             uint32_t rw[8];
-            sr_draws16(seed, step, blk_base, l, d, j0 + 16 * g, rw);
+            sr_draws16(rk, step, blk_base, l, d, j0 + 16 * g, rw);
             update16<kFp8 ? (kW5 ? 2 : 1) : 0>(r[g], rw, wrow, row, jl + 16 * g, l, d, j0 + 16 * g, lrs, Wglob);
           }
         }
@@ -1034,7 +1034,7 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
   if (e != cudaSuccess) return e;
   return launch_k(kern, grid, fp8 ? kThreads : 320, kSmemB, s, pdl, tmW, tmX, static_cast<const uint8_t*>(gbuf), h->W,
                   h->L, h->d,
-                  B, Bp, l0, l1, (const float*)h->xscale, lr, seed, step,
+                  B, Bp, l0, l1, (const float*)h->xscale, lr, philox_keys(seed), step,
                   (uint64_t)h->label_base * (uint64_t)h->d / 8, dX, g_sample_major(h, Bp) ? 1 : 0,
                   h->g_e5m2 ? 1u : 0u, h->status);
 }
