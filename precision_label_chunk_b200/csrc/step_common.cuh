@@ -124,39 +124,6 @@ __device__ __forceinline__ float grad_acc_floor(float inv_sx) {
   return __fdiv_rn(-GradWindow<kG>::kZlim, inv_sx);
 }
 
-// The rare path of grad_codes16: elements that are padding (code 0),
-// positives, near a midpoint or below the fast path's logit range get the
-// exact code.  The values are copied to a local array first, so that the
-// loop over elements can stay rolled (one call site of the exact function)
-// while the caller's arrays stay in registers.
-template <int kG>
-__device__ __forceinline__ void grad_codes16_fix(const uint32_t* acc, const float* x, float inv_sx, float acc_lo,
-                                                 uint32_t ybits, uint32_t vbits, uint32_t* out) {
-  using Wd = GradWindow<kG>;
-  constexpr int kPer = kG ? 4 : 2;
-  constexpr int kBits = 32 / kPer;
-  constexpr uint32_t kKeep = 0xFFFFFFFFu;
-  uint32_t al[16], xl[16], patch[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) { al[i] = acc[i]; xl[i] = __float_as_uint(x[i]); }
-#pragma unroll 1
-  for (int i = 0; i < 16; ++i) {
-    const float a = __uint_as_float(al[i]);
-    const uint32_t off = (xl[i] - (Wd::kMid - Wd::kT)) & Wd::kMask;
-    const bool v = (vbits >> i) & 1u, y = (ybits >> i) & 1u;
-    uint32_t c = kKeep;
-    if (!v) c = 0u;
-    else if (y || off <= 2u * Wd::kT || !(a >= acc_lo)) c = grad_code_exact<kG>(a, inv_sx, y);
-    patch[i] = c;
-  }
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int q = i / kPer, sh = (i % kPer) * kBits;
-    const uint32_t m = (kG ? 0xFFu : 0xFFFFu) << sh;
-    if (patch[i] != kKeep) out[q] = (out[q] & ~m) | (patch[i] << sh);
-  }
-}
-
 template <int kG>
 __device__ __forceinline__ void grad_codes16(const uint32_t* acc, float inv_sx, float acc_lo, uint32_t ybits,
                                              uint32_t vbits, uint32_t* out) {
@@ -176,7 +143,22 @@ __device__ __forceinline__ void grad_codes16(const uint32_t* acc, float inv_sx, 
   for (int q = 0; q < (kG ? 4 : 8); ++q)
     out[q] = kG ? grad_pack2<kG>(x[4 * q + 1], x[4 * q]) | (grad_pack2<kG>(x[4 * q + 3], x[4 * q + 2]) << 16)
                 : grad_pack2<kG>(x[2 * q + 1], x[2 * q]);
-  if (slow) grad_codes16_fix<kG>(acc, x, inv_sx, acc_lo, ybits, vbits, out);
+  if (slow) {                                  // rare: positives, padding, near-midpoint or low logits
+    constexpr int kPer = kG ? 4 : 2;
+    constexpr int kBits = 32 / kPer;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {             // unrolled: x and acc stay in registers
+      const float a = __uint_as_float(acc[i]);
+      const uint32_t off = (__float_as_uint(x[i]) - (Wd::kMid - Wd::kT)) & Wd::kMask;
+      const bool v = (vbits >> i) & 1u, y = (ybits >> i) & 1u;
+      if (!v || y || off <= 2u * Wd::kT || !(a >= acc_lo)) {
+        const uint32_t c = v ? grad_code_exact<kG>(a, inv_sx, y) : 0u;
+        const int q = i / kPer, sh = (i % kPer) * kBits;
+        const uint32_t m = (kG ? 0xFFu : 0xFFFFu) << sh;
+        out[q] = (out[q] & ~m) | (c << sh);
+      }
+    }
+  }
 }
 
 // The operand value of code `c` (G, with 2^-8 undone for the 8-bit formats).

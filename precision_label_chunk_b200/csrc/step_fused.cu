@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     const int nmb = nprod == 2 ? 1 : (Bp + 127) / 128;        // M-blocks computed here: 1 or 2
     if (threadIdx.x == 0) {
       for (int s = 0; s < kFStagesA; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
-      for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], nmb == 2 ? 8 : kFEpi); }
+      for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], kFEpi); }
       mbar_init(&S->xready, kFEpi);
       for (int i = 0; i < 4; ++i) S->arrivals[i] = 0;
       S->abort = 0;
@@ -242,16 +242,13 @@ __global__ void __launch_bounds__(kFThreads, 1)
         }
       }
     } else {
-      // Epilogue: warp (q = warp % 4, h = (warp - 2) / 4).  Two M-blocks: warp
-      // h takes M-block h / 2, label columns 32 (h % 2) .. +31 of each 64-label
-      // half-tile; one M-block: label columns 16 h .. 16 h + 15.
+      // Epilogue: warp (q = warp % 4, h = (warp - 2) / 4) takes TMEM lanes
+      // 32 q .. 32 q + 31 of every accumulator slot (samples mb * 128 + 32 q +
+      // lane of M-block mb) and label columns 16 h .. 16 h + 15 of each 64-label
+      // half: all 16 warps drain each slot, so that the MMAs into one slot
+      // overlap the epilogue of the other.
       const int q = warp & 3, h = (warp - 2) >> 2;
-      const int mb = nmb == 2 ? h >> 1 : 0;
-      const int c_lo = nmb == 2 ? 32 * (h & 1) : 16 * h;
-      const int ncol = nmb == 2 ? 32 : 16;
-      const int b = (amb + mb) * 128 + q * 32 + lane;        // sample
-      const bool bvalid = b < B;
-      const bool bstore = b < Bp;
+      const int c_lo = 16 * h;
       const float inv_sx = kFp8 ? xscale[1] : 1.0f;
       const float acc_lo = grad_acc_floor<kFp8 ? (kG5 ? 2 : 1) : 0>(inv_sx);
       constexpr int kG = kFp8 ? (kG5 ? 2 : 1) : 0;
@@ -270,61 +267,56 @@ __global__ void __launch_bounds__(kFThreads, 1)
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) { if (lane == 0) record_timeout(status, abort, 85); break; }
         }
-        // positives of sample b among this warp's label columns of the tile
-        // (c_lo .. c_lo + ncol - 1 of each 64-label half; bit 32 hf + c of pm2
-        // for column c of half hf), from the tile's keys: the warp reads them
-        // together (a frequent label's tile holds hundreds) and scatters each
-        // into the mask of its sample when that sample is one of the warp's
+        // positives among this thread's elements of the tile: bit 32 mb + 16 hf
+        // + c for sample (amb + mb) 128 + 32 q + lane and label column
+        // 64 hf + 16 h + c, from the tile's keys: the warp reads them together
+        // (a frequent label's tile holds hundreds) and scatters each into the
+        // mask of its sample's lane
         uint64_t pm2;
         {
           const int k0 = __ldg(tile_ptr + t);
           const int k1 = __ldg(tile_ptr + t + 1);
           wm[lane] = 0;
           __syncwarp();
-          const int wb = b - lane;
           const int64_t lbase = (int64_t)t * 128 + c_lo;
           for (int i = k0 + lane; i < k1; i += 32) {
             const uint32_t key = __ldg(keys + i);
-            const int sb = (int)(key & 0xFFu) - wb;
-            const int64_t dl = (int64_t)(key >> 8) - lbase;      // column in the first half, or 64 + column
+            const int smp = (int)(key & 0xFFu);
+            const int mk = (smp >> 7) - amb;                       // M-block of the sample here
+            const int sl = (smp & 127) - 32 * q;                   // its lane
+            const int64_t dl = (int64_t)(key >> 8) - lbase;        // column in the first half, or 64 + column
             const int64_t c = dl >= kFN ? dl - kFN : dl;
-            if (sb >= 0 && sb < 32 && dl >= 0 && c < ncol) atomicOr(wm + sb, 1ull << (c + (dl >= kFN ? 32 : 0)));
+            if (mk >= 0 && mk < nmb && sl >= 0 && sl < 32 && dl >= 0 && c < 16)
+              atomicOr(wm + sl, 1ull << (32 * mk + (dl >= kFN ? 16 : 0) + c));
           }
           __syncwarp();
           pm2 = wm[lane];
           __syncwarp();
         }
         bool stop = false;
-        for (int hf = 0; hf < 2; ++hf) {
-          const uint32_t uu = nmb == 2 ? 2 * use + (uint32_t)mb : use;   // this thread's use of the slots
-          ++use;
-          const uint32_t buf = uu & 1;
-          if (!mbar_wait(&S->tfull[buf], (uu >> 1) & 1, abort, kWaitCycles)) {
-            record_timeout(status, abort, 86);
-            stop = true;
-            break;
-          }
-          tc_fence_after();
-          uint32_t v[32];
-          const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + kFAcc + buf * kFN + (uint32_t)c_lo;
-          if (ncol == 32) tmem_ld32(taddr, v);
-          else tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(v));
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S->tempty[buf]);
-          const int64_t lc0 = (int64_t)t * 128 + hf * kFN + c_lo;
-          const uint64_t pm = pm2 >> (32 * hf);
-          const int lt0 = hf * kFN + c_lo;                      // first label column within the tile
-#pragma unroll
-          for (int j = 0; j < 32; j += 16) {
-            if (j >= ncol) break;
-            const int64_t nv = L - (lc0 + j);
-            const uint32_t vbits = !bvalid || nv <= 0 ? 0u : (nv >= 16 ? 0xFFFFu : (1u << nv) - 1u);
+        for (int hf = 0; hf < 2 && !stop; ++hf) {
+          for (int mb = 0; mb < nmb; ++mb) {
+            const uint32_t buf = use & 1, ph = (use >> 1) & 1;
+            ++use;
+            if (!mbar_wait(&S->tfull[buf], ph, abort, kWaitCycles)) {
+              record_timeout(status, abort, 86);
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            uint32_t v[16];
+            tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + kFAcc + buf * kFN + (uint32_t)c_lo, v);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S->tempty[buf]);
+            const int b = (amb + mb) * 128 + q * 32 + lane;     // sample
+            const int64_t nv = L - ((int64_t)t * 128 + hf * kFN + c_lo);
+            const uint32_t vbits = b >= B || nv <= 0 ? 0u : (nv >= 16 ? 0xFFFFu : (1u << nv) - 1u);
             uint32_t pk[8];
-            grad_codes16<kG>(v + j, inv_sx, acc_lo, (uint32_t)(pm >> j) & 0xFFFFu, vbits, pk);
-            if (bstore) {
-              const int lc = (lt0 + j) / kChunk;
+            grad_codes16<kG>(v, inv_sx, acc_lo, (uint32_t)(pm2 >> (32 * mb + 16 * hf)) & 0xFFFFu, vbits, pk);
+            if (b < Bp) {
+              const int lc = (hf * kFN + c_lo) / kChunk;
               *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =
                   make_uint4(pk[0], pk[1], pk[2], pk[3]);
               if (!kFp8)

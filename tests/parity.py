@@ -243,7 +243,9 @@ def check_step(orc, W, X, rowptr, cols, lr, seed, step, dtype, Wg, dXg, Zg, Gg, 
     False: the GPU stepped from its own earlier weights (a trajectory), which
     differ from W by stochastic-rounding decisions; the logits are then not
     compared (a weight one grid step apart moves a logit by x ulp(w), which a
-    relative error against the row's rms floor does not absorb)."""
+    relative error against the row's rms floor does not absorb).  Returns the
+    oracle's step (with W_ref, its weights with the flipped rows re-stepped:
+    the start of the oracle's next step in a trajectory) and the flip count."""
     r = orc.train_step(W, X, rowptr, cols, lr, seed, step, dtype, want_zg=True)
     L, B = r["Z"].shape
     Y = positives(rowptr, cols, L, B)
@@ -260,4 +262,5 @@ def check_step(orc, W, X, rowptr, cols, lr, seed, step, dtype, Wg, dXg, Zg, Gg, 
         assert steps.size == 0 or int(steps.max()) <= 1, "the sides' gradient operands differ by more than one step"
     assert_rel_close(dXg, dx_ref, dtype, what="dX")
     assert_weights_close(Wg, w_ref, weight_dtype(dtype), chunk_rows=chunk_rows)
+    r["W_ref"] = w_ref
     return r, flips
