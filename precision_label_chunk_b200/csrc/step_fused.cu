@@ -10,13 +10,15 @@
 // CTAs split into two roles that run at the same time on different SMs:
 //
 //   role A (the first nA CTAs): Z = X W_tile^T and G = sigmoid(Z) - Y for
-//     128-label tiles t = a, a + nA, ...: X stays in TMEM as the MMA's A
-//     operand, 64-label W k-blocks stream through a 16-stage TMA ring, and the
-//     16 epilogue warps write G (the next contractions' operand, sample-major)
-////     into slot t % R of a ring of R tiles in global memory, then count
-//     themselves in ready[slot] (bf16 with more than 128 samples: two CTAs,
-//     one M-block of X each, write the two halves of a tile);
-//   role B (the other CTAs, nG groups x nD d-slices): the CTA of group g and
+//     128-label tiles t = a, a + nA', ...: one M-block of X (128 samples) stays
+//     in TMEM as the MMA's A operand, W k-blocks stream through a 128 KB TMA
+//     ring, and the 16 epilogue warps write G (the next contractions'
+//     operand, sample-major) into slot t % R of a ring of R tiles in global
+//     memory, then count themselves in ready[slot].  With more than 128
+//     samples two neighbouring CTAs form a tile, one M-block each.  E4M3: one
+//     MMA chain of N = 128 labels per tile (X takes 192 TMEM columns, two
+//     128-column accumulator slots follow); bf16: two of N = 64 (X takes 384);
+////   role B (the other CTAs, nG groups x nD d-slices): the CTA of group g and
 //     slice s runs the units (t, s) for t = g, g + nG, ...: it waits for
 //     ready, copies G_t into shared memory (and counts itself in consumed[slot],
 //     which role A waits on before it reuses the slot), and issues
@@ -33,7 +35,7 @@
 // ELMO_ETIMEOUT in the status word, and the other CTAs stop at their next wait.
 //
 // Used for B <= 256, d <= 768, d a multiple of 64 (one M-block of X fits the
-// 384 TMEM columns below role A's accumulators); other shapes run the
+// TMEM columns below role A's accumulators); other shapes run the
 // range-by-range kernels of step_tc.cu.
 #include <stdlib.h>
 
@@ -46,10 +48,18 @@ namespace {
 
 constexpr int kFThreads = 576;              // warp 0 TMA, warp 1 MMA + TMEM, warps 2-17 epilogue
 constexpr int kFEpi = 16;
-constexpr int kFStagesA = 16;               // role A: W k-block ring
-constexpr int kFN = 64;                     // role A: labels per MMA tile
-constexpr uint32_t kFBoxA = kFN * 128;      // one W k-block: 64 labels x 128 bytes
-constexpr uint32_t kFAcc = 384;             // role A: first accumulator column (X below it)
+constexpr int kFStagesA = 16;               // role A: most W k-block stages (bf16: 16 x 8 KB, E4M3: 8 x 16 KB)
+constexpr uint32_t kFRingA = 128 * 1024;    // role A: bytes of the W ring
+// role A: labels per accumulator slot (the MMA's N), its W stage, its first
+// accumulator column (one M-block of X below it: E4M3 192 columns at d = 768,
+// bf16 384)
+template <int kFp8> struct RoleA {
+  static constexpr int kN = kFp8 ? 128 : 64;
+  static constexpr int kHalves = 128 / kN;
+  static constexpr uint32_t kStage = (uint32_t)kN * 128;
+  static constexpr int kStages = (int)(kFRingA / kStage);
+  static constexpr uint32_t kAcc = kFp8 ? 256 : 384;
+};
 constexpr int kFGSlots = 3;                 // role B: G tiles in shared memory
 constexpr uint32_t kFGSlotBytes = 2 * kBox; // one G tile: 128 labels x up to 256 samples (E4M3) or 128 (bf16)
 constexpr uint32_t kFXBytes = 2 * 32768;    // role B: X[:, slice]
@@ -75,12 +85,17 @@ struct SmemFB {
 
 constexpr size_t kSmemF = 1024 + kFXBytes + kFWBytes + kFGSlots * kFGSlotBytes + 1024;
 static_assert(kSmemF <= 232448, "fused step shared memory");
-static_assert(kFStagesA * kFBoxA + sizeof(SmemFA) + 1024 <= kSmemF, "role A layout");
+static_assert(kFRingA + sizeof(SmemFA) + 1024 <= kSmemF, "role A layout");
 static_assert(sizeof(SmemFB) <= 1024, "role B barriers");
 
 __device__ __forceinline__ int32_t ld_acquire(const int32_t* p) {
   int32_t v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int32_t ld_relaxed(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 __device__ __forceinline__ void st_release(int32_t* p, int32_t v) {
@@ -128,23 +143,24 @@ __global__ void __launch_bounds__(kFThreads, 1)
 
   if ((int)blockIdx.x < nA) {
     // ======================================================== role A
+    using RA = RoleA<kFp8>;
     uint8_t* ring = base;
-    SmemFA* S = reinterpret_cast<SmemFA*>(base + kFStagesA * kFBoxA);
+    SmemFA* S = reinterpret_cast<SmemFA*>(base + kFRingA);
     volatile int* abort = &S->abort;
     const int kbe = kFp8 ? 128 : 64;                          // elements of one 128-byte k-block
     const int nkb = (d + kbe - 1) / kbe;
     const uint32_t opcols = (uint32_t)nkb * 32;               // TMEM columns of one M-block of X
-    // Producers of a tile: one CTA holds every M-block of X (E4M3 up to 256
-    // samples, bf16 up to 128), or, for bf16 with more than 128 samples, two
-    // neighbouring CTAs hold one M-block each and write their halves of G.
-    const int nprod = (!kFp8 && Bp > 128) ? 2 : 1;
-    const int amb = nprod == 2 ? (int)(blockIdx.x & 1) : 0;   // first M-block held here
+    // Producers of a tile: one CTA holds the single M-block of X (up to 128
+    // samples), or two neighbouring CTAs hold one M-block each and write
+    // their halves of G.
+    const int nprod = Bp > 128 ? 2 : 1;
+    const int amb = nprod == 2 ? (int)(blockIdx.x & 1) : 0;   // the M-block held here
     const int a = nprod == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
     const int aN = nprod == 2 ? (nA >> 1) : nA;               // tile stride of the producers
-    const int nmb = nprod == 2 ? 1 : (Bp + 127) / 128;        // M-blocks computed here: 1 or 2
     if (threadIdx.x == 0) {
-      for (int s = 0; s < kFStagesA; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
-      for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], kFEpi); }
+      for (int s = 0; s < RA::kStages; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
+      // each slot is drained by one group: both groups of eight (E4M3) or all sixteen warps (bf16)
+      for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], kFEpi / (RA::kHalves == 1 ? 2 : 1)); }
       mbar_init(&S->xready, kFEpi);
       for (int i = 0; i < 4; ++i) S->arrivals[i] = 0;
       S->abort = 0;
@@ -157,30 +173,29 @@ __global__ void __launch_bounds__(kFThreads, 1)
     const uint32_t tmem = S->tmem_base;
 
     if (warp >= 2) {
-      // X into TMEM: sample h*128 + r of M-block h in lane r, columns h*opcols ...
+      // X into TMEM: sample amb*128 + r in lane r; warp (q, h) copies the
+      // 64-column chunks c0 = 64 h, 64 h + 256, ... of its quadrant's lanes
       const int q = warp & 3, h = (warp - 2) >> 2;
-      if (h < nmb) {
-        const int b = (amb + h) * 128 + q * 32 + lane;
-        const size_t rowbytes = (size_t)d * kEl;
-        // E4M3: xop holds the codes by 16-byte column chunk (chunk c of row b at
-        // (c * 256 + b) * 16); bf16: xop is X itself, row-major
-        const uint8_t* src = kFp8 ? xop + (size_t)b * 16 : xop + (size_t)b * rowbytes;
-        for (uint32_t c0 = 0; c0 < opcols; c0 += 64) {
-          uint32_t v[2][32];
+      const int b = amb * 128 + q * 32 + lane;
+      const size_t rowbytes = (size_t)d * kEl;
+      // E4M3: xop holds the codes by 16-byte column chunk (chunk c of row b at
+      // (c * 256 + b) * 16); bf16: xop is X itself, row-major
+      const uint8_t* src = kFp8 ? xop + (size_t)b * 16 : xop + (size_t)b * rowbytes;
+      for (uint32_t c0 = 64u * (uint32_t)h; c0 < opcols; c0 += 256) {
+        uint32_t v[2][32];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const size_t off = (size_t)(c0 + 4 * u) * 4;
-            uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
-            if (b < B && off < rowbytes)
-              w4 = *reinterpret_cast<const uint4*>(kFp8 ? src + (off >> 4) * (ELMO_MAX_BATCH * 16) : src + off);
-            v[u >> 3][4 * (u & 7)] = w4.x; v[u >> 3][4 * (u & 7) + 1] = w4.y;
-            v[u >> 3][4 * (u & 7) + 2] = w4.z; v[u >> 3][4 * (u & 7) + 3] = w4.w;
-          }
-          tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)h * opcols + c0, v[0]);
-          if (c0 + 32 < opcols) tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)h * opcols + c0 + 32, v[1]);
+        for (int u = 0; u < 16; ++u) {
+          const size_t off = (size_t)(c0 + 4 * u) * 4;
+          uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
+          if (b < B && off < rowbytes)
+            w4 = *reinterpret_cast<const uint4*>(kFp8 ? src + (off >> 4) * (ELMO_MAX_BATCH * 16) : src + off);
+          v[u >> 3][4 * (u & 7)] = w4.x; v[u >> 3][4 * (u & 7) + 1] = w4.y;
+          v[u >> 3][4 * (u & 7) + 2] = w4.z; v[u >> 3][4 * (u & 7) + 3] = w4.w;
         }
-        tmem_wait_st();
+        tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + c0, v[0]);
+        if (c0 + 32 < opcols) tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + c0 + 32, v[1]);
       }
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->xready);
@@ -191,151 +206,178 @@ __global__ void __launch_bounds__(kFThreads, 1)
         tma_prefetch_desc(&tmWa);
         uint32_t it = 0;
         for (int t = a; t < T && !*abort; t += aN) {
-          for (int hf = 0; hf < 2; ++hf) {
+          for (int hf = 0; hf < RA::kHalves; ++hf) {
             for (int kb = 0; kb < nkb; ++kb, ++it) {
-              const int s = (int)(it % kFStagesA);
-              const uint32_t ph = (it / kFStagesA) & 1;
+              const int s = (int)(it % RA::kStages);
+              const uint32_t ph = (it / RA::kStages) & 1;
               if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 81); break; }
-              mbar_arrive_expect_tx(&S->wfull[s], kFBoxA);
-              tma_load_2d(ring + s * kFBoxA, &tmWa, &S->wfull[s], kb * kbe, t * 128 + hf * kFN);
+              mbar_arrive_expect_tx(&S->wfull[s], RA::kStage);
+              tma_load_2d(ring + s * RA::kStage, &tmWa, &S->wfull[s], kb * kbe, t * 128 + hf * RA::kN);
             }
           }
         }
       }
     } else if (warp == 1) {
       if (elect_one()) {
-        const uint32_t idesc = kFp8 ? make_idesc(0, kW5, 0, 0, 128, kFN) : make_idesc(1, 1, 0, 0, 128, kFN);
+        const uint32_t idesc =
+            kFp8 ? make_idesc(0, kW5, 0, 0, 128, RA::kN) : make_idesc(1, 1, 0, 0, 128, RA::kN);
         uint32_t it = 0, u = 0;
         if (!mbar_wait(&S->xready, 0, abort, kWaitCycles)) record_timeout(status, abort, 82);
         tc_fence_after();
         for (int t = a; t < T && !*abort; t += aN) {
-          for (int hf = 0; hf < 2 && !*abort; ++hf) {
-            for (int mb = 0; mb < nmb && !*abort; ++mb, ++u) {
-              const uint32_t slot = u & 1, ph = (u >> 1) & 1;
-              if (!mbar_wait(&S->tempty[slot], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 83); break; }
-              tc_fence_after();
-              const uint32_t dcol = tmem + kFAcc + slot * kFN;
-              for (int kb = 0; kb < nkb; ++kb) {
-                const uint32_t its = it + (uint32_t)kb;
-                const int s = (int)(its % kFStagesA);
-                if (mb == 0) {
-                  if (!mbar_wait(&S->wfull[s], (its / kFStagesA) & 1, abort, kWaitCycles)) {
-                    record_timeout(status, abort, 84);
-                    break;
-                  }
-                  tc_fence_after();
-                }
-                const uint32_t bsm = smem_u32(ring + s * kFBoxA);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  const uint32_t aa = tmem + (uint32_t)mb * opcols + (uint32_t)kb * 32 + (uint32_t)k * 8;
-                  const uint64_t bd = sw128_desc(bsm + k * 32, 16, 1024);
-                  if (kFp8) mma_e4m3_ts(dcol, aa, bd, idesc, (kb | k) != 0);
-                  else mma_bf16_ts(dcol, aa, bd, idesc, (kb | k) != 0);
-                }
-                if (mb == nmb - 1) mma_commit(&S->wempty[s]);
+          for (int hf = 0; hf < RA::kHalves && !*abort; ++hf, ++u) {
+            const uint32_t slot = u & 1, ph = (u >> 1) & 1;
+            if (!mbar_wait(&S->tempty[slot], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 83); break; }
+            tc_fence_after();
+            const uint32_t dcol = tmem + RA::kAcc + slot * RA::kN;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+              const int s = (int)(it % RA::kStages);
+              if (!mbar_wait(&S->wfull[s], (it / RA::kStages) & 1, abort, kWaitCycles)) {
+                record_timeout(status, abort, 84);
+                break;
               }
-              mma_commit(&S->tfull[slot]);
+              tc_fence_after();
+              const uint32_t bsm = smem_u32(ring + s * RA::kStage);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t aa = tmem + (uint32_t)kb * 32 + (uint32_t)k * 8;
+                const uint64_t bd = sw128_desc(bsm + k * 32, 16, 1024);
+                if (kFp8) mma_e4m3_ts(dcol, aa, bd, idesc, (kb | k) != 0);
+                else mma_bf16_ts(dcol, aa, bd, idesc, (kb | k) != 0);
+              }
+              mma_commit(&S->wempty[s]);
             }
-            it += (uint32_t)nkb;
+            mma_commit(&S->tfull[slot]);
           }
         }
       }
     } else {
-      // Epilogue: warp (q = warp % 4, h = (warp - 2) / 4) takes TMEM lanes
-      // 32 q .. 32 q + 31 of every accumulator slot (samples mb * 128 + 32 q +
-      // lane of M-block mb) and label columns 16 h .. 16 h + 15 of each 64-label
-      // half: all 16 warps drain each slot, so that the MMAs into one slot
-      // overlap the epilogue of the other.
-      const int q = warp & 3, h = (warp - 2) >> 2;
-      const int c_lo = 16 * h;
+      // Epilogue.  E4M3 (one accumulator slot per tile): two groups of eight
+      // warps take alternate tiles, group g always slot g, so that one group's
+      // waits (ring slot, positives, MMA) overlap the other's arithmetic.
+      // bf16 (two 64-label slots per tile): one group of sixteen.  Warp
+      // (q = warp % 4, hh) of a group takes TMEM lanes 32 q .. 32 q + 31
+      // (samples amb * 128 + 32 q + lane) and label columns kColW hh .. +kColW-1
+      // of each slot.
+      constexpr int kGroups = RA::kHalves == 1 ? 2 : 1;
+      constexpr int kWarpsG = kFEpi / kGroups;
+      constexpr int kColW = RA::kN / (kWarpsG / 4);           // 64 (E4M3) or 16 (bf16)
+      const int gp = (warp - 2) / kWarpsG, wg = (warp - 2) % kWarpsG;
+      const int q = warp & 3, hh = wg >> 2;
+      const int c_lo = kColW * hh;
       const float inv_sx = kFp8 ? xscale[1] : 1.0f;
       const float acc_lo = grad_acc_floor<kFp8 ? (kG5 ? 2 : 1) : 0>(inv_sx);
       constexpr int kG = kFp8 ? (kG5 ? 2 : 1) : 0;
       constexpr int kChunk = 16 / kEl;                        // labels per 16-byte chunk
       constexpr int kNlc = 128 / kChunk;                      // chunks per 128-label tile
       unsigned long long* wm = reinterpret_cast<unsigned long long*>(S->pmask[warp - 2]);
+      const int b = amb * 128 + q * 32 + lane;               // this thread's sample
+      const int tstep = kGroups * aN;
       uint32_t use = 0;
-      int lt = 0;
-      for (int t = a; t < T && !*abort; t += aN, ++lt) {
+      int lt = gp;
+      // the key range of this group's next tile, loaded one tile ahead
+      int nk0 = 0, nk1 = 0;
+      if (a + gp * aN < T) { nk0 = __ldg(tile_ptr + a + gp * aN); nk1 = __ldg(tile_ptr + a + gp * aN + 1); }
+      for (int t = a + gp * aN; t < T && !*abort; t += tstep, lt += kGroups) {
         const int slot = t % R, round = t / R;
         uint8_t* gtile = gring + (size_t)slot * tile_bytes;
-        // the slot is free once every d-slice's CTA has copied the tile it held
-        if (round > 0) {
-          bool ok = true;
-          if (lane == 0) ok = wait_flag(consumed + slot, nD * round, abort, status, kWaitCycles);
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok) { if (lane == 0) record_timeout(status, abort, 85); break; }
-        }
-        // positives among this thread's elements of the tile: bit 32 mb + 16 hf
-        // + c for sample (amb + mb) 128 + 32 q + lane and label column
-        // 64 hf + 16 h + c, from the tile's keys: the warp reads them together
-        // (a frequent label's tile holds hundreds) and scatters each into the
-        // mask of its sample's lane
-        uint64_t pm2;
+        // the ring slot's consumed count, read now and checked before the
+        // stores (the slot is free once every d-slice's CTA has copied the
+        // tile it held); the keys of this tile, and the range of the next
+        const int32_t cnow = round > 0 ? ld_relaxed(consumed + slot) : 0;
+        const int k0 = nk0, k1 = nk1;
+        if (t + tstep < T) { nk0 = __ldg(tile_ptr + t + tstep); nk1 = __ldg(tile_ptr + t + tstep + 1); }
+        // positives among this thread's elements of the tile (bit kColW hf + c
+        // for label column kN hf + c_lo + c), from the tile's keys: the warp
+        // reads them together (a frequent label's tile holds hundreds) and
+        // scatters each into the mask of its sample's lane
+        uint64_t pm;
         {
-          const int k0 = __ldg(tile_ptr + t);
-          const int k1 = __ldg(tile_ptr + t + 1);
           wm[lane] = 0;
           __syncwarp();
           const int64_t lbase = (int64_t)t * 128 + c_lo;
           for (int i = k0 + lane; i < k1; i += 32) {
             const uint32_t key = __ldg(keys + i);
             const int smp = (int)(key & 0xFFu);
-            const int mk = (smp >> 7) - amb;                       // M-block of the sample here
-            const int sl = (smp & 127) - 32 * q;                   // its lane
-            const int64_t dl = (int64_t)(key >> 8) - lbase;        // column in the first half, or 64 + column
-            const int64_t c = dl >= kFN ? dl - kFN : dl;
-            if (mk >= 0 && mk < nmb && sl >= 0 && sl < 32 && dl >= 0 && c < 16)
-              atomicOr(wm + sl, 1ull << (32 * mk + (dl >= kFN ? 16 : 0) + c));
+            const int sl = smp - amb * 128 - 32 * q;                // the sample's lane here
+            const int64_t dl = (int64_t)(key >> 8) - lbase;
+            const int hk = dl >= RA::kN ? 1 : 0;                     // the half (bf16)
+            const int64_t c = dl - hk * RA::kN;
+            if (sl >= 0 && sl < 32 && dl >= 0 && c < kColW) atomicOr(wm + sl, 1ull << (kColW * hk + c));
           }
           __syncwarp();
-          pm2 = wm[lane];
+          pm = wm[lane];
           __syncwarp();
         }
         bool stop = false;
-        for (int hf = 0; hf < 2 && !stop; ++hf) {
-          for (int mb = 0; mb < nmb; ++mb) {
-            const uint32_t buf = use & 1, ph = (use >> 1) & 1;
-            ++use;
-            if (!mbar_wait(&S->tfull[buf], ph, abort, kWaitCycles)) {
-              record_timeout(status, abort, 86);
-              stop = true;
-              break;
-            }
-            tc_fence_after();
-            uint32_t v[16];
-            tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + kFAcc + buf * kFN + (uint32_t)c_lo, v);
+        bool free_checked = round == 0;
+        for (int hf = 0; hf < RA::kHalves && !stop; ++hf) {
+          const uint32_t buf = kGroups == 2 ? (uint32_t)gp : (use & 1);
+          const uint32_t ph = kGroups == 2 ? (use & 1) : ((use >> 1) & 1);
+          ++use;
+          if (!mbar_wait(&S->tfull[buf], ph, abort, kWaitCycles)) {
+            record_timeout(status, abort, 86);
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + RA::kAcc + buf * RA::kN + (uint32_t)c_lo;
+#pragma unroll
+          for (int cc = 0; cc < kColW; cc += 32) {
+            constexpr int kLd = kColW < 32 ? kColW : 32;
+            uint32_t v[kLd];
+            if (kLd == 32) tmem_ld32(tbase + cc, *reinterpret_cast<uint32_t(*)[32]>(v));
+            else tmem_ld16(tbase + cc, *reinterpret_cast<uint32_t(*)[16]>(v));
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S->tempty[buf]);
-            const int b = (amb + mb) * 128 + q * 32 + lane;     // sample
-            const int64_t nv = L - ((int64_t)t * 128 + hf * kFN + c_lo);
-            const uint32_t vbits = b >= B || nv <= 0 ? 0u : (nv >= 16 ? 0xFFFFu : (1u << nv) - 1u);
-            uint32_t pk[8];
-            grad_codes16<kG>(v, inv_sx, acc_lo, (uint32_t)(pm2 >> (32 * mb + 16 * hf)) & 0xFFFFu, vbits, pk);
-            if (b < Bp) {
-              const int lc = (hf * kFN + c_lo) / kChunk;
-              *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =
-                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              if (!kFp8)
-                *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc + 1) * 128 + (b & 7) * 16) =
-                    make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            if (cc + 32 >= kColW) {                           // the last load from this slot
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&S->tempty[buf]);
+            }
+            if (!free_checked) {
+              // the slot must be free before the first store into it
+              bool ok = cnow >= nD * round;
+              if (!ok) {
+                if (lane == 0) ok = wait_flag(consumed + slot, nD * round, abort, status, kWaitCycles);
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+              }
+              if (!ok) { if (lane == 0) record_timeout(status, abort, 85); stop = true; break; }
+              free_checked = true;
+            }
+#pragma unroll
+            for (int j = 0; j < kLd; j += 16) {
+              const int col = hf * RA::kN + c_lo + cc + j;          // label column within the tile
+              const int64_t nv = L - ((int64_t)t * 128 + col);
+              const uint32_t vbits = b >= B || nv <= 0 ? 0u : (nv >= 16 ? 0xFFFFu : (1u << nv) - 1u);
+              uint32_t pk[8];
+              grad_codes16<kG>(v + j, inv_sx, acc_lo, (uint32_t)(pm >> (kColW * hf + cc + j)) & 0xFFFFu, vbits,
+                               pk);
+              if (b < Bp) {
+                const int lc = col / kChunk;
+                *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc) * 128 + (b & 7) * 16) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                if (!kFp8)
+                  *reinterpret_cast<uint4*>(gtile + ((size_t)(b >> 3) * kNlc + lc + 1) * 128 + (b & 7) * 16) =
+                      make_uint4(pk[4], pk[5], pk[6], pk[7]);
+              }
             }
           }
         }
         if (stop) break;
-        // publish the tile once all 16 epilogue warps have stored their parts:
-        // each thread orders its stores (and, for the bulk copies that read
-        // them, the async proxy) before its warp's arrival; the last warp to
-        // arrive releases the flag
+        // publish the tile once the group's warps have stored their parts:
+        // each thread orders its stores with the async proxy (the bulk copies
+        // that read them); the warp's stores are ordered before its arrival
+        // at CTA scope (__syncwarp, then a CTA fence), and the last warp to
+        // arrive makes every arrival's stores visible at GPU scope (its fence
+        // is cumulative) and releases the flag.  No thread but that one waits
+        // on a GPU-scope fence, and no barrier can be left waiting by a warp
+        // that stopped early.
         fence_proxy_async_global();
-        __threadfence();
         __syncwarp();
         if (lane == 0) {
+          __threadfence_block();
           const int old = atomicAdd(&S->arrivals[lt & 3], 1);
-          if (old == kFEpi - 1) {
+          if (old == kWarpsG - 1) {
             S->arrivals[lt & 3] = 0;
             __threadfence();
             red_release_add(ready + slot, 1);      // nprod arrivals per round make the tile ready
@@ -359,7 +401,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   constexpr int kK = kFp8 ? 32 : 16;                          // MMA K
   constexpr int kPart = kFp8 ? 256 : 128;                     // samples per G part (one 32 KB slot)
   const int nparts = (Bp + kPart - 1) / kPart;
-  const int nprod = (!kFp8 && Bp > 128) ? 2 : 1;
+  const int nprod = Bp > 128 ? 2 : 1;
   uint8_t* xs = base;
   uint8_t* ws = xs + kFXBytes;
   uint8_t* gs = ws + kFWBytes;
@@ -452,8 +494,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
           ++git;
           if (!mbar_wait(&S->gfull[sg], phg, abort, kWaitCycles)) { record_timeout(status, abort, 97); stop = true; break; }
           tc_fence_after();
-          // G_t is in shared memory once its last part is: the ring slot may be reused
-          if (p == nparts - 1) red_release_add(consumed + t % R, 1);
+          // G_t is in shared memory once its last part is: the ring slot may be
+          // reused.  The copies that read it have completed, so the count
+          // needs no release ordering (and the issuing thread no fence).
+          if (p == nparts - 1) atomicAdd(consumed + t % R, 1);
           const uint32_t ga = smem_u32(gs + sg * kFGSlotBytes);
           const int np = min(kPart, Bp - p * kPart);
           const uint32_t idesc_dx =
@@ -586,10 +630,11 @@ cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float 
   const int T = (int)((h->L + 127) / 128);
   const int nD = (h->d + 127) / 128;
   int nA = 0, nG = 0;
-  fused_split(h->num_sms, nD, T, (!fp8 && Bp > 128) ? 2 : 1, &nA, &nG);
+  fused_split(h->num_sms, nD, T, Bp > 128 ? 2 : 1, &nA, &nG);
   const int grid = nA + nG * nD;
   CUtensorMap tmWa, tmWb, tmX;
-  cudaError_t e = make_tma_map_2d(&tmWa, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, kFN);
+  cudaError_t e = make_tma_map_2d(&tmWa, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d,
+                                  fp8 ? RoleA<1>::kN : RoleA<0>::kN);
   if (e != cudaSuccess) return e;
   e = make_tma_map_2d(&tmWb, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, 128);
   if (e != cudaSuccess) return e;
