@@ -48,8 +48,8 @@ namespace {
 
 constexpr int kFThreads = 576;              // warp 0 TMA, warp 1 MMA + TMEM, warps 2-17 epilogue
 constexpr int kFEpi = 16;
-constexpr int kFStagesA = 16;               // role A: most W k-block stages (bf16: 16 x 8 KB, E4M3: 8 x 16 KB)
-constexpr uint32_t kFRingA = 128 * 1024;    // role A: bytes of the W ring
+constexpr int kFStagesA = 24;               // role A: most W k-block stages (bf16: 24 x 8 KB, E4M3: 12 x 16 KB)
+constexpr uint32_t kFRingA = 192 * 1024;    // role A: bytes of the W ring
 // role A: labels per accumulator slot (the MMA's N), its W stage, its first
 // accumulator column (one M-block of X below it: E4M3 192 columns at d = 768,
 // bf16 384)
@@ -411,9 +411,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&S->xfull, 1);
     mbar_init(&S->dxfull, 1);
-    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kFEpi); }
+    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kFEpi / 2); }
     for (int s = 0; s < kFGSlots; ++s) { mbar_init(&S->gfull[s], 1); mbar_init(&S->gempty[s], 1); }
-    for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->dwfull[b2], 1); mbar_init(&S->dwempty[b2], kFEpi); }
+    for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->dwfull[b2], 1); mbar_init(&S->dwempty[b2], kFEpi / 2); }
     S->abort = 0;
     fence_barrier_init();
   }
@@ -488,6 +488,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
         const uint32_t wa = smem_u32(ws + sw * kWSB);
         const uint32_t dwcol = tmem + 256 + db * 128;
         bool stop = false;
+        // dW first (the epilogue waits for it), then dX^T; the G parts (at
+        // most two) stay in their slots until both are issued
+        int sgs[2] = {0, 0};
         for (int p = 0; p < nparts; ++p) {
           const int sg = git % kFGSlots;
           const uint32_t phg = (git / kFGSlots) & 1;
@@ -498,7 +501,22 @@ __global__ void __launch_bounds__(kFThreads, 1)
           // reused.  The copies that read it have completed, so the count
           // needs no release ordering (and the issuing thread no fence).
           if (p == nparts - 1) atomicAdd(consumed + t % R, 1);
+          sgs[p] = sg;
           const uint32_t ga = smem_u32(gs + sg * kFGSlotBytes);
+          const int np = min(kPart, Bp - p * kPart);
+          // dW[tile, slice] += G_part^T X[part, slice] : M = 128 labels, N = 128, K = np samples
+#pragma unroll 1
+          for (int k = 0; k < np / kK; ++k) {
+            const uint64_t ad = nosw_desc(ga + k * (kK / 8) * gstride, gstride, 128);
+            const uint64_t bd = sw128_desc(xa + (p * kPart + k * kK) * 128, 32768, 1024);
+            if (kFp8) mma_e4m3(dwcol, ad, bd, idesc_dw, (p | k) != 0);
+            else mma_bf16(dwcol, ad, bd, idesc_dw, (p | k) != 0);
+          }
+        }
+        if (stop) break;
+        mma_commit(&S->dwfull[db]);
+        for (int p = 0; p < nparts; ++p) {
+          const uint32_t ga = smem_u32(gs + sgs[p] * kFGSlotBytes);
           const int np = min(kPart, Bp - p * kPart);
           const uint32_t idesc_dx =
               kFp8 ? make_idesc(kW5, gfmt, 1, 0, 128, (uint32_t)np) : make_idesc(1, 1, 1, 0, 128, (uint32_t)np);
@@ -510,63 +528,67 @@ __global__ void __launch_bounds__(kFThreads, 1)
             if (kFp8) mma_e4m3(tmem + (uint32_t)(p * kPart), ad, bd, idesc_dx, !(first && k == 0));
             else mma_bf16(tmem + (uint32_t)(p * kPart), ad, bd, idesc_dx, !(first && k == 0));
           }
-          // dW[tile, slice] += G_part^T X[part, slice] : M = 128 labels, N = 128, K = np samples
-#pragma unroll 1
-          for (int k = 0; k < np / kK; ++k) {
-            const uint64_t ad = nosw_desc(ga + k * (kK / 8) * gstride, gstride, 128);
-            const uint64_t bd = sw128_desc(xa + (p * kPart + k * kK) * 128, 32768, 1024);
-            if (kFp8) mma_e4m3(dwcol, ad, bd, idesc_dw, (p | k) != 0);
-            else mma_bf16(dwcol, ad, bd, idesc_dw, (p | k) != 0);
-          }
-          mma_commit(&S->gempty[sg]);
+          mma_commit(&S->gempty[sgs[p]]);
         }
-        if (stop) break;
-        mma_commit(&S->dwfull[db]);
         first = false;
       }
       mma_commit(&S->dxfull);
     }
   } else {
+    // Two groups of eight warps take alternate units, group g always dW slot
+    // g, so that one group's waits and TMEM loads overlap the other's SR
+    // arithmetic.  Warp (q = warp % 4, sub) of a group updates label row
+    // 32 q + lane and columns 64 sub .. 64 sub + 63 of the slice.
     const int q = warp & 3;
-    const int sub = (warp - 2) >> 2;                // columns sub * 32 .. +31 of the slice
+    const int gpb = (warp - 2) >> 3, sub = ((warp - 2) & 7) >> 2;
     const int row = q * 32 + lane;                  // label row of dW; column of d for dX^T
     const float lrs = kFp8 ? lr * (0.00390625f * xscale[1]) : lr;
     const float dx_scale = kFp8 ? 0.00390625f : 1.0f;
-    uint32_t wit = 0, dwit = 0;
-    bool any = false;
-    for (int t = g; t < T && !*abort; t += nG) {
-      any = true;
-      const int sw = wit % kWS;
-      ++wit;
-      const uint32_t db = dwit & 1, duse = dwit >> 1;
-      ++dwit;
+    constexpr int kWf = kFp8 ? (kW5 ? 2 : 1) : 0;
+    uint32_t ui = (uint32_t)gpb, use = 0;           // unit index within this CTA's run, this group's uses
+    for (int t = g + gpb * nG; t < T && !*abort; t += 2 * nG, ui += 2, ++use) {
+      const int sw = (int)(ui % kWS);
+      const uint32_t db = (uint32_t)gpb;
       const int64_t l = (int64_t)t * 128 + row;
-      const int jl = sub * 32;                      // columns jl .. jl + 31 of the 128-column slice
+      const int jl = sub * 64;                      // columns jl .. jl + 63 of the 128-column slice
       const int j0 = D0 + jl;
-      const bool valid = l < L && j0 < d;           // d is a multiple of 64: both groups or none
-      // the draws do not depend on the gradient: form them while the MMAs run
-      uint32_t rw0[8], rw1[8];
-      if (valid) {
-        sr_draws16(rk, step, blk_base, l, d, j0, rw0);
-        sr_draws16(rk, step, blk_base, l, d, j0 + 16, rw1);
-      }
-      if (!mbar_wait(&S->dwfull[db], duse & 1, abort, kWaitCycles)) { record_timeout(status, abort, 98); break; }
+      const bool valid = l < L && j0 < d;           // d is a multiple of 64: all 64 columns or none
+      // the first draws do not depend on the gradient: form them while the MMAs run
+      uint32_t rw[8];
+      if (valid) sr_draws16(rk, step, blk_base, l, d, j0, rw);
+      if (!mbar_wait(&S->dwfull[db], use & 1, abort, kWaitCycles)) { record_timeout(status, abort, 98); break; }
       tc_fence_after();
       const uint8_t* wrow = ws + sw * kWSB;
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + 256 + db * 128 + jl;
-      uint32_t r0[16], r1[16];
-      tmem_ld16(taddr, r0);
-      tmem_wait_ld();
-      tmem_ld16(taddr + 16, r1);
-      constexpr int kWf = kFp8 ? (kW5 ? 2 : 1) : 0;
-      if (valid) update16<kWf>(r0, rw0, wrow, row, jl, l, d, j0, lrs, Wglob);
-      tmem_wait_ld();
-      if (valid) update16<kWf>(r1, rw1, wrow, row, jl + 16, l, d, j0 + 16, lrs, Wglob);
-      tc_fence_before();
+      // four 16-column chunks, two register sets: the load of the next chunk
+      // is in flight during the update of this one
+      uint32_t ra[16], rb[16];
+      tmem_ld16(taddr, ra);
+#pragma unroll
+      for (int c = 0; c < 4; c += 2) {
+        tmem_wait_ld();                                         // chunk c in ra
+        tmem_ld16(taddr + 16 * (c + 1), rb);
+        if (valid) {
+          update16<kWf>(ra, rw, wrow, row, jl + 16 * c, l, d, j0 + 16 * c, lrs, Wglob);
+          sr_draws16(rk, step, blk_base, l, d, j0 + 16 * (c + 1), rw);
+        }
+        tmem_wait_ld();                                         // chunk c + 1 in rb
+        if (c + 2 < 4) {
+          tmem_ld16(taddr + 16 * (c + 2), ra);
+        } else {                                                // the last load from the dW slot
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S->dwempty[db]);
+        }
+        if (valid) {
+          update16<kWf>(rb, rw, wrow, row, jl + 16 * (c + 1), l, d, j0 + 16 * (c + 1), lrs, Wglob);
+          if (c + 2 < 4) sr_draws16(rk, step, blk_base, l, d, j0 + 16 * (c + 2), rw);
+        }
+      }
       __syncwarp();
-      if (lane == 0) { mbar_arrive(&S->dwempty[db]); mbar_arrive(&S->wempty[sw]); }
+      if (lane == 0) mbar_arrive(&S->wempty[sw]);
     }
-    if (any && !*abort) {
+    if (g < T && !*abort) {
       // flush dX^T of this CTA: lane = column j of the slice, TMEM columns = samples
       if (!mbar_wait(&S->dxfull, 0, abort, kWaitCycles)) {
         record_timeout(status, abort, 99);
@@ -574,7 +596,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         tc_fence_after();
         const int j = D0 + row;
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
-        for (int c = sub; c < Bp / 32; c += 4) {
+        for (int c = (warp - 2) >> 2; c < Bp / 32; c += 4) {
           uint32_t ra[32];
           tmem_ld32(taddr + c * 32, ra);
           tmem_wait_ld();
@@ -604,12 +626,16 @@ bool fused_step_supported(const elmo_head* h, int32_t B) {
   return h->d % 64 == 0 && h->d <= 768 && Bp <= 256;
 }
 
-// Work of one 128-label tile in each role, in the units of the split: role A
-// (Z for the tile, G) against role B (dX^T and dW for every d-slice, and the
-// SR update of every weight, which the epilogue's instruction issue bounds).
-// Measured on B200 for the workloads' shapes; ELMO_FUSED_A overrides nA.
-void fused_split(int grid, int nD, int T, int nprod, int* nA, int* nG) {
-  int a = (grid * 27 + 50) / 100;                   // about 27 % of the SMs form G
+// The split of the SMs between the roles follows their measured cost per
+// 128-label tile on B200 at the workloads' shapes (d = 768): role A (Z and G
+// of the tile; two CTAs per tile when B > 128) against role B (dX^T, dW and
+// the SR update of the tile's weights for every d-slice, bound by the
+// epilogue's instruction issue).  E4M3: role A about a quarter of the step's
+// SM time; bf16 with two producers per tile 38 %, with one 27 %.
+// ELMO_FUSED_A overrides nA.
+void fused_split(int grid, int nD, int T, int nprod, bool fp8, int* nA, int* nG) {
+  const int pct = fp8 ? 24 : (nprod == 2 ? 38 : 27);
+  int a = (grid * pct + 50) / 100;
   const char* v = getenv("ELMO_FUSED_A");
   if (v && atoi(v) > 0) a = atoi(v);
   if (a > grid - nD) a = grid - nD;
@@ -630,7 +656,7 @@ cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float 
   const int T = (int)((h->L + 127) / 128);
   const int nD = (h->d + 127) / 128;
   int nA = 0, nG = 0;
-  fused_split(h->num_sms, nD, T, Bp > 128 ? 2 : 1, &nA, &nG);
+  fused_split(h->num_sms, nD, T, Bp > 128 ? 2 : 1, fp8, &nA, &nG);
   const int grid = nA + nG * nD;
   CUtensorMap tmWa, tmWb, tmX;
   cudaError_t e = make_tma_map_2d(&tmWa, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d,
