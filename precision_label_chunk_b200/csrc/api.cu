@@ -84,10 +84,11 @@ elmo_status ensure_gbuf(elmo_head* h, size_t bytes) {
 }
 
 // The persistent step's ring: kRingTiles gradient-operand tiles of up to
-// 128 labels x 256 samples (64 KB in bf16), and its two flag arrays.
+// 128 labels x 256 samples (64 KB in bf16), its two flag arrays and the
+// step's tile counters.
 elmo_status ensure_ring(elmo_head* h) {
   const size_t tiles = elmo::kRingTiles;
-  const size_t bytes = tiles * 65536 + 2 * sizeof(int32_t) * tiles;
+  const size_t bytes = tiles * 65536 + sizeof(int32_t) * (2 * tiles + elmo::kRingCounters);
   if (h->ring_bytes >= bytes) return ELMO_OK;
   if (h->ring) cudaFree(h->ring);
   h->ring = nullptr;

@@ -40,7 +40,7 @@ struct elmo_head {
   void* gbuf = nullptr;        // per-chunk gradient operands
   size_t gbuf_bytes = 0;
   void* ring = nullptr;        // the persistent step's ring of gradient-operand tiles
-  int32_t* ring_flags = nullptr; // [2 * ring_tiles]: ready, then consumed (zeroed every step)
+  int32_t* ring_flags = nullptr; // [2 * ring_tiles]: ready, then consumed; then kRingCounters tile counters (zeroed every step)
   int32_t ring_tiles = 0;
   size_t ring_bytes = 0;
   void* cand = nullptr;        // top-k candidates
@@ -116,6 +116,7 @@ cudaError_t launch_update_tc(const elmo_head* h, const uint16_t* X, int32_t B, i
 // update), for the shapes whose X fits in TMEM
 bool fused_step_supported(const elmo_head* h, int32_t B);
 constexpr int32_t kRingTiles = 256;      // gradient-operand tiles in the ring
+constexpr int32_t kRingCounters = 16;    // after the ring's flags: the persistent step's tile counters
 cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float lr, uint64_t seed, uint64_t step,
                               float* dX, cudaStream_t s);
 

@@ -65,9 +65,13 @@ constexpr uint32_t kFGSlotBytes = 2 * kBox; // one G tile: 128 labels x up to 25
 constexpr uint32_t kFXBytes = 2 * 32768;    // role B: X[:, slice]
 constexpr uint32_t kFWBytes = 4 * kBox;     // role B: W slots (E4M3 4 x 16 KB, bf16 2 x 32 KB)
 
+constexpr int kFQ = 8;                      // entries of a CTA's tile queue
+
 struct SmemFA {
   uint64_t wfull[kFStagesA], wempty[kFStagesA], tfull[2], tempty[2];
   uint64_t xready;
+  uint64_t qfull[kFQ], qempty[kFQ];           // the tile queue: tiles taken by the TMA warp, in order
+  int tq[kFQ];
   uint64_t pmask[kFEpi][32];   // per epilogue warp: its 32 samples' positives among its labels
   int arrivals[4];             // epilogue warps done with a tile's G (by local tile index mod 4)
   uint32_t tmem_base;
@@ -76,6 +80,9 @@ struct SmemFA {
 
 struct SmemFB {
   uint64_t xfull, dxfull;
+  uint64_t qfull[kFQ], qempty[kFQ];
+  int tq[kFQ];
+  int first_t;                                // the first tile taken (negative: none)
   uint64_t wfull[4], wempty[4];
   uint64_t gfull[kFGSlots], gempty[kFGSlots];
   uint64_t dwfull[2], dwempty[2];
@@ -130,8 +137,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
                const __grid_constant__ CUtensorMap tmX, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
                int32_t Bp, const uint8_t* __restrict__ xop, const uint32_t* __restrict__ keys,
                const int32_t* __restrict__ tile_ptr, const float* __restrict__ xscale, uint8_t* __restrict__ gring,
-               int32_t R, int32_t* __restrict__ ready, int32_t* __restrict__ consumed, int32_t nA, int32_t nG,
-               float lr, const PhiloxKeys rk, uint64_t step, uint64_t blk_base, float* __restrict__ dX,
+               int32_t R, int32_t* __restrict__ ready, int32_t* __restrict__ consumed,
+               int32_t* __restrict__ sched, int32_t nA, int32_t nG, float lr, const PhiloxKeys rk, uint64_t step, uint64_t blk_base, float* __restrict__ dX,
                int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -155,9 +162,13 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // their halves of G.
     const int nprod = Bp > 128 ? 2 : 1;
     const int amb = nprod == 2 ? (int)(blockIdx.x & 1) : 0;   // the M-block held here
-    const int a = nprod == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    const int aN = nprod == 2 ? (nA >> 1) : nA;               // tile stride of the producers
+    // Tiles are handed out in order, one counter per M-block (sched[amb]): a
+    // CTA's TMA warp takes the next tile and passes it to the MMA warp and the
+    // epilogue through a queue in shared memory.
+    constexpr int kGroups = RA::kHalves == 1 ? 2 : 1;        // epilogue groups (alternate queue entries)
+    constexpr int kWarpsG = kFEpi / kGroups;
     if (threadIdx.x == 0) {
+      for (int i = 0; i < kFQ; ++i) { mbar_init(&S->qfull[i], 1); mbar_init(&S->qempty[i], 1 + kWarpsG); }
       for (int s = 0; s < RA::kStages; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
       // each slot is drained by one group: both groups of eight (E4M3) or all sixteen warps (bf16)
       for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], kFEpi / (RA::kHalves == 1 ? 2 : 1)); }
@@ -205,16 +216,45 @@ __global__ void __launch_bounds__(kFThreads, 1)
       if (elect_one()) {
         tma_prefetch_desc(&tmWa);
         uint32_t it = 0;
-        for (int t = a; t < T && !*abort; t += aN) {
-          for (int hf = 0; hf < RA::kHalves; ++hf) {
+        for (uint32_t i = 0;; ++i) {
+          const int qs = (int)(i % kFQ);
+          if (!mbar_wait(&S->qempty[qs], ((i / kFQ) & 1) ^ 1, abort, kWaitCycles)) {
+            record_timeout(status, abort, 80);
+            break;
+          }
+          int t = atomicAdd(sched + amb, 1);
+          if (t >= T || *abort) t = -1;
+          S->tq[qs] = t;
+          mbar_arrive(&S->qfull[qs]);
+          if (t < 0) {
+            // a terminator for each epilogue group (they take alternate entries)
+            for (int e = 1; e < kGroups; ++e) {
+              const uint32_t i2 = i + (uint32_t)e;
+              const int q2 = (int)(i2 % kFQ);
+              if (!mbar_wait(&S->qempty[q2], ((i2 / kFQ) & 1) ^ 1, abort, kWaitCycles)) {
+                record_timeout(status, abort, 80);
+                break;
+              }
+              S->tq[q2] = -1;
+              mbar_arrive(&S->qfull[q2]);
+            }
+            break;
+          }
+          bool stop = false;
+          for (int hf = 0; hf < RA::kHalves && !stop; ++hf) {
             for (int kb = 0; kb < nkb; ++kb, ++it) {
               const int s = (int)(it % RA::kStages);
               const uint32_t ph = (it / RA::kStages) & 1;
-              if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 81); break; }
+              if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) {
+                record_timeout(status, abort, 81);
+                stop = true;
+                break;
+              }
               mbar_arrive_expect_tx(&S->wfull[s], RA::kStage);
               tma_load_2d(ring + s * RA::kStage, &tmWa, &S->wfull[s], kb * kbe, t * 128 + hf * RA::kN);
             }
           }
+          if (stop) break;
         }
       }
     } else if (warp == 1) {
@@ -224,7 +264,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
         uint32_t it = 0, u = 0;
         if (!mbar_wait(&S->xready, 0, abort, kWaitCycles)) record_timeout(status, abort, 82);
         tc_fence_after();
-        for (int t = a; t < T && !*abort; t += aN) {
+        for (uint32_t i = 0; !*abort; ++i) {
+          const int qs = (int)(i % kFQ);
+          if (!mbar_wait(&S->qfull[qs], (i / kFQ) & 1, abort, kWaitCycles)) { record_timeout(status, abort, 87); break; }
+          const int t = S->tq[qs];
+          mbar_arrive(&S->qempty[qs]);
+          if (t < 0) break;
           for (int hf = 0; hf < RA::kHalves && !*abort; ++hf, ++u) {
             const uint32_t slot = u & 1, ph = (u >> 1) & 1;
             if (!mbar_wait(&S->tempty[slot], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 83); break; }
@@ -259,8 +304,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
       // (q = warp % 4, hh) of a group takes TMEM lanes 32 q .. 32 q + 31
       // (samples amb * 128 + 32 q + lane) and label columns kColW hh .. +kColW-1
       // of each slot.
-      constexpr int kGroups = RA::kHalves == 1 ? 2 : 1;
-      constexpr int kWarpsG = kFEpi / kGroups;
       constexpr int kColW = RA::kN / (kWarpsG / 4);           // 64 (E4M3) or 16 (bf16)
       const int gp = (warp - 2) / kWarpsG, wg = (warp - 2) % kWarpsG;
       const int q = warp & 3, hh = wg >> 2;
@@ -272,21 +315,22 @@ __global__ void __launch_bounds__(kFThreads, 1)
       constexpr int kNlc = 128 / kChunk;                      // chunks per 128-label tile
       unsigned long long* wm = reinterpret_cast<unsigned long long*>(S->pmask[warp - 2]);
       const int b = amb * 128 + q * 32 + lane;               // this thread's sample
-      const int tstep = kGroups * aN;
       uint32_t use = 0;
-      int lt = gp;
-      // the key range of this group's next tile, loaded one tile ahead
-      int nk0 = 0, nk1 = 0;
-      if (a + gp * aN < T) { nk0 = __ldg(tile_ptr + a + gp * aN); nk1 = __ldg(tile_ptr + a + gp * aN + 1); }
-      for (int t = a + gp * aN; t < T && !*abort; t += tstep, lt += kGroups) {
+      // queue entries gp, gp + kGroups, ...: this group's tiles, in the order taken
+      for (uint32_t lt = (uint32_t)gp; !*abort; lt += kGroups) {
+        const int qs = (int)(lt % kFQ);
+        if (!mbar_wait(&S->qfull[qs], (lt / kFQ) & 1, abort, kWaitCycles)) { record_timeout(status, abort, 88); break; }
+        const int t = S->tq[qs];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S->qempty[qs]);
+        if (t < 0) break;
         const int slot = t % R, round = t / R;
         uint8_t* gtile = gring + (size_t)slot * tile_bytes;
         // the ring slot's consumed count, read now and checked before the
         // stores (the slot is free once every d-slice's CTA has copied the
-        // tile it held); the keys of this tile, and the range of the next
+        // tile it held), and the tile's range of keys
         const int32_t cnow = round > 0 ? ld_relaxed(consumed + slot) : 0;
-        const int k0 = nk0, k1 = nk1;
-        if (t + tstep < T) { nk0 = __ldg(tile_ptr + t + tstep); nk1 = __ldg(tile_ptr + t + tstep + 1); }
+        const int k0 = __ldg(tile_ptr + t), k1 = __ldg(tile_ptr + t + 1);
         // positives among this thread's elements of the tile (bit kColW hf + c
         // for label column kN hf + c_lo + c), from the tile's keys: the warp
         // reads them together (a frequent label's tile holds hundreds) and
@@ -414,6 +458,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
     for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kFEpi / 2); }
     for (int s = 0; s < kFGSlots; ++s) { mbar_init(&S->gfull[s], 1); mbar_init(&S->gempty[s], 1); }
     for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->dwfull[b2], 1); mbar_init(&S->dwempty[b2], kFEpi / 2); }
+    // queue entries: read by the MMA warp and by one group of eight epilogue warps
+    for (int i = 0; i < kFQ; ++i) { mbar_init(&S->qfull[i], 1); mbar_init(&S->qempty[i], 1 + kFEpi / 2); }
+    S->first_t = -1;
     S->abort = 0;
     fence_barrier_init();
   }
@@ -432,8 +479,33 @@ __global__ void __launch_bounds__(kFThreads, 1)
       mbar_arrive_expect_tx(&S->xfull, (uint32_t)nb * (uint32_t)Bp * 128u);
       for (int qq = 0; qq < 128 / kBoxCols; ++qq)
         if (D0 + qq * kBoxCols < d) tma_load_2d(xs + qq * 32768, &tmX, &S->xfull, D0 + qq * kBoxCols, 0);
+      // units of this slice are handed out in tile order (sched[2 + slice]):
+      // take the next, pass it to the MMA warp and the epilogue, then load
+      // its W slice and copy its G tile once role A has published it
       uint32_t wit = 0, git = 0;
-      for (int t = g; t < T && !*abort; t += nG) {
+      for (uint32_t i = 0;; ++i) {
+        const int qs = (int)(i % kFQ);
+        if (!mbar_wait(&S->qempty[qs], ((i / kFQ) & 1) ^ 1, abort, kWaitCycles)) {
+          record_timeout(status, abort, 90);
+          break;
+        }
+        int t = atomicAdd(sched + 2 + sl, 1);
+        if (t >= T || *abort) t = -1;
+        if (i == 0) S->first_t = t;
+        S->tq[qs] = t;
+        mbar_arrive(&S->qfull[qs]);
+        if (t < 0) {
+          // a terminator for the other epilogue group (the groups take alternate entries)
+          const uint32_t i2 = i + 1;
+          const int q2 = (int)(i2 % kFQ);
+          if (mbar_wait(&S->qempty[q2], ((i2 / kFQ) & 1) ^ 1, abort, kWaitCycles)) {
+            S->tq[q2] = -1;
+            mbar_arrive(&S->qfull[q2]);
+          } else {
+            record_timeout(status, abort, 90);
+          }
+          break;
+        }
         {
           const int s = wit % kWS;
           const uint32_t ph = (wit / kWS) & 1;
@@ -476,7 +548,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
       if (!mbar_wait(&S->xfull, 0, abort, kWaitCycles)) record_timeout(status, abort, 94);
       tc_fence_after();
       const uint32_t xa = smem_u32(xs);
-      for (int t = g; t < T && !*abort; t += nG) {
+      for (uint32_t i = 0; !*abort; ++i) {
+        const int qs = (int)(i % kFQ);
+        if (!mbar_wait(&S->qfull[qs], (i / kFQ) & 1, abort, kWaitCycles)) { record_timeout(status, abort, 89); break; }
+        const int t = S->tq[qs];
+        mbar_arrive(&S->qempty[qs]);
+        if (t < 0) break;
         const int sw = wit % kWS;
         const uint32_t phw = (wit / kWS) & 1;
         ++wit;
@@ -545,8 +622,17 @@ __global__ void __launch_bounds__(kFThreads, 1)
     const float lrs = kFp8 ? lr * (0.00390625f * xscale[1]) : lr;
     const float dx_scale = kFp8 ? 0.00390625f : 1.0f;
     constexpr int kWf = kFp8 ? (kW5 ? 2 : 1) : 0;
-    uint32_t ui = (uint32_t)gpb, use = 0;           // unit index within this CTA's run, this group's uses
-    for (int t = g + gpb * nG; t < T && !*abort; t += 2 * nG, ui += 2, ++use) {
+    uint32_t use = 0;                               // this group's units so far
+    bool any = false;                               // the CTA took at least one unit
+    for (uint32_t ui = (uint32_t)gpb; !*abort; ui += 2, ++use) {
+      // queue entry ui (the CTA's unit index): this group's next unit
+      const int qs = (int)(ui % kFQ);
+      if (!mbar_wait(&S->qfull[qs], (ui / kFQ) & 1, abort, kWaitCycles)) { record_timeout(status, abort, 100); break; }
+      const int t = S->tq[qs];
+      if (ui == (uint32_t)gpb) any = S->first_t >= 0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S->qempty[qs]);
+      if (t < 0) break;
       const int sw = (int)(ui % kWS);
       const uint32_t db = (uint32_t)gpb;
       const int64_t l = (int64_t)t * 128 + row;
@@ -588,7 +674,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->wempty[sw]);
     }
-    if (g < T && !*abort) {
+    if (any && !*abort) {
       // flush dX^T of this CTA: lane = column j of the slice, TMEM columns = samples
       if (!mbar_wait(&S->dxfull, 0, abort, kWaitCycles)) {
         record_timeout(status, abort, 99);
@@ -630,11 +716,11 @@ bool fused_step_supported(const elmo_head* h, int32_t B) {
 // 128-label tile on B200 at the workloads' shapes (d = 768): role A (Z and G
 // of the tile; two CTAs per tile when B > 128) against role B (dX^T, dW and
 // the SR update of the tile's weights for every d-slice, bound by the
-// epilogue's instruction issue).  E4M3: role A about a quarter of the step's
-// SM time; bf16 with two producers per tile 38 %, with one 27 %.
+// epilogue's instruction issue).  E4M3 with two producers per tile: role A
+// 27 % of the SMs; bf16 with two producers 38 %, with one 20 %.
 // ELMO_FUSED_A overrides nA.
 void fused_split(int grid, int nD, int T, int nprod, bool fp8, int* nA, int* nG) {
-  const int pct = fp8 ? 24 : (nprod == 2 ? 38 : 27);
+  const int pct = fp8 ? 27 : (nprod == 2 ? 38 : 20);
   int a = (grid * pct + 50) / 100;
   const char* v = getenv("ELMO_FUSED_A");
   if (v && atoi(v) > 0) a = atoi(v);
@@ -671,8 +757,8 @@ cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float 
                   : step_fused<0, 0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemF);
   if (e != cudaSuccess) return e;
-  // the ring's flags start at zero every step
-  e = cudaMemsetAsync(h->ring_flags, 0, sizeof(int32_t) * 2 * (size_t)h->ring_tiles, s);
+  // the ring's flags and the tile counters start at zero every step
+  e = cudaMemsetAsync(h->ring_flags, 0, sizeof(int32_t) * (2 * (size_t)h->ring_tiles + kRingCounters), s);
   if (e != cudaSuccess) return e;
   const uint8_t* xop = fp8 ? h->xqt : reinterpret_cast<const uint8_t*>(X);
   cudaLaunchConfig_t cfg = {};
@@ -687,7 +773,8 @@ cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float 
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, tmWa, tmWb, tmX, h->W, h->L, h->d, B, Bp, xop, (const uint32_t*)h->keys,
                             (const int32_t*)h->tile_ptr, (const float*)h->xscale, static_cast<uint8_t*>(h->ring),
-                            h->ring_tiles, h->ring_flags, h->ring_flags + h->ring_tiles, nA, nG, lr, philox_keys(seed), step,
+                            h->ring_tiles, h->ring_flags, h->ring_flags + h->ring_tiles,
+                            h->ring_flags + 2 * h->ring_tiles, nA, nG, lr, philox_keys(seed), step,
                             (uint64_t)h->label_base * (uint64_t)h->d / 8, dX, h->status);
 }
 
