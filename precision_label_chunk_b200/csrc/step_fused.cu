@@ -455,7 +455,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&S->xfull, 1);
     mbar_init(&S->dxfull, 1);
-    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kFEpi / 2); }
+    // a W slot is free once its group's epilogue is done with it and the
+    // unit's dX^T MMAs (which read it after dW is committed) have completed
+    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kFEpi / 2 + 1); }
     for (int s = 0; s < kFGSlots; ++s) { mbar_init(&S->gfull[s], 1); mbar_init(&S->gempty[s], 1); }
     for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->dwfull[b2], 1); mbar_init(&S->dwempty[b2], kFEpi / 2); }
     // queue entries: read by the MMA warp and by one group of eight epilogue warps
@@ -607,6 +609,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
           }
           mma_commit(&S->gempty[sgs[p]]);
         }
+        mma_commit(&S->wempty[sw]);
         first = false;
       }
       mma_commit(&S->dxfull);
