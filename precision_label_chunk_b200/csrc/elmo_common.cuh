@@ -57,13 +57,20 @@ inline PhiloxKeys philox_keys(uint64_t seed) {
   return K;
 }
 
+// 32 x 32 -> 64-bit product as (lo, hi) from one wide multiply
+__device__ __forceinline__ void mul_wide_u32(uint32_t a, uint32_t b, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b64 t;\n\tmul.wide.u32 t, %2, %3;\n\tmov.b64 {%0, %1}, t;\n\t}"
+      : "=r"(lo), "=r"(hi) : "r"(a), "r"(b));
+}
+
 __device__ __forceinline__ u32x4 philox10_rk(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
                                               const PhiloxKeys& K) {
   constexpr uint32_t kMulA = 0xD2511F53u, kMulB = 0xCD9E8D57u;
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t hiA = __umulhi(kMulA, c0), loA = kMulA * c0;
-    const uint32_t hiB = __umulhi(kMulB, c2), loB = kMulB * c2;
+    uint32_t loA, hiA, loB, hiB;
+    mul_wide_u32(c0, kMulA, loA, hiA);
+    mul_wide_u32(c2, kMulB, loB, hiB);
     const uint32_t n0 = hiB ^ c1 ^ K.k0[r], n2 = hiA ^ c3 ^ K.k1[r];
     c0 = n0; c1 = loB; c2 = n2; c3 = loA;
   }
