@@ -50,12 +50,15 @@ constexpr int kFThreads = 576;              // warp 0 TMA, warp 1 MMA + TMEM, wa
 constexpr int kFEpi = 16;
 constexpr int kFStagesA = 24;               // role A: most W k-block stages (bf16: 24 x 8 KB, E4M3: 12 x 16 KB)
 constexpr uint32_t kFRingA = 192 * 1024;    // role A: bytes of the W ring
-// role A: labels per accumulator slot (the MMA's N), its W stage, its first
-// accumulator column (one M-block of X below it: E4M3 192 columns at d = 768,
-// bf16 384)
+// role A: a 128-label tile is two halves of kN = 64 labels (the MMA's N),
+// each accumulated in its own TMEM slot of 64 columns after one M-block of X
+// (E4M3 192 columns at d = 768, bf16 384).  E4M3 has room for four slots:
+// two epilogue groups, each with a slot per half; bf16 for two: one group.
 template <int kFp8> struct RoleA {
-  static constexpr int kN = kFp8 ? 128 : 64;
+  static constexpr int kN = 64;
   static constexpr int kHalves = 128 / kN;
+  static constexpr int kGroups = kFp8 ? 2 : 1;
+  static constexpr int kSlots = kGroups * kHalves;
   static constexpr uint32_t kStage = (uint32_t)kN * 128;
   static constexpr int kStages = (int)(kFRingA / kStage);
   static constexpr uint32_t kAcc = kFp8 ? 256 : 384;
@@ -68,7 +71,7 @@ constexpr uint32_t kFWBytes = 4 * kBox;     // role B: W slots (E4M3 4 x 16 KB, 
 constexpr int kFQ = 8;                      // entries of a CTA's tile queue
 
 struct SmemFA {
-  uint64_t wfull[kFStagesA], wempty[kFStagesA], tfull[2], tempty[2];
+  uint64_t wfull[kFStagesA], wempty[kFStagesA], tfull[4], tempty[4];
   uint64_t xready;
   uint64_t qfull[kFQ], qempty[kFQ];           // the tile queue: tiles taken by the TMA warp, in order
   int tq[kFQ];
@@ -165,13 +168,13 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // Tiles are handed out in order, one counter per M-block (sched[amb]): a
     // CTA's TMA warp takes the next tile and passes it to the MMA warp and the
     // epilogue through a queue in shared memory.
-    constexpr int kGroups = RA::kHalves == 1 ? 2 : 1;        // epilogue groups (alternate queue entries)
+    constexpr int kGroups = RA::kGroups;                     // epilogue groups (alternate queue entries)
     constexpr int kWarpsG = kFEpi / kGroups;
     if (threadIdx.x == 0) {
       for (int i = 0; i < kFQ; ++i) { mbar_init(&S->qfull[i], 1); mbar_init(&S->qempty[i], 1 + kWarpsG); }
       for (int s = 0; s < RA::kStages; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], 1); }
       // each slot is drained by one group: both groups of eight (E4M3) or all sixteen warps (bf16)
-      for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], kFEpi / (RA::kHalves == 1 ? 2 : 1)); }
+      for (int b2 = 0; b2 < RA::kSlots; ++b2) { mbar_init(&S->tfull[b2], 1); mbar_init(&S->tempty[b2], kWarpsG); }
       mbar_init(&S->xready, kFEpi);
       for (int i = 0; i < 4; ++i) S->arrivals[i] = 0;
       S->abort = 0;
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       if (elect_one()) {
         const uint32_t idesc =
             kFp8 ? make_idesc(0, kW5, 0, 0, 128, RA::kN) : make_idesc(1, 1, 0, 0, 128, RA::kN);
-        uint32_t it = 0, u = 0;
+        uint32_t it = 0;
         if (!mbar_wait(&S->xready, 0, abort, kWaitCycles)) record_timeout(status, abort, 82);
         tc_fence_after();
         for (uint32_t i = 0; !*abort; ++i) {
@@ -270,8 +273,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
           const int t = S->tq[qs];
           mbar_arrive(&S->qempty[qs]);
           if (t < 0) break;
-          for (int hf = 0; hf < RA::kHalves && !*abort; ++hf, ++u) {
-            const uint32_t slot = u & 1, ph = (u >> 1) & 1;
+          // tile i, half hf: slot (i % kGroups) kHalves + hf, its (i / kGroups)-th use
+          for (int hf = 0; hf < RA::kHalves && !*abort; ++hf) {
+            const uint32_t slot = (i % kGroups) * RA::kHalves + (uint32_t)hf, ph = (i / kGroups) & 1;
             if (!mbar_wait(&S->tempty[slot], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 83); break; }
             tc_fence_after();
             const uint32_t dcol = tmem + RA::kAcc + slot * RA::kN;
@@ -297,14 +301,14 @@ __global__ void __launch_bounds__(kFThreads, 1)
         }
       }
     } else {
-      // Epilogue.  E4M3 (one accumulator slot per tile): two groups of eight
-      // warps take alternate tiles, group g always slot g, so that one group's
-      // waits (ring slot, positives, MMA) overlap the other's arithmetic.
-      // bf16 (two 64-label slots per tile): one group of sixteen.  Warp
-      // (q = warp % 4, hh) of a group takes TMEM lanes 32 q .. 32 q + 31
-      // (samples amb * 128 + 32 q + lane) and label columns kColW hh .. +kColW-1
-      // of each slot.
-      constexpr int kColW = RA::kN / (kWarpsG / 4);           // 64 (E4M3) or 16 (bf16)
+      // Epilogue.  E4M3: two groups of eight warps take alternate tiles, group
+      // g the slots 2 g and 2 g + 1 (one per 64-label half), so that one
+      // group's waits (ring slot, positives, MMA) overlap the other's
+      // arithmetic and the MMAs of one half overlap the epilogue of the other.
+      // bf16: one group of sixteen with two slots.  Warp (q = warp % 4, hh) of
+      // a group takes TMEM lanes 32 q .. 32 q + 31 (samples amb * 128 + 32 q +
+      // lane) and label columns kColW hh .. kColW hh + kColW - 1 of each slot.
+      constexpr int kColW = RA::kN / (kWarpsG / 4);           // 32 (E4M3) or 16 (bf16)
       const int gp = (warp - 2) / kWarpsG, wg = (warp - 2) % kWarpsG;
       const int q = warp & 3, hh = wg >> 2;
       const int c_lo = kColW * hh;
@@ -315,7 +319,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
       constexpr int kNlc = 128 / kChunk;                      // chunks per 128-label tile
       unsigned long long* wm = reinterpret_cast<unsigned long long*>(S->pmask[warp - 2]);
       const int b = amb * 128 + q * 32 + lane;               // this thread's sample
-      uint32_t use = 0;
       // queue entries gp, gp + kGroups, ...: this group's tiles, in the order taken
       for (uint32_t lt = (uint32_t)gp; !*abort; lt += kGroups) {
         const int qs = (int)(lt % kFQ);
@@ -356,9 +359,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
         bool stop = false;
         bool free_checked = round == 0;
         for (int hf = 0; hf < RA::kHalves && !stop; ++hf) {
-          const uint32_t buf = kGroups == 2 ? (uint32_t)gp : (use & 1);
-          const uint32_t ph = kGroups == 2 ? (use & 1) : ((use >> 1) & 1);
-          ++use;
+          const uint32_t buf = (uint32_t)gp * RA::kHalves + (uint32_t)hf;
+          const uint32_t ph = (lt / kGroups) & 1;
           if (!mbar_wait(&S->tfull[buf], ph, abort, kWaitCycles)) {
             record_timeout(status, abort, 86);
             stop = true;
