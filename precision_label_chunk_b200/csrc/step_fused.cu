@@ -243,6 +243,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
             }
             break;
           }
+          // bring the W tile about two rounds of this M-block's CTAs ahead
+          // into L2 (the first M-block's CTAs only: the second finds the same
+          // tiles there), so that the ring's loads meet L2 rather than HBM latency
+          if (amb == 0) {
+            const int tp = t + 2 * (nA / nprod);
+            if (tp < T)
+              for (int hf = 0; hf < RA::kHalves; ++hf)
+                for (int kb = 0; kb < nkb; ++kb) tma_prefetch_l2(&tmWa, kb * kbe, tp * 128 + hf * RA::kN);
+          }
           bool stop = false;
           for (int hf = 0; hf < RA::kHalves && !stop; ++hf) {
             for (int kb = 0; kb < nkb; ++kb, ++it) {
