@@ -274,6 +274,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         const uint32_t idesc =
             kFp8 ? make_idesc(0, kW5, 0, 0, 128, RA::kN) : make_idesc(1, 1, 0, 0, 128, RA::kN);
         uint32_t it = 0;
+        const uint64_t bdesc0 = sw128_desc(smem_u32(ring), 16, 1024);   // stage 0, k = 0
         if (!mbar_wait(&S->xready, 0, abort, kWaitCycles)) record_timeout(status, abort, 82);
         tc_fence_after();
         for (uint32_t i = 0; !*abort; ++i) {
@@ -288,6 +289,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
             if (!mbar_wait(&S->tempty[slot], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 83); break; }
             tc_fence_after();
             const uint32_t dcol = tmem + RA::kAcc + slot * RA::kN;
+            // descriptors advance by constants (the start address field counts
+            // 16-byte units): few instructions per MMA for this thread, which
+            // shares its scheduler with four busy epilogue warps
             for (int kb = 0; kb < nkb; ++kb, ++it) {
               const int s = (int)(it % RA::kStages);
               if (!mbar_wait(&S->wfull[s], (it / RA::kStages) & 1, abort, kWaitCycles)) {
@@ -295,13 +299,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 break;
               }
               tc_fence_after();
-              const uint32_t bsm = smem_u32(ring + s * RA::kStage);
+              const uint64_t bd = bdesc0 + (uint64_t)((uint32_t)s * (RA::kStage >> 4));
+              const uint32_t aa = tmem + (uint32_t)kb * 32;
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                const uint32_t aa = tmem + (uint32_t)kb * 32 + (uint32_t)k * 8;
-                const uint64_t bd = sw128_desc(bsm + k * 32, 16, 1024);
-                if (kFp8) mma_e4m3_ts(dcol, aa, bd, idesc, (kb | k) != 0);
-                else mma_bf16_ts(dcol, aa, bd, idesc, (kb | k) != 0);
+                if (kFp8) mma_e4m3_ts(dcol, aa + (uint32_t)k * 8, bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
+                else mma_bf16_ts(dcol, aa + (uint32_t)k * 8, bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
               }
               mma_commit(&S->wempty[s]);
             }
@@ -595,12 +598,16 @@ __global__ void __launch_bounds__(kFThreads, 1)
           const uint32_t ga = smem_u32(gs + sg * kFGSlotBytes);
           const int np = min(kPart, Bp - p * kPart);
           // dW[tile, slice] += G_part^T X[part, slice] : M = 128 labels, N = 128, K = np samples
-#pragma unroll 1
-          for (int k = 0; k < np / kK; ++k) {
-            const uint64_t ad = nosw_desc(ga + k * (kK / 8) * gstride, gstride, 128);
-            const uint64_t bd = sw128_desc(xa + (p * kPart + k * kK) * 128, 32768, 1024);
-            if (kFp8) mma_e4m3(dwcol, ad, bd, idesc_dw, (p | k) != 0);
-            else mma_bf16(dwcol, ad, bd, idesc_dw, (p | k) != 0);
+          {
+            const uint64_t ad0 = nosw_desc(ga, gstride, 128);
+            const uint64_t bd0 = sw128_desc(xa + p * kPart * 128, 32768, 1024);
+#pragma unroll 4
+            for (int k = 0; k < np / kK; ++k) {
+              const uint64_t ad = ad0 + (uint64_t)(k * ((kK / 8) * gstride >> 4));
+              const uint64_t bd = bd0 + (uint64_t)(k * (kK * 128 >> 4));
+              if (kFp8) mma_e4m3(dwcol, ad, bd, idesc_dw, (p | k) != 0);
+              else mma_bf16(dwcol, ad, bd, idesc_dw, (p | k) != 0);
+            }
           }
         }
         if (stop) break;
@@ -611,12 +618,16 @@ __global__ void __launch_bounds__(kFThreads, 1)
           const uint32_t idesc_dx =
               kFp8 ? make_idesc(kW5, gfmt, 1, 0, 128, (uint32_t)np) : make_idesc(1, 1, 1, 0, 128, (uint32_t)np);
           // dX^T[slice, part] += W^T G_part^T : M = 128 (columns of d), N = np, K = 128 labels
-#pragma unroll 1
-          for (int k = 0; k < 128 / kK; ++k) {
-            const uint64_t ad = sw128_desc(wa + k * kK * 128, kBox, 1024);
-            const uint64_t bd = nosw_desc(ga + k * 2 * 128, 128, gstride);
-            if (kFp8) mma_e4m3(tmem + (uint32_t)(p * kPart), ad, bd, idesc_dx, !(first && k == 0));
-            else mma_bf16(tmem + (uint32_t)(p * kPart), ad, bd, idesc_dx, !(first && k == 0));
+          {
+            const uint64_t ad0 = sw128_desc(wa, kBox, 1024);
+            const uint64_t bd0 = nosw_desc(ga, 128, gstride);
+#pragma unroll 4
+            for (int k = 0; k < 128 / kK; ++k) {
+              const uint64_t ad = ad0 + (uint64_t)(k * (kK * 128 >> 4));
+              const uint64_t bd = bd0 + (uint64_t)(k * (2 * 128 >> 4));
+              if (kFp8) mma_e4m3(tmem + (uint32_t)(p * kPart), ad, bd, idesc_dx, !(first && k == 0));
+              else mma_bf16(tmem + (uint32_t)(p * kPart), ad, bd, idesc_dx, !(first && k == 0));
+            }
           }
           mma_commit(&S->gempty[sgs[p]]);
         }
