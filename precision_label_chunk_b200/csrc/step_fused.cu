@@ -219,14 +219,18 @@ __global__ void __launch_bounds__(kFThreads, 1)
       if (elect_one()) {
         tma_prefetch_desc(&tmWa);
         uint32_t it = 0;
+        // the next tile is taken one tile ahead, so that the counter's round
+        // trip overlaps this tile's loads
+        int t_next = atomicAdd(sched + amb, 1);
         for (uint32_t i = 0;; ++i) {
           const int qs = (int)(i % kFQ);
           if (!mbar_wait(&S->qempty[qs], ((i / kFQ) & 1) ^ 1, abort, kWaitCycles)) {
             record_timeout(status, abort, 80);
             break;
           }
-          int t = atomicAdd(sched + amb, 1);
+          int t = t_next;
           if (t >= T || *abort) t = -1;
+          else t_next = atomicAdd(sched + amb, 1);
           S->tq[qs] = t;
           mbar_arrive(&S->qfull[qs]);
           if (t < 0) {
@@ -499,14 +503,16 @@ __global__ void __launch_bounds__(kFThreads, 1)
       // take the next, pass it to the MMA warp and the epilogue, then load
       // its W slice and copy its G tile once role A has published it
       uint32_t wit = 0, git = 0;
+      int t_next = atomicAdd(sched + 2 + sl, 1);              // taken one unit ahead
       for (uint32_t i = 0;; ++i) {
         const int qs = (int)(i % kFQ);
         if (!mbar_wait(&S->qempty[qs], ((i / kFQ) & 1) ^ 1, abort, kWaitCycles)) {
           record_timeout(status, abort, 90);
           break;
         }
-        int t = atomicAdd(sched + 2 + sl, 1);
+        int t = t_next;
         if (t >= T || *abort) t = -1;
+        else t_next = atomicAdd(sched + 2 + sl, 1);
         if (i == 0) S->first_t = t;
         S->tq[qs] = t;
         mbar_arrive(&S->qfull[qs]);
