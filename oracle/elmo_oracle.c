@@ -22,13 +22,16 @@
  *     s_X = 2^floor(log2(448/max|X|)); G is quantised as E4M3(2^8 * g); both
  *     scales are undone exactly in fp32;  bf16 mode: X as is, G -> RNE bf16;
  *   - E4M3 is OCP E4M3FN (max 448, no infinities), saturating;
- *   - SR uses a 16-bit uniform draw u = k / 2^16 taken from Philox4x32-10
+ *   - SR uses a 16-bit uniform draw k taken from Philox4x32-10
  *     (Salmon et al., SC'11, "Parallel Random Numbers: As Easy as 1, 2, 3")
  *     keyed by the seed, with counter (idx >> 3, step): 8 elements share one
  *     Philox block, element idx uses 16-bit half (idx & 1) of word
  *     ((idx >> 1) & 3), low half first;
- *   - SR(v): v on the grid stays; otherwise with grid neighbours lo < v < hi,
- *     return hi iff u < (v - lo) / (hi - lo), on magnitudes (sign restored);
+ *   - SR(v): v on the grid stays; otherwise with grid neighbours lo < v < hi
+ *     and f = (v - lo) / (hi - lo), return hi iff k < floor(2^16 f): the draw
+ *     is added to the first 16 bits of the discarded fraction and the sum
+ *     truncated (exactly unbiased on bf16, whose fraction has 16 bits; on the
+ *     8-bit grids P(hi) = floor(2^16 f) / 2^16), on magnitudes (sign restored);
  *     NaN -> canonical NaN (bf16 0x7FC0, E4M3 0x7F); E4M3: |v| >= 448 and
  *     +-inf -> +-448; bf16: finite |v| above the largest finite -> largest
  *     finite, +-inf stays +-inf;
@@ -221,9 +224,15 @@ uint8_t orc_rne_e4m3(float v) {
 
 /* ------------------------------------------------------------------------ */
 /* Stochastic rounding, written from its definition: neighbours lo < v < hi */
-/* on the target grid, round to hi iff u < (v - lo) / (hi - lo).  All in    */
-/* double, where these quantities are exact for fp32 inputs.                */
+/* on the target grid, f = (v - lo) / (hi - lo), and the element's 16-bit   */
+/* draw k: round to hi iff k < floor(2^16 f), i.e. iff adding 2^16 - 1 - k  */
+/* to the first 16 bits of the discarded fraction carries.  All in double,  */
+/* where these quantities are exact for fp32 inputs.  On bf16 the fraction  */
+/* has exactly 16 bits (floor(2^16 f) = 2^16 f): unbiased; on the 8-bit     */
+/* grids the probability of hi is f less at most 2^-16.                     */
 /* ------------------------------------------------------------------------ */
+static int sr_up(double f, uint32_t k16) { return (double)k16 < floor(f * 65536.0); }
+
 uint16_t orc_sr_bf16(float v, uint32_t k16) {
   if (isnan(v)) return 0x7FC0;
   uint32_t b = bits_from_f32(v);
@@ -236,8 +245,7 @@ uint16_t orc_sr_bf16(float v, uint32_t k16) {
   if (lo + 1 >= 0x7F80) return sign | 0x7F7F;  /* above the largest finite */
   double vhi = (double)orc_bf16_value((uint16_t)(lo + 1));
   double f = (a - vlo) / (vhi - vlo);
-  double u = (double)k16 / 65536.0;
-  return sign | (uint16_t)((u < f) ? lo + 1 : lo);
+  return sign | (uint16_t)(sr_up(f, k16) ? lo + 1 : lo);
 }
 
 uint8_t orc_sr_e4m3(float v, uint32_t k16) {
@@ -251,8 +259,7 @@ uint8_t orc_sr_e4m3(float v, uint32_t k16) {
   if (e4m3_pos[lo] == a) return sign | (uint8_t)lo;
   int hi = lo + 1;
   double f = (a - e4m3_pos[lo]) / (e4m3_pos[hi] - e4m3_pos[lo]);
-  double u = (double)k16 / 65536.0;
-  return sign | (uint8_t)((u < f) ? hi : lo);
+  return sign | (uint8_t)(sr_up(f, k16) ? hi : lo);
 }
 
 /* E5M2 has infinities, like bf16: +-inf stays +-inf, a finite |v| above the
@@ -269,8 +276,7 @@ uint8_t orc_sr_e5m2(float v, uint32_t k16) {
   if (vlo == a) return sign | (uint8_t)lo;
   double vhi = (double)orc_e5m2_value((uint8_t)(lo + 1));
   double f = (a - vlo) / (vhi - vlo);
-  double u = (double)k16 / 65536.0;
-  return sign | (uint8_t)((u < f) ? lo + 1 : lo);
+  return sign | (uint8_t)(sr_up(f, k16) ? lo + 1 : lo);
 }
 
 /* out[i] = SR(in[i]) with the draw of element index_base + i. */

@@ -61,7 +61,8 @@ def test_result_is_a_neighbour(orc, dtype):
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp8", "e5m2"])
 def test_probability_of_rounding_up_closed_form(orc, dtype):
-    # over all 2^16 draws the count of "hi" is #{k : k/2^16 < f} = ceil(f 2^16)
+    # over all 2^16 draws the count of "hi" is #{k : k < floor(f 2^16)} = floor(f 2^16):
+    # the draw is added to the fraction's first 16 bits and the sum truncated
     g = _grid(dtype)
     rng = np.random.default_rng(5)
     ks = np.arange(65536, dtype=np.uint32)
@@ -74,8 +75,11 @@ def test_probability_of_rounding_up_closed_form(orc, dtype):
         out = _code_value(orc.sr_with_draws(np.full(65536, v, np.float32), ks, dtype), dtype)
         n_hi = int((out == hi).sum())
         f = (Fraction(float(v)) - Fraction(lo)) / (Fraction(hi) - Fraction(lo))
-        expect = -((-f * 65536).numerator // (f * 65536).denominator)  # ceil
+        expect = (f * 65536).numerator // (f * 65536).denominator      # floor
         assert n_hi == expect
+        # which draws round up: exactly the k below that count
+        k_hi = np.nonzero(out == hi)[0]
+        assert k_hi.tolist() == list(range(expect))
         if dtype == "bf16":
             assert Fraction(n_hi, 65536) == f   # exactly unbiased on bf16
 
