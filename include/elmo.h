@@ -146,10 +146,11 @@ elmo_status elmo_head_destroy(elmo_head* h);
  * core operands are E4M3: X is quantised with a per-step power-of-two scale
  * s_X = 2^floor(log2(448 / max|X|)) and G as E4M3(2^8 G); both scales are
  * undone exactly in fp32.  In BF16 mode G is rounded to bf16 (RNE).
- * SR of element (l, j) draws u from Philox4x32-10 with key `seed`, counter
- * (idx >> 3, step), idx = l * d + j (16-bit draw: half idx & 1 of word
- * (idx >> 1) & 3), and rounds to the upper grid neighbour iff u < f, f the
- * fractional position between the neighbours.
+ * SR of element (l, j) takes a 16-bit draw k from Philox4x32-10 with key
+ * `seed`, counter (idx >> 3, step), idx = l * d + j (half idx & 1 of word
+ * (idx >> 1) & 3), and rounds to the upper grid neighbour (in magnitude) iff
+ * k < floor(2^16 f), f the fractional position between the neighbours: the
+ * draw added to the first 16 bits of the discarded fraction carries.
  *
  *   X_dev      : bf16 [B x d] sample embeddings (device).
  *   B          : 1 <= B <= ELMO_MAX_BATCH.
@@ -305,7 +306,7 @@ elmo_status elmo_kahan_sgd(void* p_dev, void* c_dev, const void* g_dev, int64_t 
 elmo_status elmo_round_bf16(const float* in_dev, void* out_dev, int64_t n, void* stream);
 
 /*
- * elmo_sr_draws -- the 16-bit uniform draws k (u = k / 2^16) that SR uses for
+ * elmo_sr_draws -- the 16-bit uniform draws k that SR uses for
  * elements index_base .. index_base + n - 1 of stream (seed, step), as uint16
  * into out_dev [n] (device).  Philox4x32-10 of Salmon et al. (SC'11).
  */

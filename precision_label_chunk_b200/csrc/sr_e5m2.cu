@@ -3,16 +3,14 @@
 // The same rounding as the other grids ("ELMO: Efficiency via Low-precision
 // and Peak Memory Optimization in Large Output Spaces", abstract: stochastic
 // rounding in place of FP32 master weights): with grid neighbours
-// lo < |v| < hi, round to hi iff u < f = (|v| - lo) / (hi - lo), u = k / 2^16,
-// sign restored.  E5M2 has infinities, so +-inf stays +-inf, a finite |v| at
-// or above the largest finite value 57344 saturates to it, NaN -> 0x7F.
+// lo < |v| < hi and f = (|v| - lo) / (hi - lo), round to hi iff
+// k < floor(2^16 f) for the element's 16-bit draw k, sign restored.  E5M2 has
+// infinities, so +-inf stays +-inf, a finite |v| at or above the largest
+// finite value 57344 saturates to it, NaN -> 0x7F.
 //
-// The decision is exact.  Normal range (|v| >= 2^-14): E5M2 keeps 2 of fp32's
-// 23 mantissa bits, so with F the 21 discarded bits, u < f <=> 32 k < F, and
-// adding 2^21 - 1 - 32 k to the bit pattern carries into the first kept bit
-// exactly then (into the exponent where the mantissa is full).  Below 2^-14
-// the grid spacing is 2^-16: t = |v| 2^16, its integer part q and fraction
-// t - q are exact in fp32, and the result is (q + [k < 2^16 (t - q)]) 2^-16.
+// Finite values go through the stochastic conversion cvt.rs.satfinite
+// .e5m2x4.f32, which applies exactly this rule; the per-value path
+// (sr_e5m2_code) handles NaN and infinities and the unaligned edges.
 #include "elmo_common.cuh"
 #include "elmo_internal.h"
 
@@ -36,14 +34,8 @@ __global__ void __launch_bounds__(256) sr_e5m2_kernel(const float* __restrict__ 
   }
 }
 
-// Eight values with the eight draws of one Philox block, without a branch
-// per value.  Below 2^-14 a value is first moved into [2^-14, 2^-13), whose
-// spacing is also 2^-16, by adding 2^-14 rounded toward +inf: in units of the
-// 21 discarded bits that keeps ceil(F), and for an integer 32 k,
-// 32 k < F <=> 32 k < ceil(F), so the carry test stays exact; the 2^-14 is
-// taken off again exactly.  Values at or above 57344 round to at least 57344
-// and the saturating conversion brings them to 57344.  A group holding a NaN
-// or an infinity takes the per-value path.
+// Eight values with the eight draws of one Philox block: the stochastic
+// conversion when all are finite, else the per-value path.
 __device__ __forceinline__ uint2 sr8_e5m2(const float (&v)[8], const u32x4& r) {
   const uint32_t w[4] = {r.x, r.y, r.z, r.w};
   float probe = 0.0f;
@@ -55,19 +47,7 @@ __device__ __forceinline__ uint2 sr8_e5m2(const float (&v)[8], const u32x4& r) {
     for (int e = 0; e < 8; ++e) c[e] = sr_e5m2_code(v[e], (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu));
     return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
   }
-  float o[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const uint32_t k = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-    const float a = fabsf(v[e]);
-    // sub = 1 when |v| < 2^-14: (2^-14 - |v|) 2^100 is then >= 2^62, else <= 0
-    const float sub = __saturatef(__fmaf_rn(-a, 0x1p100f, 0x1p86f));
-    const float sh = __fmaf_ru(sub, 0x1p-14f, a);
-    const uint32_t t = (__float_as_uint(sh) + (0x1FFFFFu - (k << 5))) & 0xFFE00000u;
-    o[e] = copysignf(__fmaf_rn(sub, -0x1p-14f, __uint_as_float(t)), v[e]);
-  }
-  return make_uint2(pack_e5m2x2(o[1], o[0]) | (pack_e5m2x2(o[3], o[2]) << 16),
-                    pack_e5m2x2(o[5], o[4]) | (pack_e5m2x2(o[7], o[6]) << 16));
+  return make_uint2(sr_e5m2x4_hw(v[0], v[1], v[2], v[3], w[0], w[1]), sr_e5m2x4_hw(v[4], v[5], v[6], v[7], w[2], w[3]));
 }
 
 // Whole Philox blocks: thread t rounds the 8 values of block q0 + t (two

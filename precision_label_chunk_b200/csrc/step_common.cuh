@@ -230,18 +230,15 @@ __device__ __forceinline__ void sr_draws16(const PhiloxKeys& rk, uint64_t step, 
 // 128B-swizzled W tile in shared memory (row `row`, tile column jl), draws rw
 // from sr_draws16.
 //
-// v = fl(w - fl(lrs dW)) (two roundings, denormals kept), then add-and-
-// truncate: if the bits of v below the target precision hold the fraction F
-// (in units of 2^-n of a grid step), u < f  <=>  2^(n-16) k < F  <=>  adding
-// 2^n - 1 - 2^(n-16) k carries into the first kept bit.
-// bf16 (n = 16): the hardware's stochastic conversion cvt.rs.bf16x2.f32 adds
-// its 16 random bits to the 16 discarded bits of each value and truncates, so
-// passing 2^16 - 1 - k (the complemented draw) gives exactly this rounding.
-// E4M3 (n = 20) and E5M2 (n = 21): below the smallest normal value (2^-6,
-// 2^-14) the grid is uniform with the spacing of the lowest binade; |v| is
-// scaled so that fp32's denormals take the same structure (below), truncated
-// there and scaled back exactly; the sign is restored and the saturating
-// conversion maps magnitudes at or above the largest finite value to it.
+// v = fl(w - fl(lrs dW)) (two roundings, denormals kept), then stochastic
+// rounding with the element's 16-bit draw k: round away from the lower
+// neighbour iff k < floor(2^16 f), f the position of |v| between its grid
+// neighbours.  bf16: cvt.rs.bf16x2.f32 adds its 16 random bits to the 16
+// discarded bits of each value and truncates, so passing 2^16 - 1 - k (the
+// complemented draw) gives exactly this rounding; E4M3 and E5M2: the
+// stochastic conversions to the 8-bit formats apply the same rule to a 16-bit
+// field (sr_e4m3x4_hw / sr_e5m2x4_hw).  A group holding a NaN or an infinity
+// takes the exact per-element path.
 // kW: the weight grid, 0 bf16, 1 E4M3, 2 E5M2.
 template <int kW>
 __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t (&rw)[8],
@@ -285,31 +282,12 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t
   for (int i = 0; i < 16; ++i) probe = __fmaf_rn(vv[i], kW ? 0.0f : 2.0f, probe);
   if (fabsf(probe) < INFINITY) {
     if (kW) {
-      // |v| scaled by 2^-120 (E4M3) or 2^-112 (E5M2) puts the grid's smallest
-      // normal on fp32's (2^-126) and its subnormal spacing on 2^20 (2^21) of
-      // fp32's denormal steps, so one add-and-truncate covers both ranges; the
-      // scaling rounds up, which keeps ceil(F) of the fraction (for an integer
-      // k, 2^(n-16) k < F <=> 2^(n-16) k < ceil(F)), and scaling back is exact
-      constexpr float kDown = kW == 1 ? 0x1p-120f : 0x1p-112f;
-      constexpr float kUp = kW == 1 ? 0x1p120f : 0x1p112f;
-      constexpr uint32_t kMask = kW == 1 ? 0xFFF00000u : 0xFFE00000u;
-      constexpr uint32_t kOne = kW == 1 ? 0xFFFFFu : 0x1FFFFFu;
-      constexpr int kShift = kW == 1 ? 4 : 5;
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        float o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t word = rw[2 * q4 + (e >> 1)];
-          const uint32_t k16 = (e & 1) ? (word >> 16) : (word & 0xFFFFu);
-          const float v = vv[4 * q4 + e];
-          const float sm = __fmul_ru(fabsf(v), kDown);
-          const uint32_t t = (__float_as_uint(sm) + (kOne - (k16 << kShift))) & kMask;
-          o[e] = __fmul_rn(__uint_as_float(t | (__float_as_uint(v) & 0x80000000u)), kUp);
-        }
-        wnew[q4] = kW == 1 ? pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16)
-                           : pack_e5m2x2(o[1], o[0]) | (pack_e5m2x2(o[3], o[2]) << 16);
-      }
+      for (int q4 = 0; q4 < 4; ++q4)
+        wnew[q4] = kW == 1 ? sr_e4m3x4_hw(vv[4 * q4], vv[4 * q4 + 1], vv[4 * q4 + 2], vv[4 * q4 + 3], rw[2 * q4],
+                                          rw[2 * q4 + 1])
+                           : sr_e5m2x4_hw(vv[4 * q4], vv[4 * q4 + 1], vv[4 * q4 + 2], vv[4 * q4 + 3], rw[2 * q4],
+                                          rw[2 * q4 + 1]);
     } else {
 #pragma unroll
       for (int p = 0; p < 8; ++p) {

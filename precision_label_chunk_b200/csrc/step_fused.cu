@@ -475,11 +475,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
     mbar_init(&S->dxfull, 1);
     // a W slot is free once its group's epilogue is done with it and the
     // unit's dX^T MMAs (which read it after dW is committed) have completed
-    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kFEpi / 2 + 1); }
+    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kFEpi + 1); }
     for (int s = 0; s < kFGSlots; ++s) { mbar_init(&S->gfull[s], 1); mbar_init(&S->gempty[s], 1); }
-    for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->dwfull[b2], 1); mbar_init(&S->dwempty[b2], kFEpi / 2); }
-    // queue entries: read by the MMA warp and by one group of eight epilogue warps
-    for (int i = 0; i < kFQ; ++i) { mbar_init(&S->qfull[i], 1); mbar_init(&S->qempty[i], 1 + kFEpi / 2); }
+    for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->dwfull[b2], 1); mbar_init(&S->dwempty[b2], kFEpi); }
+    // queue entries: read by the MMA warp and by every epilogue warp
+    for (int i = 0; i < kFQ; ++i) { mbar_init(&S->qfull[i], 1); mbar_init(&S->qempty[i], 1 + kFEpi); }
     S->first_t = -1;
     S->abort = 0;
     fence_barrier_init();
@@ -516,18 +516,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         if (i == 0) S->first_t = t;
         S->tq[qs] = t;
         mbar_arrive(&S->qfull[qs]);
-        if (t < 0) {
-          // a terminator for the other epilogue group (the groups take alternate entries)
-          const uint32_t i2 = i + 1;
-          const int q2 = (int)(i2 % kFQ);
-          if (mbar_wait(&S->qempty[q2], ((i2 / kFQ) & 1) ^ 1, abort, kWaitCycles)) {
-            S->tq[q2] = -1;
-            mbar_arrive(&S->qfull[q2]);
-          } else {
-            record_timeout(status, abort, 90);
-          }
-          break;
-        }
+        if (t < 0) break;
         {
           const int s = wit % kWS;
           const uint32_t ph = (wit / kWS) & 1;
@@ -643,33 +632,32 @@ __global__ void __launch_bounds__(kFThreads, 1)
       mma_commit(&S->dxfull);
     }
   } else {
-    // Two groups of eight warps take alternate units, group g always dW slot
-    // g, so that one group's waits and TMEM loads overlap the other's SR
-    // arithmetic.  Warp (q = warp % 4, sub) of a group updates label row
-    // 32 q + lane and columns 64 sub .. 64 sub + 63 of the slice.
+    // All sixteen warps take every unit: warp (q = warp % 4, sub) updates
+    // label row 32 q + lane and columns 32 sub .. 32 sub + 31 of the slice.
+    // The unit's dW slot (units alternate between two) is released as soon
+    // as the warps have loaded it, so the MMA warp can form the next unit's
+    // dW while this unit's update runs.
     const int q = warp & 3;
-    const int gpb = (warp - 2) >> 3, sub = ((warp - 2) & 7) >> 2;
+    const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;                  // label row of dW; column of d for dX^T
     const float lrs = kFp8 ? lr * (0.00390625f * xscale[1]) : lr;
     const float dx_scale = kFp8 ? 0.00390625f : 1.0f;
     constexpr int kWf = kFp8 ? (kW5 ? 2 : 1) : 0;
-    uint32_t use = 0;                               // this group's units so far
     bool any = false;                               // the CTA took at least one unit
-    for (uint32_t ui = (uint32_t)gpb; !*abort; ui += 2, ++use) {
-      // queue entry ui (the CTA's unit index): this group's next unit
+    for (uint32_t ui = 0; !*abort; ++ui) {
       const int qs = (int)(ui % kFQ);
       if (!mbar_wait(&S->qfull[qs], (ui / kFQ) & 1, abort, kWaitCycles)) { record_timeout(status, abort, 100); break; }
       const int t = S->tq[qs];
-      if (ui == (uint32_t)gpb) any = S->first_t >= 0;
+      if (ui == 0) any = S->first_t >= 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->qempty[qs]);
       if (t < 0) break;
       const int sw = (int)(ui % kWS);
-      const uint32_t db = (uint32_t)gpb;
+      const uint32_t db = ui & 1, use = ui >> 1;
       const int64_t l = (int64_t)t * 128 + row;
-      const int jl = sub * 64;                      // columns jl .. jl + 63 of the 128-column slice
+      const int jl = sub * 32;                      // columns jl .. jl + 31 of the 128-column slice
       const int j0 = D0 + jl;
-      const bool valid = l < L && j0 < d;           // d is a multiple of 64: all 64 columns or none
+      const bool valid = l < L && j0 < d;           // d is a multiple of 64: all 32 columns or none
       // the first draws do not depend on the gradient: form them while the MMAs run
       uint32_t rw[8];
       if (valid) sr_draws16(rk, step, blk_base, l, d, j0, rw);
@@ -677,30 +665,17 @@ __global__ void __launch_bounds__(kFThreads, 1)
       tc_fence_after();
       const uint8_t* wrow = ws + sw * kWSB;
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + 256 + db * 128 + jl;
-      // four 16-column chunks, two register sets: the load of the next chunk
-      // is in flight during the update of this one
       uint32_t ra[16], rb[16];
       tmem_ld16(taddr, ra);
-#pragma unroll
-      for (int c = 0; c < 4; c += 2) {
-        tmem_wait_ld();                                         // chunk c in ra
-        tmem_ld16(taddr + 16 * (c + 1), rb);
-        if (valid) {
-          update16<kWf>(ra, rw, wrow, row, jl + 16 * c, l, d, j0 + 16 * c, lrs, Wglob);
-          sr_draws16(rk, step, blk_base, l, d, j0 + 16 * (c + 1), rw);
-        }
-        tmem_wait_ld();                                         // chunk c + 1 in rb
-        if (c + 2 < 4) {
-          tmem_ld16(taddr + 16 * (c + 2), ra);
-        } else {                                                // the last load from the dW slot
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S->dwempty[db]);
-        }
-        if (valid) {
-          update16<kWf>(rb, rw, wrow, row, jl + 16 * (c + 1), l, d, j0 + 16 * (c + 1), lrs, Wglob);
-          if (c + 2 < 4) sr_draws16(rk, step, blk_base, l, d, j0 + 16 * (c + 2), rw);
-        }
+      tmem_ld16(taddr + 16, rb);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S->dwempty[db]);
+      if (valid) {
+        update16<kWf>(ra, rw, wrow, row, jl, l, d, j0, lrs, Wglob);
+        sr_draws16(rk, step, blk_base, l, d, j0 + 16, rw);
+        update16<kWf>(rb, rw, wrow, row, jl + 16, l, d, j0 + 16, lrs, Wglob);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->wempty[sw]);
