@@ -721,12 +721,15 @@ bool fused_step_supported(const elmo_head* h, int32_t B) {
 // The split of the SMs between the roles follows their measured cost per
 // 128-label tile on B200 at the workloads' shapes (d = 768): role A (Z and G
 // of the tile; two CTAs per tile when B > 128) against role B (dX^T, dW and
-// the SR update of the tile's weights for every d-slice, bound by the
-// epilogue's instruction issue).  E4M3 with two producers per tile: role A
-// 27 % of the SMs; bf16 with two producers 38 %, with one 20 %.
-// ELMO_FUSED_A overrides nA.
+// the SR update of the tile's weights for every d-slice).  Measured optima:
+// E4M3 with two producers per tile 31 % of the SMs for role A (46 of 148; the
+// 3M-label step at 2.53 ms against 2.58 at 44 and 2.67 at 48); bf16 with two
+// producers 27 % (40; the 500K-label step at 0.87 ms against 0.96 at 36 and
+// 0.90 at 44), with one 22 % (the 8.6M-label step at 10.7 ms at 32, 11.2 at 26
+// and 38).  E4M3 with one producer (no workload measured) 19 %, from the same
+// per-tile costs.  ELMO_FUSED_A overrides nA.
 void fused_split(int grid, int nD, int T, int nprod, bool fp8, int* nA, int* nG) {
-  const int pct = fp8 ? 27 : (nprod == 2 ? 38 : 20);
+  const int pct = fp8 ? (nprod == 2 ? 31 : 19) : (nprod == 2 ? 27 : 22);
   int a = (grid * pct + 50) / 100;
   const char* v = getenv("ELMO_FUSED_A");
   if (v && atoi(v) > 0) a = atoi(v);
