@@ -217,10 +217,12 @@ __device__ __forceinline__ uint8_t sr_e4m3(float v, uint32_t k) {
   return (uint8_t)(pack_e4m3x2(0.0f, sr_e4m3_value(v, k)) & 0xFF);
 }
 
-// Four finite fp32 values -> four codes (byte i = value i) by the stochastic
+// Four fp32 values -> four codes (byte i = value i) by the stochastic
 // conversions: values 0 and 1 take the low and high 16-bit draws of w01,
-// values 2 and 3 those of w23.  Saturating.  NaN and infinities are for the
-// per-element functions (a NaN's sign, and E5M2's infinities, are kept there).
+// values 2 and 3 those of w23.  Saturating: E4M3 maps NaN of either sign to
+// 0x7F and +-inf to +-448, +-0 and fp32 denormals to +-0 (checked on B200
+// against the rounding's definition); E5M2's infinities must stay infinite,
+// so E5M2 callers send NaN and infinities to sr_e5m2_code.
 __device__ __forceinline__ uint32_t sr_e4m3x4_hw(float v0, float v1, float v2, float v3, uint32_t w01,
                                                  uint32_t w23) {
   uint32_t a, b;
@@ -244,9 +246,9 @@ __device__ __forceinline__ uint32_t sr_e5m2x4_hw(float v0, float v1, float v2, f
 // Eight values rounded with the eight 16-bit draws of one Philox block (draw
 // e is half e & 1 of word e >> 1).  bf16: add-and-truncate on the fp32 bit
 // pattern (adding 2^16 - 1 - k carries into the first kept bit exactly when
-// k < F, F the 16 discarded bits); E4M3: the stochastic conversion.  A group
-// holding a NaN or an infinity (bf16: or a magnitude of 2^127 or more, where
-// the carry could reach the exponent's top) takes the per-element path.
+// k < F, F the 16 discarded bits); E4M3: the stochastic conversion.  A bf16
+// group holding a NaN, an infinity or a magnitude of 2^127 or more (where the
+// carry could reach the exponent's top) takes the per-element path.
 __device__ __forceinline__ uint4 sr8_bf16(const float (&v)[8], const u32x4& r) {
   const uint32_t w[4] = {r.x, r.y, r.z, r.w};
   float probe = 0.0f;
@@ -268,18 +270,10 @@ __device__ __forceinline__ uint4 sr8_bf16(const float (&v)[8], const u32x4& r) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// E4M3: the stochastic conversion for every value, NaN (0x7F), +-inf
+// (+-448), +-0 and fp32 denormals included (the rounding's own results there).
 __device__ __forceinline__ uint2 sr8_e4m3(const float (&v)[8], const u32x4& r) {
-  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-  float probe = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) probe = __fmaf_rn(v[i], 0.0f, probe);
-  if (probe == 0.0f)
-    return make_uint2(sr_e4m3x4_hw(v[0], v[1], v[2], v[3], w[0], w[1]), sr_e4m3x4_hw(v[4], v[5], v[6], v[7], w[2], w[3]));
-  float o[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) o[e] = sr_e4m3_value(v[e], (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu));
-  return make_uint2(pack_e4m3x2(o[1], o[0]) | (pack_e4m3x2(o[3], o[2]) << 16),
-                    pack_e4m3x2(o[5], o[4]) | (pack_e4m3x2(o[7], o[6]) << 16));
+  return make_uint2(sr_e4m3x4_hw(v[0], v[1], v[2], v[3], r.x, r.y), sr_e4m3x4_hw(v[4], v[5], v[6], v[7], r.z, r.w));
 }
 
 // Stochastic rounding of v onto the OCP E5M2 grid with a 16-bit draw k, as

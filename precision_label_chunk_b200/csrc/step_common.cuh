@@ -273,14 +273,19 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t
 #pragma unroll
   for (int i = 0; i < 16; ++i) vv[i] = __fsub_rn(wv[i], __fmul_rn(lrs, __uint_as_float(r[i])));
   uint32_t wnew[8];
-  // a probe that is not finite when some v is NaN or infinite (8-bit grids:
-  // the sum of 0 v; bf16: the sum of 2 v, which also overflows once some
-  // |v| >= 2^127, where rounding could pass the largest finite value) sends
-  // the group to the exact per-element path
+  // E4M3: the stochastic conversion also gives the rounding's results for
+  // NaN (0x7F, either sign), +-inf (+-448), +-0 and fp32 denormals (+-0), as
+  // checked on B200, so every group takes it.  bf16 and E5M2: a probe that is
+  // not finite when some v is NaN or infinite (E5M2: the sum of 0 v, whose
+  // infinities must stay infinite; bf16: the sum of 2 v, which also overflows
+  // once some |v| >= 2^127, where rounding could pass the largest finite
+  // value) sends the group to the exact per-element path.
   float probe = 0.0f;
+  if (kW != 1) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) probe = __fmaf_rn(vv[i], kW ? 0.0f : 2.0f, probe);
-  if (fabsf(probe) < INFINITY) {
+    for (int i = 0; i < 16; ++i) probe = __fmaf_rn(vv[i], kW ? 0.0f : 2.0f, probe);
+  }
+  if (kW == 1 || fabsf(probe) < INFINITY) {
     if (kW) {
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4)
