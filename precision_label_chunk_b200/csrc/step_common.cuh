@@ -239,8 +239,10 @@ __device__ __forceinline__ void sr_draws16(const PhiloxKeys& rk, uint64_t step, 
 // stochastic conversions to the 8-bit formats apply the same rule to a 16-bit
 // field (sr_e4m3x4_hw / sr_e5m2x4_hw).  A group holding a NaN or an infinity
 // takes the exact per-element path.
-// kW: the weight grid, 0 bf16, 1 E4M3, 2 E5M2.
-template <int kW>
+// kW: the weight grid, 0 bf16, 1 E4M3, 2 E5M2.  kInPlace: the new codes go
+// back into the shared-memory tile where the old ones were read (for a bulk
+// store of the whole tile), else to Wglob[l, j0 ..].
+template <int kW, bool kInPlace = false>
 __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t (&rw)[8],
                                          const uint8_t* __restrict__ wtile, int row, int jl, int64_t l, int32_t d,
                                          int j0, float lrs, void* __restrict__ Wglob) {
@@ -323,9 +325,24 @@ __device__ __forceinline__ void update16(const uint32_t (&r)[16], const uint32_t
       }
     }
   }
-  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(Wglob) + ((size_t)l * d + j0) * (kW ? 1 : 2));
-  dst[0] = make_uint4(wnew[0], wnew[1], wnew[2], wnew[3]);
-  if (!kW) dst[1] = make_uint4(wnew[4], wnew[5], wnew[6], wnew[7]);
+  if (kInPlace) {
+    uint8_t* wt = const_cast<uint8_t*>(wtile);
+    if (kW) {
+      *reinterpret_cast<uint4*>(wt + row * 128 + (((jl >> 4) ^ (row & 7)) << 4)) =
+          make_uint4(wnew[0], wnew[1], wnew[2], wnew[3]);
+    } else {
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        const int c16 = ((jl & 63) >> 3) + v;
+        *reinterpret_cast<uint4*>(wt + (jl >> 6) * kBox + row * 128 + ((c16 ^ (row & 7)) << 4)) =
+            make_uint4(wnew[4 * v], wnew[4 * v + 1], wnew[4 * v + 2], wnew[4 * v + 3]);
+      }
+    }
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(Wglob) + ((size_t)l * d + j0) * (kW ? 1 : 2));
+    dst[0] = make_uint4(wnew[0], wnew[1], wnew[2], wnew[3]);
+    if (!kW) dst[1] = make_uint4(wnew[4], wnew[5], wnew[6], wnew[7]);
+  }
 }
 
 }  // namespace

@@ -458,6 +458,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
   const int g = bid / nD, sl = bid % nD;
   if (g >= nG) return;                                        // spare CTA
   constexpr int kWS = kFp8 ? 4 : 2;
+  // bf16: the epilogue writes the new weights back into the W slot and the
+  // TMA warp stores the slot (measured: 8.6M-label step 10.5 -> 8.9 ms, 500K
+  // 0.86 -> 0.69 ms); E4M3: each thread stores its 16 codes (1 to 2 % faster
+  // there, its slices being half as wide)
+  constexpr bool kWB = !kFp8;
   constexpr uint32_t kWSB = kFp8 ? kBox : 2 * kBox;
   constexpr int kBoxCols = 128 / kEl;                         // elements per 128-byte box row
   constexpr int kK = kFp8 ? 32 : 16;                          // MMA K
@@ -473,9 +478,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&S->xfull, 1);
     mbar_init(&S->dxfull, 1);
-    // a W slot is free once its group's epilogue is done with it and the
-    // unit's dX^T MMAs (which read it after dW is committed) have completed
-    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kFEpi + 1); }
+    // a W slot holds the unit's new weights once all sixteen epilogue warps
+    // have written them back (the unit's MMAs, which read the old ones, have
+    // completed before the epilogue starts); the TMA warp then stores it
+    // (E4M3: free once the epilogue is done with it and the unit's dX^T MMAs
+    // have completed: an mma_commit counts too)
+    for (int s = 0; s < kWS; ++s) { mbar_init(&S->wfull[s], 1); mbar_init(&S->wempty[s], kWB ? kFEpi : kFEpi + 1); }
     for (int s = 0; s < kFGSlots; ++s) { mbar_init(&S->gfull[s], 1); mbar_init(&S->gempty[s], 1); }
     for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&S->dwfull[b2], 1); mbar_init(&S->dwempty[b2], kFEpi); }
     // queue entries: read by the MMA warp and by every epilogue warp
@@ -503,6 +511,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
       // take the next, pass it to the MMA warp and the epilogue, then load
       // its W slice and copy its G tile once role A has published it
       uint32_t wit = 0, git = 0;
+      int slot_t[kWS];                                        // the tile whose W slice a slot holds
+      for (int s = 0; s < kWS; ++s) slot_t[s] = -1;
+      // the new weights of the tile that slot s held go back to W with one
+      // bulk tensor store per 128-byte column box (rows past L are clipped)
+      auto store_slot = [&](int s) {
+        for (int qq = 0; qq < 128 / kBoxCols; ++qq)
+          if (D0 + qq * kBoxCols < d) tma_store_2d(&tmWb, ws + s * kWSB + qq * kBox, D0 + qq * kBoxCols, slot_t[s] * 128);
+        bulk_commit_group();
+      };
       int t_next = atomicAdd(sched + 2 + sl, 1);              // taken one unit ahead
       for (uint32_t i = 0;; ++i) {
         const int qs = (int)(i % kFQ);
@@ -522,6 +539,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
           const uint32_t ph = (wit / kWS) & 1;
           ++wit;
           if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) { record_timeout(status, abort, 91); break; }
+          if (kWB && slot_t[s] >= 0) {
+            store_slot(s);
+            bulk_wait_read_all();                             // the store has read the slot
+          }
+          slot_t[s] = t;
           mbar_arrive_expect_tx(&S->wfull[s], (uint32_t)nb * kBox);
           for (int qq = 0; qq < 128 / kBoxCols; ++qq)
             if (D0 + qq * kBoxCols < d) tma_load_2d(ws + s * kWSB + qq * kBox, &tmWb, &S->wfull[s], D0 + qq * kBoxCols, t * 128);
@@ -547,6 +569,14 @@ __global__ void __launch_bounds__(kFThreads, 1)
         }
         if (stop) break;
       }
+      // the last unit of each slot: its epilogue's completion is use
+      // (n / kWS) of the slot's barrier, n the unit's index
+      for (uint32_t n = wit > (uint32_t)kWS ? wit - kWS : 0u; kWB && n < wit && !*abort; ++n) {
+        const int s = (int)(n % kWS);
+        if (!mbar_wait(&S->wempty[s], (n / kWS) & 1, abort, kWaitCycles)) { record_timeout(status, abort, 91); break; }
+        store_slot(s);
+      }
+      bulk_wait_all();
     }
   } else if (warp == 1) {
     if (elect_one()) {
@@ -576,8 +606,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
         const uint32_t wa = smem_u32(ws + sw * kWSB);
         const uint32_t dwcol = tmem + 256 + db * 128;
         bool stop = false;
-        // dW first (the epilogue waits for it), then dX^T; the G parts (at
-        // most two) stay in their slots until both are issued
+        // dW, then dX^T (which reads the old W in the slot).  bf16: the
+        // epilogue waits for both, since it writes the new W into the same
+        // slot; E4M3: for dW only.  The G parts (at most two) stay in their
+        // slots until both are issued
         int sgs[2] = {0, 0};
         for (int p = 0; p < nparts; ++p) {
           const int sg = git % kFGSlots;
@@ -606,7 +638,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
           }
         }
         if (stop) break;
-        mma_commit(&S->dwfull[db]);
+        if (!kWB) mma_commit(&S->dwfull[db]);
         for (int p = 0; p < nparts; ++p) {
           const uint32_t ga = smem_u32(gs + sgs[p] * kFGSlotBytes);
           const int np = min(kPart, Bp - p * kPart);
@@ -626,7 +658,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
           }
           mma_commit(&S->gempty[sgs[p]]);
         }
-        mma_commit(&S->wempty[sw]);
+        mma_commit(kWB ? &S->dwfull[db] : &S->wempty[sw]);
         first = false;
       }
       mma_commit(&S->dxfull);
@@ -658,9 +690,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
       const int jl = sub * 32;                      // columns jl .. jl + 31 of the 128-column slice
       const int j0 = D0 + jl;
       const bool valid = l < L && j0 < d;           // d is a multiple of 64: all 32 columns or none
-      // the first draws do not depend on the gradient: form them while the MMAs run
-      uint32_t rw[8];
-      if (valid) sr_draws16(rk, step, blk_base, l, d, j0, rw);
+      // the draws do not depend on the gradient: form them while the MMAs run
+      // (bf16: both chunks' four Philox blocks here, measured 4 % faster on the
+      // 8.6M-label step; E4M3: the second chunk's after the first update,
+      // 9 % faster on the 3M-label step)
+      uint32_t rw[8], rw1[8];
+      if (valid) {
+        sr_draws16(rk, step, blk_base, l, d, j0, rw);
+        if (!kFp8) sr_draws16(rk, step, blk_base, l, d, j0 + 16, rw1);
+      }
       if (!mbar_wait(&S->dwfull[db], use & 1, abort, kWaitCycles)) { record_timeout(status, abort, 98); break; }
       tc_fence_after();
       const uint8_t* wrow = ws + sw * kWSB;
@@ -673,9 +711,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->dwempty[db]);
       if (valid) {
-        update16<kWf>(ra, rw, wrow, row, jl, l, d, j0, lrs, Wglob);
-        sr_draws16(rk, step, blk_base, l, d, j0 + 16, rw);
-        update16<kWf>(rb, rw, wrow, row, jl + 16, l, d, j0 + 16, lrs, Wglob);
+        // bf16: the new codes go back into the slot, in place of the old ones
+        update16<kWf, kWB>(ra, rw, wrow, row, jl, l, d, j0, lrs, Wglob);
+        if (kFp8) sr_draws16(rk, step, blk_base, l, d, j0 + 16, rw1);
+        update16<kWf, kWB>(rb, rw1, wrow, row, jl + 16, l, d, j0 + 16, lrs, Wglob);
+        if (kWB) fence_proxy_async_smem();            // visible to the bulk store that reads the slot
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->wempty[sw]);
@@ -723,13 +763,13 @@ bool fused_step_supported(const elmo_head* h, int32_t B) {
 // of the tile; two CTAs per tile when B > 128) against role B (dX^T, dW and
 // the SR update of the tile's weights for every d-slice).  Measured optima:
 // E4M3 with two producers per tile 31 % of the SMs for role A (46 of 148; the
-// 3M-label step at 2.53 ms against 2.58 at 44 and 2.67 at 48); bf16 with two
-// producers 27 % (40; the 500K-label step at 0.87 ms against 0.96 at 36 and
-// 0.90 at 44), with one 22 % (the 8.6M-label step at 10.7 ms at 32, 11.2 at 26
-// and 38).  E4M3 with one producer (no workload measured) 19 %, from the same
+// 3M-label step at 2.48 ms against 2.55 at 44 and 2.63 at 48); bf16 with two
+// producers 35 % (52; the 500K-label step at 0.70 ms against 0.72 at 48 and
+// 0.75 at 56), with one 23 % (34; the 8.6M-label step at 8.8 ms, 9.1 at 32,
+// 9.3 at 38).  E4M3 with one producer (no workload measured) 19 %, from the same
 // per-tile costs.  ELMO_FUSED_A overrides nA.
 void fused_split(int grid, int nD, int T, int nprod, bool fp8, int* nA, int* nG) {
-  const int pct = fp8 ? (nprod == 2 ? 31 : 19) : (nprod == 2 ? 27 : 22);
+  const int pct = fp8 ? (nprod == 2 ? 31 : 19) : (nprod == 2 ? 35 : 23);
   int a = (grid * pct + 50) / 100;
   const char* v = getenv("ELMO_FUSED_A");
   if (v && atoi(v) > 0) a = atoi(v);
