@@ -29,7 +29,10 @@ def test_committed_summaries_match_their_sources():
     """Every summary the bench reads belongs to the current kernel code (else
     its traffic would be reported as null)."""
     bench = _bench()
-    for kernel, workload in [("kahan_sgd_vec", "kahan_sgd")]:
+    for kernel, workload in [("kahan_sgd_vec", "kahan_sgd"), ("sr_round_vec", "sr_round"),
+                             ("step_fused", "product3m_fp8"), ("step_fused", "product3m_fp8_ge5m2"),
+                             ("step_fused", "product3m_e5m2"), ("step_fused", "text500k_bf16"),
+                             ("step_fused", "keyword8m6_bf16"), ("topk_screen_tc", "topk5_3m_fp8")]:
         tr = bench.profiled_traffic(kernel, workload)
         assert tr is not None, f"profiles/{kernel}_{workload}.md does not match its source"
         assert tr["bytes"] > 0 and tr["labels"] > 0
