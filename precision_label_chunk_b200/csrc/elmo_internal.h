@@ -100,6 +100,8 @@ cudaError_t launch_prep_step(elmo_head* h, const int32_t* rowptr, const int32_t*
 // x box_rows, 128-byte swizzle, zero fill outside the tensor.
 cudaError_t make_tma_map_2d(CUtensorMap_st* m, const void* ptr, int elem_bytes, uint64_t cols, uint64_t rows,
                             uint64_t row_stride_elems, uint32_t box_rows);
+cudaError_t make_tma_map_kb3d(CUtensorMap_st* m, const void* ptr, int elem_bytes, uint64_t cols, uint64_t rows,
+                              uint32_t box_rows, uint32_t box_kb);
 int32_t padded_batch(int32_t B, bool fp8);
 cudaError_t launch_wait_check(long long limit_cycles, int32_t* status, cudaStream_t s);
 // pdl: launch programmatically dependent on the previous kernel in the stream,

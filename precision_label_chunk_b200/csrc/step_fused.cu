@@ -39,6 +39,7 @@
 // range-by-range kernels of step_tc.cu.
 #include <stdlib.h>
 
+#include <algorithm>
 #include <utility>
 
 #include "step_common.cuh"
@@ -48,7 +49,7 @@ namespace {
 
 constexpr int kFThreads = 576;              // warp 0 TMA, warp 1 MMA + TMEM, warps 2-17 epilogue
 constexpr int kFEpi = 16;
-constexpr int kFStagesA = 24;               // role A: most W k-block stages (bf16: 24 x 8 KB, E4M3: 12 x 16 KB)
+constexpr int kFStagesA = 24;               // role A: most W ring stages (4 of 48 KB are used)
 constexpr uint32_t kFRingA = 192 * 1024;    // role A: bytes of the W ring
 // role A: a 128-label tile is two halves of kN = 64 labels (the MMA's N),
 // each accumulated in its own TMEM slot of 64 columns after one M-block of X
@@ -59,7 +60,14 @@ template <int kFp8> struct RoleA {
   static constexpr int kHalves = 128 / kN;
   static constexpr int kGroups = kFp8 ? 2 : 1;
   static constexpr int kSlots = kGroups * kHalves;
-  static constexpr uint32_t kStage = (uint32_t)kN * 128;
+  // a ring stage holds up to kKbs 128-byte k-blocks of a 64-label half
+  // (48 KB): one TMA request per stage where the W rows divide into whole
+  // k-blocks (a 3-D box), else one 2-D box per k-block.  The TMA engine's
+  // rate follows its request count: 8 KB requests streamed about 25 bytes
+  // per clock per SM on B200, 48 KB requests 75 (the HBM bound at 46 SMs).
+  static constexpr int kKbs = 6;
+  static constexpr uint32_t kKb = (uint32_t)kN * 128;       // one k-block of the half
+  static constexpr uint32_t kStage = kKb * kKbs;
   static constexpr int kStages = (int)(kFRingA / kStage);
   static constexpr uint32_t kAcc = kFp8 ? 256 : 384;
 };
@@ -136,7 +144,8 @@ __device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t target, v
 
 template <int kFp8, int kG5, int kW5 = 0>
 __global__ void __launch_bounds__(kFThreads, 1)
-    step_fused(const __grid_constant__ CUtensorMap tmWa, const __grid_constant__ CUtensorMap tmWb,
+    step_fused(const __grid_constant__ CUtensorMap tmWa, const __grid_constant__ CUtensorMap tmWa3, int32_t wa3,
+               const __grid_constant__ CUtensorMap tmWb,
                const __grid_constant__ CUtensorMap tmX, void* __restrict__ Wglob, int64_t L, int32_t d, int32_t B,
                int32_t Bp, const uint8_t* __restrict__ xop, const uint32_t* __restrict__ keys,
                const int32_t* __restrict__ tile_ptr, const float* __restrict__ xscale, uint8_t* __restrict__ gring,
@@ -159,6 +168,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     volatile int* abort = &S->abort;
     const int kbe = kFp8 ? 128 : 64;                          // elements of one 128-byte k-block
     const int nkb = (d + kbe - 1) / kbe;
+    const int kbs = nkb < RA::kKbs ? nkb : RA::kKbs;          // k-blocks of one 3-D box
     const uint32_t opcols = (uint32_t)nkb * 32;               // TMEM columns of one M-block of X
     // Producers of a tile: one CTA holds the single M-block of X (up to 128
     // samples), or two neighbouring CTAs hold one M-block each and write
@@ -253,12 +263,16 @@ __global__ void __launch_bounds__(kFThreads, 1)
           if (amb == 0) {
             const int tp = t + 2 * (nA / nprod);
             if (tp < T)
-              for (int hf = 0; hf < RA::kHalves; ++hf)
-                for (int kb = 0; kb < nkb; ++kb) tma_prefetch_l2(&tmWa, kb * kbe, tp * 128 + hf * RA::kN);
+              for (int hf = 0; hf < RA::kHalves; ++hf) {
+                if (wa3)
+                  for (int k0 = 0; k0 < nkb; k0 += RA::kKbs) tma_prefetch_l2_3d(&tmWa3, 0, tp * 128 + hf * RA::kN, k0);
+                else
+                  for (int kb = 0; kb < nkb; ++kb) tma_prefetch_l2(&tmWa, kb * kbe, tp * 128 + hf * RA::kN);
+              }
           }
           bool stop = false;
           for (int hf = 0; hf < RA::kHalves && !stop; ++hf) {
-            for (int kb = 0; kb < nkb; ++kb, ++it) {
+            for (int k0 = 0; k0 < nkb; k0 += RA::kKbs, ++it) {
               const int s = (int)(it % RA::kStages);
               const uint32_t ph = (it / RA::kStages) & 1;
               if (!mbar_wait(&S->wempty[s], ph ^ 1, abort, kWaitCycles)) {
@@ -266,8 +280,17 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 stop = true;
                 break;
               }
-              mbar_arrive_expect_tx(&S->wfull[s], RA::kStage);
-              tma_load_2d(ring + s * RA::kStage, &tmWa, &S->wfull[s], kb * kbe, t * 128 + hf * RA::kN);
+              const int nk = min(RA::kKbs, nkb - k0);        // k-blocks in this stage
+              if (wa3) {
+                // one box of kbs k-blocks (past the last k-block: zero fill, still counted)
+                mbar_arrive_expect_tx(&S->wfull[s], (uint32_t)kbs * RA::kKb);
+                tma_load_3d(ring + s * RA::kStage, &tmWa3, &S->wfull[s], 0, t * 128 + hf * RA::kN, k0);
+              } else {
+                mbar_arrive_expect_tx(&S->wfull[s], (uint32_t)nk * RA::kKb);
+                for (int j = 0; j < nk; ++j)
+                  tma_load_2d(ring + s * RA::kStage + j * RA::kKb, &tmWa, &S->wfull[s], (k0 + j) * kbe,
+                              t * 128 + hf * RA::kN);
+              }
             }
           }
           if (stop) break;
@@ -296,19 +319,23 @@ __global__ void __launch_bounds__(kFThreads, 1)
             // descriptors advance by constants (the start address field counts
             // 16-byte units): few instructions per MMA for this thread, which
             // shares its scheduler with four busy epilogue warps
-            for (int kb = 0; kb < nkb; ++kb, ++it) {
+            for (int k0 = 0; k0 < nkb; k0 += RA::kKbs, ++it) {
               const int s = (int)(it % RA::kStages);
               if (!mbar_wait(&S->wfull[s], (it / RA::kStages) & 1, abort, kWaitCycles)) {
                 record_timeout(status, abort, 84);
                 break;
               }
               tc_fence_after();
-              const uint64_t bd = bdesc0 + (uint64_t)((uint32_t)s * (RA::kStage >> 4));
-              const uint32_t aa = tmem + (uint32_t)kb * 32;
+              const int k1 = min(nkb, k0 + RA::kKbs);
+              for (int kb = k0; kb < k1; ++kb) {
+                // k-block kb - k0 of the stage: kKb bytes further in
+                const uint64_t bd = bdesc0 + (uint64_t)((uint32_t)s * (RA::kStage >> 4) + (uint32_t)(kb - k0) * (RA::kKb >> 4));
+                const uint32_t aa = tmem + (uint32_t)kb * 32;
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                if (kFp8) mma_e4m3_ts(dcol, aa + (uint32_t)k * 8, bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
-                else mma_bf16_ts(dcol, aa + (uint32_t)k * 8, bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
+                for (int k = 0; k < 4; ++k) {
+                  if (kFp8) mma_e4m3_ts(dcol, aa + (uint32_t)k * 8, bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
+                  else mma_bf16_ts(dcol, aa + (uint32_t)k * 8, bd + (uint64_t)(k * 2), idesc, (kb | k) != 0);
+                }
               }
               mma_commit(&S->wempty[s]);
             }
@@ -793,10 +820,21 @@ cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float 
   int nA = 0, nG = 0;
   fused_split(h->num_sms, nD, T, Bp > 128 ? 2 : 1, fp8, &nA, &nG);
   const int grid = nA + nG * nD;
-  CUtensorMap tmWa, tmWb, tmX;
+  CUtensorMap tmWa, tmWa3, tmWb, tmX;
   cudaError_t e = make_tma_map_2d(&tmWa, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d,
                                   fp8 ? RoleA<1>::kN : RoleA<0>::kN);
   if (e != cudaSuccess) return e;
+  // role A's 3-D view needs rows of whole 128-byte k-blocks (else the view
+  // would run into the next row): then one request per ring stage
+  const int nkb = (int)((h->d * eb + 127) / 128);
+  const int wa3 = (h->d * eb) % 128 == 0 ? 1 : 0;
+  if (wa3) {
+    e = make_tma_map_kb3d(&tmWa3, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, RoleA<1>::kN,
+                          (uint32_t)std::min(nkb, RoleA<1>::kKbs));
+    if (e != cudaSuccess) return e;
+  } else {
+    tmWa3 = tmWa;                                   // not read
+  }
   e = make_tma_map_2d(&tmWb, h->W, eb, (uint64_t)h->d, (uint64_t)h->L, (uint64_t)h->d, 128);
   if (e != cudaSuccess) return e;
   e = make_tma_map_2d(&tmX, fp8 ? static_cast<const void*>(h->xq) : static_cast<const void*>(X), eb, (uint64_t)h->d,
@@ -820,7 +858,7 @@ cudaError_t launch_step_fused(elmo_head* h, const uint16_t* X, int32_t B, float 
   at[0].val.cooperative = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tmWa, tmWb, tmX, h->W, h->L, h->d, B, Bp, xop, (const uint32_t*)h->keys,
+  return cudaLaunchKernelEx(&cfg, kern, tmWa, tmWa3, wa3, tmWb, tmX, h->W, h->L, h->d, B, Bp, xop, (const uint32_t*)h->keys,
                             (const int32_t*)h->tile_ptr, (const float*)h->xscale, static_cast<uint8_t*>(h->ring),
                             h->ring_tiles, h->ring_flags, h->ring_flags + h->ring_tiles,
                             h->ring_flags + 2 * h->ring_tiles, nA, nG, lr, philox_keys(seed), step,

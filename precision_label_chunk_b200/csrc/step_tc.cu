@@ -911,6 +911,26 @@ cudaError_t make_tma_map_2d(CUtensorMap* m, const void* ptr, int elem_bytes, uin
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// A row-major matrix seen as (128-byte k-block column, row, k-block): box
+// {128 bytes, box_rows, box_kb} lands in shared memory as box_kb blocks of
+// box_rows x 128 bytes, each in the 128B-swizzled K-major operand layout.
+// One request per box (the W stream's rate follows the request count).
+cudaError_t make_tma_map_kb3d(CUtensorMap* m, const void* ptr, int elem_bytes, uint64_t cols, uint64_t rows,
+                              uint32_t box_rows, uint32_t box_kb) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const uint64_t kbe = 128 / elem_bytes;                       // elements per k-block
+  const cuuint64_t dims[3] = {kbe, rows, (cols + kbe - 1) / kbe};
+  const cuuint64_t strides[2] = {cols * (uint64_t)elem_bytes, 128};
+  const cuuint32_t box[3] = {(cuuint32_t)kbe, box_rows, box_kb};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                        const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // Samples are padded to whole 128-byte swizzle atoms of the operand type
 // (64 bf16 or 128 E4M3 values): padded rows of X are zero-filled by TMA and
 // the padded gradient entries are written as 0.
