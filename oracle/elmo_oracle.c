@@ -30,8 +30,10 @@
  *   - SR(v): v on the grid stays; otherwise with grid neighbours lo < v < hi
  *     and f = (v - lo) / (hi - lo), return hi iff k < floor(2^16 f): the draw
  *     is added to the first 16 bits of the discarded fraction and the sum
- *     truncated (exactly unbiased on bf16, whose fraction has 16 bits; on the
- *     8-bit grids P(hi) = floor(2^16 f) / 2^16), on magnitudes (sign restored);
+ *     truncated; equivalently hi iff u <= f for u = (k + 1) / 2^16 on the
+ *     16-bit grid of (0, 1] (exactly unbiased on bf16, whose fraction has 16
+ *     bits; on the 8-bit grids P(hi) = floor(2^16 f) / 2^16), on magnitudes
+ *     (sign restored);
  *     NaN -> canonical NaN (bf16 0x7FC0, E4M3 0x7F); E4M3: |v| >= 448 and
  *     +-inf -> +-448; bf16: finite |v| above the largest finite -> largest
  *     finite, +-inf stays +-inf;
