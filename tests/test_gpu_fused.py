@@ -62,3 +62,25 @@ def test_fused_step_special_weights(orc):
     b = _run(elmo, W, w, 1, fused=True)[0][0]
     bad = np.argwhere(a.view(np.uint16) != b.view(np.uint16))
     assert bad.size == 0, f"{len(bad)} weights differ: first {bad[:10].tolist()}"
+
+
+@pytest.mark.parametrize("dtype,B,split", [("fp8", 256, "2"), ("fp8", 256, "140"), ("bf16", 128, "1"),
+                                           ("bf16", 256, "142"), ("fp8", 96, "3")])
+def test_fused_step_extreme_role_splits(orc, dtype, B, split, monkeypatch):
+    """The dynamic tile queues and the ring under extreme splits of the SMs:
+    one or two producer CTAs against all the rest, and almost every SM a
+    producer (the split is clamped to leave one CTA per d-slice); the weights
+    must not depend on it."""
+    need_gpu()
+    import precision_label_chunk_b200 as elmo
+    w = workload("tiny", dtype=dtype, L=20000, d=256, B=B)
+    W = make_W_bf16(w) if dtype == "bf16" else orc.sr_round(make_W_f32(w), "fp8", 0, 2**64 - 1)
+    a = _run(elmo, W, w, 2, fused=False)
+    monkeypatch.setenv("ELMO_FUSED_A", split)
+    b = _run(elmo, W, w, 2, fused=True)
+    for s, ((wa, xa), (wb, xb)) in enumerate(zip(a, b)):
+        assert np.array_equal(wa, wb), f"step {s}: {int((wa != wb).sum())} weights differ"
+        # dX sums 20,000 labels' terms in an order that follows the split: fp32
+        # reordering only, well inside 1e-4 of the rms
+        rms = float(np.sqrt(np.mean(xb.astype(np.float64) ** 2)))
+        assert np.allclose(xa, xb, rtol=1e-4, atol=1e-4 * rms), f"step {s}: dX differs"
