@@ -36,7 +36,10 @@ def _run(elmo, W, w, steps, fused, specials=None):
                                          ("bf16", 700, 768, 256), ("fp8", 1000, 768, 256), ("bf16", 900, 256, 100),
                                          # rows of a partial 128-byte k-block (E4M3 d = 704: one 2-D box per
                                          # k-block) and a last ring stage past the k-blocks (bf16 d = 640)
-                                         ("fp8", 900, 704, 256), ("bf16", 800, 640, 128)])
+                                         ("fp8", 900, 704, 256), ("bf16", 800, 640, 128),
+                                         # bf16 with a last d-slice of 64 columns (one box in the W
+                                         # slot the bulk store writes back)
+                                         ("bf16", 700, 704, 64)])
 def test_fused_step_matches_range_kernels(orc, dtype, L, d, B):
     need_gpu()
     import precision_label_chunk_b200 as elmo
